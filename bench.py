@@ -1,0 +1,353 @@
+"""Benchmark of the fused sharded optimizer step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = zero_step over the whole workload: the ring reduce-scatter of every bucket
+fused with the unscale + AdamW + fp16 update (and, for ZeRO-3, the all-gather of every
+gather unit), with inputs resident in HBM.  With N GPUs every GPU runs its own replica of
+the workload (the simulated ranks all live in one GPU's memory, so nothing is exchanged
+between GPUs); the value is the total over GPUs, timed as the max over ranks.
+
+--impl reference times the CPU oracle on a bounded sample of the same workload (rank 0
+only; other ranks exit without work).
+"""
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "params updated/sec per zero_step and achieved HBM GB/s vs peak (1×B200)"
+UNIT = "params/s"
+DEFAULT_WORKLOAD = "flat1p3b_n4_zero1"
+FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "fused_step_flat1p3b_n4.md")
+KERNEL_SOURCE = os.path.join(ROOT, "zero_sharded_optimizer_ring_b200", "csrc", "kernels.cu")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=4)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--kernel", type=int, default=0, help="fused kernel: 0 auto, 1 register, 2 bulk")
+    ap.add_argument("--psi", type=int, default=0,
+                    help="flat workloads only: run the same shape with this many parameters "
+                         "(small cases for profiler captures; not a bench line)")
+    a = ap.parse_args()
+    if a.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    return a
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)), int(os.environ.get("WORLD_SIZE", 1))
+
+
+def ideal_bytes_per_param(wl):
+    # grads 2N read; master, m, v read + write 24; fp16 write 2; ZeRO-3 gather 2 + 2
+    return 2 * wl.n_ranks + 24 + 2 + (4 if wl.stage == 3 else 0)
+
+
+def fused_bytes_per_param(wl):
+    return 2 * wl.n_ranks + 24 + 2
+
+
+def hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        return float(json.load(open(p))["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def profiled_traffic(workload):
+    """dram bytes per parameter of the fused kernel from the committed ncu summary, if
+    it was taken on this workload with the current kernel source; else None."""
+    try:
+        text = open(PROFILE_SUMMARY).read()
+        sha = hashlib.sha256(open(KERNEL_SOURCE, "rb").read()).hexdigest()[:16]
+        m_sha = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
+        m_wl = re.search(r"workload:\s*(\S+)", text)
+        m_tr = re.search(r"dram_bytes_per_param:\s*([0-9.]+)", text)
+        if m_sha and m_tr and m_wl and m_sha.group(1) == sha and m_wl.group(1) == workload:
+            return float(m_tr.group(1))
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = str(gpu_index)
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                       "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except Exception:
+            self.p.kill()
+        self.f.flush()
+        rows = [r.split(",") for r in open(self.f.name).read().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        rows = [[c.strip() for c in r] for r in rows if len(r) >= 9 and r[0].strip() == self.gpu]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[j] for r in rows for j in range(4) if r[5 + j].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def workload_config(wl, world):
+    return {"workload": wl.name, "description": wl.description, "psi": wl.psi, "n_ranks_simulated": wl.n_ranks,
+            "zero_stage": wl.stage, "bucket_elems": wl.bucket_elems, "loss_scale": wl.loss_scale,
+            "inputs": "seeded synthetic (Philox4x32-10), resident in HBM",
+            "l2": "working set far above the 126 MB L2; no flush needed",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU (ranks simulated in HBM)"}
+
+
+# ---------------------------------------------------------------- CPU oracle sample
+
+def oracle_sample_run(wl, psi_s, steps=1):
+    """Run the oracle on the first psi_s parameters of the workload (same N, stage, input
+    distributions, hyper-parameters); returns seconds spent in the oracle."""
+    import oracle
+    import seeded_inputs as si
+    from oracle.layout import make_layout
+    B = wl.bucket_elems if wl.bucket_elems > 0 else 0
+    lay = make_layout([psi_s], wl.n_ranks, B, wl.pad_align)
+    P = lay.padded
+    g = si.fill_grads(wl.n_ranks, P, psi_s, wl.seed, wl.grad_sigma, wl.loss_scale, wl.heavy_frac, wl.heavy_mult)
+    master = si.fill_f32(P, psi_s, wl.seed, si.STREAM_MASTER, wl.master_sigma)
+    m = si.fill_f32(P, psi_s, wl.seed, si.STREAM_M, wl.m_sigma) if wl.m_sigma else np.zeros(P, np.float32)
+    v = si.fill_f32(P, psi_s, wl.seed, si.STREAM_V, wl.v_sigma, True) if wl.v_sigma else np.zeros(P, np.float32)
+    hp = oracle.Hyper(wl.lr, wl.beta1, wl.beta2, wl.eps, wl.weight_decay, wl.loss_scale)
+    t0 = time.perf_counter()
+    oracle.run_steps(lay, wl.stage, g, master, m, v, hp, steps)
+    return time.perf_counter() - t0
+
+
+def size_sample(wl, seconds):
+    """Largest power-of-two sample whose one-step oracle run fits `seconds`."""
+    psi_s = 1 << 16
+    t = oracle_sample_run(wl, psi_s)
+    while t * 2 < seconds and psi_s < (1 << 27):
+        psi_s *= 2
+        t = t * 2
+    return psi_s
+
+
+def cpu_baseline(wl, seconds):
+    psi_s = size_sample(wl, seconds)
+    t = oracle_sample_run(wl, psi_s)
+    return {"value": psi_s / t, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"first {psi_s} parameters of {wl.name} (same N={wl.n_ranks}, stage {wl.stage}, "
+                      f"inputs, AdamW), one step, single-threaded C oracle, {t:.1f} s"}
+
+
+def run_reference(a, wl):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return
+    per_step = 120.0 / (a.steps + a.warmup)
+    psi_s = size_sample(wl, per_step)
+    for _ in range(a.warmup):
+        oracle_sample_run(wl, psi_s)
+    ts = [oracle_sample_run(wl, psi_s) for _ in range(a.steps)]
+    t = sum(ts) / len(ts)
+    value = psi_s / t
+    sample = (f"each step: first {psi_s} parameters of {wl.name} (same N={wl.n_ranks}, stage {wl.stage}, inputs, "
+              f"AdamW), single-threaded C oracle")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": a.gpus, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": workload_config(wl, 1),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+# ---------------------------------------------------------------- the GPU arm
+
+def run_ours(a, wl):
+    import torch
+    import torch.distributed as dist
+    import seeded_inputs as si
+    import zero_sharded_optimizer_ring_b200 as zs
+
+    rank, local, world = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier(device_ids=[local])
+        torch.cuda.synchronize()
+
+    lay = zs.Layout(list(wl.tensors), wl.n_ranks, wl.stage, wl.bucket_elems, wl.pad_align, list(wl.units))
+    lay.to_device()
+    if a.kernel:
+        lay.set_impl(a.kernel)
+    P, psi, N = lay.padded, lay.psi, wl.n_ranks
+    g = torch.empty((N, P), dtype=torch.int16, device="cuda")
+    si.fill_grads_cuda(g, psi, wl.seed, wl.grad_sigma, wl.loss_scale, wl.heavy_frac, wl.heavy_mult)
+    master = torch.empty(P, dtype=torch.float32, device="cuda")
+    si.fill_f32_cuda(master, psi, wl.seed, si.STREAM_MASTER, wl.master_sigma)
+    m = torch.zeros(P, dtype=torch.float32, device="cuda")
+    v = torch.zeros(P, dtype=torch.float32, device="cuda")
+    if wl.m_sigma:
+        si.fill_f32_cuda(m, psi, wl.seed, si.STREAM_M, wl.m_sigma)
+    if wl.v_sigma:
+        si.fill_f32_cuda(v, psi, wl.seed, si.STREAM_V, wl.v_sigma, absval=True)
+    p16_full = torch.zeros(P, dtype=torch.int16, device="cuda")
+    p16_shard = torch.zeros(P, dtype=torch.int16, device="cuda") if wl.stage == 3 else None
+    nonfinite = torch.zeros(max(1, lay.n_buckets), dtype=torch.int32, device="cuda")
+
+    def hp(t):
+        return zs.AdamW(wl.lr, wl.beta1, wl.beta2, wl.eps, wl.weight_decay, wl.loss_scale, t)
+
+    t = 0
+    for _ in range(a.warmup):
+        t += 1
+        zs.step(lay, g, master, m, v, p16_shard, p16_full, hp(t), nonfinite=nonfinite)
+    zs.get_error(lay)
+
+    K = a.steps
+    ev = [{k: torch.cuda.Event(enable_timing=True) for k in ("update_begin", "update_end", "gather_begin", "gather_end")}
+          for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    time.sleep(0.3)
+    barrier()
+    start.record()
+    for i in range(K):
+        t += 1
+        zs.step(lay, g, master, m, v, p16_shard, p16_full, hp(t), nonfinite=nonfinite, events=ev[i])
+    end.record()
+    barrier()
+    clocks = sampler.stop() if sampler else None
+    zs.get_error(lay)
+    ms = max_over_ranks(start.elapsed_time(end) / K)
+    upd_ms = max_over_ranks(sum(e["update_begin"].elapsed_time(e["update_end"]) for e in ev) / K)
+    gat_ms = None
+    if wl.stage == 3:
+        gat_ms = max_over_ranks(sum(e["gather_begin"].elapsed_time(e["gather_end"]) for e in ev) / K)
+    launches_per_step = 2 if wl.stage == 3 else 1
+
+    # end to end through the host-buffer entry point: gradients from pinned host memory
+    # in, fp16 parameters to pinned host memory out, every step
+    e2e = None
+    if a.e2e_steps > 0:
+        del g
+        torch.cuda.empty_cache()
+        g_host = torch.empty((N, P), dtype=torch.int16).pin_memory()
+        ge = torch.empty((N, P), dtype=torch.int16, device="cuda")
+        si.fill_grads_cuda(ge, psi, wl.seed, wl.grad_sigma, wl.loss_scale, wl.heavy_frac, wl.heavy_mult)
+        g_host.copy_(ge)
+        p16_host = torch.empty(P, dtype=torch.int16).pin_memory()
+        t += 1
+        zs.step_host(lay, g_host, ge, master, m, v, p16_shard, p16_full, p16_host, hp(t))
+        barrier()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record()
+        for _ in range(a.e2e_steps):
+            t += 1
+            zs.step_host(lay, g_host, ge, master, m, v, p16_shard, p16_full, p16_host, hp(t))
+        e2.record()
+        barrier()
+        e2e_ms = max_over_ranks(s2.elapsed_time(e2) / a.e2e_steps)
+        e2e = {"value": psi * world / (e2e_ms / 1e3), "unit": UNIT, "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": 2 * N * P, "d2h_bytes_per_step": 2 * P,
+               "steps": a.e2e_steps, "path": "zero_step_host (pinned host grads in, fp16 params out)"}
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peak, peak_kind = hbm_peak()
+    fused_bytes = fused_bytes_per_param(wl) * P
+    achieved = fused_bytes / (upd_ms / 1e3) / 1e9
+    traffic_pp = profiled_traffic(wl.name)
+    step_bytes = ideal_bytes_per_param(wl) * P
+    out = {
+        "metric": METRIC, "value": psi * world / (ms / 1e3), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": workload_config(wl, world),
+        "hbm": {"achieved_gbs_step": step_bytes / (ms / 1e3) / 1e9, "ideal_bytes_per_param": ideal_bytes_per_param(wl),
+                "frac_of_measured_peak": step_bytes / (ms / 1e3) / 1e9 / peak,
+                "frac_of_nominal_8tbs": step_bytes / (ms / 1e3) / 1e9 / NOMINAL_HBM_GBS},
+        "roofline": {"bound": "hbm", "kernel": "fused reduce-scatter + AdamW (tile_kernel)",
+                     "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": achieved / peak, "kernel_ms": upd_ms,
+                     "algorithmic_bytes_per_launch": fused_bytes,
+                     "traffic": traffic_pp * P if traffic_pp else None},
+        "gpu_launches": K * launches_per_step,
+        "e2e": e2e,
+        "clocks": clocks,
+    }
+    if gat_ms is not None:
+        out["gather_kernel_ms"] = gat_ms
+        out["gather_gbs"] = 4 * P / (gat_ms / 1e3) / 1e9
+    if world == 1 and a.cpu_seconds > 0:
+        out["cpu_baseline"] = cpu_baseline(wl, a.cpu_seconds)
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    a = parse()
+    from seeded_inputs.workloads import full_workloads
+    wl = full_workloads()[a.workload]
+    if a.psi:
+        if len(wl.tensors) != 1:
+            raise SystemExit("--psi applies to flat (single-tensor) workloads only")
+        wl = wl.with_(tensors=(a.psi,), name=f"{wl.name}_psi{a.psi}")
+    if a.impl == "reference":
+        run_reference(a, wl)
+    else:
+        run_ours(a, wl)
+
+
+if __name__ == "__main__":
+    main()

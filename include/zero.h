@@ -1,0 +1,200 @@
+/*
+ * zero.h -- C ABI of the sharded data-parallel optimizer step (DDP, ZeRO-1/2/3) on one
+ * B200: N data-parallel ranks are simulated as N gradient buffers in one GPU's HBM.
+ *
+ * Sources (page address, then section):
+ *   P1 = rkmt.cn/news/44736           (sections DP, DDP, Deepspeed ZeRO, ZeRO-1/-2/-3, 总结)
+ *   P2 = wangyh.co PaperReading:DeepSpeed (sections 1.1-1.5, 2.1-2.6, 3)
+ *   P3 = en.pswp.cn/web/84187          (sections DP, DDP, FSDP)
+ *
+ * Conventions shared by every call:
+ *  - psi  = number of parameters (sum of the tensor sizes), N = ranks,
+ *    S    = shard = roundup(ceil(psi / N), pad_align), P = padded = N * S.
+ *    All flat buffers are indexed by the flat parameter index 0 .. P-1; tensors are
+ *    concatenated in list order with no per-tensor padding; [psi, P) is tail padding,
+ *    which must hold zeros in gradients and state on entry (it then stays zero).
+ *  - Shard k is [k*S, (k+1)*S) (P1 Deepspeed ZeRO-1: each of 3 GPUs is responsible for
+ *    one third).  Buckets are fixed ranges of bucket_elems elements cut from the TAIL of
+ *    the padded buffer: bucket 0 = [P - B, P), the gradients a backward pass produces
+ *    first (P1 DDP and ZeRO-1/-2: gradients are computed back to front and synced group
+ *    by group; P3 DDP: parameters are reduced bucket by bucket).  A segment is a bucket
+ *    intersected with a shard: chunk k of that bucket's ring.
+ *  - fp16 values are passed as uint16_t bit patterns.  Device pointers are caller-owned
+ *    device memory (e.g. from PyTorch), 16-byte aligned; element strides are multiples
+ *    of 8.  The library never frees or retains caller memory.
+ *  - Every device call is asynchronous on `stream` (a cudaStream_t, NULL = legacy
+ *    default stream) of the CUDA device the layout was uploaded to, which must be the
+ *    current device.  Argument errors return before anything is launched.  Launch
+ *    failures return ZERO_ERR_CUDA.  A kernel that gives up a bounded wait records
+ *    ZERO_ERR_TIMEOUT in a device error word that zero_get_error() reports.
+ *  - Arithmetic: every reduction and update step is one IEEE-754 binary32 operation,
+ *    rounded to nearest even, no fused multiply-add, no flush of subnormals.
+ */
+#ifndef ZERO_H
+#define ZERO_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ZERO_OK = 0,
+    ZERO_ERR_INVALID = 1,   /* bad argument: NULL where required, size or index out of range */
+    ZERO_ERR_ALIGN = 2,     /* a device pointer not 16-byte aligned, or a stride not a multiple of 8 */
+    ZERO_ERR_CUDA = 3,      /* a CUDA runtime call or kernel launch failed */
+    ZERO_ERR_OOM = 4,       /* allocation of the layout's own tables failed */
+    ZERO_ERR_TIMEOUT = 5,   /* a bounded wait inside a kernel gave up (see zero_get_error) */
+    ZERO_ERR_STATE = 6      /* layout not uploaded, or uploaded to another device */
+} zero_status;
+
+typedef struct zero_layout zero_layout;   /* opaque; owned by the library */
+
+/* Layout description: what a DeepSpeed-style config names (P2 section 2.2-2.4:
+ * zero_optimization.stage), plus the model's parameter list and the bucket size. */
+typedef struct {
+    int32_t n_ranks;                    /* N >= 1 simulated data-parallel ranks */
+    int32_t stage;                      /* 0 = DDP (ZeRO-0), 1, 2, 3 (P2 section 1) */
+    int64_t n_tensors;                  /* >= 0 */
+    const int64_t *tensor_numel;        /* [n_tensors], each >= 0 (host memory, copied) */
+    int64_t bucket_elems;               /* bucket size in elements; <= 0: one bucket */
+    int64_t pad_align;                  /* shard rounding in elements, >= 1 (128 typical) */
+    int64_t n_units;                    /* stage-3 gather units (layers); 0 = one unit */
+    const int64_t *unit_first_tensor;   /* [n_units]: first tensor of each unit; [0] == 0,
+                                           strictly increasing (host memory, copied) */
+} zero_layout_desc;
+
+typedef struct {
+    int64_t psi, shard, padded;         /* psi, S, P */
+    int64_t n_buckets, n_segments, n_units;
+    int64_t tile_elems, n_tiles;        /* the kernels' work decomposition of the segments */
+} zero_layout_info;
+
+/* AdamW hyper-parameters of one step (step >= 1, counted from 1 for every run). */
+typedef struct {
+    double lr, beta1, beta2, eps, weight_decay;
+    double loss_scale;                  /* L > 0: gradients arrive multiplied by L */
+    int64_t step;
+} zero_adamw_hparams;
+
+/* Modelled per-rank memory (bytes) and communication (elements) of one training step.
+ * Memory: P1 Deepspeed ZeRO (2B fp16 params + 2B fp16 grads + 12B optimizer state per
+ * parameter for DDP; ZeRO-1 shards the optimizer state, ZeRO-2 also the gradients,
+ * ZeRO-3 also the parameters).  Communication: P1 DDP (N-1 rounds of psi/N per phase,
+ * two phases), ZeRO-1/-2 (same as DDP), ZeRO-3 (a third phase: 3 psi, 1.5x DDP). */
+typedef struct {
+    int64_t mem_p16, mem_g16, mem_os, mem_total;
+    int64_t sent_elems, recv_elems;
+} zero_counters;
+
+/* Optional CUDA events (cudaEvent_t, created by the caller; any may be NULL) that
+ * zero_step records on `stream` around its kernels, for per-kernel timing. */
+typedef struct {
+    void *update_begin, *update_end;    /* the fused reduce-scatter + update kernel */
+    void *gather_begin, *gather_end;    /* the stage-3 all-gather kernel */
+} zero_step_events;
+
+/* ---- layout (host) ------------------------------------------------------------ */
+
+/* Partition the flat parameter buffer into shards, buckets, segments and gather units.
+ * Host-only work; no CUDA call.  *out must be released with zero_layout_destroy. */
+zero_status zero_layout_create(const zero_layout_desc *desc, zero_layout **out);
+void zero_layout_destroy(zero_layout *layout);
+zero_status zero_layout_get_info(const zero_layout *layout, zero_layout_info *info);
+
+/* Host copies of the tables (any pointer may be NULL):
+ *   tensor_off [n_tensors]        flat offset of each tensor
+ *   bucket_lohi [n_buckets][2]    bucket ranges, bucket order (bucket 0 = tail)
+ *   segments [n_segments][4]      bucket, shard, lo, hi; bucket order, then shard order
+ *   unit_lohi [n_units][2]        gather-unit ranges, ascending, covering [0, P) */
+zero_status zero_layout_get_tables(const zero_layout *layout, int64_t *tensor_off,
+                                   int64_t *bucket_lohi, int64_t *segments, int64_t *unit_lohi);
+zero_status zero_layout_counters(const zero_layout *layout, zero_counters *out);
+
+/* Upload the segment table to the current CUDA device and build the tile index on it
+ * (a one-warp prefix scan of the segments' tile counts).  Allocates the layout's small
+ * device tables (about 40 bytes per segment); must precede every device call. */
+zero_status zero_layout_to_device(zero_layout *layout, void *stream);
+
+/* Copy back the device-built table: [n_segments + 1][5] = bucket, shard, lo, hi,
+ * first tile (the last row holds -1, -1, P, P, total tiles).  Synchronises `stream`. */
+zero_status zero_layout_device_segments(const zero_layout *layout, int64_t *host_out, void *stream);
+
+/* ---- the hot path (device) ------------------------------------------------------ */
+
+/* Ring reduce-scatter of bucket `bucket` (-1 = every bucket, in bucket order).
+ * P3 DDP (three-GPU walk-through) and P1 DDP (scatter-reduce: values passed on and
+ * added): chunk k of the bucket starts at rank k and accumulates ranks k+1, k+2, ...
+ * (mod N).  For each flat index i of the bucket, in shard k:
+ *     reduced[i] = (...((f32(g_k[i]) + f32(g_{k+1}[i])) + f32(g_{k+2}[i])) ...)
+ * with g_r[i] = grads[r * rank_stride + i] (fp16, rank_stride >= P, multiple of 8).
+ * reduced: fp32 [P] (only the bucket's indices are written).
+ * nonfinite: optional device int32 [n_buckets]; each bucket's count of non-finite sums
+ * is ADDED to its entry (zero it first). */
+zero_status zero_reduce_scatter(const zero_layout *layout, int64_t bucket, const uint16_t *grads,
+                                int64_t rank_stride, float *reduced, int32_t *nonfinite,
+                                void *stream);
+
+/* Shard update of shard `shard` (-1 = every shard), P1 Deepspeed ZeRO-1 update step:
+ * the reduced fp32 sum is scaled by 1/(N * loss_scale), then AdamW updates the fp32
+ * first and second moments and the fp32 master weights, then the fp16 parameters:
+ *     g = s * fp32(1/(N L));  p = p * fp32(1 - lr wd)
+ *     m = fp32(b1) m + fp32(1 - b1) g;  v = fp32(b2) v + fp32(1 - b2) (g g)
+ *     p = p - fp32(lr / (1 - b1^t)) * (m / (sqrt(v) / fp32(sqrt(1 - b2^t)) + fp32(eps)))
+ *     p16_out[i] = fp16_rne(p)
+ * (scalars computed on the host in double, each rounded once to fp32).
+ * reduced, master, m, v: fp32 [P]; p16_out: fp16 [P] (the full buffer for stages 0-2,
+ * the shard buffer for stage 3); only the shard's indices are touched. */
+zero_status zero_adamw_shard_step(const zero_layout *layout, int32_t shard, const float *reduced,
+                                  float *master, float *m, float *v, uint16_t *p16_out,
+                                  const zero_adamw_hparams *hp, void *stream);
+
+/* All-gather of gather unit `unit` (-1 = all units): every shard's fp16 parameters of the
+ * unit are written into the full flat buffer, p16_full[i] = p16_shard[i] for i in the
+ * unit (P1 ZeRO-1 broadcast step; P2 section 2.5: the full parameter is the
+ * concatenation of all ranks' partitions; P1 ZeRO-3: parameters are gathered layer by
+ * layer for the forward and again for the backward pass).  Both fp16 [P]. */
+zero_status zero_allgather(const zero_layout *layout, int64_t unit, const uint16_t *p16_shard,
+                           uint16_t *p16_full, void *stream);
+
+/* One whole optimizer step of the layout's stage: the reduce-scatter of every bucket
+ * fused with the shard update, each gradient and state byte crossing HBM once; the
+ * reduced sums stay in registers.  Stages 0-2 write the fp16 parameters straight into
+ * p16_full (the owner's slice of the replicated buffer: the broadcast is the write
+ * itself; p16_shard may be NULL).  Stage 3 writes p16_shard, then runs the all-gather
+ * of every unit into p16_full.  Results are bit-identical to zero_reduce_scatter +
+ * zero_adamw_shard_step (+ zero_allgather).  nonfinite and events may be NULL. */
+zero_status zero_step(const zero_layout *layout, const uint16_t *grads, int64_t rank_stride,
+                      float *master, float *m, float *v, uint16_t *p16_shard, uint16_t *p16_full,
+                      const zero_adamw_hparams *hp, int32_t *nonfinite,
+                      const zero_step_events *events, void *stream);
+
+/* zero_step for gradients that live in HOST memory (page-locked), with the fp16
+ * parameters returned to host memory: per bucket, the N gradient slices are copied to
+ * the device staging buffer grads_dev on an internal copy stream, the bucket's fused
+ * update runs on `stream` as soon as they land, and (stages 0-2) the bucket's new fp16
+ * parameters are copied back to p16_host on a second internal stream, so transfers and
+ * compute overlap bucket by bucket.  Stage 3 copies p16_full back after the gather.
+ *   grads_host: [N][rank_stride] page-locked; grads_dev: device [N][rank_stride];
+ *   p16_host: page-locked fp16 [P].  Completion: synchronise `stream`. */
+zero_status zero_step_host(const zero_layout *layout, const uint16_t *grads_host,
+                           uint16_t *grads_dev, int64_t rank_stride, float *master, float *m,
+                           float *v, uint16_t *p16_shard, uint16_t *p16_full, uint16_t *p16_host,
+                           const zero_adamw_hparams *hp, int32_t *nonfinite, void *stream);
+
+/* Select the fused kernel's implementation: 0 = automatic, 1 = register streaming
+ * (vectorised 16-byte loads held in registers), 2 = bulk-copy pipeline (cp.async.bulk
+ * into a shared-memory ring, warp-specialised).  Results are identical. */
+zero_status zero_set_impl(zero_layout *layout, int32_t impl);
+
+/* Synchronise `stream`, read and clear the layout's device error word. */
+zero_status zero_get_error(const zero_layout *layout, void *stream);
+
+const char *zero_status_string(zero_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ZERO_H */

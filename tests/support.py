@@ -1,0 +1,112 @@
+"""Helpers shared by the GPU parity tests: seeded inputs for both sides, the oracle's
+answers, and the comparison rules.
+
+Both sides get their inputs from seeded_inputs (host fill for the oracle, device fill
+for the CUDA path; the two fills are checked bit-identical in test_inputs_gen.py).
+Nothing the CUDA path computes ever feeds the oracle.
+
+Comparison bar: ring sums bit-exact; fp32 master / moments within 1e-6 relative;
+fp16 parameters within 1 ulp.  The arithmetic on both sides is the same sequence of
+correctly rounded IEEE operations, so bit-exact agreement is also checked separately.
+"""
+import numpy as np
+
+import oracle
+import seeded_inputs as si
+from oracle.layout import make_layout
+
+F32_REL = 1e-6
+F16_ULPS = 1
+
+
+def oracle_layout(wl):
+    return make_layout(list(wl.tensors), wl.n_ranks, wl.bucket_elems, wl.pad_align, list(wl.units))
+
+
+def hyper(wl):
+    return oracle.Hyper(wl.lr, wl.beta1, wl.beta2, wl.eps, wl.weight_decay, wl.loss_scale)
+
+
+def host_inputs(wl, P):
+    """grads uint16 [N, P]; master, m, v float32 [P] (zero tail padding)."""
+    psi = wl.psi
+    g = si.fill_grads(wl.n_ranks, P, psi, wl.seed, wl.grad_sigma, wl.loss_scale, wl.heavy_frac, wl.heavy_mult)
+    master = si.fill_f32(P, psi, wl.seed, si.STREAM_MASTER, wl.master_sigma)
+    m = si.fill_f32(P, psi, wl.seed, si.STREAM_M, wl.m_sigma) if wl.m_sigma else np.zeros(P, np.float32)
+    v = si.fill_f32(P, psi, wl.seed, si.STREAM_V, wl.v_sigma, True) if wl.v_sigma else np.zeros(P, np.float32)
+    return g, master, m, v
+
+
+def device_inputs(wl, P, rank_stride=None):
+    """The same inputs generated directly in device memory (torch tensors)."""
+    import torch
+    stride = rank_stride or P
+    psi = wl.psi
+    g = torch.empty((wl.n_ranks, stride), dtype=torch.int16, device="cuda")
+    si.fill_grads_cuda(g, psi, wl.seed, wl.grad_sigma, wl.loss_scale, wl.heavy_frac, wl.heavy_mult)
+    master = torch.empty(P, dtype=torch.float32, device="cuda")
+    si.fill_f32_cuda(master, psi, wl.seed, si.STREAM_MASTER, wl.master_sigma)
+    m = torch.zeros(P, dtype=torch.float32, device="cuda")
+    v = torch.zeros(P, dtype=torch.float32, device="cuda")
+    if wl.m_sigma:
+        si.fill_f32_cuda(m, psi, wl.seed, si.STREAM_M, wl.m_sigma)
+    if wl.v_sigma:
+        si.fill_f32_cuda(v, psi, wl.seed, si.STREAM_V, wl.v_sigma, absval=True)
+    return g, master, m, v
+
+
+def sampled_oracle(wl, lay, idx, steps):
+    """Oracle values at flat indices idx after `steps` steps (per-element path)."""
+    psi = wl.psi
+    g = si.gather_grads(idx, wl.n_ranks, psi, wl.seed, wl.grad_sigma, wl.loss_scale, wl.heavy_frac,
+                        wl.heavy_mult)
+    master = si.gather_f32(idx, psi, wl.seed, si.STREAM_MASTER, wl.master_sigma)
+    m = si.gather_f32(idx, psi, wl.seed, si.STREAM_M, wl.m_sigma) if wl.m_sigma else np.zeros(len(idx), np.float32)
+    v = (si.gather_f32(idx, psi, wl.seed, si.STREAM_V, wl.v_sigma, True) if wl.v_sigma
+         else np.zeros(len(idx), np.float32))
+    sc = np.stack([oracle.adamw_scalars(wl.n_ranks, hyper(wl), t) for t in range(1, steps + 1)])
+    reduced, p16 = oracle.sampled(g, idx // lay.shard, steps, sc, master, m, v)
+    return reduced, master, m, v, p16
+
+
+def sample_indices(lay, n_random=16384, seed=0):
+    """Random indices plus every segment, shard, bucket and unit edge, and the tail."""
+    P = lay.padded
+    rng = np.random.default_rng(seed)
+    pts = [rng.integers(0, P, n_random)]
+    edges = []
+    for _, _, lo, hi in lay.segments:
+        edges += [lo, lo + 1, lo + 7, lo + 8, hi - 1, hi - 2, hi - 8, hi - 9]
+    for lo, hi in lay.units:
+        edges += [lo, lo + 1, hi - 1]
+    edges += [lay.psi - 1, lay.psi, P - 1, 0]
+    pts.append(np.array(edges, dtype=np.int64))
+    idx = np.unique(np.concatenate(pts))
+    return idx[(idx >= 0) & (idx < P)]
+
+
+def f16_ordered(bits):
+    """Map fp16 bit patterns to integers that preserve numeric order (ulp distance)."""
+    b = bits.astype(np.int32)
+    return np.where(b & 0x8000, -(b & 0x7FFF), b)
+
+
+def assert_f32_close(got, want, what, rel=F32_REL):
+    got = np.asarray(got, np.float32)
+    want = np.asarray(want, np.float32)
+    same = (got.view(np.uint32) == want.view(np.uint32)) | (np.isnan(got) & np.isnan(want))
+    bad = ~same & ~(np.abs(got.astype(np.float64) - want) <= rel * np.abs(want.astype(np.float64)))
+    assert not bad.any(), f"{what}: {bad.sum()} elements beyond {rel} relative, first at {np.flatnonzero(bad)[:5]}"
+
+
+def assert_f16_ulp(got, want, what, ulps=F16_ULPS):
+    d = np.abs(f16_ordered(np.asarray(got, np.uint16)) - f16_ordered(np.asarray(want, np.uint16)))
+    assert d.max(initial=0) <= ulps, f"{what}: max {d.max()} ulp"
+
+
+def assert_bits_equal(got, want, what):
+    got = np.ascontiguousarray(got)
+    want = np.ascontiguousarray(want)
+    diff = got.view(np.uint8).reshape(got.size, -1) != want.view(np.uint8).reshape(want.size, -1)
+    n = int(diff.any(axis=1).sum())
+    assert n == 0, f"{what}: {n} elements differ bitwise"

@@ -1,0 +1,108 @@
+"""CPU checks of the C ABI: the library loads and exports every function include/zero.h
+declares; its host partitioner and counters equal the oracle's; bad arguments are
+rejected before anything runs.  No kernel is launched here."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle.layout import make_layout
+from seeded_inputs.workloads import full_workloads, reduced_workloads
+import zero_sharded_optimizer_ring_b200 as zs
+from zero_sharded_optimizer_ring_b200 import _abi, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    build.build()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "zero.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(zero_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_exports_every_declared_function():
+    names = _declared()
+    assert len(names) >= 15
+    lib = ctypes.CDLL(_abi.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(_abi.SIGNATURES)
+
+
+def _compare(tensors, N, stage, B, A, units):
+    ref = make_layout(tensors, N, B, A, units)
+    lay = zs.Layout(tensors, N, stage, B, A, units)
+    assert (lay.psi, lay.shard, lay.padded) == (ref.psi, ref.shard, ref.padded)
+    t, b, s, u = lay.tables()
+    assert list(t) == ref.tensor_off
+    assert [tuple(x) for x in b] == ref.buckets
+    assert [tuple(x) for x in s] == [tuple(x) for x in ref.segments]
+    assert [tuple(x) for x in u] == ref.units
+    c = lay.counters()
+    rc = oracle.counters(ref, stage)
+    assert (c["mem_p16"], c["mem_g16"], c["mem_os"], c["mem_total"], c["sent_elems"], c["recv_elems"]) == \
+        (rc.mem_p16, rc.mem_g16, rc.mem_os, rc.mem_total, rc.sent_elems, rc.recv_elems)
+    # tile numbering: each segment's tiles are the kTileElems cells it overlaps
+    T = lay.tile_elems
+    assert lay.n_tiles == sum(-(-hi // T) - lo // T for _, _, lo, hi in ref.segments)
+    lay.close()
+
+
+def test_layout_matches_oracle_random():
+    rng = np.random.default_rng(21)
+    for _ in range(300):
+        N = int(rng.integers(1, 20))
+        nt = int(rng.integers(0, 8))
+        tensors = [int(x) for x in rng.integers(0, 5000, nt)]
+        units = sorted({0} | {int(x) for x in rng.integers(0, max(1, nt), 3)}) if nt and rng.random() < 0.5 else []
+        _compare(tensors, N, int(rng.integers(0, 4)), int(rng.integers(-5, 9000)),
+                 int(rng.choice([1, 3, 8, 128])), units)
+
+
+def test_layout_matches_oracle_workloads():
+    for wl in list(reduced_workloads().values()) + list(full_workloads().values()):
+        _compare(list(wl.tensors), wl.n_ranks, wl.stage, wl.bucket_elems, wl.pad_align, list(wl.units))
+
+
+def test_config_sizes():
+    # shard and padding of the flat 1.3e9 workload and the Llama-shaped list
+    w = full_workloads()
+    lay = zs.Layout(w["flat1p3b_n4_zero1"].tensors, 4, 1, 50_000_000)
+    assert (lay.shard, lay.padded, lay.n_buckets) == (325_000_064, 1_300_000_256, 27)
+    ll = w["llama3b_n8_zero3"]
+    lay = zs.Layout(ll.tensors, 8, 3, 50_000_000, 128, ll.units)
+    assert (lay.psi, lay.padded, lay.n_units) == (3_042_868_224, 3_042_868_224, 28)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(n_ranks=0), dict(stage=4), dict(stage=-1), dict(pad_align=0),
+    dict(tensors=[5, -1]), dict(units=[1]), dict(units=[0, 0]), dict(units=[0, 9]),
+])
+def test_invalid_descriptions_rejected(kw):
+    args = dict(tensors=[100, 50], n_ranks=2, stage=1, bucket_elems=10, pad_align=8, units=())
+    args.update(kw)
+    with pytest.raises(zs.ZeroError) as e:
+        zs.Layout(**args)
+    assert e.value.status == 1
+
+
+def test_device_calls_need_upload():
+    lay = zs.Layout([1000], 2, 1, 100)
+    with pytest.raises(zs.ZeroError) as e:
+        zs.reduce_scatter(lay, -1, 0, 0, rank_stride=1024, stream=0)
+    assert e.value.status == 6           # ZERO_ERR_STATE, nothing launched
+
+
+def test_empty_layout():
+    lay = zs.Layout([], 4, 2, 100)
+    assert (lay.psi, lay.padded, lay.n_buckets, lay.n_segments, lay.n_units, lay.n_tiles) == (0, 0, 0, 0, 0, 0)
+    lay = zs.Layout([0, 0], 3, 3, 0)
+    assert lay.padded == 0

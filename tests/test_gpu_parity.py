@@ -1,0 +1,307 @@
+"""GPU parity: the CUDA path, through the C ABI, against the CPU oracle.
+
+- reduced-size twins of every workload: every element of every output after all steps;
+- the full-size workloads in the launch configuration the benchmark times: sampled
+  elements (every segment, shard, bucket and unit edge plus random ones) against the
+  oracle's per-element path;
+- edge cases: one rank, unaligned segment edges (shard rounding 1), one-element
+  buckets, a rank count without a compiled specialisation, empty layouts, non-finite
+  gradients, per-bucket / per-shard / per-unit calls, the host-buffer step.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import seeded_inputs as si
+from seeded_inputs.workloads import Workload, full_workloads, reduced_workloads
+import zero_sharded_optimizer_ring_b200 as zs
+import support as S
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+def _hp(wl, t):
+    return zs.AdamW(wl.lr, wl.beta1, wl.beta2, wl.eps, wl.weight_decay, wl.loss_scale, t)
+
+
+def _layout(wl):
+    return zs.Layout(list(wl.tensors), wl.n_ranks, wl.stage, wl.bucket_elems, wl.pad_align,
+                     list(wl.units)).to_device()
+
+
+def _bufs(lay, wl, rank_stride=None):
+    g, master, m, v = S.device_inputs(wl, lay.padded, rank_stride)
+    p16_shard = torch.zeros(lay.padded, dtype=torch.int16, device="cuda")
+    p16_full = torch.zeros(lay.padded, dtype=torch.int16, device="cuda")
+    nonfinite = torch.zeros(max(1, lay.n_buckets), dtype=torch.int32, device="cuda")
+    return dict(g=g, master=master, m=m, v=v, p16_shard=p16_shard, p16_full=p16_full, nonfinite=nonfinite)
+
+
+def _run(lay, wl, b, steps):
+    for t in range(1, steps + 1):
+        b["nonfinite"].zero_()
+        zs.step(lay, b["g"], b["master"], b["m"], b["v"], b["p16_shard"], b["p16_full"], _hp(wl, t),
+                nonfinite=b["nonfinite"])
+    zs.get_error(lay)
+    torch.cuda.synchronize()
+
+
+def _np(t):
+    a = t.cpu().numpy()
+    return a.view(np.uint16) if a.dtype == np.int16 else a
+
+
+def _check_full(wl, lay, b, ref, exact=True):
+    S.assert_f32_close(_np(b["master"]), ref.master, "master")
+    S.assert_f32_close(_np(b["m"]), ref.m, "m")
+    S.assert_f32_close(_np(b["v"]), ref.v, "v")
+    S.assert_f16_ulp(_np(b["p16_full"]), ref.p16_full, "p16_full")
+    if wl.stage == 3:
+        S.assert_f16_ulp(_np(b["p16_shard"]), ref.p16_shard, "p16_shard")
+    assert list(_np(b["nonfinite"])[:lay.n_buckets]) == list(ref.nonfinite)
+    if exact:
+        S.assert_bits_equal(_np(b["master"]), ref.master, "master")
+        S.assert_bits_equal(_np(b["m"]), ref.m, "m")
+        S.assert_bits_equal(_np(b["v"]), ref.v, "v")
+        S.assert_bits_equal(_np(b["p16_full"]), ref.p16_full, "p16_full")
+
+
+def _oracle(wl, steps=None):
+    lay = S.oracle_layout(wl)
+    g, master, m, v = S.host_inputs(wl, lay.padded)
+    return oracle.run_steps(lay, wl.stage, g, master, m, v, S.hyper(wl), steps or wl.steps), lay
+
+
+@pytest.fixture(autouse=True)
+def _free():
+    yield
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+# ------------------------------------------------------------- reduced-size, every element
+
+@pytest.mark.parametrize("key", list(reduced_workloads()))
+def test_reduced_workload_all_elements(key):
+    wl = reduced_workloads()[key]
+    ref, olay = _oracle(wl)
+    lay = _layout(wl)
+    assert lay.n_tiles >= 8 and lay.n_buckets >= 1     # several tiles, ragged edges
+    b = _bufs(lay, wl)
+    _run(lay, wl, b, wl.steps)
+    _check_full(wl, lay, b, ref)
+
+    # ring sums: bit-exact
+    red = torch.zeros(lay.padded, dtype=torch.float32, device="cuda")
+    nf = torch.zeros(max(1, lay.n_buckets), dtype=torch.int32, device="cuda")
+    zs.reduce_scatter(lay, -1, b["g"], red, nonfinite=nf)
+    S.assert_bits_equal(_np(red), ref.reduced, "reduced")
+    assert list(_np(nf)[:lay.n_buckets]) == list(ref.nonfinite)
+
+
+@pytest.mark.parametrize("key", list(reduced_workloads()))
+def test_unfused_path_equals_fused(key):
+    wl = reduced_workloads()[key]
+    lay = _layout(wl)
+    a = _bufs(lay, wl)
+    b = _bufs(lay, wl)
+    red = torch.zeros(lay.padded, dtype=torch.float32, device="cuda")
+    for t in range(1, 3):
+        zs.step(lay, a["g"], a["master"], a["m"], a["v"], a["p16_shard"], a["p16_full"], _hp(wl, t))
+        # per bucket, per shard, per unit
+        for bk in range(lay.n_buckets):
+            zs.reduce_scatter(lay, bk, b["g"], red)
+        for k in range(lay.n_ranks):
+            out = b["p16_shard"] if wl.stage == 3 else b["p16_full"]
+            zs.adamw_shard_step(lay, k, red, b["master"], b["m"], b["v"], out, _hp(wl, t))
+        if wl.stage == 3:
+            for u in range(lay.n_units):
+                zs.allgather(lay, u, b["p16_shard"], b["p16_full"])
+    torch.cuda.synchronize()
+    for name in ("master", "m", "v", "p16_full"):
+        S.assert_bits_equal(_np(a[name]), _np(b[name]), name)
+
+
+def test_deterministic_rerun():
+    wl = reduced_workloads()["ragged2000_n16_zero2"]
+    lay = _layout(wl)
+    outs = []
+    for _ in range(2):
+        b = _bufs(lay, wl)
+        _run(lay, wl, b, 2)
+        outs.append({k: _np(v) for k, v in b.items() if k != "g"})
+    for k in outs[0]:
+        S.assert_bits_equal(outs[0][k], outs[1][k], k)
+
+
+def test_device_tile_index_matches_host():
+    for wl in list(reduced_workloads().values()) + list(full_workloads().values()):
+        lay = _layout(wl)
+        dev = lay.device_segments()
+        _, _, segs, _ = lay.tables()
+        T = lay.tile_elems
+        assert np.array_equal(dev[:-1, :4], segs)
+        counts = [-(-hi // T) - lo // T for _, _, lo, hi in segs]
+        assert list(dev[:-1, 4]) == list(np.cumsum([0] + counts)[:-1])
+        assert dev[-1, 4] == lay.n_tiles == sum(counts)
+
+
+# ------------------------------------------------------------- edge cases
+
+def _edge(tensors, N, stage, B, A, steps=2, units=(), L=1024.0, **kw):
+    return Workload(name="edge", description="edge", tensors=tuple(tensors), units=tuple(units), n_ranks=N,
+                    stage=stage, bucket_elems=B, steps=steps, loss_scale=L, pad_align=A, **kw)
+
+
+EDGES = {
+    "ring3_trace": _edge([3], 3, 1, 0, 1),
+    "one_rank": _edge([10_001], 1, 1, 999, 8),
+    "two_ranks_unaligned": _edge([4097, 3, 7, 12_289], 2, 2, 37, 1),
+    "five_ranks": _edge([77_777], 5, 0, 9_999, 1),
+    "one_elem_buckets": _edge([301], 4, 2, 1, 1),
+    "seven_elem_buckets": _edge([5_000], 6, 3, 7, 1, units=()),
+    "seventeen_ranks_runtime_n": _edge([33_333, 1, 2], 17, 2, 4_111, 4, heavy_frac=0.05, heavy_mult=100.0),
+    "stage3_units_unaligned": _edge([13, 4099, 8190, 5], 3, 3, 1_000, 1, units=(0, 1, 3)),
+    "ddp_many_tiles": _edge([3 * 4096 * 148 + 5], 3, 0, 100_003, 128, m_sigma=1e-4, v_sigma=1e-6),
+}
+
+
+@pytest.mark.parametrize("key", list(EDGES))
+def test_edge_cases(key):
+    wl = EDGES[key]
+    ref, _ = _oracle(wl)
+    lay = _layout(wl)
+    b = _bufs(lay, wl)
+    _run(lay, wl, b, wl.steps)
+    _check_full(wl, lay, b, ref)
+
+
+def test_padded_rank_stride():
+    wl = _edge([50_000], 4, 1, 7_000, 128)
+    ref, _ = _oracle(wl)
+    lay = _layout(wl)
+    b = _bufs(lay, wl, rank_stride=lay.padded + 4096)
+    _run(lay, wl, b, wl.steps)
+    _check_full(wl, lay, b, ref)
+
+
+def test_empty_layout_is_noop():
+    lay = zs.Layout([], 4, 2, 100).to_device()
+    zs.step(lay, 0, 0, 0, 0, 0, 0, zs.AdamW(), rank_stride=0)
+    zs.reduce_scatter(lay, -1, 0, 0, rank_stride=0)
+    zs.allgather(lay, -1, 0, 0)
+    zs.get_error(lay)
+
+
+def test_order_probe_on_gpu():
+    # chunk k: ranks k, k+1 hold 2^-24, rank k+2 holds 1: only the ring order k, k+1, k+2
+    # gives 1 + 2^-23
+    lay = zs.Layout([3], 3, 1, 0, 1).to_device()
+    g = np.zeros((3, 8), np.uint16)
+    for k in range(3):
+        g[k, k] = 1
+        g[(k + 1) % 3, k] = 1
+        g[(k + 2) % 3, k] = 0x3C00
+    gd = torch.from_numpy(g.view(np.int16)).cuda()
+    red = torch.zeros(8, dtype=torch.float32, device="cuda")
+    zs.reduce_scatter(lay, -1, gd, red)
+    assert np.all(_np(red)[:3] == np.float32(1) + np.float32(2 ** -23))
+
+
+def test_nonfinite_counts_per_bucket():
+    wl = _edge([30_000], 4, 2, 7_001, 8)
+    olay = S.oracle_layout(wl)
+    P = olay.padded
+    g = np.zeros((4, P), np.uint16)
+    marks = {3: 0x7C00, 7_000: 0xFC00, 7_001: 0x7E00, 22_222: 0x7C00, 29_999: 0x7C00}
+    for i, bits in marks.items():
+        g[i % 4, i] = bits
+    g[0, 29_999] = 0xFC00
+    master = np.zeros(P, np.float32)
+    ref = oracle.run_steps(olay, 2, g, master, master, master, S.hyper(wl), 1)
+    lay = _layout(wl)
+    gd = torch.from_numpy(g.view(np.int16)).cuda()
+    bufs = [torch.zeros(P, dtype=torch.float32, device="cuda") for _ in range(3)]
+    p16 = torch.zeros(P, dtype=torch.int16, device="cuda")
+    nf = torch.zeros(lay.n_buckets, dtype=torch.int32, device="cuda")
+    zs.step(lay, gd, *bufs, None, p16, _hp(wl, 1), nonfinite=nf)
+    assert list(_np(nf)) == list(ref.nonfinite)
+    assert sum(ref.nonfinite) == len(marks)
+    S.assert_f16_ulp(_np(p16), ref.p16_full, "p16")
+
+
+def test_bad_arguments_rejected():
+    wl = _edge([10_000], 2, 1, 1_000, 8)
+    lay = _layout(wl)
+    b = _bufs(lay, wl)
+    with pytest.raises(zs.ZeroError) as e:
+        zs.step(lay, b["g"], b["master"], b["m"], b["v"], None, b["p16_full"], _hp(wl, 0))
+    assert e.value.status == 1
+    with pytest.raises(zs.ZeroError) as e:
+        zs.step(lay, b["g"], b["master"][1:], b["m"], b["v"], None, b["p16_full"], _hp(wl, 1))
+    assert e.value.status == 2
+    with pytest.raises(zs.ZeroError) as e:
+        zs.step(lay, b["g"], b["master"], b["m"], b["v"], None, b["p16_full"], _hp(wl, 1),
+                rank_stride=lay.padded - 8)
+    assert e.value.status == 1
+    with pytest.raises(zs.ZeroError):
+        zs.reduce_scatter(lay, lay.n_buckets, b["g"], b["master"])
+    with pytest.raises(zs.ZeroError):
+        zs.allgather(lay, 5, b["p16_shard"], b["p16_full"])
+    with pytest.raises(zs.ZeroError):
+        zs.step(lay, b["g"], b["master"], b["m"], b["v"], None, b["p16_full"],
+                zs.AdamW(loss_scale=0.0, step=1))
+
+
+def test_host_buffer_step_equals_device_step():
+    for key in ("flat1p3b_n4_zero1", "llama3b_n8_zero3", "ragged2000_n16_zero2"):
+        wl = reduced_workloads()[key]
+        lay = _layout(wl)
+        a = _bufs(lay, wl)
+        b = _bufs(lay, wl)
+        g_host = a["g"].cpu().pin_memory()
+        b["g"].zero_()
+        p16_host = torch.zeros(lay.padded, dtype=torch.int16).pin_memory()
+        for t in range(1, 3):
+            zs.step(lay, a["g"], a["master"], a["m"], a["v"], a["p16_shard"], a["p16_full"], _hp(wl, t))
+            zs.step_host(lay, g_host, b["g"], b["master"], b["m"], b["v"], b["p16_shard"], b["p16_full"],
+                         p16_host, _hp(wl, t))
+        torch.cuda.synchronize()
+        for name in ("master", "m", "v", "p16_full"):
+            S.assert_bits_equal(_np(a[name]), _np(b[name]), name)
+        S.assert_bits_equal(p16_host.numpy().view(np.uint16), _np(a["p16_full"]), "p16_host")
+
+
+# ------------------------------------------------------------- full size, sampled
+
+@pytest.mark.parametrize("key", list(full_workloads()))
+def test_full_size_sampled(key):
+    wl = full_workloads()[key]
+    olay = S.oracle_layout(wl)
+    lay = _layout(wl)
+    b = _bufs(lay, wl)
+    _run(lay, wl, b, wl.steps)
+    idx = S.sample_indices(olay)
+    it = torch.from_numpy(idx).cuda()
+    red_ref, master, m, v, p16 = S.sampled_oracle(wl, olay, idx, wl.steps)
+    got = {k: _np(b[k][it]) for k in ("master", "m", "v", "p16_full", "p16_shard")}
+    S.assert_f32_close(got["master"], master, "master")
+    S.assert_f32_close(got["m"], m, "m")
+    S.assert_f32_close(got["v"], v, "v")
+    S.assert_f16_ulp(got["p16_full"], p16, "p16_full")
+    S.assert_bits_equal(got["master"], master, "master")
+    S.assert_bits_equal(got["m"], m, "m")
+    S.assert_bits_equal(got["v"], v, "v")
+    S.assert_bits_equal(got["p16_full"], p16, "p16_full")
+    if wl.stage == 3:
+        S.assert_bits_equal(got["p16_shard"], p16, "p16_shard")
+    assert int(b["nonfinite"].sum()) == 0
+    # ring sums at the sampled indices
+    del b["m"], b["v"], b["p16_shard"]
+    red = torch.empty(lay.padded, dtype=torch.float32, device="cuda")
+    zs.reduce_scatter(lay, -1, b["g"], red)
+    S.assert_bits_equal(_np(red[it]), red_ref, "reduced")
+    # the padding stayed zero
+    assert int(torch.count_nonzero(b["p16_full"][lay.psi:])) == 0
+    assert int(torch.count_nonzero(b["master"][lay.psi:])) == 0

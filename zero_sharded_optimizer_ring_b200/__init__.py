@@ -1,0 +1,186 @@
+"""Sharded data-parallel optimizer step (DDP, ZeRO-1/2/3) for one B200.
+
+A thin binding over the C ABI of include/zero.h: it turns torch tensors into device
+pointers and a CUDA stream handle, and status codes into exceptions.  Every step of
+the computation runs in the library's CUDA kernels (libzero_b200.so).
+
+    lay = Layout(tensor_sizes, n_ranks=8, stage=2, bucket_elems=25_000_000)
+    lay.to_device()
+    step(lay, grads, master, m, v, None, p16_full, AdamW(lr=1e-3, loss_scale=1024, step=t))
+"""
+import ctypes
+from dataclasses import dataclass
+
+import numpy as np
+
+from . import _abi
+
+__all__ = ["ZeroError", "Layout", "AdamW", "reduce_scatter", "adamw_shard_step", "allgather",
+           "step", "step_host", "get_error", "IMPL_AUTO", "IMPL_REGISTER", "IMPL_BULK"]
+
+IMPL_AUTO, IMPL_REGISTER, IMPL_BULK = 0, 1, 2
+
+
+class ZeroError(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        msg = _abi.lib().zero_status_string(status).decode()
+        super().__init__(f"{what}: {_abi.STATUS_NAMES.get(status, status)} ({msg})")
+
+
+def _check(status, what):
+    if status != _abi.ZERO_OK:
+        raise ZeroError(status, what)
+
+
+def _ptr(t):
+    """Device (or host) address of a torch tensor, an int address, or None."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+@dataclass
+class AdamW:
+    lr: float = 1e-3
+    beta1: float = 0.9
+    beta2: float = 0.999
+    eps: float = 1e-8
+    weight_decay: float = 0.01
+    loss_scale: float = 1.0
+    step: int = 1
+
+    def c(self):
+        return _abi.AdamWHparams(self.lr, self.beta1, self.beta2, self.eps, self.weight_decay,
+                                 self.loss_scale, self.step)
+
+
+class Layout:
+    """Flat buffer, shards, buckets, segments and gather units (zero_layout_create)."""
+
+    def __init__(self, tensors, n_ranks, stage, bucket_elems=0, pad_align=128, units=()):
+        lib = _abi.lib()
+        self._numel = (ctypes.c_int64 * max(1, len(tensors)))(*[int(x) for x in tensors])
+        self._units = (ctypes.c_int64 * max(1, len(units)))(*[int(x) for x in units])
+        desc = _abi.LayoutDesc(int(n_ranks), int(stage), len(tensors), self._numel, int(bucket_elems),
+                               int(pad_align), len(units), self._units)
+        h = ctypes.c_void_p()
+        _check(lib.zero_layout_create(ctypes.byref(desc), ctypes.byref(h)), "zero_layout_create")
+        self._h = h
+        self.n_ranks = int(n_ranks)
+        self.stage = int(stage)
+        self.n_tensors = len(tensors)
+        info = _abi.LayoutInfo()
+        _check(lib.zero_layout_get_info(self._h, ctypes.byref(info)), "zero_layout_get_info")
+        self.psi, self.shard, self.padded = info.psi, info.shard, info.padded
+        self.n_buckets, self.n_segments, self.n_units = info.n_buckets, info.n_segments, info.n_units
+        self.tile_elems, self.n_tiles = info.tile_elems, info.n_tiles
+
+    @property
+    def handle(self):
+        return self._h
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            _abi.lib().zero_layout_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def tables(self):
+        """Host copies: tensor_off [T], buckets [B,2], segments [S,4], units [U,2]."""
+        t = np.zeros(max(1, self.n_tensors), np.int64)
+        b = np.zeros((max(1, self.n_buckets), 2), np.int64)
+        s = np.zeros((max(1, self.n_segments), 4), np.int64)
+        u = np.zeros((max(1, self.n_units), 2), np.int64)
+        _check(_abi.lib().zero_layout_get_tables(self._h, t.ctypes.data, b.ctypes.data, s.ctypes.data,
+                                                 u.ctypes.data), "zero_layout_get_tables")
+        return t[:self.n_tensors], b[:self.n_buckets], s[:self.n_segments], u[:self.n_units]
+
+    def counters(self):
+        c = _abi.Counters()
+        _check(_abi.lib().zero_layout_counters(self._h, ctypes.byref(c)), "zero_layout_counters")
+        return {f: getattr(c, f) for f, _ in _abi.Counters._fields_}
+
+    def to_device(self, stream=None):
+        _check(_abi.lib().zero_layout_to_device(self._h, _stream(stream)), "zero_layout_to_device")
+        return self
+
+    def device_segments(self, stream=None):
+        out = np.zeros((self.n_segments + 1, 5), np.int64)
+        _check(_abi.lib().zero_layout_device_segments(self._h, out.ctypes.data, _stream(stream)),
+               "zero_layout_device_segments")
+        return out
+
+    def set_impl(self, impl):
+        _check(_abi.lib().zero_set_impl(self._h, int(impl)), "zero_set_impl")
+
+
+def _stride(grads, layout, rank_stride):
+    if rank_stride is not None:
+        return int(rank_stride)
+    if grads.dim() == 2:
+        return int(grads.stride(0))
+    return int(layout.padded)
+
+
+def reduce_scatter(layout, bucket, grads, reduced, nonfinite=None, rank_stride=None, stream=None):
+    _check(_abi.lib().zero_reduce_scatter(layout.handle, int(bucket), _ptr(grads),
+                                          _stride(grads, layout, rank_stride), _ptr(reduced),
+                                          _ptr(nonfinite), _stream(stream)), "zero_reduce_scatter")
+
+
+def adamw_shard_step(layout, shard, reduced, master, m, v, p16_out, hp, stream=None):
+    h = hp.c()
+    _check(_abi.lib().zero_adamw_shard_step(layout.handle, int(shard), _ptr(reduced), _ptr(master), _ptr(m),
+                                            _ptr(v), _ptr(p16_out), ctypes.byref(h), _stream(stream)),
+           "zero_adamw_shard_step")
+
+
+def allgather(layout, unit, p16_shard, p16_full, stream=None):
+    _check(_abi.lib().zero_allgather(layout.handle, int(unit), _ptr(p16_shard), _ptr(p16_full),
+                                     _stream(stream)), "zero_allgather")
+
+
+def step(layout, grads, master, m, v, p16_shard, p16_full, hp, nonfinite=None, events=None,
+         rank_stride=None, stream=None):
+    """events: optional dict of torch.cuda.Event (enable_timing) under the keys
+    update_begin, update_end, gather_begin, gather_end."""
+    h = hp.c()
+    ev = None
+    if events:
+        ev = _abi.StepEvents(*[events[k].cuda_event if k in events else None
+                               for k in ("update_begin", "update_end", "gather_begin", "gather_end")])
+    _check(_abi.lib().zero_step(layout.handle, _ptr(grads), _stride(grads, layout, rank_stride), _ptr(master),
+                                _ptr(m), _ptr(v), _ptr(p16_shard), _ptr(p16_full), ctypes.byref(h),
+                                _ptr(nonfinite), ctypes.byref(ev) if ev is not None else None,
+                                _stream(stream)), "zero_step")
+
+
+def step_host(layout, grads_host, grads_dev, master, m, v, p16_shard, p16_full, p16_host, hp,
+              nonfinite=None, rank_stride=None, stream=None):
+    """grads_host / p16_host: page-locked (pinned) host tensors."""
+    h = hp.c()
+    _check(_abi.lib().zero_step_host(layout.handle, _ptr(grads_host), _ptr(grads_dev),
+                                     _stride(grads_dev, layout, rank_stride), _ptr(master), _ptr(m), _ptr(v),
+                                     _ptr(p16_shard), _ptr(p16_full), _ptr(p16_host), ctypes.byref(h),
+                                     _ptr(nonfinite), _stream(stream)), "zero_step_host")
+
+
+def get_error(layout, stream=None):
+    _check(_abi.lib().zero_get_error(layout.handle, _stream(stream)), "zero_get_error")

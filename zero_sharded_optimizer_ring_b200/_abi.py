@@ -1,0 +1,81 @@
+"""ctypes declarations of the C ABI in include/zero.h (argument marshalling only)."""
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libzero_b200.so")
+
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_i32 = ctypes.c_int32
+_p_i64 = ctypes.POINTER(ctypes.c_int64)
+
+ZERO_OK = 0
+STATUS_NAMES = {0: "ZERO_OK", 1: "ZERO_ERR_INVALID", 2: "ZERO_ERR_ALIGN", 3: "ZERO_ERR_CUDA",
+                4: "ZERO_ERR_OOM", 5: "ZERO_ERR_TIMEOUT", 6: "ZERO_ERR_STATE"}
+
+
+class LayoutDesc(ctypes.Structure):
+    _fields_ = [("n_ranks", _i32), ("stage", _i32), ("n_tensors", _i64),
+                ("tensor_numel", _p_i64), ("bucket_elems", _i64), ("pad_align", _i64),
+                ("n_units", _i64), ("unit_first_tensor", _p_i64)]
+
+
+class LayoutInfo(ctypes.Structure):
+    _fields_ = [("psi", _i64), ("shard", _i64), ("padded", _i64), ("n_buckets", _i64),
+                ("n_segments", _i64), ("n_units", _i64), ("tile_elems", _i64), ("n_tiles", _i64)]
+
+
+class AdamWHparams(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_double), ("beta1", ctypes.c_double), ("beta2", ctypes.c_double),
+                ("eps", ctypes.c_double), ("weight_decay", ctypes.c_double),
+                ("loss_scale", ctypes.c_double), ("step", _i64)]
+
+
+class Counters(ctypes.Structure):
+    _fields_ = [("mem_p16", _i64), ("mem_g16", _i64), ("mem_os", _i64), ("mem_total", _i64),
+                ("sent_elems", _i64), ("recv_elems", _i64)]
+
+
+class StepEvents(ctypes.Structure):
+    _fields_ = [("update_begin", _vp), ("update_end", _vp), ("gather_begin", _vp), ("gather_end", _vp)]
+
+
+# name -> (restype, argtypes); every function declared in include/zero.h
+SIGNATURES = {
+    "zero_layout_create": (_i32, [ctypes.POINTER(LayoutDesc), ctypes.POINTER(_vp)]),
+    "zero_layout_destroy": (None, [_vp]),
+    "zero_layout_get_info": (_i32, [_vp, ctypes.POINTER(LayoutInfo)]),
+    "zero_layout_get_tables": (_i32, [_vp, _vp, _vp, _vp, _vp]),
+    "zero_layout_counters": (_i32, [_vp, ctypes.POINTER(Counters)]),
+    "zero_layout_to_device": (_i32, [_vp, _vp]),
+    "zero_layout_device_segments": (_i32, [_vp, _vp, _vp]),
+    "zero_reduce_scatter": (_i32, [_vp, _i64, _vp, _i64, _vp, _vp, _vp]),
+    "zero_adamw_shard_step": (_i32, [_vp, _i32, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(AdamWHparams), _vp]),
+    "zero_allgather": (_i32, [_vp, _i64, _vp, _vp, _vp]),
+    "zero_step": (_i32, [_vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(AdamWHparams), _vp,
+                         ctypes.POINTER(StepEvents), _vp]),
+    "zero_step_host": (_i32, [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp,
+                              ctypes.POINTER(AdamWHparams), _vp, _vp]),
+    "zero_set_impl": (_i32, [_vp, _i32]),
+    "zero_get_error": (_i32, [_vp, _vp]),
+    "zero_status_string": (ctypes.c_char_p, [_i32]),
+}
+
+_LIB = None
+
+
+def lib():
+    """Load libzero_b200.so.  There is no fallback: without the library nothing runs."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m zero_sharded_optimizer_ring_b200.build` (nvcc, sm_100a)")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = L
+    return _LIB

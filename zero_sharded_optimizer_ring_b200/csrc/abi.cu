@@ -1,0 +1,364 @@
+// extern "C" entry points: argument checks, the AdamW step scalars, kernel launches.
+#include <math.h>
+#include <stdint.h>
+
+#include <vector>
+
+#include "internal.h"
+
+using zero::AdamScalars;
+using zero::Seg;
+using zero::TileWork;
+
+namespace {
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+zero_status check_device(const zero_layout *L)
+{
+    if (!L) return ZERO_ERR_INVALID;
+    if (L->dev.device < 0 || !L->dev.segs) return ZERO_ERR_STATE;
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess) return ZERO_ERR_CUDA;
+    return cur == L->dev.device ? ZERO_OK : ZERO_ERR_STATE;
+}
+
+zero_status cuda_status(cudaError_t e) { return e == cudaSuccess ? ZERO_OK : ZERO_ERR_CUDA; }
+
+bool finite(double x) { return isfinite(x) != 0; }
+
+zero_status check_hparams(const zero_adamw_hparams *h)
+{
+    if (!h) return ZERO_ERR_INVALID;
+    if (h->step < 1 || !finite(h->lr) || !finite(h->eps) || !finite(h->weight_decay) ||
+        !finite(h->loss_scale) || !(h->loss_scale > 0.0) || !(h->beta1 >= 0.0 && h->beta1 < 1.0) ||
+        !(h->beta2 >= 0.0 && h->beta2 < 1.0))
+        return ZERO_ERR_INVALID;
+    return ZERO_OK;
+}
+
+// The step's fp32 scalars, each evaluated in double and rounded once.
+AdamScalars step_scalars(int32_t n_ranks, const zero_adamw_hparams &h)
+{
+    AdamScalars c;
+    const double t = (double)h.step;
+    c.inv_scale = (float)(1.0 / ((double)n_ranks * h.loss_scale));
+    c.decay = (float)(1.0 - h.lr * h.weight_decay);
+    c.beta1 = (float)h.beta1;
+    c.omb1 = (float)(1.0 - h.beta1);
+    c.beta2 = (float)h.beta2;
+    c.omb2 = (float)(1.0 - h.beta2);
+    c.step_size = (float)(h.lr / (1.0 - pow(h.beta1, t)));
+    c.sqrt_bc2 = (float)sqrt(1.0 - pow(h.beta2, t));
+    c.eps = (float)h.eps;
+    return c;
+}
+
+TileWork all_tiles(const zero_layout *L)
+{
+    TileWork w;
+    w.segs = L->dev.segs;
+    w.seg_first = 0;
+    w.tile_first = 0;
+    w.n_tiles = L->n_tiles;
+    return w;
+}
+
+TileWork bucket_tiles(const zero_layout *L, int64_t b)
+{
+    TileWork w;
+    w.segs = L->dev.segs;
+    w.seg_first = L->bucket_seg_begin[(size_t)b];
+    const int64_t seg_end = L->bucket_seg_begin[(size_t)b + 1];
+    w.tile_first = L->segs[(size_t)w.seg_first].tile_begin;
+    const int64_t tile_end = seg_end < (int64_t)L->segs.size() ? L->segs[(size_t)seg_end].tile_begin : L->n_tiles;
+    w.n_tiles = tile_end - w.tile_first;
+    return w;
+}
+
+zero_status check_grads(const zero_layout *L, const void *grads, int64_t rank_stride)
+{
+    if (!grads) return ZERO_ERR_INVALID;
+    if (rank_stride < L->padded) return ZERO_ERR_INVALID;
+    if (!aligned16(grads) || rank_stride % 8 != 0) return ZERO_ERR_ALIGN;
+    return ZERO_OK;
+}
+
+zero_status check_state(const float *master, const float *m, const float *v)
+{
+    if (!master || !m || !v) return ZERO_ERR_INVALID;
+    if (!aligned16(master) || !aligned16(m) || !aligned16(v)) return ZERO_ERR_ALIGN;
+    return ZERO_OK;
+}
+
+void release_device(zero_layout *L)
+{
+    if (L->dev.device < 0) return;
+    int cur = -1;
+    cudaGetDevice(&cur);
+    if (cur != L->dev.device) cudaSetDevice(L->dev.device);
+    for (cudaEvent_t e : L->dev.landed) cudaEventDestroy(e);
+    for (cudaEvent_t e : L->dev.updated) cudaEventDestroy(e);
+    L->dev.landed.clear();
+    L->dev.updated.clear();
+    if (L->dev.begin) cudaEventDestroy(L->dev.begin);
+    if (L->dev.done) cudaEventDestroy(L->dev.done);
+    if (L->dev.copy_in) cudaStreamDestroy(L->dev.copy_in);
+    if (L->dev.copy_out) cudaStreamDestroy(L->dev.copy_out);
+    if (L->dev.segs) cudaFree(L->dev.segs);
+    if (L->dev.error) cudaFree(L->dev.error);
+    if (cur >= 0 && cur != L->dev.device) cudaSetDevice(cur);
+    L->dev = zero::DeviceState();
+}
+
+}  // namespace
+
+extern "C" void zero_layout_destroy(zero_layout *L)
+{
+    if (!L) return;
+    release_device(L);
+    delete L;
+}
+
+extern "C" const char *zero_status_string(zero_status s)
+{
+    switch (s) {
+        case ZERO_OK: return "ok";
+        case ZERO_ERR_INVALID: return "invalid argument";
+        case ZERO_ERR_ALIGN: return "misaligned pointer or stride (need 16-byte pointers, strides multiple of 8)";
+        case ZERO_ERR_CUDA: return "CUDA error";
+        case ZERO_ERR_OOM: return "out of memory";
+        case ZERO_ERR_TIMEOUT: return "a bounded wait in a kernel timed out";
+        case ZERO_ERR_STATE: return "layout not uploaded to the current device";
+    }
+    return "unknown status";
+}
+
+extern "C" zero_status zero_layout_to_device(zero_layout *L, void *stream)
+{
+    if (!L) return ZERO_ERR_INVALID;
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess) return ZERO_ERR_CUDA;
+    if (L->dev.device >= 0) return L->dev.device == cur ? ZERO_OK : ZERO_ERR_STATE;
+    cudaStream_t st = (cudaStream_t)stream;
+    zero::DeviceState &d = L->dev;
+    d.device = cur;
+    if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, cur) != cudaSuccess) {
+        release_device(L);
+        return ZERO_ERR_CUDA;
+    }
+    // rows 0..n_seg-1 from the host partitioner with the tile numbers left blank (-1):
+    // the device builds them; row n_seg is the sentinel.
+    std::vector<Seg> rows(L->segs);
+    for (Seg &s : rows) s.tile_begin = -1;
+    Seg sentinel;
+    sentinel.lo = sentinel.hi = L->padded;
+    sentinel.tile_begin = -1;
+    sentinel.shard = sentinel.bucket = -1;
+    rows.push_back(sentinel);
+    if (cudaMalloc(&d.segs, rows.size() * sizeof(Seg)) != cudaSuccess ||
+        cudaMalloc(&d.error, sizeof(int32_t)) != cudaSuccess) {
+        cudaGetLastError();
+        release_device(L);
+        return ZERO_ERR_OOM;
+    }
+    cudaError_t e = cudaMemcpyAsync(d.segs, rows.data(), rows.size() * sizeof(Seg), cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(d.error, 0, sizeof(int32_t), st);
+    if (e == cudaSuccess) e = zero::launch_tile_index(d.segs, (int64_t)L->segs.size(), st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&d.copy_in, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&d.copy_out, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&d.begin, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&d.done, cudaEventDisableTiming);
+    for (size_t b = 0; e == cudaSuccess && b < L->bucket_lo.size(); ++b) {
+        cudaEvent_t a = nullptr, u = nullptr;
+        e = cudaEventCreateWithFlags(&a, cudaEventDisableTiming);
+        if (e == cudaSuccess) d.landed.push_back(a);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&u, cudaEventDisableTiming);
+        if (e == cudaSuccess) d.updated.push_back(u);
+    }
+    if (e != cudaSuccess) {
+        release_device(L);
+        return ZERO_ERR_CUDA;
+    }
+    return ZERO_OK;
+}
+
+extern "C" zero_status zero_layout_device_segments(const zero_layout *L, int64_t *out, void *stream)
+{
+    zero_status s = check_device(L);
+    if (s != ZERO_OK) return s;
+    if (!out) return ZERO_ERR_INVALID;
+    std::vector<Seg> rows(L->segs.size() + 1);
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = cudaMemcpyAsync(rows.data(), L->dev.segs, rows.size() * sizeof(Seg), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return ZERO_ERR_CUDA;
+    for (size_t i = 0; i < rows.size(); ++i) {
+        out[5 * i + 0] = rows[i].bucket;
+        out[5 * i + 1] = rows[i].shard;
+        out[5 * i + 2] = rows[i].lo;
+        out[5 * i + 3] = rows[i].hi;
+        out[5 * i + 4] = rows[i].tile_begin;
+    }
+    return ZERO_OK;
+}
+
+extern "C" zero_status zero_reduce_scatter(const zero_layout *L, int64_t bucket, const uint16_t *grads,
+                                           int64_t rank_stride, float *reduced, int32_t *nonfinite,
+                                           void *stream)
+{
+    zero_status s = check_device(L);
+    if (s != ZERO_OK) return s;
+    if (bucket < -1 || bucket >= (int64_t)L->bucket_lo.size()) return ZERO_ERR_INVALID;
+    if (L->padded == 0) return ZERO_OK;
+    if ((s = check_grads(L, grads, rank_stride)) != ZERO_OK) return s;
+    if (!reduced) return ZERO_ERR_INVALID;
+    if (!aligned16(reduced)) return ZERO_ERR_ALIGN;
+    const TileWork w = bucket < 0 ? all_tiles(L) : bucket_tiles(L, bucket);
+    return cuda_status(zero::launch_reduce_scatter(*L, w, grads, rank_stride, reduced, nonfinite,
+                                                   (cudaStream_t)stream));
+}
+
+extern "C" zero_status zero_adamw_shard_step(const zero_layout *L, int32_t shard, const float *reduced,
+                                             float *master, float *m, float *v, uint16_t *p16_out,
+                                             const zero_adamw_hparams *hp, void *stream)
+{
+    zero_status s = check_device(L);
+    if (s != ZERO_OK) return s;
+    if (shard < -1 || shard >= L->n_ranks) return ZERO_ERR_INVALID;
+    if ((s = check_hparams(hp)) != ZERO_OK) return s;
+    if (L->padded == 0) return ZERO_OK;
+    if ((s = check_state(master, m, v)) != ZERO_OK) return s;
+    if (!reduced || !p16_out) return ZERO_ERR_INVALID;
+    if (!aligned16(reduced) || !aligned16(p16_out)) return ZERO_ERR_ALIGN;
+    const int64_t lo = shard < 0 ? 0 : (int64_t)shard * L->shard;
+    const int64_t hi = shard < 0 ? L->padded : lo + L->shard;
+    return cuda_status(zero::launch_adamw_range(*L, lo, hi, reduced, master, m, v, p16_out,
+                                                step_scalars(L->n_ranks, *hp), (cudaStream_t)stream));
+}
+
+extern "C" zero_status zero_allgather(const zero_layout *L, int64_t unit, const uint16_t *p16_shard,
+                                      uint16_t *p16_full, void *stream)
+{
+    zero_status s = check_device(L);
+    if (s != ZERO_OK) return s;
+    if (unit < -1 || unit >= (int64_t)L->unit_lo.size()) return ZERO_ERR_INVALID;
+    if (L->padded == 0) return ZERO_OK;
+    if (!p16_shard || !p16_full) return ZERO_ERR_INVALID;
+    if (!aligned16(p16_shard) || !aligned16(p16_full)) return ZERO_ERR_ALIGN;
+    const int64_t lo = unit < 0 ? 0 : L->unit_lo[(size_t)unit];
+    const int64_t hi = unit < 0 ? L->padded : L->unit_hi[(size_t)unit];
+    return cuda_status(zero::launch_copy_range(*L, lo, hi, p16_shard, p16_full, (cudaStream_t)stream));
+}
+
+namespace {
+
+zero_status check_step(const zero_layout *L, const uint16_t *grads, int64_t rank_stride, float *master,
+                       float *m, float *v, uint16_t *p16_shard, uint16_t *p16_full,
+                       const zero_adamw_hparams *hp)
+{
+    zero_status s = check_device(L);
+    if (s != ZERO_OK) return s;
+    if ((s = check_hparams(hp)) != ZERO_OK) return s;
+    if (L->padded == 0) return ZERO_OK;
+    if ((s = check_grads(L, grads, rank_stride)) != ZERO_OK) return s;
+    if ((s = check_state(master, m, v)) != ZERO_OK) return s;
+    if (!p16_full || (L->stage == 3 && !p16_shard)) return ZERO_ERR_INVALID;
+    if (!aligned16(p16_full) || (p16_shard && !aligned16(p16_shard))) return ZERO_ERR_ALIGN;
+    return ZERO_OK;
+}
+
+void record(void *ev, cudaStream_t st)
+{
+    if (ev) cudaEventRecord((cudaEvent_t)ev, st);
+}
+
+}  // namespace
+
+extern "C" zero_status zero_step(const zero_layout *L, const uint16_t *grads, int64_t rank_stride,
+                                 float *master, float *m, float *v, uint16_t *p16_shard,
+                                 uint16_t *p16_full, const zero_adamw_hparams *hp,
+                                 int32_t *nonfinite, const zero_step_events *ev, void *stream)
+{
+    zero_status s = check_step(L, grads, rank_stride, master, m, v, p16_shard, p16_full, hp);
+    if (s != ZERO_OK || L->padded == 0) return s;
+    cudaStream_t st = (cudaStream_t)stream;
+    const AdamScalars c = step_scalars(L->n_ranks, *hp);
+    uint16_t *p16 = L->stage == 3 ? p16_shard : p16_full;
+    if (ev) record(ev->update_begin, st);
+    cudaError_t e = zero::launch_fused_step(*L, all_tiles(L), grads, rank_stride, master, m, v, p16, c,
+                                            nonfinite, st);
+    if (ev) record(ev->update_end, st);
+    if (e == cudaSuccess && L->stage == 3) {
+        if (ev) record(ev->gather_begin, st);
+        e = zero::launch_copy_range(*L, 0, L->padded, p16_shard, p16_full, st);
+        if (ev) record(ev->gather_end, st);
+    }
+    return cuda_status(e);
+}
+
+extern "C" zero_status zero_step_host(const zero_layout *L, const uint16_t *grads_host, uint16_t *grads_dev,
+                                      int64_t rank_stride, float *master, float *m, float *v,
+                                      uint16_t *p16_shard, uint16_t *p16_full, uint16_t *p16_host,
+                                      const zero_adamw_hparams *hp, int32_t *nonfinite, void *stream)
+{
+    zero_status s = check_step(L, grads_dev, rank_stride, master, m, v, p16_shard, p16_full, hp);
+    if (s != ZERO_OK || L->padded == 0) return s;
+    if (!grads_host || !p16_host) return ZERO_ERR_INVALID;
+    cudaStream_t st = (cudaStream_t)stream;
+    const zero::DeviceState &d = L->dev;
+    const AdamScalars c = step_scalars(L->n_ranks, *hp);
+    const size_t nb = L->bucket_lo.size();
+    uint16_t *p16 = L->stage == 3 ? p16_shard : p16_full;
+
+    // the staging buffer may still be read by earlier work on `stream`
+    cudaError_t e = cudaEventRecord(d.begin, st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(d.copy_in, d.begin, 0);
+    for (size_t b = 0; e == cudaSuccess && b < nb; ++b) {
+        const int64_t lo = L->bucket_lo[b], bytes = 2 * (L->bucket_hi[b] - lo);
+        for (int32_t r = 0; e == cudaSuccess && r < L->n_ranks; ++r) {
+            const int64_t off = (int64_t)r * rank_stride + lo;
+            e = cudaMemcpyAsync(grads_dev + off, grads_host + off, (size_t)bytes, cudaMemcpyHostToDevice,
+                                d.copy_in);
+        }
+        if (e == cudaSuccess) e = cudaEventRecord(d.landed[b], d.copy_in);
+    }
+    for (size_t b = 0; e == cudaSuccess && b < nb; ++b) {
+        e = cudaStreamWaitEvent(st, d.landed[b], 0);
+        if (e == cudaSuccess)
+            e = zero::launch_fused_step(*L, bucket_tiles(L, (int64_t)b), grads_dev, rank_stride, master, m, v,
+                                        p16, c, nonfinite, st);
+        if (e == cudaSuccess && L->stage != 3) {
+            e = cudaEventRecord(d.updated[b], st);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(d.copy_out, d.updated[b], 0);
+            const int64_t lo = L->bucket_lo[b], bytes = 2 * (L->bucket_hi[b] - lo);
+            if (e == cudaSuccess)
+                e = cudaMemcpyAsync(p16_host + lo, p16_full + lo, (size_t)bytes, cudaMemcpyDeviceToHost,
+                                    d.copy_out);
+        }
+    }
+    if (e == cudaSuccess && L->stage == 3) {
+        e = zero::launch_copy_range(*L, 0, L->padded, p16_shard, p16_full, st);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(p16_host, p16_full, (size_t)(2 * L->padded), cudaMemcpyDeviceToHost, st);
+    } else if (e == cudaSuccess) {
+        // `stream` completes only after the last parameter copy has landed
+        e = cudaEventRecord(d.done, d.copy_out);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(st, d.done, 0);
+    }
+    return cuda_status(e);
+}
+
+extern "C" zero_status zero_get_error(const zero_layout *L, void *stream)
+{
+    zero_status s = check_device(L);
+    if (s != ZERO_OK) return s;
+    cudaStream_t st = (cudaStream_t)stream;
+    int32_t word = 0;
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e == cudaSuccess) e = cudaMemcpy(&word, L->dev.error, sizeof word, cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess && word != 0) e = cudaMemset(L->dev.error, 0, sizeof word);
+    if (e != cudaSuccess) return ZERO_ERR_CUDA;
+    return word == 0 ? ZERO_OK : (zero_status)word;
+}

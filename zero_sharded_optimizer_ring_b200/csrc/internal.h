@@ -1,0 +1,85 @@
+// Internal definitions shared by the library's translation units (not installed).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <vector>
+
+#include "zero.h"
+
+namespace zero {
+
+// Elements per tile: the unit of work one CTA picks up.  A multiple of 8 so that
+// tile boundaries fall on 16-byte fp16 vectors.
+constexpr int64_t kTileElems = 4096;
+
+// One row of the segment table: chunk `shard` of bucket `bucket`, flat range [lo, hi),
+// whose tiles are numbered tile_begin .. next row's tile_begin - 1.
+struct Seg {
+    int64_t lo, hi, tile_begin;
+    int32_t shard, bucket;
+};
+static_assert(sizeof(Seg) == 32, "device table row is 32 bytes");
+
+// fp32 scalars of one AdamW step, each computed on the host in double and rounded once.
+struct AdamScalars {
+    float inv_scale;   // 1 / (N * loss_scale)
+    float decay;       // 1 - lr * weight_decay
+    float beta1, omb1; // beta1, 1 - beta1
+    float beta2, omb2; // beta2, 1 - beta2
+    float step_size;   // lr / (1 - beta1^t)
+    float sqrt_bc2;    // sqrt(1 - beta2^t)
+    float eps;
+};
+
+// Launch arguments of the tile-walking kernels (reduce-scatter, fused step).
+struct TileWork {
+    const Seg *segs;       // device segment table (n_seg + 1 rows, last = sentinel)
+    int64_t seg_first;     // first row of the launch's range
+    int64_t tile_first;    // first global tile of the launch
+    int64_t n_tiles;       // tiles in the launch
+};
+
+struct DeviceState {
+    int device = -1;
+    Seg *segs = nullptr;          // n_seg + 1 rows
+    int32_t *error = nullptr;     // device error word (timeouts)
+    int num_sms = 0;
+    size_t smem_optin = 0;
+    cudaStream_t copy_in = nullptr, copy_out = nullptr;   // zero_step_host
+    std::vector<cudaEvent_t> landed, updated;              // per bucket
+    cudaEvent_t begin = nullptr, done = nullptr;           // per zero_step_host call
+};
+
+}  // namespace zero
+
+struct zero_layout {
+    int32_t n_ranks = 0, stage = 0;
+    int64_t psi = 0, shard = 0, padded = 0, pad_align = 1, bucket_elems = 0;
+    std::vector<int64_t> tensor_off;
+    std::vector<int64_t> bucket_lo, bucket_hi;
+    std::vector<int64_t> bucket_seg_begin;     // n_buckets + 1: first segment of each bucket
+    std::vector<zero::Seg> segs;               // host copy, tile_begin filled on the host too
+    std::vector<int64_t> unit_lo, unit_hi;
+    int64_t n_tiles = 0;
+    int32_t impl = 0;
+    zero::DeviceState dev;
+};
+
+namespace zero {
+
+// kernels.cu
+cudaError_t launch_tile_index(Seg *segs, int64_t n_seg, cudaStream_t s);
+cudaError_t launch_reduce_scatter(const zero_layout &L, const TileWork &w, const uint16_t *grads,
+                                  int64_t stride, float *reduced, int32_t *nonfinite, cudaStream_t s);
+cudaError_t launch_adamw_range(const zero_layout &L, int64_t lo, int64_t hi, const float *reduced,
+                               float *master, float *m, float *v, uint16_t *p16,
+                               const AdamScalars &c, cudaStream_t s);
+cudaError_t launch_copy_range(const zero_layout &L, int64_t lo, int64_t hi, const uint16_t *src,
+                              uint16_t *dst, cudaStream_t s);
+cudaError_t launch_fused_step(const zero_layout &L, const TileWork &w, const uint16_t *grads,
+                              int64_t stride, float *master, float *m, float *v, uint16_t *p16,
+                              const AdamScalars &c, int32_t *nonfinite, cudaStream_t s);
+
+}  // namespace zero

@@ -1,0 +1,417 @@
+// Device kernels of the sharded optimizer step (sm_100a).
+//
+// Everything here is HBM-bound streaming work: no dense contraction, so no tensor
+// cores.  The kernels move 16-byte vectors (8 fp16 or 4 fp32 values) per thread per
+// access, walk the segment table tile by tile with a persistent grid sized to the SM
+// count, and do every floating-point step as one explicitly rounded IEEE operation
+// (__fadd_rn / __fmul_rn / __fdiv_rn / __fsqrt_rn, no contraction into FMA).
+//
+// Ring order (en.pswp.cn/web/84187, "DDP" walk-through; rkmt.cn/news/44736 "DDP"):
+// chunk k of a bucket starts at rank k and each later rank of the ring adds its own
+// fp32-converted gradient, so the sum for an element of shard k is folded in the fixed
+// order k, k+1, ..., k+N-1 (mod N).  All N ranks' slices are loaded before the fold;
+// only the order of the additions matters for the result.
+//
+// Update (rkmt.cn/news/44736, "Deepspeed ZeRO-1", update step): fp16 -> fp32 without
+// storing it, scale, fp32 first and second moments, fp32 master weights, fp16 params.
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "internal.h"
+
+namespace zero {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kVec = 8;   // elements per 16-byte fp16 vector
+
+__device__ __forceinline__ float h2f(uint32_t bits16)
+{
+    return __half2float(__ushort_as_half((unsigned short)(bits16 & 0xffffu)));
+}
+
+__device__ __forceinline__ uint32_t f2h(float f)
+{
+    return (uint32_t)__half_as_ushort(__float2half_rn(f));
+}
+
+__device__ __forceinline__ void unpack8(const uint4 u, float (&f)[8])
+{
+    f[0] = h2f(u.x); f[1] = h2f(u.x >> 16);
+    f[2] = h2f(u.y); f[3] = h2f(u.y >> 16);
+    f[4] = h2f(u.z); f[5] = h2f(u.z >> 16);
+    f[6] = h2f(u.w); f[7] = h2f(u.w >> 16);
+}
+
+__device__ __forceinline__ void add8(float (&acc)[8], const uint4 u)
+{
+    float f[8];
+    unpack8(u, f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = __fadd_rn(acc[e], f[e]);
+}
+
+// One element of the shard update.  Order of operations as documented in zero.h.
+__device__ __forceinline__ void adamw_elem(float s, const AdamScalars &c, float &p, float &m,
+                                           float &v, uint32_t &h)
+{
+    const float g = __fmul_rn(s, c.inv_scale);
+    const float pd = __fmul_rn(p, c.decay);
+    m = __fadd_rn(__fmul_rn(m, c.beta1), __fmul_rn(g, c.omb1));
+    v = __fadd_rn(__fmul_rn(v, c.beta2), __fmul_rn(__fmul_rn(g, g), c.omb2));
+    const float denom = __fadd_rn(__fdiv_rn(__fsqrt_rn(v), c.sqrt_bc2), c.eps);
+    p = __fsub_rn(pd, __fmul_rn(c.step_size, __fdiv_rn(m, denom)));
+    h = f2h(p);
+}
+
+__device__ __forceinline__ int is_nonfinite(float x) { return !isfinite(x); }
+
+// Adds this thread's non-finite count into counts[bucket]: one atomic per warp.
+__device__ __forceinline__ void flush_nonfinite(int32_t *counts, int32_t bucket, int mine)
+{
+    if (counts == nullptr) return;
+    const unsigned full = 0xffffffffu;
+    if (__any_sync(full, mine != 0)) {
+        const int total = __reduce_add_sync(full, mine);
+        if ((threadIdx.x & 31) == 0) atomicAdd(counts + bucket, total);
+    }
+}
+
+struct TileRange {
+    int64_t a, b;      // [a, b): the tile's elements
+    int32_t shard, bucket;
+};
+
+// Locate tile t: advance the segment cursor s (tiles are visited in increasing order
+// by each CTA, so the cursor only moves forward), then clip the tile's cell of the
+// global kTileElems grid to the segment.
+__device__ __forceinline__ TileRange locate_tile(const Seg *__restrict__ segs, int64_t &s, int64_t t)
+{
+    while (__ldg(&segs[s + 1].tile_begin) <= t) ++s;
+    const int64_t lo = __ldg(&segs[s].lo), hi = __ldg(&segs[s].hi);
+    const int64_t cell = lo / kTileElems + (t - __ldg(&segs[s].tile_begin));
+    TileRange r;
+    r.a = cell * kTileElems > lo ? cell * kTileElems : lo;
+    r.b = (cell + 1) * kTileElems < hi ? (cell + 1) * kTileElems : hi;
+    r.shard = __ldg(&segs[s].shard);
+    r.bucket = __ldg(&segs[s].bucket);
+    return r;
+}
+
+// Rank at position j of the ring fold that starts at rank k.
+__device__ __forceinline__ int ring_rank(int k, int j, int n)
+{
+    const int r = k + j;
+    return r >= n ? r - n : r;
+}
+
+// Scalar ring fold of one element (ragged tile edges, runtime-N path).
+__device__ __forceinline__ float fold_scalar(const uint16_t *__restrict__ grads, int64_t stride,
+                                             int k, int n, int64_t i)
+{
+    float acc = h2f(__ldcs(grads + (int64_t)k * stride + i));
+    for (int j = 1; j < n; ++j)
+        acc = __fadd_rn(acc, h2f(__ldcs(grads + (int64_t)ring_rank(k, j, n) * stride + i)));
+    return acc;
+}
+
+// ---------------------------------------------------------------------------------
+// Tile kernel: ring reduce-scatter of every tile of the launch, then either the
+// fused shard update (kFused) or a store of the fp32 sums.
+//   NT = compile-time rank count (0 = runtime n_ranks), U = vectors per thread whose
+//   loads are in flight together.
+template <int NT, int U, bool kFused>
+__global__ void __launch_bounds__(kThreads)
+tile_kernel(TileWork w, int n_ranks, const uint16_t *__restrict__ grads, int64_t stride,
+            float *__restrict__ reduced, float *__restrict__ master, float *__restrict__ mom1,
+            float *__restrict__ mom2, uint16_t *__restrict__ p16, AdamScalars c,
+            int32_t *__restrict__ nonfinite)
+{
+    const int n = NT > 0 ? NT : n_ranks;
+    int64_t s = w.seg_first;
+    const int64_t t_end = w.tile_first + w.n_tiles;
+    for (int64_t t = w.tile_first + blockIdx.x; t < t_end; t += gridDim.x) {
+        const TileRange tr = locate_tile(w.segs, s, t);
+        const int k = tr.shard;
+        int bad = 0;
+        const int64_t va = (tr.a + kVec - 1) / kVec * kVec;
+        const int64_t vb = tr.b / kVec * kVec;
+
+        // aligned body: 8 elements per vector, U vectors per thread in flight
+        for (int64_t q0 = va + (int64_t)threadIdx.x * kVec; q0 < vb; q0 += (int64_t)U * kThreads * kVec) {
+            float acc[U][8];
+            if constexpr (NT > 0) {
+                uint4 g[U][NT];
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int64_t q = q0 + (int64_t)u * kThreads * kVec;
+                    if (q < vb) {
+#pragma unroll
+                        for (int j = 0; j < NT; ++j)
+                            g[u][j] = __ldcs(reinterpret_cast<const uint4 *>(
+                                grads + (int64_t)ring_rank(k, j, NT) * stride + q));
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    unpack8(g[u][0], acc[u]);
+#pragma unroll
+                    for (int j = 1; j < NT; ++j) add8(acc[u], g[u][j]);
+                }
+            } else {
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int64_t q = q0 + (int64_t)u * kThreads * kVec;
+                    if (q < vb) {
+                        unpack8(__ldcs(reinterpret_cast<const uint4 *>(grads + (int64_t)k * stride + q)), acc[u]);
+#pragma unroll 4
+                        for (int j = 1; j < n; ++j)
+                            add8(acc[u], __ldcs(reinterpret_cast<const uint4 *>(
+                                             grads + (int64_t)ring_rank(k, j, n) * stride + q)));
+                    }
+                }
+            }
+
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int64_t q = q0 + (int64_t)u * kThreads * kVec;
+                if (q >= vb) continue;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) bad += is_nonfinite(acc[u][e]);
+                if constexpr (kFused) {
+                    float4 *pp = reinterpret_cast<float4 *>(master + q);
+                    float4 *mp = reinterpret_cast<float4 *>(mom1 + q);
+                    float4 *vp = reinterpret_cast<float4 *>(mom2 + q);
+                    float4 p4[2] = {__ldcs(pp), __ldcs(pp + 1)};
+                    float4 m4[2] = {__ldcs(mp), __ldcs(mp + 1)};
+                    float4 v4[2] = {__ldcs(vp), __ldcs(vp + 1)};
+                    float *pf = reinterpret_cast<float *>(p4);
+                    float *mf = reinterpret_cast<float *>(m4);
+                    float *vf = reinterpret_cast<float *>(v4);
+                    uint32_t h[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) adamw_elem(acc[u][e], c, pf[e], mf[e], vf[e], h[e]);
+                    __stcs(pp, p4[0]); __stcs(pp + 1, p4[1]);
+                    __stcs(mp, m4[0]); __stcs(mp + 1, m4[1]);
+                    __stcs(vp, v4[0]); __stcs(vp + 1, v4[1]);
+                    __stcs(reinterpret_cast<uint4 *>(p16 + q),
+                           make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16),
+                                      h[4] | (h[5] << 16), h[6] | (h[7] << 16)));
+                } else {
+                    float4 *rp = reinterpret_cast<float4 *>(reduced + q);
+                    __stcs(rp, make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]));
+                    __stcs(rp + 1, make_float4(acc[u][4], acc[u][5], acc[u][6], acc[u][7]));
+                }
+            }
+        }
+
+        // ragged edges of the tile (segment boundaries that are not 8-aligned)
+        const int64_t head_end = va < tr.b ? va : tr.b;
+        const int64_t tail_begin = vb > head_end ? vb : head_end;
+        const int64_t n_head = head_end - tr.a, n_tail = tr.b - tail_begin;
+        if (threadIdx.x < n_head + n_tail) {
+            const int64_t i = threadIdx.x < n_head ? tr.a + threadIdx.x : tail_begin + (threadIdx.x - n_head);
+            const float acc = fold_scalar(grads, stride, k, n, i);
+            bad += is_nonfinite(acc);
+            if constexpr (kFused) {
+                float p = master[i], m = mom1[i], v = mom2[i];
+                uint32_t h;
+                adamw_elem(acc, c, p, m, v, h);
+                master[i] = p;
+                mom1[i] = m;
+                mom2[i] = v;
+                p16[i] = (uint16_t)h;
+            } else {
+                reduced[i] = acc;
+            }
+        }
+        flush_nonfinite(nonfinite, tr.bucket, bad);
+    }
+}
+
+// ---------------------------------------------------------------------------------
+// Range kernels over [lo, hi) with an aligned 16-byte body and scalar edges.
+
+__global__ void __launch_bounds__(kThreads)
+adamw_range_kernel(int64_t lo, int64_t hi, const float *__restrict__ reduced, float *__restrict__ master,
+                   float *__restrict__ mom1, float *__restrict__ mom2, uint16_t *__restrict__ p16,
+                   AdamScalars c)
+{
+    const int64_t va = (lo + kVec - 1) / kVec * kVec, vb = hi / kVec * kVec;
+    const int64_t stride = (int64_t)gridDim.x * kThreads * kVec;
+    for (int64_t q = va + ((int64_t)blockIdx.x * kThreads + threadIdx.x) * kVec; q < vb; q += stride) {
+        const float4 *rp = reinterpret_cast<const float4 *>(reduced + q);
+        float4 *pp = reinterpret_cast<float4 *>(master + q);
+        float4 *mp = reinterpret_cast<float4 *>(mom1 + q);
+        float4 *vp = reinterpret_cast<float4 *>(mom2 + q);
+        float4 r4[2] = {__ldcs(rp), __ldcs(rp + 1)};
+        float4 p4[2] = {__ldcs(pp), __ldcs(pp + 1)};
+        float4 m4[2] = {__ldcs(mp), __ldcs(mp + 1)};
+        float4 v4[2] = {__ldcs(vp), __ldcs(vp + 1)};
+        const float *rf = reinterpret_cast<const float *>(r4);
+        float *pf = reinterpret_cast<float *>(p4);
+        float *mf = reinterpret_cast<float *>(m4);
+        float *vf = reinterpret_cast<float *>(v4);
+        uint32_t h[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) adamw_elem(rf[e], c, pf[e], mf[e], vf[e], h[e]);
+        __stcs(pp, p4[0]); __stcs(pp + 1, p4[1]);
+        __stcs(mp, m4[0]); __stcs(mp + 1, m4[1]);
+        __stcs(vp, v4[0]); __stcs(vp + 1, v4[1]);
+        __stcs(reinterpret_cast<uint4 *>(p16 + q),
+               make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16)));
+    }
+    if (blockIdx.x == 0) {
+        const int64_t head_end = va < hi ? va : hi;
+        const int64_t tail_begin = vb > head_end ? vb : head_end;
+        const int64_t n_head = head_end - lo, n_tail = hi - tail_begin;
+        if (threadIdx.x < n_head + n_tail) {
+            const int64_t i = threadIdx.x < n_head ? lo + threadIdx.x : tail_begin + (threadIdx.x - n_head);
+            float p = master[i], m = mom1[i], v = mom2[i];
+            uint32_t h;
+            adamw_elem(reduced[i], c, p, m, v, h);
+            master[i] = p;
+            mom1[i] = m;
+            mom2[i] = v;
+            p16[i] = (uint16_t)h;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kThreads)
+copy_range_kernel(int64_t lo, int64_t hi, const uint16_t *__restrict__ src, uint16_t *__restrict__ dst)
+{
+    const int64_t va = (lo + kVec - 1) / kVec * kVec, vb = hi / kVec * kVec;
+    const int64_t stride = (int64_t)gridDim.x * kThreads * kVec;
+    for (int64_t q = va + ((int64_t)blockIdx.x * kThreads + threadIdx.x) * kVec; q < vb; q += stride)
+        __stcs(reinterpret_cast<uint4 *>(dst + q), __ldcs(reinterpret_cast<const uint4 *>(src + q)));
+    if (blockIdx.x == 0) {
+        const int64_t head_end = va < hi ? va : hi;
+        const int64_t tail_begin = vb > head_end ? vb : head_end;
+        const int64_t n_head = head_end - lo, n_tail = hi - tail_begin;
+        if (threadIdx.x < n_head + n_tail) {
+            const int64_t i = threadIdx.x < n_head ? lo + threadIdx.x : tail_begin + (threadIdx.x - n_head);
+            dst[i] = src[i];
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------------
+// Tile index: one warp scans the segments' tile counts (exclusive prefix sum with
+// __shfl_up_sync, 32 segments per pass, carried across passes).  Row n_seg receives
+// the total, closing the table.
+__global__ void tile_index_kernel(Seg *segs, int64_t n_seg)
+{
+    const unsigned full = 0xffffffffu;
+    const int lane = threadIdx.x;
+    int64_t carry = 0;
+    for (int64_t base = 0; base < n_seg; base += 32) {
+        const int64_t i = base + lane;
+        int64_t cnt = 0;
+        if (i < n_seg) {
+            const int64_t lo = segs[i].lo, hi = segs[i].hi;
+            cnt = (hi + kTileElems - 1) / kTileElems - lo / kTileElems;
+        }
+        int64_t x = cnt;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int64_t y = __shfl_up_sync(full, x, off);
+            if (lane >= off) x += y;
+        }
+        if (i < n_seg) segs[i].tile_begin = carry + x - cnt;
+        carry += __shfl_sync(full, x, 31);
+    }
+    if (lane == 0) segs[n_seg].tile_begin = carry;
+}
+
+template <class K>
+int grid_for(K kernel, int64_t work_items, int num_sms)
+{
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0) != cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    int64_t g = (int64_t)per_sm * (num_sms > 0 ? num_sms : 148);
+    if (g > work_items) g = work_items;
+    return (int)(g < 1 ? 1 : g);
+}
+
+template <int NT, int U, bool kFused>
+cudaError_t launch_tiles(const zero_layout &L, const TileWork &w, const uint16_t *grads, int64_t stride,
+                         float *reduced, float *master, float *m, float *v, uint16_t *p16,
+                         const AdamScalars &c, int32_t *nonfinite, cudaStream_t st)
+{
+    auto kern = tile_kernel<NT, U, kFused>;
+    const int grid = grid_for(kern, w.n_tiles, L.dev.num_sms);
+    kern<<<grid, kThreads, 0, st>>>(w, L.n_ranks, grads, stride, reduced, master, m, v, p16, c, nonfinite);
+    return cudaGetLastError();
+}
+
+template <bool kFused>
+cudaError_t dispatch_tiles(const zero_layout &L, const TileWork &w, const uint16_t *grads, int64_t stride,
+                           float *reduced, float *master, float *m, float *v, uint16_t *p16,
+                           const AdamScalars &c, int32_t *nonfinite, cudaStream_t st)
+{
+    if (w.n_tiles <= 0) return cudaSuccess;
+#define ZERO_CASE(NV, UV) \
+    case NV: return launch_tiles<NV, UV, kFused>(L, w, grads, stride, reduced, master, m, v, p16, c, nonfinite, st);
+    switch (L.n_ranks) {
+        ZERO_CASE(1, 2)
+        ZERO_CASE(2, 2)
+        ZERO_CASE(3, 2)
+        ZERO_CASE(4, 2)
+        ZERO_CASE(5, 1)
+        ZERO_CASE(6, 1)
+        ZERO_CASE(7, 1)
+        ZERO_CASE(8, 1)
+        ZERO_CASE(16, 1)
+        default:
+            return launch_tiles<0, 1, kFused>(L, w, grads, stride, reduced, master, m, v, p16, c, nonfinite, st);
+    }
+#undef ZERO_CASE
+}
+
+}  // namespace
+
+cudaError_t launch_tile_index(Seg *segs, int64_t n_seg, cudaStream_t s)
+{
+    tile_index_kernel<<<1, 32, 0, s>>>(segs, n_seg);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_reduce_scatter(const zero_layout &L, const TileWork &w, const uint16_t *grads,
+                                  int64_t stride, float *reduced, int32_t *nonfinite, cudaStream_t s)
+{
+    return dispatch_tiles<false>(L, w, grads, stride, reduced, nullptr, nullptr, nullptr, nullptr,
+                                 AdamScalars{}, nonfinite, s);
+}
+
+cudaError_t launch_fused_step(const zero_layout &L, const TileWork &w, const uint16_t *grads,
+                              int64_t stride, float *master, float *m, float *v, uint16_t *p16,
+                              const AdamScalars &c, int32_t *nonfinite, cudaStream_t s)
+{
+    return dispatch_tiles<true>(L, w, grads, stride, nullptr, master, m, v, p16, c, nonfinite, s);
+}
+
+cudaError_t launch_adamw_range(const zero_layout &L, int64_t lo, int64_t hi, const float *reduced,
+                               float *master, float *m, float *v, uint16_t *p16,
+                               const AdamScalars &c, cudaStream_t s)
+{
+    if (hi <= lo) return cudaSuccess;
+    const int grid = grid_for(adamw_range_kernel, (hi - lo + kThreads * kVec - 1) / (kThreads * kVec),
+                              L.dev.num_sms);
+    adamw_range_kernel<<<grid, kThreads, 0, s>>>(lo, hi, reduced, master, m, v, p16, c);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_copy_range(const zero_layout &L, int64_t lo, int64_t hi, const uint16_t *src,
+                              uint16_t *dst, cudaStream_t s)
+{
+    if (hi <= lo) return cudaSuccess;
+    const int grid = grid_for(copy_range_kernel, (hi - lo + kThreads * kVec - 1) / (kThreads * kVec),
+                              L.dev.num_sms);
+    copy_range_kernel<<<grid, kThreads, 0, s>>>(lo, hi, src, dst);
+    return cudaGetLastError();
+}
+
+}  // namespace zero
