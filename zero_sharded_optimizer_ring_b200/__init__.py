@@ -164,8 +164,13 @@ def step(layout, grads, master, m, v, p16_shard, p16_full, hp, nonfinite=None, e
     h = hp.c()
     ev = None
     if events:
-        ev = _abi.StepEvents(*[events[k].cuda_event if k in events else None
-                               for k in ("update_begin", "update_end", "gather_begin", "gather_end")])
+        handles = []
+        for k in ("update_begin", "update_end", "gather_begin", "gather_end"):
+            e = events.get(k)
+            if e is not None and e.cuda_event == 0:
+                e.record()          # torch creates the cudaEvent_t on first record
+            handles.append(e.cuda_event if e is not None else None)
+        ev = _abi.StepEvents(*handles)
     _check(_abi.lib().zero_step(layout.handle, _ptr(grads), _stride(grads, layout, rank_stride), _ptr(master),
                                 _ptr(m), _ptr(v), _ptr(p16_shard), _ptr(p16_full), ctypes.byref(h),
                                 _ptr(nonfinite), ctypes.byref(ev) if ev is not None else None,
