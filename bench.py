@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=4)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-seconds", type=float, default=120.0,
+                    help="--impl reference: oracle time budget of the whole run")
     ap.add_argument("--kernel", type=int, default=0, help="fused kernel: 0 auto, 1 register, 2 bulk")
     ap.add_argument("--psi", type=int, default=0,
                     help="flat workloads only: run the same shape with this many parameters "
@@ -57,6 +59,22 @@ def parse():
 
 def dist_env():
     return int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)), int(os.environ.get("WORLD_SIZE", 1))
+
+
+def max_over_ranks(x, world, device):
+    """The largest of the ranks' values (timing: the slowest rank defines the step)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def throughput(psi, world, ms):
+    """Whole-job parameters per second: every rank updates its own replica of psi."""
+    return psi * world / (ms / 1e3)
 
 
 def ideal_bytes_per_param(wl):
@@ -180,7 +198,7 @@ def run_reference(a, wl):
     rank, _, world = dist_env()
     if rank != 0:
         return
-    per_step = 120.0 / (a.steps + a.warmup)
+    per_step = a.ref_seconds / (a.steps + a.warmup)
     psi_s = size_sample(wl, per_step)
     for _ in range(a.warmup):
         oracle_sample_run(wl, psi_s)
@@ -211,13 +229,6 @@ def run_ours(a, wl):
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
-
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     def barrier():
         torch.cuda.synchronize()
@@ -268,11 +279,11 @@ def run_ours(a, wl):
     barrier()
     clocks = sampler.stop() if sampler else None
     zs.get_error(lay)
-    ms = max_over_ranks(start.elapsed_time(end) / K)
-    upd_ms = max_over_ranks(sum(e["update_begin"].elapsed_time(e["update_end"]) for e in ev) / K)
+    ms = max_over_ranks(start.elapsed_time(end) / K, world, "cuda")
+    upd_ms = max_over_ranks(sum(e["update_begin"].elapsed_time(e["update_end"]) for e in ev) / K, world, "cuda")
     gat_ms = None
     if wl.stage == 3:
-        gat_ms = max_over_ranks(sum(e["gather_begin"].elapsed_time(e["gather_end"]) for e in ev) / K)
+        gat_ms = max_over_ranks(sum(e["gather_begin"].elapsed_time(e["gather_end"]) for e in ev) / K, world, "cuda")
     launches_per_step = 2 if wl.stage == 3 else 1
 
     # end to end through the host-buffer entry point: gradients from pinned host memory
@@ -296,8 +307,8 @@ def run_ours(a, wl):
             zs.step_host(lay, g_host, ge, master, m, v, p16_shard, p16_full, p16_host, hp(t))
         e2.record()
         barrier()
-        e2e_ms = max_over_ranks(s2.elapsed_time(e2) / a.e2e_steps)
-        e2e = {"value": psi * world / (e2e_ms / 1e3), "unit": UNIT, "ms_per_step": e2e_ms,
+        e2e_ms = max_over_ranks(s2.elapsed_time(e2) / a.e2e_steps, world, "cuda")
+        e2e = {"value": throughput(psi, world, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": 2 * N * P, "d2h_bytes_per_step": 2 * P,
                "steps": a.e2e_steps, "path": "zero_step_host (pinned host grads in, fp16 params out)"}
 
@@ -306,19 +317,21 @@ def run_ours(a, wl):
     if rank != 0:
         return
 
+    impl_name = {0: "automatic choice", 1: "register streaming (tile_kernel)",
+                 2: "bulk-copy pipeline (bulk_step_kernel)"}[a.kernel]
     peak, peak_kind = hbm_peak()
     fused_bytes = fused_bytes_per_param(wl) * P
     achieved = fused_bytes / (upd_ms / 1e3) / 1e9
     traffic_pp = profiled_traffic(wl.name)
     step_bytes = ideal_bytes_per_param(wl) * P
     out = {
-        "metric": METRIC, "value": psi * world / (ms / 1e3), "unit": UNIT, "n_gpus": world, "steps": K,
+        "metric": METRIC, "value": throughput(psi, world, ms), "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": workload_config(wl, world),
         "hbm": {"achieved_gbs_step": step_bytes / (ms / 1e3) / 1e9, "ideal_bytes_per_param": ideal_bytes_per_param(wl),
                 "frac_of_measured_peak": step_bytes / (ms / 1e3) / 1e9 / peak,
                 "frac_of_nominal_8tbs": step_bytes / (ms / 1e3) / 1e9 / NOMINAL_HBM_GBS},
-        "roofline": {"bound": "hbm", "kernel": "fused reduce-scatter + AdamW (tile_kernel)",
+        "roofline": {"bound": "hbm", "kernel": "fused reduce-scatter + AdamW, " + impl_name,
                      "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": achieved / peak, "kernel_ms": upd_ms,
                      "algorithmic_bytes_per_launch": fused_bytes,

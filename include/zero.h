@@ -188,6 +188,14 @@ zero_status zero_step_host(const zero_layout *layout, const uint16_t *grads_host
  * into a shared-memory ring, warp-specialised).  Results are identical. */
 zero_status zero_set_impl(zero_layout *layout, int32_t impl);
 
+/* Test hook of the bulk-copy pipeline's bounded waits: every in-kernel wait gives up
+ * after wait_limit_ns nanoseconds (default 2e9) and records ZERO_ERR_TIMEOUT.  With
+ * skip_first_fill = 1 the pipeline never posts its first chunk, so the consumers' wait
+ * for it expires: the kernel then drains its own copies and returns, and
+ * zero_get_error() reports ZERO_ERR_TIMEOUT (the GPU context stays usable).  Set
+ * skip_first_fill back to 0 for normal use.  Requires an uploaded layout. */
+zero_status zero_debug_set_wait(zero_layout *layout, int64_t wait_limit_ns, int32_t skip_first_fill);
+
 /* Synchronise `stream`, read and clear the layout's device error word. */
 zero_status zero_get_error(const zero_layout *layout, void *stream);
 

@@ -25,9 +25,14 @@ def _hp(wl, t):
     return zs.AdamW(wl.lr, wl.beta1, wl.beta2, wl.eps, wl.weight_decay, wl.loss_scale, t)
 
 
-def _layout(wl):
-    return zs.Layout(list(wl.tensors), wl.n_ranks, wl.stage, wl.bucket_elems, wl.pad_align,
-                     list(wl.units)).to_device()
+def _layout(wl, impl=zs.IMPL_REGISTER):
+    lay = zs.Layout(list(wl.tensors), wl.n_ranks, wl.stage, wl.bucket_elems, wl.pad_align,
+                    list(wl.units)).to_device()
+    lay.set_impl(impl)
+    return lay
+
+
+IMPLS = [zs.IMPL_REGISTER, zs.IMPL_BULK]
 
 
 def _bufs(lay, wl, rank_stride=None):
@@ -82,11 +87,12 @@ def _free():
 
 # ------------------------------------------------------------- reduced-size, every element
 
+@pytest.mark.parametrize("impl", IMPLS)
 @pytest.mark.parametrize("key", list(reduced_workloads()))
-def test_reduced_workload_all_elements(key):
+def test_reduced_workload_all_elements(key, impl):
     wl = reduced_workloads()[key]
     ref, olay = _oracle(wl)
-    lay = _layout(wl)
+    lay = _layout(wl, impl)
     assert lay.n_tiles >= 8 and lay.n_buckets >= 1     # several tiles, ragged edges
     b = _bufs(lay, wl)
     _run(lay, wl, b, wl.steps)
@@ -167,11 +173,12 @@ EDGES = {
 }
 
 
+@pytest.mark.parametrize("impl", IMPLS)
 @pytest.mark.parametrize("key", list(EDGES))
-def test_edge_cases(key):
+def test_edge_cases(key, impl):
     wl = EDGES[key]
     ref, _ = _oracle(wl)
-    lay = _layout(wl)
+    lay = _layout(wl, impl)
     b = _bufs(lay, wl)
     _run(lay, wl, b, wl.steps)
     _check_full(wl, lay, b, ref)
@@ -275,11 +282,12 @@ def test_host_buffer_step_equals_device_step():
 
 # ------------------------------------------------------------- full size, sampled
 
+@pytest.mark.parametrize("impl", IMPLS)
 @pytest.mark.parametrize("key", list(full_workloads()))
-def test_full_size_sampled(key):
+def test_full_size_sampled(key, impl):
     wl = full_workloads()[key]
     olay = S.oracle_layout(wl)
-    lay = _layout(wl)
+    lay = _layout(wl, impl)
     b = _bufs(lay, wl)
     _run(lay, wl, b, wl.steps)
     idx = S.sample_indices(olay)
@@ -305,3 +313,23 @@ def test_full_size_sampled(key):
     # the padding stayed zero
     assert int(torch.count_nonzero(b["p16_full"][lay.psi:])) == 0
     assert int(torch.count_nonzero(b["master"][lay.psi:])) == 0
+
+
+def test_bulk_pipeline_bounded_wait_reports_timeout():
+    """The bulk pipeline's waits are bounded: with its first chunk never posted, the
+    consumers' wait expires after 1 ms, the kernel drains and returns, the host reads
+    ZERO_ERR_TIMEOUT, and the same context then runs a correct step."""
+    wl = reduced_workloads()["flat1p3b_n4_zero1"]
+    ref, _ = _oracle(wl, steps=1)
+    lay = _layout(wl, zs.IMPL_BULK)
+    b = _bufs(lay, wl)
+    lay.debug_set_wait(1_000_000, skip_first_fill=1)
+    zs.step(lay, b["g"], b["master"], b["m"], b["v"], b["p16_shard"], b["p16_full"], _hp(wl, 1))
+    with pytest.raises(zs.ZeroError) as e:
+        zs.get_error(lay)
+    assert e.value.status == 5
+    zs.get_error(lay)                        # the word was cleared
+    lay.debug_set_wait(2_000_000_000, skip_first_fill=0)
+    b = _bufs(lay, wl)
+    _run(lay, wl, b, 1)
+    _check_full(wl, lay, b, ref)

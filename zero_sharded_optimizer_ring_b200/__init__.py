@@ -130,6 +130,10 @@ class Layout:
     def set_impl(self, impl):
         _check(_abi.lib().zero_set_impl(self._h, int(impl)), "zero_set_impl")
 
+    def debug_set_wait(self, wait_limit_ns, skip_first_fill=0):
+        _check(_abi.lib().zero_debug_set_wait(self._h, int(wait_limit_ns), int(skip_first_fill)),
+               "zero_debug_set_wait")
+
 
 def _stride(grads, layout, rank_stride):
     if rank_stride is not None:

@@ -58,6 +58,7 @@ SIGNATURES = {
     "zero_step_host": (_i32, [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp,
                               ctypes.POINTER(AdamWHparams), _vp, _vp]),
     "zero_set_impl": (_i32, [_vp, _i32]),
+    "zero_debug_set_wait": (_i32, [_vp, _i64, _i32]),
     "zero_get_error": (_i32, [_vp, _vp]),
     "zero_status_string": (ctypes.c_char_p, [_i32]),
 }

@@ -143,10 +143,13 @@ extern "C" zero_status zero_layout_to_device(zero_layout *L, void *stream)
     cudaStream_t st = (cudaStream_t)stream;
     zero::DeviceState &d = L->dev;
     d.device = cur;
-    if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, cur) != cudaSuccess) {
+    int optin = 0;
+    if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, cur) != cudaSuccess ||
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, cur) != cudaSuccess) {
         release_device(L);
         return ZERO_ERR_CUDA;
     }
+    d.smem_optin = (size_t)optin;
     // rows 0..n_seg-1 from the host partitioner with the tile numbers left blank (-1):
     // the device builds them; row n_seg is the sentinel.
     std::vector<Seg> rows(L->segs);
@@ -274,6 +277,17 @@ void record(void *ev, cudaStream_t st)
     if (ev) cudaEventRecord((cudaEvent_t)ev, st);
 }
 
+// The fused reduce-scatter + update over the tiles of `w`, in the selected implementation.
+cudaError_t fused(const zero_layout *L, const TileWork &w, const uint16_t *grads, int64_t stride, float *master,
+                  float *m, float *v, uint16_t *p16, const AdamScalars &c, int32_t *nonfinite, cudaStream_t st)
+{
+    const bool bulk = L->impl == 2 && zero::bulk_supported(L->n_ranks);
+    if (bulk)
+        return zero::launch_bulk_step(*L, w, grads, stride, master, m, v, p16, c, nonfinite, L->dev.wait_limit_ns,
+                                      L->dev.skip_first_fill, st);
+    return zero::launch_fused_step(*L, w, grads, stride, master, m, v, p16, c, nonfinite, st);
+}
+
 }  // namespace
 
 extern "C" zero_status zero_step(const zero_layout *L, const uint16_t *grads, int64_t rank_stride,
@@ -287,8 +301,7 @@ extern "C" zero_status zero_step(const zero_layout *L, const uint16_t *grads, in
     const AdamScalars c = step_scalars(L->n_ranks, *hp);
     uint16_t *p16 = L->stage == 3 ? p16_shard : p16_full;
     if (ev) record(ev->update_begin, st);
-    cudaError_t e = zero::launch_fused_step(*L, all_tiles(L), grads, rank_stride, master, m, v, p16, c,
-                                            nonfinite, st);
+    cudaError_t e = fused(L, all_tiles(L), grads, rank_stride, master, m, v, p16, c, nonfinite, st);
     if (ev) record(ev->update_end, st);
     if (e == cudaSuccess && L->stage == 3) {
         if (ev) record(ev->gather_begin, st);
@@ -327,8 +340,7 @@ extern "C" zero_status zero_step_host(const zero_layout *L, const uint16_t *grad
     for (size_t b = 0; e == cudaSuccess && b < nb; ++b) {
         e = cudaStreamWaitEvent(st, d.landed[b], 0);
         if (e == cudaSuccess)
-            e = zero::launch_fused_step(*L, bucket_tiles(L, (int64_t)b), grads_dev, rank_stride, master, m, v,
-                                        p16, c, nonfinite, st);
+            e = fused(L, bucket_tiles(L, (int64_t)b), grads_dev, rank_stride, master, m, v, p16, c, nonfinite, st);
         if (e == cudaSuccess && L->stage != 3) {
             e = cudaEventRecord(d.updated[b], st);
             if (e == cudaSuccess) e = cudaStreamWaitEvent(d.copy_out, d.updated[b], 0);
@@ -361,4 +373,13 @@ extern "C" zero_status zero_get_error(const zero_layout *L, void *stream)
     if (e == cudaSuccess && word != 0) e = cudaMemset(L->dev.error, 0, sizeof word);
     if (e != cudaSuccess) return ZERO_ERR_CUDA;
     return word == 0 ? ZERO_OK : (zero_status)word;
+}
+
+extern "C" zero_status zero_debug_set_wait(zero_layout *L, int64_t wait_limit_ns, int32_t skip_first_fill)
+{
+    if (!L || wait_limit_ns <= 0 || skip_first_fill < 0 || skip_first_fill > 1) return ZERO_ERR_INVALID;
+    if (L->dev.device < 0) return ZERO_ERR_STATE;
+    L->dev.wait_limit_ns = (uint64_t)wait_limit_ns;
+    L->dev.skip_first_fill = skip_first_fill;
+    return ZERO_OK;
 }

@@ -1,0 +1,383 @@
+// Fused step, bulk-copy pipeline variant (sm_100a).
+//
+// Same computation as the register-streaming tile kernel (ring-order fp32 fold of the N
+// ranks' fp16 gradients, scale, AdamW, fp16 write; rkmt.cn/news/44736 "DDP" and
+// "Deepspeed ZeRO-1", en.pswp.cn/web/84187 "DDP"), staged differently:
+//
+//   warp 0, lane 0 (producer): for each 2048-element chunk of its tiles, waits for a free
+//     stage of a shared-memory ring, posts the stage's byte count on the stage's "full"
+//     mbarrier and issues one cp.async.bulk (global -> shared, no tensor map, no
+//     multicast) per gradient slice (ranks in ring order) and per state array;
+//   warps 1..8 (consumers): wait for the stage to fill, fold / update from shared memory
+//     (16-byte vectors, conflict-free for the gradients), store results with 16-byte
+//     streaming stores, and release the stage on its "empty" mbarrier.
+//
+// Up to `stages` chunks are in flight per SM without holding any of them in registers,
+// which is what the register-streaming variant lacks at high register counts.
+//
+// Every wait is bounded by the global timer.  When a wait expires the kernel writes
+// ZERO_ERR_TIMEOUT to the error word, raises a CTA-wide abort flag that every other
+// wait polls, the producer waits (again bounded) for the copies it has issued to land,
+// and all threads return.  No trap, no unbounded spin.
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "internal.h"
+
+namespace zero {
+namespace {
+
+constexpr int kConsumerWarps = 8;
+constexpr int kBulkThreads = 32 * (1 + kConsumerWarps);
+constexpr int kChunk = 2048;                 // elements per pipeline stage
+constexpr int kVec = 8;
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p)
+{
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ uint64_t global_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Bounded wait for the phase of `parity` to complete.  Returns false when the wait
+// gave up (time limit, or another thread of the CTA raised the abort flag).
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                           int32_t *error, uint64_t limit_ns)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 63u) == 0) {
+            if (*abort_flag) return false;
+            if (global_ns() - t0 > limit_ns) {
+                atomicExch(error, (int32_t)ZERO_ERR_TIMEOUT);
+                *abort_flag = 1;
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ float h2f(uint32_t bits16)
+{
+    return __half2float(__ushort_as_half((unsigned short)(bits16 & 0xffffu)));
+}
+
+__device__ __forceinline__ uint32_t f2h(float f)
+{
+    return (uint32_t)__half_as_ushort(__float2half_rn(f));
+}
+
+__device__ __forceinline__ void add8(float (&acc)[8], const uint4 u)
+{
+    acc[0] = __fadd_rn(acc[0], h2f(u.x)); acc[1] = __fadd_rn(acc[1], h2f(u.x >> 16));
+    acc[2] = __fadd_rn(acc[2], h2f(u.y)); acc[3] = __fadd_rn(acc[3], h2f(u.y >> 16));
+    acc[4] = __fadd_rn(acc[4], h2f(u.z)); acc[5] = __fadd_rn(acc[5], h2f(u.z >> 16));
+    acc[6] = __fadd_rn(acc[6], h2f(u.w)); acc[7] = __fadd_rn(acc[7], h2f(u.w >> 16));
+}
+
+__device__ __forceinline__ void adamw_elem(float s, const AdamScalars &c, float &p, float &m, float &v,
+                                           uint32_t &h)
+{
+    const float g = __fmul_rn(s, c.inv_scale);
+    const float pd = __fmul_rn(p, c.decay);
+    m = __fadd_rn(__fmul_rn(m, c.beta1), __fmul_rn(g, c.omb1));
+    v = __fadd_rn(__fmul_rn(v, c.beta2), __fmul_rn(__fmul_rn(g, g), c.omb2));
+    const float denom = __fadd_rn(__fdiv_rn(__fsqrt_rn(v), c.sqrt_bc2), c.eps);
+    p = __fsub_rn(pd, __fmul_rn(c.step_size, __fdiv_rn(m, denom)));
+    h = f2h(p);
+}
+
+__device__ __forceinline__ int ring_rank(int k, int j, int n)
+{
+    const int r = k + j;
+    return r >= n ? r - n : r;
+}
+
+struct TileRange {
+    int64_t a, b;
+    int32_t shard, bucket;
+};
+
+__device__ __forceinline__ TileRange locate_tile(const Seg *__restrict__ segs, int64_t &s, int64_t t)
+{
+    while (__ldg(&segs[s + 1].tile_begin) <= t) ++s;
+    const int64_t lo = __ldg(&segs[s].lo), hi = __ldg(&segs[s].hi);
+    const int64_t cell = lo / kTileElems + (t - __ldg(&segs[s].tile_begin));
+    TileRange r;
+    r.a = cell * kTileElems > lo ? cell * kTileElems : lo;
+    r.b = (cell + 1) * kTileElems < hi ? (cell + 1) * kTileElems : hi;
+    r.shard = __ldg(&segs[s].shard);
+    r.bucket = __ldg(&segs[s].bucket);
+    return r;
+}
+
+struct BulkArgs {
+    TileWork w;
+    const uint16_t *grads;
+    int64_t stride;
+    float *master, *mom1, *mom2;
+    uint16_t *p16;
+    AdamScalars c;
+    int32_t *nonfinite;
+    int32_t *error;
+    uint64_t wait_limit_ns;
+    int32_t stages;
+    int32_t skip_first_fill;   // test hook: never post chunk 0, so its consumers' wait expires
+};
+
+// Shared memory: [full[S], empty[S] mbarriers][abort flag] ... stage ring (128-B aligned):
+// stage s = N gradient slices of kChunk fp16, then master, m, v slices of kChunk fp32.
+template <int N>
+__global__ void __launch_bounds__(kBulkThreads, 1) bulk_step_kernel(BulkArgs A)
+{
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem);
+    uint64_t *empty = full + A.stages;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + A.stages);
+    unsigned char *ring = smem + ((16 * A.stages + 4 + 127) / 128) * 128;
+    constexpr uint32_t kStageBytes = (uint32_t)kChunk * (2 * N + 12);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < A.stages; ++s) {
+            mbar_init(smem_addr(&full[s]), 1);
+            mbar_init(smem_addr(&empty[s]), kConsumerWarps);
+        }
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+
+    const int64_t t_end = A.w.tile_first + A.w.n_tiles;
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane != 0) return;
+        int64_t s = A.w.seg_first;
+        uint32_t it = 0;          // chunks issued (or deliberately skipped by the test hook)
+        uint32_t posted = 0;      // chunks whose copies were issued
+        bool ok = true;
+        for (int64_t t = A.w.tile_first + blockIdx.x; ok && t < t_end; t += gridDim.x) {
+            const TileRange tr = locate_tile(A.w.segs, s, t);
+            const int64_t va = (tr.a + kVec - 1) / kVec * kVec, vb = tr.b / kVec * kVec;
+            for (int64_t q0 = va; ok && q0 < vb; q0 += kChunk, ++it) {
+                const uint32_t st = it % (uint32_t)A.stages, ph = (it / (uint32_t)A.stages) & 1u;
+                if (!wait_phase(smem_addr(&empty[st]), ph ^ 1u, abort_flag, A.error, A.wait_limit_ns)) {
+                    ok = false;
+                    break;
+                }
+                if (A.skip_first_fill && it == 0) continue;
+                const uint32_t n = (uint32_t)((vb - q0) < kChunk ? (vb - q0) : kChunk);
+                const uint32_t bar = smem_addr(&full[st]);
+                unsigned char *base = ring + (size_t)st * kStageBytes;
+                mbar_arrive_expect_tx(bar, n * (2u * N + 12u));
+#pragma unroll
+                for (int j = 0; j < N; ++j)
+                    bulk_load(smem_addr(base + (size_t)j * kChunk * 2),
+                              A.grads + (int64_t)ring_rank(tr.shard, j, N) * A.stride + q0, n * 2u, bar);
+                unsigned char *st_base = base + (size_t)N * kChunk * 2;
+                bulk_load(smem_addr(st_base), A.master + q0, n * 4u, bar);
+                bulk_load(smem_addr(st_base + kChunk * 4), A.mom1 + q0, n * 4u, bar);
+                bulk_load(smem_addr(st_base + kChunk * 8), A.mom2 + q0, n * 4u, bar);
+                posted = it + 1;
+            }
+        }
+        // Drain: every stage whose copies were issued must have landed before the CTA's
+        // shared memory goes away (normally the consumers have already seen them).
+        const uint32_t first = posted > (uint32_t)A.stages ? posted - (uint32_t)A.stages : 0u;
+        for (uint32_t i = first; i < posted; ++i) {
+            if (A.skip_first_fill && i == 0) continue;
+            const uint32_t st = i % (uint32_t)A.stages, ph = (i / (uint32_t)A.stages) & 1u;
+            const uint64_t t0 = global_ns();
+            while (!mbar_try_wait(smem_addr(&full[st]), ph) && global_ns() - t0 < A.wait_limit_ns) {
+            }
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------------- consumers
+    const int ct = threadIdx.x - 32;            // 0 .. 255
+    int64_t s = A.w.seg_first;
+    uint32_t it = 0;
+    for (int64_t t = A.w.tile_first + blockIdx.x; t < t_end; t += gridDim.x) {
+        const TileRange tr = locate_tile(A.w.segs, s, t);
+        const int64_t va = (tr.a + kVec - 1) / kVec * kVec, vb = tr.b / kVec * kVec;
+        int bad = 0;
+        for (int64_t q0 = va; q0 < vb; q0 += kChunk, ++it) {
+            const uint32_t st = it % (uint32_t)A.stages, ph = (it / (uint32_t)A.stages) & 1u;
+            // every lane waits (acquiring the stage's data); the warp leaves together
+            const bool got = wait_phase(smem_addr(&full[st]), ph, abort_flag, A.error, A.wait_limit_ns);
+            if (!__all_sync(0xffffffffu, got)) return;
+            const int64_t n = (vb - q0) < kChunk ? (vb - q0) : kChunk;
+            const unsigned char *base = ring + (size_t)st * kStageBytes;
+            for (int64_t vi = ct; vi * kVec < n; vi += 32 * kConsumerWarps) {
+                const int64_t e0 = vi * kVec;
+                float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+                {
+                    const uint4 u = *reinterpret_cast<const uint4 *>(base + e0 * 2);
+                    acc[0] = h2f(u.x); acc[1] = h2f(u.x >> 16); acc[2] = h2f(u.y); acc[3] = h2f(u.y >> 16);
+                    acc[4] = h2f(u.z); acc[5] = h2f(u.z >> 16); acc[6] = h2f(u.w); acc[7] = h2f(u.w >> 16);
+                }
+#pragma unroll
+                for (int j = 1; j < N; ++j)
+                    add8(acc, *reinterpret_cast<const uint4 *>(base + ((size_t)j * kChunk + e0) * 2));
+                const float *sp = reinterpret_cast<const float *>(base + (size_t)N * kChunk * 2);
+                float4 p4[2] = {*reinterpret_cast<const float4 *>(sp + e0), *reinterpret_cast<const float4 *>(sp + e0 + 4)};
+                float4 m4[2] = {*reinterpret_cast<const float4 *>(sp + kChunk + e0),
+                                *reinterpret_cast<const float4 *>(sp + kChunk + e0 + 4)};
+                float4 v4[2] = {*reinterpret_cast<const float4 *>(sp + 2 * kChunk + e0),
+                                *reinterpret_cast<const float4 *>(sp + 2 * kChunk + e0 + 4)};
+                float *pf = reinterpret_cast<float *>(p4);
+                float *mf = reinterpret_cast<float *>(m4);
+                float *vf = reinterpret_cast<float *>(v4);
+                uint32_t h[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    bad += !isfinite(acc[e]);
+                    adamw_elem(acc[e], A.c, pf[e], mf[e], vf[e], h[e]);
+                }
+                const int64_t q = q0 + e0;
+                float4 *pp = reinterpret_cast<float4 *>(A.master + q);
+                float4 *mp = reinterpret_cast<float4 *>(A.mom1 + q);
+                float4 *vp = reinterpret_cast<float4 *>(A.mom2 + q);
+                __stcs(pp, p4[0]); __stcs(pp + 1, p4[1]);
+                __stcs(mp, m4[0]); __stcs(mp + 1, m4[1]);
+                __stcs(vp, v4[0]); __stcs(vp + 1, v4[1]);
+                __stcs(reinterpret_cast<uint4 *>(A.p16 + q),
+                       make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16)));
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&empty[st]));
+        }
+
+        // ragged edges of the tile, straight from global memory
+        const int64_t head_end = va < tr.b ? va : tr.b;
+        const int64_t tail_begin = vb > head_end ? vb : head_end;
+        const int64_t n_head = head_end - tr.a, n_tail = tr.b - tail_begin;
+        if (ct < n_head + n_tail) {
+            const int64_t i = ct < n_head ? tr.a + ct : tail_begin + (ct - n_head);
+            float acc = h2f(A.grads[(int64_t)tr.shard * A.stride + i]);
+            for (int j = 1; j < N; ++j)
+                acc = __fadd_rn(acc, h2f(A.grads[(int64_t)ring_rank(tr.shard, j, N) * A.stride + i]));
+            bad += !isfinite(acc);
+            float p = A.master[i], m = A.mom1[i], v = A.mom2[i];
+            uint32_t h;
+            adamw_elem(acc, A.c, p, m, v, h);
+            A.master[i] = p;
+            A.mom1[i] = m;
+            A.mom2[i] = v;
+            A.p16[i] = (uint16_t)h;
+        }
+        if (A.nonfinite) {
+            if (__any_sync(0xffffffffu, bad != 0)) {
+                const int total = __reduce_add_sync(0xffffffffu, bad);
+                if (lane == 0) atomicAdd(A.nonfinite + tr.bucket, total);
+            }
+        }
+    }
+}
+
+template <int N>
+cudaError_t launch_bulk_n(const zero_layout &L, BulkArgs &a, cudaStream_t st)
+{
+    constexpr size_t stage_bytes = (size_t)kChunk * (2 * N + 12);
+    const size_t budget = L.dev.smem_optin > 0 ? L.dev.smem_optin : 227 * 1024;
+    int stages = (int)((budget - 256) / stage_bytes);
+    if (stages > 8) stages = 8;
+    if (stages < 2) return cudaErrorInvalidConfiguration;
+    a.stages = stages;
+    const size_t smem = ((16 * (size_t)stages + 4 + 127) / 128) * 128 + (size_t)stages * stage_bytes;
+    auto kern = bulk_step_kernel<N>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int64_t grid = L.dev.num_sms > 0 ? L.dev.num_sms : 148;
+    if (grid > a.w.n_tiles) grid = a.w.n_tiles;
+    kern<<<(unsigned)grid, kBulkThreads, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool bulk_supported(int n_ranks)
+{
+    switch (n_ranks) {
+        case 1: case 2: case 3: case 4: case 5: case 6: case 7: case 8: case 16: return true;
+        default: return false;
+    }
+}
+
+cudaError_t launch_bulk_step(const zero_layout &L, const TileWork &w, const uint16_t *grads, int64_t stride,
+                             float *master, float *m, float *v, uint16_t *p16, const AdamScalars &c,
+                             int32_t *nonfinite, uint64_t wait_limit_ns, int skip_first_fill, cudaStream_t st)
+{
+    if (w.n_tiles <= 0) return cudaSuccess;
+    BulkArgs a;
+    a.w = w;
+    a.grads = grads;
+    a.stride = stride;
+    a.master = master;
+    a.mom1 = m;
+    a.mom2 = v;
+    a.p16 = p16;
+    a.c = c;
+    a.nonfinite = nonfinite;
+    a.error = L.dev.error;
+    a.wait_limit_ns = wait_limit_ns;
+    a.stages = 0;
+    a.skip_first_fill = skip_first_fill;
+    switch (L.n_ranks) {
+        case 1: return launch_bulk_n<1>(L, a, st);
+        case 2: return launch_bulk_n<2>(L, a, st);
+        case 3: return launch_bulk_n<3>(L, a, st);
+        case 4: return launch_bulk_n<4>(L, a, st);
+        case 5: return launch_bulk_n<5>(L, a, st);
+        case 6: return launch_bulk_n<6>(L, a, st);
+        case 7: return launch_bulk_n<7>(L, a, st);
+        case 8: return launch_bulk_n<8>(L, a, st);
+        case 16: return launch_bulk_n<16>(L, a, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace zero

@@ -50,6 +50,8 @@ struct DeviceState {
     cudaStream_t copy_in = nullptr, copy_out = nullptr;   // zero_step_host
     std::vector<cudaEvent_t> landed, updated;              // per bucket
     cudaEvent_t begin = nullptr, done = nullptr;           // per zero_step_host call
+    uint64_t wait_limit_ns = 2000000000ull;   // bound of every in-kernel wait (2 s)
+    int32_t skip_first_fill = 0;              // test hook of the bulk pipeline (see zero.h)
 };
 
 }  // namespace zero
@@ -81,5 +83,11 @@ cudaError_t launch_copy_range(const zero_layout &L, int64_t lo, int64_t hi, cons
 cudaError_t launch_fused_step(const zero_layout &L, const TileWork &w, const uint16_t *grads,
                               int64_t stride, float *master, float *m, float *v, uint16_t *p16,
                               const AdamScalars &c, int32_t *nonfinite, cudaStream_t s);
+
+// bulk_step.cu
+bool bulk_supported(int n_ranks);
+cudaError_t launch_bulk_step(const zero_layout &L, const TileWork &w, const uint16_t *grads, int64_t stride,
+                             float *master, float *m, float *v, uint16_t *p16, const AdamScalars &c,
+                             int32_t *nonfinite, uint64_t wait_limit_ns, int skip_first_fill, cudaStream_t st);
 
 }  // namespace zero
