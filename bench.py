@@ -32,8 +32,8 @@ UNIT = "params/s"
 DEFAULT_WORKLOAD = "flat1p3b_n4_zero1"
 FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "fused_step_flat1p3b_n4.md")
-KERNEL_SOURCE = os.path.join(ROOT, "zero_sharded_optimizer_ring_b200", "csrc", "kernels.cu")
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "bulk_step_flat1p3b_n4.md")
+KERNEL_SOURCE = os.path.join(ROOT, "zero_sharded_optimizer_ring_b200", "csrc", "bulk_step.cu")
 
 
 def parse():
@@ -317,7 +317,7 @@ def run_ours(a, wl):
     if rank != 0:
         return
 
-    impl_name = {0: "automatic choice", 1: "register streaming (tile_kernel)",
+    impl_name = {0: "bulk-copy pipeline (bulk_step_kernel, automatic choice)", 1: "register streaming (tile_kernel)",
                  2: "bulk-copy pipeline (bulk_step_kernel)"}[a.kernel]
     peak, peak_kind = hbm_peak()
     fused_bytes = fused_bytes_per_param(wl) * P

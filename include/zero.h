@@ -183,9 +183,10 @@ zero_status zero_step_host(const zero_layout *layout, const uint16_t *grads_host
                            float *v, uint16_t *p16_shard, uint16_t *p16_full, uint16_t *p16_host,
                            const zero_adamw_hparams *hp, int32_t *nonfinite, void *stream);
 
-/* Select the fused kernel's implementation: 0 = automatic, 1 = register streaming
- * (vectorised 16-byte loads held in registers), 2 = bulk-copy pipeline (cp.async.bulk
- * into a shared-memory ring, warp-specialised).  Results are identical. */
+/* Select the fused kernel's implementation: 0 = automatic (the bulk-copy pipeline for
+ * N in 1..8 and 16, register streaming otherwise), 1 = register streaming (vectorised
+ * 16-byte loads held in registers), 2 = bulk-copy pipeline (cp.async.bulk into a
+ * shared-memory ring, warp-specialised).  Results are bit-identical. */
 zero_status zero_set_impl(zero_layout *layout, int32_t impl);
 
 /* Test hook of the bulk-copy pipeline's bounded waits: every in-kernel wait gives up
