@@ -183,6 +183,37 @@ zero_status zero_step_host(const zero_layout *layout, const uint16_t *grads_host
                            float *v, uint16_t *p16_shard, uint16_t *p16_full, uint16_t *p16_host,
                            const zero_adamw_hparams *hp, int32_t *nonfinite, void *stream);
 
+/* The step for callers that cannot allocate device memory.  The pages have no
+ * counterpart: this entry point exists for the library's users, not for the method.
+ *
+ * zero_step needs zero_layout_to_device, which obtains device memory with cudaMalloc for
+ * the segment table and its tile index.  Callers whose device memory belongs to another
+ * allocator (a framework's caching allocator or a fixed pool that has reserved the GPU),
+ * whose loop cannot take the device-wide synchronisation an allocation may imply, or
+ * that run where allocating is not allowed can call this instead: it computes exactly
+ * what zero_step computes (register-streaming kernel, results bit-identical), with that
+ * scratch held in a static device array of the library instead of allocated memory.
+ *   - The layout does not need zero_layout_to_device.  Inputs and outputs are the
+ *     caller's, as for zero_step.  Nothing is allocated and nothing is freed.
+ *   - Limit: layouts of at most ZERO_NOALLOC_MAX_SEGMENTS segments (bucket x shard
+ *     pieces); larger layouts return ZERO_ERR_INVALID before anything runs.  The array
+ *     takes (ZERO_NOALLOC_MAX_SEGMENTS + 1) x 32 bytes = 256 KiB on every GPU that
+ *     loads the library, until the process exits.
+ *   - The first call on each device looks up the array's device address (which can load
+ *     the library's device code onto that device); make that first call before any
+ *     stream capture begins.
+ *   - All calls on a device share the one array, and it keeps whatever the last call
+ *     wrote.  Each call rewrites every row it reads (the rows are copied from the
+ *     layout's host table, which waits for earlier work on `stream` to finish, and the
+ *     tile index is rebuilt on the device), so no clearing is needed; but two calls
+ *     whose work overlaps on the GPU (different streams, different layouts) race on
+ *     the array and may compute garbage.  Serialise them.
+ *   - nonfinite (optional) is added to, as in zero_step. */
+#define ZERO_NOALLOC_MAX_SEGMENTS 8191
+zero_status zero_step_noalloc(const zero_layout *layout, const uint16_t *grads, int64_t rank_stride,
+                              float *master, float *m, float *v, uint16_t *p16_shard, uint16_t *p16_full,
+                              const zero_adamw_hparams *hp, int32_t *nonfinite, void *stream);
+
 /* Select the fused kernel's implementation: 0 = automatic (the bulk-copy pipeline for
  * N in 1..8 and 16, register streaming otherwise), 1 = register streaming (vectorised
  * 16-byte loads held in registers), 2 = bulk-copy pipeline (cp.async.bulk into a

@@ -16,7 +16,7 @@ import numpy as np
 from . import _abi
 
 __all__ = ["ZeroError", "Layout", "AdamW", "reduce_scatter", "adamw_shard_step", "allgather",
-           "step", "step_host", "get_error", "IMPL_AUTO", "IMPL_REGISTER", "IMPL_BULK"]
+           "step", "step_host", "step_noalloc", "get_error", "IMPL_AUTO", "IMPL_REGISTER", "IMPL_BULK"]
 
 IMPL_AUTO, IMPL_REGISTER, IMPL_BULK = 0, 1, 2
 
@@ -189,6 +189,18 @@ def step_host(layout, grads_host, grads_dev, master, m, v, p16_shard, p16_full, 
                                      _stride(grads_dev, layout, rank_stride), _ptr(master), _ptr(m), _ptr(v),
                                      _ptr(p16_shard), _ptr(p16_full), _ptr(p16_host), ctypes.byref(h),
                                      _ptr(nonfinite), _stream(stream)), "zero_step_host")
+
+
+def step_noalloc(layout, grads, master, m, v, p16_shard, p16_full, hp, nonfinite=None, rank_stride=None,
+                 stream=None):
+    """zero_step for callers that cannot allocate device memory: same result, with the
+    step's scratch in the library's static device array (at most
+    _abi.NOALLOC_MAX_SEGMENTS segments; calls that overlap on the GPU race).  The layout
+    need not be uploaded with to_device()."""
+    h = hp.c()
+    _check(_abi.lib().zero_step_noalloc(layout.handle, _ptr(grads), _stride(grads, layout, rank_stride),
+                                        _ptr(master), _ptr(m), _ptr(v), _ptr(p16_shard), _ptr(p16_full),
+                                        ctypes.byref(h), _ptr(nonfinite), _stream(stream)), "zero_step_noalloc")
 
 
 def get_error(layout, stream=None):

@@ -11,6 +11,7 @@ _i32 = ctypes.c_int32
 _p_i64 = ctypes.POINTER(ctypes.c_int64)
 
 ZERO_OK = 0
+NOALLOC_MAX_SEGMENTS = 8191   # ZERO_NOALLOC_MAX_SEGMENTS in include/zero.h
 STATUS_NAMES = {0: "ZERO_OK", 1: "ZERO_ERR_INVALID", 2: "ZERO_ERR_ALIGN", 3: "ZERO_ERR_CUDA",
                 4: "ZERO_ERR_OOM", 5: "ZERO_ERR_TIMEOUT", 6: "ZERO_ERR_STATE"}
 
@@ -57,6 +58,7 @@ SIGNATURES = {
                          ctypes.POINTER(StepEvents), _vp]),
     "zero_step_host": (_i32, [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp,
                               ctypes.POINTER(AdamWHparams), _vp, _vp]),
+    "zero_step_noalloc": (_i32, [_vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(AdamWHparams), _vp, _vp]),
     "zero_set_impl": (_i32, [_vp, _i32]),
     "zero_debug_set_wait": (_i32, [_vp, _i64, _i32]),
     "zero_get_error": (_i32, [_vp, _vp]),

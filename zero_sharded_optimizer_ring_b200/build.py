@@ -16,7 +16,7 @@ LIB = os.path.join(HERE, "libzero_b200.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
-SOURCES = ["layout.cpp", "kernels.cu", "bulk_step.cu", "abi.cu"]
+SOURCES = ["layout.cpp", "kernels.cu", "bulk_step.cu", "abi.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-fmad=false", "-prec-div=true", "-prec-sqrt=true",
          "-ftz=false", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC]
