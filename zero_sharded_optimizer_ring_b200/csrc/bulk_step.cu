@@ -4,11 +4,11 @@
 // ranks' fp16 gradients, scale, AdamW, fp16 write; rkmt.cn/news/44736 "DDP" and
 // "Deepspeed ZeRO-1", en.pswp.cn/web/84187 "DDP"), staged differently:
 //
-//   warp 0, lane 0 (producer): for each 2048-element chunk of its tiles, waits for a free
+//   warp 0, lane 0 (producer): for each chunk (2048 or 4096 elements) of its tiles, waits for a free
 //     stage of a shared-memory ring, posts the stage's byte count on the stage's "full"
 //     mbarrier and issues one cp.async.bulk (global -> shared, no tensor map, no
 //     multicast) per gradient slice (ranks in ring order) and per state array;
-//   warps 1..8 (consumers): wait for the stage to fill, fold / update from shared memory
+//   warps 1..8 or 1..16 (consumers): wait for the stage to fill, fold / update from shared memory
 //     (16-byte vectors, conflict-free for the gradients), store results with 16-byte
 //     streaming stores, and release the stage on its "empty" mbarrier.
 //
@@ -27,10 +27,21 @@
 namespace zero {
 namespace {
 
-constexpr int kConsumerWarps = 8;
-constexpr int kBulkThreads = 32 * (1 + kConsumerWarps);
-constexpr int kChunk = 2048;                 // elements per pipeline stage
 constexpr int kVec = 8;
+
+// Pipeline shape per rank count, measured on B200 (kernel GB/s of the full step on the
+// flat N=4, GPT-2 N=8, Llama N=8 and ragged N=16 workloads): larger single copies pay,
+// but more than about 120-170 KB in flight per SM costs DRAM efficiency.  Few ranks:
+// 4096-element chunks (one tile), 16 consumer warps, 2-3 stages.  More ranks: 2048-element
+// chunks, 8 consumer warps, at most 3 stages.
+template <int N>
+struct BulkShape {
+    static constexpr int kChunk = N <= 4 ? 4096 : 2048;        // elements per stage
+    static constexpr int kConsumerWarps = N <= 4 ? 16 : 8;
+    static constexpr int kThreads = 32 * (1 + kConsumerWarps);
+    static constexpr int kMaxStages = 3;
+    static constexpr uint32_t kStageBytes = (uint32_t)kChunk * (2 * N + 12);
+};
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p)
 {
@@ -170,14 +181,16 @@ struct BulkArgs {
 // Shared memory: [full[S], empty[S] mbarriers][abort flag] ... stage ring (128-B aligned):
 // stage s = N gradient slices of kChunk fp16, then master, m, v slices of kChunk fp32.
 template <int N>
-__global__ void __launch_bounds__(kBulkThreads, 1) bulk_step_kernel(BulkArgs A)
+__global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(BulkArgs A)
 {
+    constexpr int kChunk = BulkShape<N>::kChunk;
+    constexpr int kConsumerWarps = BulkShape<N>::kConsumerWarps;
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem);
     uint64_t *empty = full + A.stages;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + A.stages);
     unsigned char *ring = smem + ((16 * A.stages + 4 + 127) / 128) * 128;
-    constexpr uint32_t kStageBytes = (uint32_t)kChunk * (2 * N + 12);
+    constexpr uint32_t kStageBytes = BulkShape<N>::kStageBytes;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -237,7 +250,7 @@ __global__ void __launch_bounds__(kBulkThreads, 1) bulk_step_kernel(BulkArgs A)
     }
 
     // ---------------------------------------------------------------- consumers
-    const int ct = threadIdx.x - 32;            // 0 .. 255
+    const int ct = threadIdx.x - 32;            // 0 .. 32 * kConsumerWarps - 1
     int64_t s = A.w.seg_first;
     uint32_t it = 0;
     for (int64_t t = A.w.tile_first + blockIdx.x; t < t_end; t += gridDim.x) {
@@ -321,10 +334,10 @@ __global__ void __launch_bounds__(kBulkThreads, 1) bulk_step_kernel(BulkArgs A)
 template <int N>
 cudaError_t launch_bulk_n(const zero_layout &L, BulkArgs &a, cudaStream_t st)
 {
-    constexpr size_t stage_bytes = (size_t)kChunk * (2 * N + 12);
+    constexpr size_t stage_bytes = BulkShape<N>::kStageBytes;
     const size_t budget = L.dev.smem_optin > 0 ? L.dev.smem_optin : 227 * 1024;
     int stages = (int)((budget - 256) / stage_bytes);
-    if (stages > 8) stages = 8;
+    if (stages > BulkShape<N>::kMaxStages) stages = BulkShape<N>::kMaxStages;
     if (stages < 2) return cudaErrorInvalidConfiguration;
     a.stages = stages;
     const size_t smem = ((16 * (size_t)stages + 4 + 127) / 128) * 128 + (size_t)stages * stage_bytes;
@@ -333,7 +346,7 @@ cudaError_t launch_bulk_n(const zero_layout &L, BulkArgs &a, cudaStream_t st)
     if (e != cudaSuccess) return e;
     int64_t grid = L.dev.num_sms > 0 ? L.dev.num_sms : 148;
     if (grid > a.w.n_tiles) grid = a.w.n_tiles;
-    kern<<<(unsigned)grid, kBulkThreads, smem, st>>>(a);
+    kern<<<(unsigned)grid, BulkShape<N>::kThreads, smem, st>>>(a);
     return cudaGetLastError();
 }
 
