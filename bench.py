@@ -111,19 +111,38 @@ def profiled_traffic(workload):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi clock / throttle-reason samples; only those taken between mark_start()
+    and mark_end() (the timed region) are summarised."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, gpu_index):
         self.gpu = str(gpu_index)
+        self.t0 = self.t1 = None
         self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
         try:
             self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                                        "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.p = None
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    @staticmethod
+    def _when(stamp):
+        from datetime import datetime
+        for fmt in ("%Y/%m/%d %H:%M:%S.%f", "%Y/%m/%d %H:%M:%S"):
+            try:
+                return datetime.strptime(stamp, fmt).timestamp()
+            except ValueError:
+                pass
+        return None
 
     def stop(self):
         if self.p is None:
@@ -134,17 +153,19 @@ class ClockSampler:
         except Exception:
             self.p.kill()
         self.f.flush()
-        rows = [r.split(",") for r in open(self.f.name).read().splitlines() if r.strip()]
+        rows = [[c.strip() for c in r.split(",")] for r in open(self.f.name).read().splitlines() if r.strip()]
         os.unlink(self.f.name)
-        rows = [[c.strip() for c in r] for r in rows if len(r) >= 9 and r[0].strip() == self.gpu]
+        rows = [r for r in rows if len(r) >= 10 and r[1] == self.gpu]
+        inside = [r for r in rows if self.t0 is not None and self._when(r[0]) is not None
+                  and self.t0 - 0.05 <= self._when(r[0]) <= (self.t1 or 1e18) + 0.05]
+        rows = inside or rows
         if not rows:
             return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[j] for r in rows for j in range(4) if r[5 + j].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
-                "reasons": reasons, "samples": len(rows)}
+        num = lambda x: float(x) if x.replace(".", "", 1).isdigit() else None
+        sm = [num(r[2]) for r in rows if num(r[2]) is not None]
+        reasons = sorted({self.REASONS[j] for r in rows for j in range(4) if r[6 + j].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": num(rows[0][3]),
+                "reasons": reasons, "samples": len(rows), "in_timed_region": bool(inside)}
 
 
 def workload_config(wl, world):
@@ -271,12 +292,16 @@ def run_ours(a, wl):
     sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
     time.sleep(0.3)
     barrier()
+    if sampler:
+        sampler.mark_start()
     start.record()
     for i in range(K):
         t += 1
         zs.step(lay, g, master, m, v, p16_shard, p16_full, hp(t), nonfinite=nonfinite, events=ev[i])
     end.record()
     barrier()
+    if sampler:
+        sampler.mark_end()
     clocks = sampler.stop() if sampler else None
     zs.get_error(lay)
     ms = max_over_ranks(start.elapsed_time(end) / K, world, "cuda")

@@ -38,25 +38,29 @@ def lib():
     global _LIB
     if _LIB is None:
         _build.build()
-        L = ctypes.CDLL(_build.LIB)
-        L.oracle_half_to_float.argtypes = [ctypes.c_uint16]
-        L.oracle_half_to_float.restype = ctypes.c_float
-        L.oracle_float_to_half.argtypes = [ctypes.c_float]
-        L.oracle_float_to_half.restype = ctypes.c_uint16
-        L.oracle_halfs_to_floats.argtypes = [_vp, _vp, _i64]
-        L.oracle_floats_to_halfs.argtypes = [_vp, _vp, _i64]
-        L.oracle_ring_reduce_scatter.argtypes = [_vp, _i32, _i64, _i64, _i64, _i64, _i32,
-                                                 _vp, _vp, _vp, _vp, _vp]
-        L.oracle_ring_reduce_scatter.restype = _i64
-        L.oracle_ring_allgather.argtypes = [_vp, _i32, _i32, _i64, _i64, _i64, _i64, _vp, _vp, _vp]
-        L.oracle_ring_allgather.restype = _i64
-        L.oracle_adamw_scalars.argtypes = [_vp, _i32, _dbl, _dbl, _dbl, _dbl, _dbl, _dbl, _i64]
-        L.oracle_adamw.argtypes = [_i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]
-        L.oracle_count_nonfinite.argtypes = [_vp, _i64, _i64]
-        L.oracle_count_nonfinite.restype = _i64
-        L.oracle_sampled.argtypes = [_i64, _i32, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp]
-        _LIB = L
+        _LIB = configure(ctypes.CDLL(_build.LIB))
     return _LIB
+
+
+def configure(L):
+    """Declare the C functions' signatures on a loaded oracle library."""
+    L.oracle_half_to_float.argtypes = [ctypes.c_uint16]
+    L.oracle_half_to_float.restype = ctypes.c_float
+    L.oracle_float_to_half.argtypes = [ctypes.c_float]
+    L.oracle_float_to_half.restype = ctypes.c_uint16
+    L.oracle_halfs_to_floats.argtypes = [_vp, _vp, _i64]
+    L.oracle_floats_to_halfs.argtypes = [_vp, _vp, _i64]
+    L.oracle_ring_reduce_scatter.argtypes = [_vp, _i32, _i64, _i64, _i64, _i64, _i32,
+                                             _vp, _vp, _vp, _vp, _vp]
+    L.oracle_ring_reduce_scatter.restype = _i64
+    L.oracle_ring_allgather.argtypes = [_vp, _i32, _i32, _i64, _i64, _i64, _i64, _vp, _vp, _vp]
+    L.oracle_ring_allgather.restype = _i64
+    L.oracle_adamw_scalars.argtypes = [_vp, _i32, _dbl, _dbl, _dbl, _dbl, _dbl, _dbl, _i64]
+    L.oracle_adamw.argtypes = [_i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]
+    L.oracle_count_nonfinite.argtypes = [_vp, _i64, _i64]
+    L.oracle_count_nonfinite.restype = _i64
+    L.oracle_sampled.argtypes = [_i64, _i32, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp]
+    return L
 
 
 def _p(a):

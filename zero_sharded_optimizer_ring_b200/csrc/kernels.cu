@@ -278,13 +278,28 @@ adamw_range_kernel(int64_t lo, int64_t hi, const float *__restrict__ reduced, fl
     }
 }
 
+// Copy [lo, hi): each thread keeps kCopyUnroll 16-byte loads in flight before storing;
+// the block's vectors stay contiguous (thread t takes vectors t, t + 256, ...).
+constexpr int kCopyUnroll = 4;
+
 __global__ void __launch_bounds__(kThreads)
 copy_range_kernel(int64_t lo, int64_t hi, const uint16_t *__restrict__ src, uint16_t *__restrict__ dst)
 {
     const int64_t va = (lo + kVec - 1) / kVec * kVec, vb = hi / kVec * kVec;
-    const int64_t stride = (int64_t)gridDim.x * kThreads * kVec;
-    for (int64_t q = va + ((int64_t)blockIdx.x * kThreads + threadIdx.x) * kVec; q < vb; q += stride)
-        __stcs(reinterpret_cast<uint4 *>(dst + q), __ldcs(reinterpret_cast<const uint4 *>(src + q)));
+    const int64_t block_span = (int64_t)kThreads * kVec * kCopyUnroll;
+    for (int64_t base = va + (int64_t)blockIdx.x * block_span; base < vb; base += (int64_t)gridDim.x * block_span) {
+        uint4 x[kCopyUnroll];
+#pragma unroll
+        for (int u = 0; u < kCopyUnroll; ++u) {
+            const int64_t q = base + ((int64_t)u * kThreads + threadIdx.x) * kVec;
+            if (q < vb) x[u] = __ldcs(reinterpret_cast<const uint4 *>(src + q));
+        }
+#pragma unroll
+        for (int u = 0; u < kCopyUnroll; ++u) {
+            const int64_t q = base + ((int64_t)u * kThreads + threadIdx.x) * kVec;
+            if (q < vb) __stcs(reinterpret_cast<uint4 *>(dst + q), x[u]);
+        }
+    }
     if (blockIdx.x == 0) {
         const int64_t head_end = va < hi ? va : hi;
         const int64_t tail_begin = vb > head_end ? vb : head_end;
@@ -408,8 +423,8 @@ cudaError_t launch_copy_range(const zero_layout &L, int64_t lo, int64_t hi, cons
                               uint16_t *dst, cudaStream_t s)
 {
     if (hi <= lo) return cudaSuccess;
-    const int grid = grid_for(copy_range_kernel, (hi - lo + kThreads * kVec - 1) / (kThreads * kVec),
-                              L.dev.num_sms);
+    const int grid = grid_for(copy_range_kernel, (hi - lo + kThreads * kVec * kCopyUnroll - 1) /
+                                                     (kThreads * kVec * kCopyUnroll), L.dev.num_sms);
     copy_range_kernel<<<grid, kThreads, 0, s>>>(lo, hi, src, dst);
     return cudaGetLastError();
 }
