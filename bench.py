@@ -48,6 +48,9 @@ def parse():
     ap.add_argument("--ref-seconds", type=float, default=120.0,
                     help="--impl reference: oracle time budget of the whole run")
     ap.add_argument("--kernel", type=int, default=0, help="fused kernel: 0 auto, 1 register, 2 bulk")
+    ap.add_argument("--overlap", action="store_true",
+                    help="measure the bucket-pipelined step behind a simulated backward pass "
+                         "(its own JSON line; not the headline)")
     ap.add_argument("--psi", type=int, default=0,
                     help="flat workloads only: run the same shape with this many parameters "
                          "(small cases for profiler captures; not a bench line)")
@@ -373,6 +376,94 @@ def run_ours(a, wl):
     print(json.dumps(out), flush=True)
 
 
+def run_overlap(a, wl):
+    """The step overlapped with a simulated backward pass.  The backward writes every
+    rank's gradients one bucket at a time, tail bucket first (seeded generator kernels:
+    ALU-heavy, like a backward pass, and writing the 2N bytes per parameter a backward
+    pass writes), on its own stream, recording an event per bucket; zero_step_overlapped
+    runs each bucket's fused update on the compute stream as soon as its event fires."""
+    import torch
+    import seeded_inputs as si
+    import zero_sharded_optimizer_ring_b200 as zs
+
+    torch.cuda.set_device(dist_env()[1])
+    lay = zs.Layout(list(wl.tensors), wl.n_ranks, wl.stage, wl.bucket_elems, wl.pad_align, list(wl.units))
+    lay.to_device()
+    P, psi, N = lay.padded, lay.psi, wl.n_ranks
+    g = torch.zeros((N, P), dtype=torch.int16, device="cuda")
+    master = torch.empty(P, dtype=torch.float32, device="cuda")
+    si.fill_f32_cuda(master, psi, wl.seed, si.STREAM_MASTER, wl.master_sigma)
+    m = torch.zeros(P, dtype=torch.float32, device="cuda")
+    v = torch.zeros(P, dtype=torch.float32, device="cuda")
+    p16_full = torch.zeros(P, dtype=torch.int16, device="cuda")
+    p16_shard = torch.zeros(P, dtype=torch.int16, device="cuda") if wl.stage == 3 else None
+    _, buckets, _, _ = lay.tables()
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    hi_pri = torch.cuda.Stream.priority_range()[1]       # numerically lowest = highest priority
+
+    def backward_fn(producer):
+        def backward(events=None):
+            for b, (lo, hi) in enumerate(buckets):
+                si.fill_grads_range_cuda(g, int(lo), int(hi), psi, wl.seed, wl.grad_sigma, wl.loss_scale,
+                                         wl.heavy_frac, wl.heavy_mult, cuda_stream=producer.cuda_stream)
+                if events is not None:
+                    events[b].record(producer)
+        return backward
+
+    t = 0
+
+    reps = max(3, a.steps // 20)
+    for prio_name, prio in (("default", 0), ("high", hi_pri)):
+        producer, compute = torch.cuda.Stream(), torch.cuda.Stream(priority=prio)
+        t = _overlap_reps(a, wl, lay, g, master, m, v, p16_shard, p16_full, backward_fn(producer), producer,
+                          compute, ev, reps, t, prio_name)
+    zs.get_error(lay)
+
+
+def _overlap_reps(a, wl, lay, g, master, m, v, p16_shard, p16_full, backward, producer, compute, ev, reps, t,
+                  prio_name):
+    import torch
+    import zero_sharded_optimizer_ring_b200 as zs
+
+    def hp():
+        return zs.AdamW(wl.lr, wl.beta1, wl.beta2, wl.eps, wl.weight_decay, wl.loss_scale, t)
+
+    res = {"bwd": [], "step": [], "pipe": []}
+    for rep in range(a.warmup + reps):
+        torch.cuda.synchronize()
+        s0, e0 = ev(), ev()
+        s0.record(producer)
+        backward()
+        e0.record(producer)
+        torch.cuda.synchronize()
+        t += 1
+        s1, e1 = ev(), ev()
+        s1.record(compute)
+        zs.step(lay, g, master, m, v, p16_shard, p16_full, hp(), stream=compute)
+        e1.record(compute)
+        torch.cuda.synchronize()
+        t += 1
+        ready = [torch.cuda.Event() for _ in range(lay.n_buckets)]
+        s2, e2 = ev(), ev()
+        s2.record(producer)
+        backward(ready)
+        zs.step_overlapped(lay, ready, g, master, m, v, p16_shard, p16_full, hp(), stream=compute)
+        e2.record(compute)
+        torch.cuda.synchronize()
+        if rep >= a.warmup:
+            res["bwd"].append(s0.elapsed_time(e0))
+            res["step"].append(s1.elapsed_time(e1))
+            res["pipe"].append(s2.elapsed_time(e2))
+    tb, ts, tp = (statistics.median(res[k]) for k in ("bwd", "step", "pipe"))
+    print(json.dumps({
+        "metric": "bucket-pipelined step behind a simulated backward (overlap)", "workload": wl.name,
+        "compute_stream_priority": prio_name, "buckets": lay.n_buckets, "reps": reps, "t_backward_ms": tb,
+        "t_step_ms": ts, "t_pipelined_ms": tp, "exposed_step_ms": tp - tb, "overlap_efficiency": (tb + ts - tp) / ts,
+        "note": "overlap_efficiency = share of the step hidden behind the backward (1 = fully hidden)"}),
+        flush=True)
+    return t
+
+
 def main():
     a = parse()
     from seeded_inputs.workloads import full_workloads
@@ -383,6 +474,8 @@ def main():
         wl = wl.with_(tensors=(a.psi,), name=f"{wl.name}_psi{a.psi}")
     if a.impl == "reference":
         run_reference(a, wl)
+    elif a.overlap:
+        run_overlap(a, wl)
     else:
         run_ours(a, wl)
 

@@ -170,6 +170,30 @@ zero_status zero_step(const zero_layout *layout, const uint16_t *grads, int64_t 
                       const zero_adamw_hparams *hp, int32_t *nonfinite,
                       const zero_step_events *events, void *stream);
 
+/* One bucket's share of zero_step: the fused reduce-scatter + update of bucket `bucket`
+ * only, so that it can start as soon as that bucket's gradients exist (P1 DDP: the first
+ * group of gradients computed starts its ring while the next group is still being
+ * computed; P1 ZeRO-2: each bucket goes to its owner as soon as it is complete; P3 DDP:
+ * buckets).  Running every bucket once, in any order, gives exactly zero_step's result.
+ * Stage 3 writes p16_shard only: call zero_allgather after the last bucket. */
+zero_status zero_step_bucket(const zero_layout *layout, int64_t bucket, const uint16_t *grads,
+                             int64_t rank_stride, float *master, float *m, float *v, uint16_t *p16_shard,
+                             uint16_t *p16_full, const zero_adamw_hparams *hp, int32_t *nonfinite,
+                             void *stream);
+
+/* zero_step overlapped with the backward pass that produces the gradients: for each
+ * bucket b in bucket order (the order a backward pass completes them), `stream` waits
+ * for ready_events[b] (a cudaEvent_t the caller records once bucket b's gradients are
+ * written, typically on another stream), then runs bucket b's fused update.  Stage 3
+ * then runs the all-gather.  ready_events: host array [n_buckets], none NULL.  As for
+ * any cudaStreamWaitEvent, each wait takes the event's most recent record at the time of
+ * this call: enqueue the producer's records first (the producer's work itself may still
+ * be running).  Result identical to zero_step. */
+zero_status zero_step_overlapped(const zero_layout *layout, void *const *ready_events,
+                                 const uint16_t *grads, int64_t rank_stride, float *master, float *m,
+                                 float *v, uint16_t *p16_shard, uint16_t *p16_full,
+                                 const zero_adamw_hparams *hp, int32_t *nonfinite, void *stream);
+
 /* zero_step for gradients that live in HOST memory (page-locked), with the fp16
  * parameters returned to host memory: per bucket, the N gradient slices are copied to
  * the device staging buffer grads_dev on an internal copy stream, the bucket's fused

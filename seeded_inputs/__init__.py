@@ -49,13 +49,15 @@ def _host():
 def _cuda():
     global _CUDA
     if _CUDA is None:
-        if not os.path.exists(_build.CUDA_LIB):
-            _build.build()
+        _build.build()
         lib = ctypes.CDLL(_build.CUDA_LIB)
         lib.si_fill_f32_cuda.argtypes = [_vp, _i64, _i64, _u32, _u32, _dbl, ctypes.c_int, _vp]
         lib.si_fill_f32_cuda.restype = ctypes.c_int
         lib.si_fill_grads_cuda.argtypes = [_vp, _i32, _i64, _i64, _u32, _dbl, _dbl, _u32, _dbl, _vp]
         lib.si_fill_grads_cuda.restype = ctypes.c_int
+        lib.si_fill_grads_range_cuda.argtypes = [_vp, _i32, _i64, _i64, _i64, _i64, _u32, _dbl, _dbl, _u32,
+                                                 _dbl, _vp]
+        lib.si_fill_grads_range_cuda.restype = ctypes.c_int
         _CUDA = lib
     return _CUDA
 
@@ -151,3 +153,14 @@ def fill_grads_cuda(t, valid, seed, sigma, loss_scale, heavy_frac=0.0, heavy_mul
     _check(_cuda().si_fill_grads_cuda(t.data_ptr(), t.shape[0], t.shape[1], valid, seed, sigma,
                                       loss_scale, heavy_q32(heavy_frac), heavy_mult, s),
            "si_fill_grads_cuda")
+
+
+def fill_grads_range_cuda(t, lo, hi, valid, seed, sigma, loss_scale, heavy_frac=0.0, heavy_mult=1.0,
+                          cuda_stream=None):
+    """Fill flat indices [lo, hi) of every rank's row of t [n_ranks, rank_stride]."""
+    import torch
+    s = cuda_stream if cuda_stream is not None else torch.cuda.current_stream(t.device).cuda_stream
+    assert t.is_cuda and t.dim() == 2 and t.is_contiguous() and t.element_size() == 2
+    _check(_cuda().si_fill_grads_range_cuda(t.data_ptr(), t.shape[0], t.shape[1], lo, hi, valid, seed, sigma,
+                                            loss_scale, heavy_q32(heavy_frac), heavy_mult, s),
+           "si_fill_grads_range_cuda")

@@ -1,0 +1,97 @@
+"""Bucket pipelining: the per-bucket step and the event-gated step against zero_step.
+
+A simulated backward pass writes one bucket of gradients at a time, last bucket of the
+flat buffer first (the order a backward pass completes them), on its own stream and
+records an event per bucket; zero_step_overlapped runs each bucket's fused update on
+another stream as soon as its event fires.  Results must equal zero_step's bit for bit.
+"""
+import numpy as np
+import pytest
+
+from seeded_inputs.workloads import reduced_workloads
+import seeded_inputs as si
+import zero_sharded_optimizer_ring_b200 as zs
+import support as S
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+def _hp(wl, t):
+    return zs.AdamW(wl.lr, wl.beta1, wl.beta2, wl.eps, wl.weight_decay, wl.loss_scale, t)
+
+
+def _setup(wl):
+    lay = zs.Layout(list(wl.tensors), wl.n_ranks, wl.stage, wl.bucket_elems, wl.pad_align,
+                    list(wl.units)).to_device()
+    P = lay.padded
+
+    def bufs():
+        g, master, m, v = S.device_inputs(wl, P)
+        return dict(g=g, master=master, m=m, v=v,
+                    p16_shard=torch.zeros(P, dtype=torch.int16, device="cuda"),
+                    p16_full=torch.zeros(P, dtype=torch.int16, device="cuda"),
+                    nonfinite=torch.zeros(max(1, lay.n_buckets), dtype=torch.int32, device="cuda"))
+    return lay, bufs
+
+
+def _same(a, b):
+    torch.cuda.synchronize()
+    for k in ("master", "m", "v", "p16_full", "p16_shard", "nonfinite"):
+        S.assert_bits_equal(a[k].cpu().numpy(), b[k].cpu().numpy(), k)
+
+
+@pytest.mark.parametrize("key", list(reduced_workloads()))
+@pytest.mark.parametrize("order", ["bucket", "reverse"])
+def test_step_bucket_equals_step(key, order):
+    wl = reduced_workloads()[key]
+    lay, bufs = _setup(wl)
+    a, b = bufs(), bufs()
+    _, buckets, _, _ = lay.tables()
+    seq = list(range(lay.n_buckets))
+    if order == "reverse":
+        seq.reverse()
+    for t in (1, 2):
+        zs.step(lay, a["g"], a["master"], a["m"], a["v"], a["p16_shard"], a["p16_full"], _hp(wl, t),
+                nonfinite=a["nonfinite"])
+        for bk in seq:
+            zs.step_bucket(lay, bk, b["g"], b["master"], b["m"], b["v"], b["p16_shard"], b["p16_full"], _hp(wl, t),
+                           nonfinite=b["nonfinite"])
+        if wl.stage == 3:
+            zs.allgather(lay, -1, b["p16_shard"], b["p16_full"])
+    _same(a, b)
+
+
+@pytest.mark.parametrize("key", ["flat1p3b_n4_zero1", "llama3b_n8_zero3", "ragged2000_n16_zero2"])
+def test_overlapped_step_with_simulated_backward(key):
+    wl = reduced_workloads()[key]
+    lay, bufs = _setup(wl)
+    a, b = bufs(), bufs()
+    _, buckets, _, _ = lay.tables()
+    producer, consumer = torch.cuda.Stream(), torch.cuda.Stream()
+    for t in (1, 2):
+        zs.step(lay, a["g"], a["master"], a["m"], a["v"], a["p16_shard"], a["p16_full"], _hp(wl, t),
+                nonfinite=a["nonfinite"])
+        torch.cuda.synchronize()
+        b["g"].zero_()
+        torch.cuda.synchronize()
+        ready = [torch.cuda.Event() for _ in range(lay.n_buckets)]
+        for bk, (lo, hi) in enumerate(buckets):            # the backward: bucket 0 (the tail) first
+            si.fill_grads_range_cuda(b["g"], int(lo), int(hi), wl.psi, wl.seed, wl.grad_sigma, wl.loss_scale,
+                                     wl.heavy_frac, wl.heavy_mult, cuda_stream=producer.cuda_stream)
+            ready[bk].record(producer)
+        zs.step_overlapped(lay, ready, b["g"], b["master"], b["m"], b["v"], b["p16_shard"], b["p16_full"],
+                           _hp(wl, t), nonfinite=b["nonfinite"], stream=consumer)
+    zs.get_error(lay)
+    _same(a, b)
+
+
+def test_overlapped_rejects_unrecorded_events():
+    wl = reduced_workloads()["flat1p3b_n4_zero1"]
+    lay, bufs = _setup(wl)
+    b = bufs()
+    with pytest.raises(ValueError):
+        zs.step_overlapped(lay, [torch.cuda.Event() for _ in range(lay.n_buckets)], b["g"], b["master"], b["m"],
+                           b["v"], None, b["p16_full"], _hp(wl, 1))
+    with pytest.raises(zs.ZeroError):
+        zs.step_bucket(lay, lay.n_buckets, b["g"], b["master"], b["m"], b["v"], None, b["p16_full"], _hp(wl, 1))

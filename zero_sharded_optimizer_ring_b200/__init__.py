@@ -16,7 +16,7 @@ import numpy as np
 from . import _abi
 
 __all__ = ["ZeroError", "Layout", "AdamW", "reduce_scatter", "adamw_shard_step", "allgather",
-           "step", "step_host", "step_noalloc", "get_error", "IMPL_AUTO", "IMPL_REGISTER", "IMPL_BULK"]
+           "step", "step_bucket", "step_overlapped", "step_host", "step_noalloc", "get_error", "IMPL_AUTO", "IMPL_REGISTER", "IMPL_BULK"]
 
 IMPL_AUTO, IMPL_REGISTER, IMPL_BULK = 0, 1, 2
 
@@ -179,6 +179,31 @@ def step(layout, grads, master, m, v, p16_shard, p16_full, hp, nonfinite=None, e
                                 _ptr(m), _ptr(v), _ptr(p16_shard), _ptr(p16_full), ctypes.byref(h),
                                 _ptr(nonfinite), ctypes.byref(ev) if ev is not None else None,
                                 _stream(stream)), "zero_step")
+
+
+def step_bucket(layout, bucket, grads, master, m, v, p16_shard, p16_full, hp, nonfinite=None, rank_stride=None,
+                stream=None):
+    """The fused reduce-scatter + update of one bucket (zero_step_bucket)."""
+    h = hp.c()
+    _check(_abi.lib().zero_step_bucket(layout.handle, int(bucket), _ptr(grads), _stride(grads, layout, rank_stride),
+                                       _ptr(master), _ptr(m), _ptr(v), _ptr(p16_shard), _ptr(p16_full),
+                                       ctypes.byref(h), _ptr(nonfinite), _stream(stream)), "zero_step_bucket")
+
+
+def step_overlapped(layout, ready_events, grads, master, m, v, p16_shard, p16_full, hp, nonfinite=None,
+                    rank_stride=None, stream=None):
+    """zero_step with bucket b gated on ready_events[b] (torch.cuda.Event, recorded by the
+    producer of bucket b's gradients)."""
+    assert len(ready_events) == layout.n_buckets
+    handles = (ctypes.c_void_p * max(1, layout.n_buckets))()
+    for b, e in enumerate(ready_events):
+        if e.cuda_event == 0:
+            raise ValueError(f"ready event of bucket {b} was never recorded")
+        handles[b] = e.cuda_event
+    h = hp.c()
+    _check(_abi.lib().zero_step_overlapped(layout.handle, handles, _ptr(grads), _stride(grads, layout, rank_stride),
+                                           _ptr(master), _ptr(m), _ptr(v), _ptr(p16_shard), _ptr(p16_full),
+                                           ctypes.byref(h), _ptr(nonfinite), _stream(stream)), "zero_step_overlapped")
 
 
 def step_host(layout, grads_host, grads_dev, master, m, v, p16_shard, p16_full, p16_host, hp,

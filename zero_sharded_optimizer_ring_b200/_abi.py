@@ -56,6 +56,10 @@ SIGNATURES = {
     "zero_allgather": (_i32, [_vp, _i64, _vp, _vp, _vp]),
     "zero_step": (_i32, [_vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(AdamWHparams), _vp,
                          ctypes.POINTER(StepEvents), _vp]),
+    "zero_step_bucket": (_i32, [_vp, _i64, _vp, _i64, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(AdamWHparams),
+                                _vp, _vp]),
+    "zero_step_overlapped": (_i32, [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(AdamWHparams),
+                                    _vp, _vp]),
     "zero_step_host": (_i32, [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp,
                               ctypes.POINTER(AdamWHparams), _vp, _vp]),
     "zero_step_noalloc": (_i32, [_vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(AdamWHparams), _vp, _vp]),

@@ -313,6 +313,42 @@ extern "C" zero_status zero_step(const zero_layout *L, const uint16_t *grads, in
     return cuda_status(e);
 }
 
+extern "C" zero_status zero_step_bucket(const zero_layout *L, int64_t bucket, const uint16_t *grads,
+                                        int64_t rank_stride, float *master, float *m, float *v,
+                                        uint16_t *p16_shard, uint16_t *p16_full, const zero_adamw_hparams *hp,
+                                        int32_t *nonfinite, void *stream)
+{
+    zero_status s = check_step(L, grads, rank_stride, master, m, v, p16_shard, p16_full, hp);
+    if (s != ZERO_OK || L->padded == 0) return s;
+    if (bucket < 0 || bucket >= (int64_t)L->bucket_lo.size()) return ZERO_ERR_INVALID;
+    uint16_t *p16 = L->stage == 3 ? p16_shard : p16_full;
+    return cuda_status(fused(L, bucket_tiles(L, bucket), grads, rank_stride, master, m, v, p16,
+                             step_scalars(L->n_ranks, *hp), nonfinite, (cudaStream_t)stream));
+}
+
+extern "C" zero_status zero_step_overlapped(const zero_layout *L, void *const *ready_events, const uint16_t *grads,
+                                            int64_t rank_stride, float *master, float *m, float *v,
+                                            uint16_t *p16_shard, uint16_t *p16_full, const zero_adamw_hparams *hp,
+                                            int32_t *nonfinite, void *stream)
+{
+    zero_status s = check_step(L, grads, rank_stride, master, m, v, p16_shard, p16_full, hp);
+    if (s != ZERO_OK || L->padded == 0) return s;
+    if (!ready_events) return ZERO_ERR_INVALID;
+    for (size_t b = 0; b < L->bucket_lo.size(); ++b)
+        if (!ready_events[b]) return ZERO_ERR_INVALID;
+    cudaStream_t st = (cudaStream_t)stream;
+    const AdamScalars c = step_scalars(L->n_ranks, *hp);
+    uint16_t *p16 = L->stage == 3 ? p16_shard : p16_full;
+    cudaError_t e = cudaSuccess;
+    for (size_t b = 0; e == cudaSuccess && b < L->bucket_lo.size(); ++b) {
+        e = cudaStreamWaitEvent(st, (cudaEvent_t)ready_events[b], 0);
+        if (e == cudaSuccess)
+            e = fused(L, bucket_tiles(L, (int64_t)b), grads, rank_stride, master, m, v, p16, c, nonfinite, st);
+    }
+    if (e == cudaSuccess && L->stage == 3) e = zero::launch_copy_range(*L, 0, L->padded, p16_shard, p16_full, st);
+    return cuda_status(e);
+}
+
 extern "C" zero_status zero_step_host(const zero_layout *L, const uint16_t *grads_host, uint16_t *grads_dev,
                                       int64_t rank_stride, float *master, float *m, float *v,
                                       uint16_t *p16_shard, uint16_t *p16_full, uint16_t *p16_host,

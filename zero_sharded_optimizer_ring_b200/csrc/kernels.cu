@@ -278,27 +278,27 @@ adamw_range_kernel(int64_t lo, int64_t hi, const float *__restrict__ reduced, fl
     }
 }
 
-// Copy [lo, hi): each thread keeps kCopyUnroll 16-byte loads in flight before storing;
-// the block's vectors stay contiguous (thread t takes vectors t, t + 256, ...).
+// Copy [lo, hi): one block per 4 x 256 16-byte vectors, each thread holding its 4 loads in
+// flight before storing.  A grid of short blocks keeps the blocks in flight on a compact
+// window of the buffer (a persistent grid-stride loop lets the blocks drift apart over
+// the buffer and costs ~15 % of copy bandwidth on B200: 5.9 vs 6.9 TB/s measured).
 constexpr int kCopyUnroll = 4;
 
 __global__ void __launch_bounds__(kThreads)
 copy_range_kernel(int64_t lo, int64_t hi, const uint16_t *__restrict__ src, uint16_t *__restrict__ dst)
 {
     const int64_t va = (lo + kVec - 1) / kVec * kVec, vb = hi / kVec * kVec;
-    const int64_t block_span = (int64_t)kThreads * kVec * kCopyUnroll;
-    for (int64_t base = va + (int64_t)blockIdx.x * block_span; base < vb; base += (int64_t)gridDim.x * block_span) {
-        uint4 x[kCopyUnroll];
+    const int64_t base = va + (int64_t)blockIdx.x * kThreads * kVec * kCopyUnroll;
+    uint4 x[kCopyUnroll];
 #pragma unroll
-        for (int u = 0; u < kCopyUnroll; ++u) {
-            const int64_t q = base + ((int64_t)u * kThreads + threadIdx.x) * kVec;
-            if (q < vb) x[u] = __ldcs(reinterpret_cast<const uint4 *>(src + q));
-        }
+    for (int u = 0; u < kCopyUnroll; ++u) {
+        const int64_t q = base + ((int64_t)u * kThreads + threadIdx.x) * kVec;
+        if (q < vb) x[u] = *reinterpret_cast<const uint4 *>(src + q);
+    }
 #pragma unroll
-        for (int u = 0; u < kCopyUnroll; ++u) {
-            const int64_t q = base + ((int64_t)u * kThreads + threadIdx.x) * kVec;
-            if (q < vb) __stcs(reinterpret_cast<uint4 *>(dst + q), x[u]);
-        }
+    for (int u = 0; u < kCopyUnroll; ++u) {
+        const int64_t q = base + ((int64_t)u * kThreads + threadIdx.x) * kVec;
+        if (q < vb) *reinterpret_cast<uint4 *>(dst + q) = x[u];
     }
     if (blockIdx.x == 0) {
         const int64_t head_end = va < hi ? va : hi;
@@ -423,9 +423,11 @@ cudaError_t launch_copy_range(const zero_layout &L, int64_t lo, int64_t hi, cons
                               uint16_t *dst, cudaStream_t s)
 {
     if (hi <= lo) return cudaSuccess;
-    const int grid = grid_for(copy_range_kernel, (hi - lo + kThreads * kVec * kCopyUnroll - 1) /
-                                                     (kThreads * kVec * kCopyUnroll), L.dev.num_sms);
-    copy_range_kernel<<<grid, kThreads, 0, s>>>(lo, hi, src, dst);
+    const int64_t per_block = (int64_t)kThreads * kVec * kCopyUnroll;
+    const int64_t va = (lo + kVec - 1) / kVec * kVec, vb = hi / kVec * kVec;
+    const int64_t blocks = vb > va ? (vb - va + per_block - 1) / per_block : 1;
+    (void)L;
+    copy_range_kernel<<<(unsigned)blocks, kThreads, 0, s>>>(lo, hi, src, dst);
     return cudaGetLastError();
 }
 
