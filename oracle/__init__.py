@@ -50,7 +50,9 @@ def configure(L):
     L.oracle_float_to_half.restype = ctypes.c_uint16
     L.oracle_halfs_to_floats.argtypes = [_vp, _vp, _i64]
     L.oracle_floats_to_halfs.argtypes = [_vp, _vp, _i64]
-    L.oracle_ring_reduce_scatter.argtypes = [_vp, _i32, _i64, _i64, _i64, _i64, _i32,
+    L.oracle_double_to_half.argtypes = [_dbl]
+    L.oracle_double_to_half.restype = ctypes.c_uint16
+    L.oracle_ring_reduce_scatter.argtypes = [_vp, _i32, _i64, _i64, _i64, _i64, _i32, _i32,
                                              _vp, _vp, _vp, _vp, _vp]
     L.oracle_ring_reduce_scatter.restype = _i64
     L.oracle_ring_allgather.argtypes = [_vp, _i32, _i32, _i64, _i64, _i64, _i64, _vp, _vp, _vp]
@@ -59,7 +61,7 @@ def configure(L):
     L.oracle_adamw.argtypes = [_i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]
     L.oracle_count_nonfinite.argtypes = [_vp, _i64, _i64]
     L.oracle_count_nonfinite.restype = _i64
-    L.oracle_sampled.argtypes = [_i64, _i32, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp]
+    L.oracle_sampled.argtypes = [_i64, _i32, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp]
     return L
 
 
@@ -106,15 +108,16 @@ def adamw_scalars(n_ranks, hp, t):
 
 
 def ring_reduce_scatter(grads, shard, blo, bhi, hops=None, reduced=None, sent=None, recv=None,
-                        want_log=False):
+                        want_log=False, wire16=False):
     """Scatter-reduce of bucket [blo, bhi).  grads: uint16 [N, rank_stride] fp16 bits.
+    wire16: partials travel as fp16 (each hop's sum rounded to fp16).
     Returns (work [N, bhi-blo] running partials per rank, log [n, 4] or None)."""
     _need(grads, np.uint16)
     N, stride = grads.shape
     hops = N - 1 if hops is None else hops
     work = np.zeros((N, bhi - blo), dtype=np.float32)
     log = np.zeros((max(1, N * hops), 4), dtype=np.int64) if want_log else None
-    n = lib().oracle_ring_reduce_scatter(_p(grads), N, stride, shard, blo, bhi, hops, _p(work),
+    n = lib().oracle_ring_reduce_scatter(_p(grads), N, stride, shard, blo, bhi, hops, int(wire16), _p(work),
                                          _p(reduced), _p(log), _p(sent), _p(recv))
     return work, (log[:n] if want_log else None)
 
@@ -140,7 +143,11 @@ def count_nonfinite(reduced, lo, hi):
     return int(lib().oracle_count_nonfinite(_p(_need(reduced, np.float32)), lo, hi))
 
 
-def sampled(g, shard_of, steps, scalars, master, m, v):
+def double_to_half(x):
+    return int(lib().oracle_double_to_half(float(x)))
+
+
+def sampled(g, shard_of, steps, scalars, master, m, v, wire16=False):
     """Per-element path: g uint16 [n, N]; shard_of int64 [n]; scalars float32 [steps, 9];
     master/m/v float32 [n] (updated in place).  Returns (reduced, p16)."""
     g = np.ascontiguousarray(g, dtype=np.uint16)
@@ -151,7 +158,7 @@ def sampled(g, shard_of, steps, scalars, master, m, v):
         _need(a, np.float32)
     reduced = np.zeros(n, dtype=np.float32)
     p16 = np.zeros(n, dtype=np.uint16)
-    lib().oracle_sampled(n, N, _p(g), _p(shard_of), steps, _p(scalars), _p(reduced),
+    lib().oracle_sampled(n, N, _p(g), _p(shard_of), int(wire16), steps, _p(scalars), _p(reduced),
                          _p(master), _p(m), _p(v), _p(p16))
     return reduced, p16
 
@@ -172,7 +179,7 @@ class StepResult:
     replicas_identical: bool  # with replicas=True: every rank ended with the same values
 
 
-def run_steps(lay, stage, grads, master, m, v, hp, steps, replicas=False):
+def run_steps(lay, stage, grads, master, m, v, hp, steps, replicas=False, wire16=False, first_step=1):
     """Run `steps` optimizer steps of ZeRO stage `stage` (0 = DDP) on the oracle.
 
     grads: uint16 [N, rank_stride >= P] fp16 bits (the same at every step);
@@ -194,11 +201,11 @@ def run_steps(lay, stage, grads, master, m, v, hp, steps, replicas=False):
     reduced = np.zeros(P, dtype=np.float32)
     nonfinite = np.zeros(len(lay.buckets), dtype=np.int64)
 
-    for t in range(1, steps + 1):
+    for t in range(first_step, first_step + steps):
         sc = adamw_scalars(N, hp, t)
         reduced[:] = 0
         for b, (lo, hi) in enumerate(lay.buckets):
-            ring_reduce_scatter(grads, S, lo, hi, reduced=reduced, sent=sent, recv=recv)
+            ring_reduce_scatter(grads, S, lo, hi, reduced=reduced, sent=sent, recv=recv, wire16=wire16)
             nonfinite[b] = count_nonfinite(reduced, lo, hi)
 
         if stage == 0:
@@ -244,3 +251,60 @@ def run_steps(lay, stage, grads, master, m, v, hp, steps, replicas=False):
         p16_shard = p16_full[0].copy()
     return StepResult(master, m, v, p16_full[0].copy(), p16_shard, reduced.copy(), nonfinite,
                       sent, recv, same)
+
+
+# ---------------------------------------------------------------- dynamic loss scaling
+
+@dataclass
+class LossScaler:
+    """Dynamic loss scaling (mixed-precision training practice; the pages do not spell it
+    out): gradients arrive multiplied by `scale`.  A step whose reduced gradients hold a
+    non-finite value is skipped (no state changes) and the scale is divided by `factor`
+    (not below `min_scale`); after `window` consecutive applied steps it is multiplied by
+    `factor`.  `step` counts applied AdamW steps (the next applied step uses step + 1)."""
+    scale: float
+    factor: float = 2.0
+    window: int = 1000
+    min_scale: float = 1.0
+    clean_steps: int = 0
+    step: int = 0
+    skipped: int = 0
+
+    def update(self, overflow):
+        if overflow:
+            self.scale = max(self.scale / self.factor, self.min_scale)
+            self.clean_steps = 0
+            self.skipped += 1
+        else:
+            self.step += 1
+            self.clean_steps += 1
+            if self.clean_steps == self.window:
+                self.scale *= self.factor
+                self.clean_steps = 0
+
+
+def run_steps_dynamic(lay, stage, grads_at, master, m, v, hp, steps, scaler, wire16=False):
+    """`steps` training steps under dynamic loss scaling.  grads_at(scale, i) gives step i's
+    fp16 gradients [N, >= P] produced at loss scale `scale`.  Each step reduces every
+    bucket (ring order, fp32 or fp16 wire), and applies the update with the scale the
+    gradients carry only if no reduced value is non-finite.  Returns (result of the last
+    applied step or None, trace of (scale used, overflow, AdamW step or 0) per step)."""
+    N, S = lay.n_ranks, lay.shard
+    state = [np.array(x, dtype=np.float32, copy=True) for x in (master, m, v)]
+    last = None
+    trace = []
+    for i in range(steps):
+        g = grads_at(scaler.scale, i)
+        reduced = np.zeros(lay.padded, dtype=np.float32)
+        bad = 0
+        for lo, hi in lay.buckets:
+            ring_reduce_scatter(g, S, lo, hi, reduced=reduced, wire16=wire16)
+            bad += count_nonfinite(reduced, lo, hi)
+        used = scaler.scale
+        if bad == 0:
+            h = Hyper(hp.lr, hp.beta1, hp.beta2, hp.eps, hp.weight_decay, used)
+            last = run_steps(lay, stage, g, *state, h, 1, wire16=wire16, first_step=scaler.step + 1)
+            state = [last.master, last.m, last.v]
+        scaler.update(bad > 0)
+        trace.append((used, bad > 0, scaler.step if bad == 0 else 0))
+    return last, trace

@@ -47,10 +47,10 @@ ORACLE_API float oracle_half_to_float(uint16_t h)
     return (float)(sign ? -mag : mag);
 }
 
-ORACLE_API uint16_t oracle_float_to_half(float x)
+ORACLE_API uint16_t oracle_double_to_half(double x)
 {
     const uint16_t sign = signbit(x) ? 0x8000 : 0;
-    const double a = fabs((double)x);
+    const double a = fabs(x);
     if (isnan(x)) return (uint16_t)(sign | 0x7e00);
     if (a == 0.0) return sign;
     /* spacing of halfs at |x|: 2^-24 below 2^-14, else 2^(floor(log2|x|) - 10) */
@@ -68,6 +68,21 @@ ORACLE_API uint16_t oracle_float_to_half(float x)
     const int er = ex - 1;
     const uint16_t frac = (uint16_t)(r / ldexp(1.0, er - 10) - 1024.0);
     return (uint16_t)(sign | (uint16_t)((er + 15) << 10) | frac);
+}
+
+/* fp32 -> fp16: the fp32 value is exact in double, so one rounding, as above. */
+ORACLE_API uint16_t oracle_float_to_half(float x)
+{
+    return oracle_double_to_half((double)x);
+}
+
+/* One hop of the fp16 wire: the receiver adds its own fp16 gradient to the fp16 partial
+ * it received and sends the sum on as fp16.  Two fp16 values have at most 11 significant
+ * bits each within exponents -24..15, so their sum is exact in double; rounding it once
+ * gives the correctly rounded fp16 sum. */
+static float wire16_add(float incoming, float own)
+{
+    return oracle_half_to_float(oracle_double_to_half((double)incoming + (double)own));
 }
 
 ORACLE_API void oracle_halfs_to_floats(const uint16_t *in, float *out, int64_t n)
@@ -109,10 +124,13 @@ static void chunk_range(int64_t k, int64_t shard, int64_t lo, int64_t hi, int64_
  * its own partial to it (page 3's trace: a0 goes to GPU1, which forms a0+a1, ...).
  * After N-1 hops chunk k's full sum, folded in the order k, k+1, ..., k+N-1, sits at
  * rank (k - 1) mod N.  Returns the number of log records written.
+ *   wire16   0: partials travel as fp32 (every add one fp32 rounding); 1: partials travel
+ *            as fp16, every hop's sum rounded to fp16 (rkmt.cn/news/44736 "Deepspeed
+ *            ZeRO-1": each GPU ends up with its part's gradient mean in fp16).
  */
 ORACLE_API int64_t oracle_ring_reduce_scatter(const uint16_t *grads, int32_t n_ranks,
                                               int64_t rank_stride, int64_t shard,
-                                              int64_t blo, int64_t bhi, int32_t hops,
+                                              int64_t blo, int64_t bhi, int32_t hops, int32_t wire16,
                                               float *work, float *reduced, int64_t *log,
                                               int64_t *sent, int64_t *recv)
 {
@@ -130,7 +148,8 @@ ORACLE_API int64_t oracle_ring_reduce_scatter(const uint16_t *grads, int32_t n_r
             chunk_range(k, shard, blo, bhi, &clo, &chi);
             for (int64_t i = clo; i < chi; ++i) {
                 const float incoming = work[r * n + (i - blo)];
-                work[dst * n + (i - blo)] = incoming + work[dst * n + (i - blo)];
+                const float own = work[dst * n + (i - blo)];
+                work[dst * n + (i - blo)] = wire16 ? wire16_add(incoming, own) : incoming + own;
             }
             if (log) {
                 log[4 * nlog + 0] = h;
@@ -271,7 +290,7 @@ ORACLE_API int64_t oracle_count_nonfinite(const float *reduced, int64_t lo, int6
  * are the same at every step.  reduced[j] receives the ring sum.
  */
 ORACLE_API void oracle_sampled(int64_t n, int32_t n_ranks, const uint16_t *g, const int64_t *shard_of,
-                               int32_t steps, const float *scalars, float *reduced,
+                               int32_t wire16, int32_t steps, const float *scalars, float *reduced,
                                float *master, float *m, float *v, uint16_t *p16)
 {
     for (int64_t j = 0; j < n; ++j) {
@@ -279,7 +298,8 @@ ORACLE_API void oracle_sampled(int64_t n, int32_t n_ranks, const uint16_t *g, co
         float partial = oracle_half_to_float(g[j * n_ranks + k]);      /* starts at rank k */
         for (int32_t h = 0; h < n_ranks - 1; ++h) {
             const int64_t receiver = imod(k + h + 1, n_ranks);
-            partial = partial + oracle_half_to_float(g[j * n_ranks + receiver]);
+            const float own = oracle_half_to_float(g[j * n_ranks + receiver]);
+            partial = wire16 ? wire16_add(partial, own) : partial + own;
         }
         reduced[j] = partial;
         for (int32_t t = 0; t < steps; ++t)

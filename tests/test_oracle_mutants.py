@@ -20,6 +20,7 @@ import test_oracle_adamw as T_adamw
 import test_oracle_fp16 as T_fp16
 import test_oracle_ring as T_ring
 import test_oracle_stages as T_stages
+import test_oracle_wire as T_wire
 
 ORACLE_DIR = os.path.dirname(oracle.__file__)
 
@@ -33,13 +34,16 @@ PINS = [
     T_stages.test_allgather_is_concatenation_of_partitions, T_stages.test_literal_send_counts_match_closed_form,
     T_stages.test_memory_and_comm_closed_forms_match_pages, T_stages.test_layout_brute_force,
     T_stages.test_three_gpu_thirds,
+    T_wire.test_one_wire_hop_is_the_rounded_fp16_sum, T_wire.test_wire_rounds_at_every_hop,
+    T_wire.test_wire_overflow_depends_on_ring_order, T_wire.test_scaler_follows_hand_trace,
+    T_wire.test_dynamic_run_skips_overflowing_steps,
 ]
 
 # (name, original text, mutated text) in oracle.c
 C_MUTANTS = [
     ("fold starts one rank late", "const int64_t k = imod(r - h, n_ranks);", "const int64_t k = imod(r - h + 1, n_ranks);"),
-    ("receiver drops its own value", "work[dst * n + (i - blo)] = incoming + work[dst * n + (i - blo)];",
-     "work[dst * n + (i - blo)] = incoming;"),
+    ("receiver drops its own value", "wire16 ? wire16_add(incoming, own) : incoming + own;",
+     "wire16 ? wire16_add(incoming, own) : incoming;"),
     ("sum read from the wrong rank", "const int64_t holder = imod(k - 1, n_ranks);", "const int64_t holder = imod(k, n_ranks);"),
     ("all-gather passes the wrong chunk", "const int64_t k = imod(r + 1 - h, n_ranks);", "const int64_t k = imod(r - h, n_ranks);"),
     ("no weight decay", "float pp = *p * s[1];", "float pp = *p;"),
@@ -55,6 +59,10 @@ C_MUTANTS = [
     ("fp16 exponent bias off", "mag = ldexp((double)(1024 + f), e - 25);", "mag = ldexp((double)(1024 + f), e - 24);"),
     ("non-finite count misses inf", "if (!isfinite(reduced[i])) ++c;", "if (isnan(reduced[i])) ++c;"),
     ("sender counter not kept", "if (sent) sent[r] += chi - clo;", "if (sent) sent[r] += 0;"),
+    ("wire sum not rounded to fp16", "return oracle_half_to_float(oracle_double_to_half((double)incoming + (double)own));",
+     "return incoming + own;"),
+    ("wire sum rounded through fp32", "oracle_double_to_half((double)incoming + (double)own)",
+     "oracle_double_to_half((double)(float)((double)incoming + (double)own) * 1.0000001)"),
 ]
 
 # (name, original, mutated) in layout.py
@@ -66,6 +74,14 @@ PY_MUTANTS = [
     ("ZeRO-3 without the backward gather", "phases = 3 if stage == 3 else 2", "phases = 2"),
     ("ZeRO-2 keeps full gradients", "p16, g16, os_ = 2 * psi, 2 * S, 12 * S", "p16, g16, os_ = 2 * psi, 2 * psi, 12 * S"),
     ("DDP optimizer state sharded", "p16, g16, os_ = 2 * psi, 2 * psi, 12 * psi", "p16, g16, os_ = 2 * psi, 2 * psi, 12 * S"),
+]
+
+# (name, original, mutated) in the oracle's Python composition (oracle/__init__.py)
+INIT_MUTANTS = [
+    ("scaler never grows", "                self.scale *= self.factor\n", "                self.scale *= 1.0\n"),
+    ("scaler counts skipped steps as applied", "            self.skipped += 1\n", "            self.skipped += 1\n            self.step += 1\n"),
+    ("overflow step still updates", "        if bad == 0:\n            h = Hyper(", "        if True:\n            h = Hyper("),
+    ("scale window not reset", "                self.clean_steps = 0\n", "                pass\n"),
 ]
 
 
@@ -116,3 +132,16 @@ def test_layout_mutant_is_caught(name, old, new, workdir, monkeypatch):
 
 def test_unmutated_oracle_passes_every_pin():
     assert not _some_pin_fails()
+
+
+@pytest.mark.parametrize("name,old,new", INIT_MUTANTS, ids=[m[0] for m in INIT_MUTANTS])
+def test_composition_mutant_is_caught(name, old, new, monkeypatch):
+    src = open(os.path.join(ORACLE_DIR, "__init__.py")).read()
+    assert old in src, name
+    ns = {"__name__": "oracle_mutant"}
+    mutated = src.replace(old, new, 1).replace("from . import build as _build", "from oracle import build as _build")
+    mutated = mutated.replace("from .layout import", "from oracle.layout import")
+    exec(compile(mutated, "oracle_mutant", "exec"), ns)
+    monkeypatch.setattr(oracle, "LossScaler", ns["LossScaler"])
+    monkeypatch.setattr(oracle, "run_steps_dynamic", ns["run_steps_dynamic"])
+    assert _some_pin_fails(), f"no pin caught the planted mistake: {name}"
