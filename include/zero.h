@@ -63,6 +63,11 @@ typedef struct {
     int64_t n_units;                    /* stage-3 gather units (layers); 0 = one unit */
     const int64_t *unit_first_tensor;   /* [n_units]: first tensor of each unit; [0] == 0,
                                            strictly increasing (host memory, copied) */
+    int32_t wire_fp16;                  /* 0: the ring's partial sums are fp32 (one fp32
+                                           rounding per add); 1: they travel as fp16, each
+                                           hop's sum rounded to fp16 (P1 Deepspeed ZeRO-1:
+                                           each GPU ends with its part's gradient mean in
+                                           fp16); sums beyond 65504 then overflow to inf */
 } zero_layout_desc;
 
 typedef struct {
@@ -87,6 +92,21 @@ typedef struct {
     int64_t mem_p16, mem_g16, mem_os, mem_total;
     int64_t sent_elems, recv_elems;
 } zero_counters;
+
+/* Dynamic loss scaling state (host memory, updated by zero_step_dynamic).  Mixed-precision
+ * practice (the pages do not spell it out): gradients arrive multiplied by `scale`; a
+ * step whose reduced gradients hold a non-finite value is skipped and the scale divided by
+ * `factor` (not below `min_scale`); after `window` applied steps in a row it is multiplied
+ * by `factor`.  `step` counts applied AdamW steps: the next applied step uses step + 1. */
+typedef struct {
+    double scale;           /* > 0 */
+    double factor;          /* > 1 */
+    int64_t window;         /* >= 1 */
+    double min_scale;       /* > 0 */
+    int64_t clean_steps;    /* state: applied steps since the scale last changed */
+    int64_t step;           /* state: applied AdamW steps so far */
+    int64_t skipped;        /* state: steps skipped for overflow */
+} zero_loss_scaler;
 
 /* Optional CUDA events (cudaEvent_t, created by the caller; any may be NULL) that
  * zero_step records on `stream` around its kernels, for per-kernel timing. */
@@ -237,6 +257,21 @@ zero_status zero_step_host(const zero_layout *layout, const uint16_t *grads_host
 zero_status zero_step_noalloc(const zero_layout *layout, const uint16_t *grads, int64_t rank_stride,
                               float *master, float *m, float *v, uint16_t *p16_shard, uint16_t *p16_full,
                               const zero_adamw_hparams *hp, int32_t *nonfinite, void *stream);
+
+/* One step under dynamic loss scaling (see zero_loss_scaler).  The gradients must carry
+ * the scaler's current scale.  Runs the reduce-scatter of every bucket into `reduced`
+ * (fp32 [P], caller's scratch) with per-bucket non-finite counts in `nonfinite` (device
+ * int32 [n_buckets], required, zeroed here), copies the counts back and synchronises
+ * `stream`; then, if every count is zero, applies the shard update with loss_scale =
+ * scale and step = scaler->step + 1 (hp's loss_scale and step are ignored) and, for
+ * stage 3, the all-gather; otherwise skips the update, leaving master, m, v and the fp16
+ * parameters untouched.  Finally advances the scaler.  *applied = 1 if the update ran.
+ * With the fp16 wire (zero_layout_desc.wire_fp16) a partial sum beyond 65504 overflows
+ * and triggers a skip; with fp32 partials only non-finite inputs do. */
+zero_status zero_step_dynamic(const zero_layout *layout, const uint16_t *grads, int64_t rank_stride,
+                              float *reduced, float *master, float *m, float *v, uint16_t *p16_shard,
+                              uint16_t *p16_full, const zero_adamw_hparams *hp, zero_loss_scaler *scaler,
+                              int32_t *nonfinite, int32_t *applied, void *stream);
 
 /* Select the fused kernel's implementation: 0 = automatic (the bulk-copy pipeline for
  * N in 1..8 and 16, register streaming otherwise), 1 = register streaming (vectorised

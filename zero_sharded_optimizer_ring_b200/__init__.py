@@ -16,7 +16,8 @@ import numpy as np
 from . import _abi
 
 __all__ = ["ZeroError", "Layout", "AdamW", "reduce_scatter", "adamw_shard_step", "allgather",
-           "step", "step_bucket", "step_overlapped", "step_host", "step_noalloc", "get_error", "IMPL_AUTO", "IMPL_REGISTER", "IMPL_BULK"]
+           "step", "step_bucket", "step_overlapped", "step_dynamic", "LossScaler", "step_host",
+           "step_noalloc", "get_error", "IMPL_AUTO", "IMPL_REGISTER", "IMPL_BULK"]
 
 IMPL_AUTO, IMPL_REGISTER, IMPL_BULK = 0, 1, 2
 
@@ -69,12 +70,12 @@ class AdamW:
 class Layout:
     """Flat buffer, shards, buckets, segments and gather units (zero_layout_create)."""
 
-    def __init__(self, tensors, n_ranks, stage, bucket_elems=0, pad_align=128, units=()):
+    def __init__(self, tensors, n_ranks, stage, bucket_elems=0, pad_align=128, units=(), wire_fp16=False):
         lib = _abi.lib()
         self._numel = (ctypes.c_int64 * max(1, len(tensors)))(*[int(x) for x in tensors])
         self._units = (ctypes.c_int64 * max(1, len(units)))(*[int(x) for x in units])
         desc = _abi.LayoutDesc(int(n_ranks), int(stage), len(tensors), self._numel, int(bucket_elems),
-                               int(pad_align), len(units), self._units)
+                               int(pad_align), len(units), self._units, int(bool(wire_fp16)))
         h = ctypes.c_void_p()
         _check(lib.zero_layout_create(ctypes.byref(desc), ctypes.byref(h)), "zero_layout_create")
         self._h = h
@@ -204,6 +205,28 @@ def step_overlapped(layout, ready_events, grads, master, m, v, p16_shard, p16_fu
     _check(_abi.lib().zero_step_overlapped(layout.handle, handles, _ptr(grads), _stride(grads, layout, rank_stride),
                                            _ptr(master), _ptr(m), _ptr(v), _ptr(p16_shard), _ptr(p16_full),
                                            ctypes.byref(h), _ptr(nonfinite), _stream(stream)), "zero_step_overlapped")
+
+
+class LossScaler:
+    """Dynamic loss scaling state (zero_loss_scaler); advanced by step_dynamic()."""
+
+    def __init__(self, scale, factor=2.0, window=1000, min_scale=1.0):
+        self.c = _abi.LossScaler(float(scale), float(factor), int(window), float(min_scale), 0, 0, 0)
+
+    def __getattr__(self, name):
+        return getattr(self.__dict__["c"], name)
+
+
+def step_dynamic(layout, grads, reduced, master, m, v, p16_shard, p16_full, hp, scaler, nonfinite,
+                 rank_stride=None, stream=None):
+    """One step under dynamic loss scaling; returns True if the update was applied."""
+    h = hp.c()
+    applied = ctypes.c_int32(0)
+    _check(_abi.lib().zero_step_dynamic(layout.handle, _ptr(grads), _stride(grads, layout, rank_stride),
+                                        _ptr(reduced), _ptr(master), _ptr(m), _ptr(v), _ptr(p16_shard),
+                                        _ptr(p16_full), ctypes.byref(h), ctypes.byref(scaler.c), _ptr(nonfinite),
+                                        ctypes.byref(applied), _stream(stream)), "zero_step_dynamic")
+    return bool(applied.value)
 
 
 def step_host(layout, grads_host, grads_dev, master, m, v, p16_shard, p16_full, p16_host, hp,

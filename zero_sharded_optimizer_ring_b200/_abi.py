@@ -19,7 +19,7 @@ STATUS_NAMES = {0: "ZERO_OK", 1: "ZERO_ERR_INVALID", 2: "ZERO_ERR_ALIGN", 3: "ZE
 class LayoutDesc(ctypes.Structure):
     _fields_ = [("n_ranks", _i32), ("stage", _i32), ("n_tensors", _i64),
                 ("tensor_numel", _p_i64), ("bucket_elems", _i64), ("pad_align", _i64),
-                ("n_units", _i64), ("unit_first_tensor", _p_i64)]
+                ("n_units", _i64), ("unit_first_tensor", _p_i64), ("wire_fp16", _i32)]
 
 
 class LayoutInfo(ctypes.Structure):
@@ -36,6 +36,11 @@ class AdamWHparams(ctypes.Structure):
 class Counters(ctypes.Structure):
     _fields_ = [("mem_p16", _i64), ("mem_g16", _i64), ("mem_os", _i64), ("mem_total", _i64),
                 ("sent_elems", _i64), ("recv_elems", _i64)]
+
+
+class LossScaler(ctypes.Structure):
+    _fields_ = [("scale", ctypes.c_double), ("factor", ctypes.c_double), ("window", _i64),
+                ("min_scale", ctypes.c_double), ("clean_steps", _i64), ("step", _i64), ("skipped", _i64)]
 
 
 class StepEvents(ctypes.Structure):
@@ -60,6 +65,8 @@ SIGNATURES = {
                                 _vp, _vp]),
     "zero_step_overlapped": (_i32, [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(AdamWHparams),
                                     _vp, _vp]),
+    "zero_step_dynamic": (_i32, [_vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(AdamWHparams),
+                                 ctypes.POINTER(LossScaler), _vp, ctypes.POINTER(_i32), _vp]),
     "zero_step_host": (_i32, [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp,
                               ctypes.POINTER(AdamWHparams), _vp, _vp]),
     "zero_step_noalloc": (_i32, [_vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(AdamWHparams), _vp, _vp]),

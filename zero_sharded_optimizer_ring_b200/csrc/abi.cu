@@ -25,13 +25,13 @@ zero_status check_device(const zero_layout *L)
 
 zero_status cuda_status(cudaError_t e) { return e == cudaSuccess ? ZERO_OK : ZERO_ERR_CUDA; }
 
-bool finite(double x) { return isfinite(x) != 0; }
+bool finite_d(double x) { return isfinite(x) != 0; }
 
 zero_status check_hparams(const zero_adamw_hparams *h)
 {
     if (!h) return ZERO_ERR_INVALID;
-    if (h->step < 1 || !finite(h->lr) || !finite(h->eps) || !finite(h->weight_decay) ||
-        !finite(h->loss_scale) || !(h->loss_scale > 0.0) || !(h->beta1 >= 0.0 && h->beta1 < 1.0) ||
+    if (h->step < 1 || !finite_d(h->lr) || !finite_d(h->eps) || !finite_d(h->weight_decay) ||
+        !finite_d(h->loss_scale) || !(h->loss_scale > 0.0) || !(h->beta1 >= 0.0 && h->beta1 < 1.0) ||
         !(h->beta2 >= 0.0 && h->beta2 < 1.0))
         return ZERO_ERR_INVALID;
     return ZERO_OK;
@@ -347,6 +347,55 @@ extern "C" zero_status zero_step_overlapped(const zero_layout *L, void *const *r
     }
     if (e == cudaSuccess && L->stage == 3) e = zero::launch_copy_range(*L, 0, L->padded, p16_shard, p16_full, st);
     return cuda_status(e);
+}
+
+extern "C" zero_status zero_step_dynamic(const zero_layout *L, const uint16_t *grads, int64_t rank_stride,
+                                         float *reduced, float *master, float *m, float *v, uint16_t *p16_shard,
+                                         uint16_t *p16_full, const zero_adamw_hparams *hp, zero_loss_scaler *sc,
+                                         int32_t *nonfinite, int32_t *applied, void *stream)
+{
+    if (!L || !hp || !sc || !applied) return ZERO_ERR_INVALID;
+    if (!(sc->scale > 0.0) || !finite_d(sc->scale) || !(sc->factor > 1.0) || !finite_d(sc->factor) ||
+        sc->window < 1 || !(sc->min_scale > 0.0) || !finite_d(sc->min_scale) || sc->step < 0)
+        return ZERO_ERR_INVALID;
+    zero_adamw_hparams h = *hp;
+    h.loss_scale = sc->scale;
+    h.step = sc->step + 1;
+    zero_status s = check_step(L, grads, rank_stride, master, m, v, p16_shard, p16_full, &h);
+    if (s != ZERO_OK) return s;
+    *applied = 0;
+    if (L->padded == 0) return ZERO_OK;
+    if (!reduced || !nonfinite) return ZERO_ERR_INVALID;
+    if (!aligned16(reduced)) return ZERO_ERR_ALIGN;
+    cudaStream_t st = (cudaStream_t)stream;
+    const size_t nb = L->bucket_lo.size();
+    std::vector<int32_t> counts(nb, 0);
+    cudaError_t e = cudaMemsetAsync(nonfinite, 0, nb * sizeof(int32_t), st);
+    if (e == cudaSuccess) e = zero::launch_reduce_scatter(*L, all_tiles(L), grads, rank_stride, reduced, nonfinite, st);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(counts.data(), nonfinite, nb * sizeof(int32_t), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return ZERO_ERR_CUDA;
+    int64_t bad = 0;
+    for (int32_t c : counts) bad += c;
+    if (bad == 0) {
+        uint16_t *p16 = L->stage == 3 ? p16_shard : p16_full;
+        e = zero::launch_adamw_range(*L, 0, L->padded, reduced, master, m, v, p16, step_scalars(L->n_ranks, h), st);
+        if (e == cudaSuccess && L->stage == 3) e = zero::launch_copy_range(*L, 0, L->padded, p16_shard, p16_full, st);
+        if (e != cudaSuccess) return ZERO_ERR_CUDA;
+        *applied = 1;
+        sc->step += 1;
+        sc->clean_steps += 1;
+        if (sc->clean_steps == sc->window) {
+            sc->scale *= sc->factor;
+            sc->clean_steps = 0;
+        }
+    } else {
+        const double lowered = sc->scale / sc->factor;
+        sc->scale = lowered > sc->min_scale ? lowered : sc->min_scale;
+        sc->clean_steps = 0;
+        sc->skipped += 1;
+    }
+    return ZERO_OK;
 }
 
 extern "C" zero_status zero_step_host(const zero_layout *L, const uint16_t *grads_host, uint16_t *grads_dev,

@@ -22,12 +22,10 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
-#include "internal.h"
+#include "device_common.cuh"
 
 namespace zero {
 namespace {
-
-constexpr int kVec = 8;
 
 // Pipeline shape per rank count, measured on B200 (kernel GB/s of the full step on the
 // flat N=4, GPT-2 N=8, Llama N=8 and ragged N=16 workloads): larger single copies pay,
@@ -110,60 +108,6 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volati
     }
 }
 
-__device__ __forceinline__ float h2f(uint32_t bits16)
-{
-    return __half2float(__ushort_as_half((unsigned short)(bits16 & 0xffffu)));
-}
-
-__device__ __forceinline__ uint32_t f2h(float f)
-{
-    return (uint32_t)__half_as_ushort(__float2half_rn(f));
-}
-
-__device__ __forceinline__ void add8(float (&acc)[8], const uint4 u)
-{
-    acc[0] = __fadd_rn(acc[0], h2f(u.x)); acc[1] = __fadd_rn(acc[1], h2f(u.x >> 16));
-    acc[2] = __fadd_rn(acc[2], h2f(u.y)); acc[3] = __fadd_rn(acc[3], h2f(u.y >> 16));
-    acc[4] = __fadd_rn(acc[4], h2f(u.z)); acc[5] = __fadd_rn(acc[5], h2f(u.z >> 16));
-    acc[6] = __fadd_rn(acc[6], h2f(u.w)); acc[7] = __fadd_rn(acc[7], h2f(u.w >> 16));
-}
-
-__device__ __forceinline__ void adamw_elem(float s, const AdamScalars &c, float &p, float &m, float &v,
-                                           uint32_t &h)
-{
-    const float g = __fmul_rn(s, c.inv_scale);
-    const float pd = __fmul_rn(p, c.decay);
-    m = __fadd_rn(__fmul_rn(m, c.beta1), __fmul_rn(g, c.omb1));
-    v = __fadd_rn(__fmul_rn(v, c.beta2), __fmul_rn(__fmul_rn(g, g), c.omb2));
-    const float denom = __fadd_rn(__fdiv_rn(__fsqrt_rn(v), c.sqrt_bc2), c.eps);
-    p = __fsub_rn(pd, __fmul_rn(c.step_size, __fdiv_rn(m, denom)));
-    h = f2h(p);
-}
-
-__device__ __forceinline__ int ring_rank(int k, int j, int n)
-{
-    const int r = k + j;
-    return r >= n ? r - n : r;
-}
-
-struct TileRange {
-    int64_t a, b;
-    int32_t shard, bucket;
-};
-
-__device__ __forceinline__ TileRange locate_tile(const Seg *__restrict__ segs, int64_t &s, int64_t t)
-{
-    while (__ldg(&segs[s + 1].tile_begin) <= t) ++s;
-    const int64_t lo = __ldg(&segs[s].lo), hi = __ldg(&segs[s].hi);
-    const int64_t cell = lo / kTileElems + (t - __ldg(&segs[s].tile_begin));
-    TileRange r;
-    r.a = cell * kTileElems > lo ? cell * kTileElems : lo;
-    r.b = (cell + 1) * kTileElems < hi ? (cell + 1) * kTileElems : hi;
-    r.shard = __ldg(&segs[s].shard);
-    r.bucket = __ldg(&segs[s].bucket);
-    return r;
-}
-
 struct BulkArgs {
     TileWork w;
     const uint16_t *grads;
@@ -180,7 +124,7 @@ struct BulkArgs {
 
 // Shared memory: [full[S], empty[S] mbarriers][abort flag] ... stage ring (128-B aligned):
 // stage s = N gradient slices of kChunk fp16, then master, m, v slices of kChunk fp32.
-template <int N>
+template <int N, bool kWire>
 __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(BulkArgs A)
 {
     constexpr int kChunk = BulkShape<N>::kChunk;
@@ -266,15 +210,19 @@ __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(Bu
             const unsigned char *base = ring + (size_t)st * kStageBytes;
             for (int64_t vi = ct; vi * kVec < n; vi += 32 * kConsumerWarps) {
                 const int64_t e0 = vi * kVec;
-                float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-                {
-                    const uint4 u = *reinterpret_cast<const uint4 *>(base + e0 * 2);
-                    acc[0] = h2f(u.x); acc[1] = h2f(u.x >> 16); acc[2] = h2f(u.y); acc[3] = h2f(u.y >> 16);
-                    acc[4] = h2f(u.z); acc[5] = h2f(u.z >> 16); acc[6] = h2f(u.w); acc[7] = h2f(u.w >> 16);
-                }
+                float acc[8];
+                if constexpr (kWire) {
+                    uint4 h = *reinterpret_cast<const uint4 *>(base + e0 * 2);
 #pragma unroll
-                for (int j = 1; j < N; ++j)
-                    add8(acc, *reinterpret_cast<const uint4 *>(base + ((size_t)j * kChunk + e0) * 2));
+                    for (int j = 1; j < N; ++j)
+                        h = hadd8(h, *reinterpret_cast<const uint4 *>(base + ((size_t)j * kChunk + e0) * 2));
+                    unpack8(h, acc);
+                } else {
+                    unpack8(*reinterpret_cast<const uint4 *>(base + e0 * 2), acc);
+#pragma unroll
+                    for (int j = 1; j < N; ++j)
+                        add8(acc, *reinterpret_cast<const uint4 *>(base + ((size_t)j * kChunk + e0) * 2));
+                }
                 const float *sp = reinterpret_cast<const float *>(base + (size_t)N * kChunk * 2);
                 float4 p4[2] = {*reinterpret_cast<const float4 *>(sp + e0), *reinterpret_cast<const float4 *>(sp + e0 + 4)};
                 float4 m4[2] = {*reinterpret_cast<const float4 *>(sp + kChunk + e0),
@@ -310,9 +258,16 @@ __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(Bu
         const int64_t n_head = head_end - tr.a, n_tail = tr.b - tail_begin;
         if (ct < n_head + n_tail) {
             const int64_t i = ct < n_head ? tr.a + ct : tail_begin + (ct - n_head);
-            float acc = h2f(A.grads[(int64_t)tr.shard * A.stride + i]);
-            for (int j = 1; j < N; ++j)
-                acc = __fadd_rn(acc, h2f(A.grads[(int64_t)ring_rank(tr.shard, j, N) * A.stride + i]));
+            float acc;
+            if constexpr (kWire) {
+                uint32_t h = A.grads[(int64_t)tr.shard * A.stride + i];
+                for (int j = 1; j < N; ++j) h = hadd1(h, A.grads[(int64_t)ring_rank(tr.shard, j, N) * A.stride + i]);
+                acc = h2f(h);
+            } else {
+                acc = h2f(A.grads[(int64_t)tr.shard * A.stride + i]);
+                for (int j = 1; j < N; ++j)
+                    acc = __fadd_rn(acc, h2f(A.grads[(int64_t)ring_rank(tr.shard, j, N) * A.stride + i]));
+            }
             bad += !isfinite(acc);
             float p = A.master[i], m = A.mom1[i], v = A.mom2[i];
             uint32_t h;
@@ -341,7 +296,7 @@ cudaError_t launch_bulk_n(const zero_layout &L, BulkArgs &a, cudaStream_t st)
     if (stages < 2) return cudaErrorInvalidConfiguration;
     a.stages = stages;
     const size_t smem = ((16 * (size_t)stages + 4 + 127) / 128) * 128 + (size_t)stages * stage_bytes;
-    auto kern = bulk_step_kernel<N>;
+    auto kern = L.wire16 ? bulk_step_kernel<N, true> : bulk_step_kernel<N, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int64_t grid = L.dev.num_sms > 0 ? L.dev.num_sms : 148;

@@ -58,6 +58,7 @@ struct DeviceState {
 
 struct zero_layout {
     int32_t n_ranks = 0, stage = 0;
+    int32_t wire16 = 0;                        // 1: partials travel the ring as fp16
     int64_t psi = 0, shard = 0, padded = 0, pad_align = 1, bucket_elems = 0;
     std::vector<int64_t> tensor_off;
     std::vector<int64_t> bucket_lo, bucket_hi;

@@ -17,110 +17,36 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
-#include "internal.h"
+#include "device_common.cuh"
 
 namespace zero {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kVec = 8;   // elements per 16-byte fp16 vector
-
-__device__ __forceinline__ float h2f(uint32_t bits16)
-{
-    return __half2float(__ushort_as_half((unsigned short)(bits16 & 0xffffu)));
-}
-
-__device__ __forceinline__ uint32_t f2h(float f)
-{
-    return (uint32_t)__half_as_ushort(__float2half_rn(f));
-}
-
-__device__ __forceinline__ void unpack8(const uint4 u, float (&f)[8])
-{
-    f[0] = h2f(u.x); f[1] = h2f(u.x >> 16);
-    f[2] = h2f(u.y); f[3] = h2f(u.y >> 16);
-    f[4] = h2f(u.z); f[5] = h2f(u.z >> 16);
-    f[6] = h2f(u.w); f[7] = h2f(u.w >> 16);
-}
-
-__device__ __forceinline__ void add8(float (&acc)[8], const uint4 u)
-{
-    float f[8];
-    unpack8(u, f);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] = __fadd_rn(acc[e], f[e]);
-}
-
-// One element of the shard update.  Order of operations as documented in zero.h.
-__device__ __forceinline__ void adamw_elem(float s, const AdamScalars &c, float &p, float &m,
-                                           float &v, uint32_t &h)
-{
-    const float g = __fmul_rn(s, c.inv_scale);
-    const float pd = __fmul_rn(p, c.decay);
-    m = __fadd_rn(__fmul_rn(m, c.beta1), __fmul_rn(g, c.omb1));
-    v = __fadd_rn(__fmul_rn(v, c.beta2), __fmul_rn(__fmul_rn(g, g), c.omb2));
-    const float denom = __fadd_rn(__fdiv_rn(__fsqrt_rn(v), c.sqrt_bc2), c.eps);
-    p = __fsub_rn(pd, __fmul_rn(c.step_size, __fdiv_rn(m, denom)));
-    h = f2h(p);
-}
-
-__device__ __forceinline__ int is_nonfinite(float x) { return !isfinite(x); }
-
-// Adds this thread's non-finite count into counts[bucket]: one atomic per warp.
-__device__ __forceinline__ void flush_nonfinite(int32_t *counts, int32_t bucket, int mine)
-{
-    if (counts == nullptr) return;
-    const unsigned full = 0xffffffffu;
-    if (__any_sync(full, mine != 0)) {
-        const int total = __reduce_add_sync(full, mine);
-        if ((threadIdx.x & 31) == 0) atomicAdd(counts + bucket, total);
-    }
-}
-
-struct TileRange {
-    int64_t a, b;      // [a, b): the tile's elements
-    int32_t shard, bucket;
-};
-
-// Locate tile t: advance the segment cursor s (tiles are visited in increasing order
-// by each CTA, so the cursor only moves forward), then clip the tile's cell of the
-// global kTileElems grid to the segment.
-__device__ __forceinline__ TileRange locate_tile(const Seg *__restrict__ segs, int64_t &s, int64_t t)
-{
-    while (__ldg(&segs[s + 1].tile_begin) <= t) ++s;
-    const int64_t lo = __ldg(&segs[s].lo), hi = __ldg(&segs[s].hi);
-    const int64_t cell = lo / kTileElems + (t - __ldg(&segs[s].tile_begin));
-    TileRange r;
-    r.a = cell * kTileElems > lo ? cell * kTileElems : lo;
-    r.b = (cell + 1) * kTileElems < hi ? (cell + 1) * kTileElems : hi;
-    r.shard = __ldg(&segs[s].shard);
-    r.bucket = __ldg(&segs[s].bucket);
-    return r;
-}
-
-// Rank at position j of the ring fold that starts at rank k.
-__device__ __forceinline__ int ring_rank(int k, int j, int n)
-{
-    const int r = k + j;
-    return r >= n ? r - n : r;
-}
 
 // Scalar ring fold of one element (ragged tile edges, runtime-N path).
+template <bool kWire>
 __device__ __forceinline__ float fold_scalar(const uint16_t *__restrict__ grads, int64_t stride,
                                              int k, int n, int64_t i)
 {
-    float acc = h2f(__ldcs(grads + (int64_t)k * stride + i));
-    for (int j = 1; j < n; ++j)
-        acc = __fadd_rn(acc, h2f(__ldcs(grads + (int64_t)ring_rank(k, j, n) * stride + i)));
-    return acc;
+    if constexpr (kWire) {
+        uint32_t h = __ldcs(grads + (int64_t)k * stride + i);
+        for (int j = 1; j < n; ++j) h = hadd1(h, __ldcs(grads + (int64_t)ring_rank(k, j, n) * stride + i));
+        return h2f(h);
+    } else {
+        float acc = h2f(__ldcs(grads + (int64_t)k * stride + i));
+        for (int j = 1; j < n; ++j)
+            acc = __fadd_rn(acc, h2f(__ldcs(grads + (int64_t)ring_rank(k, j, n) * stride + i)));
+        return acc;
+    }
 }
 
 // ---------------------------------------------------------------------------------
 // Tile kernel: ring reduce-scatter of every tile of the launch, then either the
 // fused shard update (kFused) or a store of the fp32 sums.
 //   NT = compile-time rank count (0 = runtime n_ranks), U = vectors per thread whose
-//   loads are in flight together.
-template <int NT, int U, bool kFused>
+//   loads are in flight together, kWire = fp16 wire (partials rounded to fp16 per hop).
+template <int NT, int U, bool kFused, bool kWire>
 __global__ void __launch_bounds__(kThreads)
 tile_kernel(TileWork w, int n_ranks, const uint16_t *__restrict__ grads, int64_t stride,
             float *__restrict__ reduced, float *__restrict__ master, float *__restrict__ mom1,
@@ -154,20 +80,37 @@ tile_kernel(TileWork w, int n_ranks, const uint16_t *__restrict__ grads, int64_t
                 }
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
-                    unpack8(g[u][0], acc[u]);
+                    if constexpr (kWire) {
+                        uint4 h = g[u][0];
 #pragma unroll
-                    for (int j = 1; j < NT; ++j) add8(acc[u], g[u][j]);
+                        for (int j = 1; j < NT; ++j) h = hadd8(h, g[u][j]);
+                        unpack8(h, acc[u]);
+                    } else {
+                        unpack8(g[u][0], acc[u]);
+#pragma unroll
+                        for (int j = 1; j < NT; ++j) add8(acc[u], g[u][j]);
+                    }
                 }
             } else {
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
                     const int64_t q = q0 + (int64_t)u * kThreads * kVec;
                     if (q < vb) {
-                        unpack8(__ldcs(reinterpret_cast<const uint4 *>(grads + (int64_t)k * stride + q)), acc[u]);
+                        const uint4 first = __ldcs(reinterpret_cast<const uint4 *>(grads + (int64_t)k * stride + q));
+                        if constexpr (kWire) {
+                            uint4 h = first;
 #pragma unroll 4
-                        for (int j = 1; j < n; ++j)
-                            add8(acc[u], __ldcs(reinterpret_cast<const uint4 *>(
-                                             grads + (int64_t)ring_rank(k, j, n) * stride + q)));
+                            for (int j = 1; j < n; ++j)
+                                h = hadd8(h, __ldcs(reinterpret_cast<const uint4 *>(
+                                                 grads + (int64_t)ring_rank(k, j, n) * stride + q)));
+                            unpack8(h, acc[u]);
+                        } else {
+                            unpack8(first, acc[u]);
+#pragma unroll 4
+                            for (int j = 1; j < n; ++j)
+                                add8(acc[u], __ldcs(reinterpret_cast<const uint4 *>(
+                                                 grads + (int64_t)ring_rank(k, j, n) * stride + q)));
+                        }
                     }
                 }
             }
@@ -211,7 +154,7 @@ tile_kernel(TileWork w, int n_ranks, const uint16_t *__restrict__ grads, int64_t
         const int64_t n_head = head_end - tr.a, n_tail = tr.b - tail_begin;
         if (threadIdx.x < n_head + n_tail) {
             const int64_t i = threadIdx.x < n_head ? tr.a + threadIdx.x : tail_begin + (threadIdx.x - n_head);
-            const float acc = fold_scalar(grads, stride, k, n, i);
+            const float acc = fold_scalar<kWire>(grads, stride, k, n, i);
             bad += is_nonfinite(acc);
             if constexpr (kFused) {
                 float p = master[i], m = mom1[i], v = mom2[i];
@@ -356,7 +299,7 @@ cudaError_t launch_tiles(const zero_layout &L, const TileWork &w, const uint16_t
                          float *reduced, float *master, float *m, float *v, uint16_t *p16,
                          const AdamScalars &c, int32_t *nonfinite, cudaStream_t st)
 {
-    auto kern = tile_kernel<NT, U, kFused>;
+    auto kern = L.wire16 ? tile_kernel<NT, U, kFused, true> : tile_kernel<NT, U, kFused, false>;
     const int grid = grid_for(kern, w.n_tiles, L.dev.num_sms);
     kern<<<grid, kThreads, 0, st>>>(w, L.n_ranks, grads, stride, reduced, master, m, v, p16, c, nonfinite);
     return cudaGetLastError();

@@ -27,6 +27,7 @@ extern "C" zero_status zero_layout_create(const zero_layout_desc *d, zero_layout
     if (!d || !out) return ZERO_ERR_INVALID;
     *out = nullptr;
     if (d->n_ranks < 1 || d->n_ranks > 4096 || d->stage < 0 || d->stage > 3 ||
+        d->wire_fp16 < 0 || d->wire_fp16 > 1 ||
         d->n_tensors < 0 || (d->n_tensors > 0 && !d->tensor_numel) || d->pad_align < 1 ||
         d->pad_align > (int64_t(1) << 30) || d->n_units < 0 ||
         (d->n_units > 0 && !d->unit_first_tensor))
@@ -37,6 +38,7 @@ extern "C" zero_status zero_layout_create(const zero_layout_desc *d, zero_layout
     try {
         L->n_ranks = d->n_ranks;
         L->stage = d->stage;
+        L->wire16 = d->wire_fp16;
         L->pad_align = d->pad_align;
         L->bucket_elems = d->bucket_elems;
 
