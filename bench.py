@@ -48,6 +48,14 @@ def parse():
     ap.add_argument("--ref-seconds", type=float, default=120.0,
                     help="--impl reference: oracle time budget of the whole run")
     ap.add_argument("--kernel", type=int, default=0, help="fused kernel: 0 auto, 1 register, 2 bulk")
+    ap.add_argument("--wire-fp16", action="store_true",
+                    help="partial sums travel the ring as fp16 (its own line; not the headline)")
+    ap.add_argument("--dynamic", action="store_true",
+                    help="time zero_step_dynamic (reduce-scatter, overflow check, update) instead of the fused step")
+    ap.add_argument("--zero3-passes", action="store_true",
+                    help="time ZeRO-3's per-layer forward and backward gathers with 1-3 prefetch slots "
+                         "against a simulated layer compute (its own JSON line)")
+    ap.add_argument("--tokens", type=int, default=2048, help="--zero3-passes: tokens per rank")
     ap.add_argument("--overlap", action="store_true",
                     help="measure the bucket-pipelined step behind a simulated backward pass "
                          "(its own JSON line; not the headline)")
@@ -179,6 +187,15 @@ def workload_config(wl, world):
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU (ranks simulated in HBM)"}
 
 
+def variant_config(a, wl, world):
+    c = workload_config(wl, world)
+    if a.wire_fp16:
+        c["ring_partials"] = "fp16 wire"
+    if a.dynamic:
+        c["step"] = "zero_step_dynamic"
+    return c
+
+
 # ---------------------------------------------------------------- CPU oracle sample
 
 def oracle_sample_run(wl, psi_s, steps=1):
@@ -260,7 +277,8 @@ def run_ours(a, wl):
             dist.barrier(device_ids=[local])
         torch.cuda.synchronize()
 
-    lay = zs.Layout(list(wl.tensors), wl.n_ranks, wl.stage, wl.bucket_elems, wl.pad_align, list(wl.units))
+    lay = zs.Layout(list(wl.tensors), wl.n_ranks, wl.stage, wl.bucket_elems, wl.pad_align, list(wl.units),
+                    wire_fp16=a.wire_fp16)
     lay.to_device()
     if a.kernel:
         lay.set_impl(a.kernel)
@@ -282,10 +300,27 @@ def run_ours(a, wl):
     def hp(t):
         return zs.AdamW(wl.lr, wl.beta1, wl.beta2, wl.eps, wl.weight_decay, wl.loss_scale, t)
 
+    if a.dynamic:
+        # the scale the gradients carry never overflows here, so every step applies; the
+        # timed work is the reduce-scatter pass, the overflow check (a host round trip)
+        # and the update pass
+        reduced = torch.empty(P, dtype=torch.float32, device="cuda")
+        scaler = zs.LossScaler(wl.loss_scale, window=1 << 40)
+
+        def one_step(t, events=None):
+            if events:
+                events["update_begin"].record()
+            zs.step_dynamic(lay, g, reduced, master, m, v, p16_shard, p16_full, hp(t), scaler, nonfinite)
+            if events:
+                events["update_end"].record()
+    else:
+        def one_step(t, events=None):
+            zs.step(lay, g, master, m, v, p16_shard, p16_full, hp(t), nonfinite=nonfinite, events=events)
+
     t = 0
     for _ in range(a.warmup):
         t += 1
-        zs.step(lay, g, master, m, v, p16_shard, p16_full, hp(t), nonfinite=nonfinite)
+        one_step(t)
     zs.get_error(lay)
 
     K = a.steps
@@ -300,7 +335,7 @@ def run_ours(a, wl):
     start.record()
     for i in range(K):
         t += 1
-        zs.step(lay, g, master, m, v, p16_shard, p16_full, hp(t), nonfinite=nonfinite, events=ev[i])
+        one_step(t, ev[i])
     end.record()
     barrier()
     if sampler:
@@ -317,7 +352,7 @@ def run_ours(a, wl):
     # end to end through the host-buffer entry point: gradients from pinned host memory
     # in, fp16 parameters to pinned host memory out, every step
     e2e = None
-    if a.e2e_steps > 0:
+    if a.e2e_steps > 0 and not a.dynamic:
         del g
         torch.cuda.empty_cache()
         g_host = torch.empty((N, P), dtype=torch.int16).pin_memory()
@@ -347,15 +382,21 @@ def run_ours(a, wl):
 
     impl_name = {0: "bulk-copy pipeline (bulk_step_kernel, automatic choice)", 1: "register streaming (tile_kernel)",
                  2: "bulk-copy pipeline (bulk_step_kernel)"}[a.kernel]
+    if a.wire_fp16:
+        impl_name += ", fp16 wire"
+    if a.dynamic:
+        impl_name = "dynamic loss scaling: reduce-scatter + overflow check + update (two passes)"
     peak, peak_kind = hbm_peak()
     fused_bytes = fused_bytes_per_param(wl) * P
+    if a.dynamic:
+        fused_bytes = (2 * wl.n_ranks + 4 + 4 + 24 + 2) * P     # reduce pass + update pass
     achieved = fused_bytes / (upd_ms / 1e3) / 1e9
     traffic_pp = profiled_traffic(wl.name)
     step_bytes = ideal_bytes_per_param(wl) * P
     out = {
         "metric": METRIC, "value": throughput(psi, world, ms), "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": workload_config(wl, world),
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": variant_config(a, wl, world),
         "hbm": {"achieved_gbs_step": step_bytes / (ms / 1e3) / 1e9, "ideal_bytes_per_param": ideal_bytes_per_param(wl),
                 "frac_of_measured_peak": step_bytes / (ms / 1e3) / 1e9 / peak,
                 "frac_of_nominal_8tbs": step_bytes / (ms / 1e3) / 1e9 / NOMINAL_HBM_GBS},
@@ -464,6 +505,109 @@ def _overlap_reps(a, wl, lay, g, master, m, v, p16_shard, p16_full, backward, pr
     return t
 
 
+def run_zero3_passes(a, wl):
+    """ZeRO-3's gather passes over the Llama-shaped list: each layer's parameters are
+    gathered (zero_gather_unit) into one of n_slots unit-sized buffers and the layer's
+    matrices are then used by a simulated compute: one GEMM per matrix with T tokens in the
+    forward pass, two (input and weight gradients) in the backward pass (cuBLAS, standing
+    in for the model).  Reported: each pass with 1, 2 and 3 slots (1 = no prefetch), the
+    compute alone (parameters already in place) and the gathers alone."""
+    import torch
+    import zero_sharded_optimizer_ring_b200 as zs
+    from zero_sharded_optimizer_ring_b200.schedule import zero3_pass
+    from seeded_inputs.workloads import llama_tensors
+
+    torch.cuda.set_device(dist_env()[1])
+    d, ffn, vocab, layers = 3072, 8192, 32000, 26
+    tensors, units = llama_tensors(vocab, d, ffn, layers)
+    if tuple(tensors) != tuple(wl.tensors):
+        raise SystemExit("--zero3-passes needs the Llama-shaped workload")
+    lay = zs.Layout(list(tensors), wl.n_ranks, 3, wl.bucket_elems, wl.pad_align, list(units)).to_device()
+    P = lay.padded
+    shard = (torch.randn(P, device="cuda", dtype=torch.float16) * 0.02).view(torch.int16)
+    _, _, _, u = lay.tables()
+    width = int(max(hi - lo for lo, hi in u))
+    # matrices of a layer unit: (offset in the unit, rows, cols); norms carry no GEMM
+    layer_mats, off = [], d
+    for rows, cols in [(d, d)] * 4:
+        layer_mats.append((off, rows, cols))
+        off += rows * cols
+    off += d
+    for rows, cols in [(ffn, d), (ffn, d), (d, ffn)]:
+        layer_mats.append((off, rows, cols))
+        off += rows * cols
+    T = a.tokens
+    x = {d: torch.randn(T, d, device="cuda", dtype=torch.float16),
+         ffn: torch.randn(T, ffn, device="cuda", dtype=torch.float16)}
+    gy = {d: torch.randn(T, d, device="cuda", dtype=torch.float16),
+          ffn: torch.randn(T, ffn, device="cuda", dtype=torch.float16)}
+
+    def mats(unit, buf):
+        if unit == 0 or unit == lay.n_units - 1:
+            return []                                  # embedding lookup / final norm: no GEMM
+        w = buf.view(torch.float16)
+        return [w[o:o + r * c].view(r, c) for o, r, c in layer_mats]
+
+    def fwd(unit, buf):
+        for W in mats(unit, buf):
+            torch.matmul(x[W.shape[1]], W.t())
+
+    def bwd(unit, buf):
+        for W in mats(unit, buf):
+            torch.matmul(gy[W.shape[0]], W)            # input gradient
+            torch.matmul(gy[W.shape[0]].t(), x[W.shape[1]])   # weight gradient
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    gs, cs = torch.cuda.Stream(), torch.cuda.Stream()
+    slots = [torch.empty(width, dtype=torch.int16, device="cuda") for _ in range(3)]
+    full = torch.empty(P, dtype=torch.int16, device="cuda")
+    zs.allgather(lay, -1, shard, full)
+    torch.cuda.synchronize()
+    order_f = list(range(lay.n_units))
+    order_b = order_f[::-1]
+
+    def timed(fn):
+        best = None
+        for rep in range(a.warmup + 3):
+            torch.cuda.synchronize()
+            s0, e0 = ev(), ev()
+            s0.record(gs)
+            cs.wait_event(s0)
+            fn()
+            e0.record(cs)
+            torch.cuda.synchronize()
+            if rep >= a.warmup:
+                t = s0.elapsed_time(e0)
+                best = t if best is None else min(best, t)
+        return best
+
+    def compute_only(work):
+        def run():
+            with torch.cuda.stream(cs):
+                for k in order_f:
+                    lo, hi = int(u[k][0]), int(u[k][1])
+                    work(k, full[lo:hi])
+        return run
+
+    def gathers_only():
+        for k in order_f:
+            zs.gather_unit(lay, k, shard, slots[k % 3], stream=gs)
+        cs.wait_stream(gs)
+
+    res = {"gathers_only_ms": timed(gathers_only)}
+    for name, work, order in (("forward", fwd, order_f), ("backward", bwd, order_b)):
+        res[f"{name}_compute_only_ms"] = timed(compute_only(work))
+        for n in (1, 2, 3):
+            res[f"{name}_{n}slot_ms"] = timed(lambda: zero3_pass(lay, shard, slots[:n], order, work, gs, cs))
+        res[f"{name}_exposed_gather_1slot_ms"] = res[f"{name}_1slot_ms"] - res[f"{name}_compute_only_ms"]
+        res[f"{name}_exposed_gather_2slot_ms"] = res[f"{name}_2slot_ms"] - res[f"{name}_compute_only_ms"]
+    gather_bytes = 4 * P
+    print(json.dumps({"metric": "ZeRO-3 per-layer gather passes with prefetch", "workload": wl.name,
+                      "units": lay.n_units, "tokens": T, "gather_bytes_per_pass": gather_bytes,
+                      "gather_gbs": gather_bytes / (res["gathers_only_ms"] / 1e3) / 1e9,
+                      **{k: round(v, 4) for k, v in res.items()}}), flush=True)
+
+
 def main():
     a = parse()
     from seeded_inputs.workloads import full_workloads
@@ -476,6 +620,8 @@ def main():
         run_reference(a, wl)
     elif a.overlap:
         run_overlap(a, wl)
+    elif a.zero3_passes:
+        run_zero3_passes(a, wl)
     else:
         run_ours(a, wl)
 

@@ -178,6 +178,17 @@ zero_status zero_adamw_shard_step(const zero_layout *layout, int32_t shard, cons
 zero_status zero_allgather(const zero_layout *layout, int64_t unit, const uint16_t *p16_shard,
                            uint16_t *p16_full, void *stream);
 
+/* ZeRO-3's per-layer gather into a buffer of its own (P1 ZeRO-3: before a layer's
+ * forward, and again before its backward, the layer's parameters are gathered from the
+ * ranks that hold them, and released once the layer is done; P2 section 2.5).
+ * dst[j] = p16_shard[lo + j] for j < hi - lo, where [lo, hi) is unit `unit`'s range:
+ * dst receives the unit's full fp16 parameters contiguously, so a caller can keep only
+ * a few layers materialised at a time (a ring of unit-sized buffers, the next layer's
+ * gather overlapping the current layer's compute).  dst: device, 16-byte aligned,
+ * >= hi - lo elements. */
+zero_status zero_gather_unit(const zero_layout *layout, int64_t unit, const uint16_t *p16_shard,
+                             uint16_t *dst, void *stream);
+
 /* One whole optimizer step of the layout's stage: the reduce-scatter of every bucket
  * fused with the shard update, each gradient and state byte crossing HBM once; the
  * reduced sums stay in registers.  Stages 0-2 write the fp16 parameters straight into

@@ -34,7 +34,8 @@ def test_one_wire_hop_is_the_rounded_fp16_sum():
     red = _ring(a, True, shard=a.shape[1])                          # one shard: fold from rank 0
     with np.errstate(over="ignore"):
         want = (a[0].astype(np.float64) + a[1].astype(np.float64)).astype(np.float16)
-    assert np.array_equal(red.astype(np.float16).view(np.uint16), want.view(np.uint16))
+        got = red.astype(np.float16)
+    assert np.array_equal(got.view(np.uint16), want.view(np.uint16))
 
 
 def test_wire_rounds_at_every_hop():

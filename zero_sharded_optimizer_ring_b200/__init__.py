@@ -15,7 +15,7 @@ import numpy as np
 
 from . import _abi
 
-__all__ = ["ZeroError", "Layout", "AdamW", "reduce_scatter", "adamw_shard_step", "allgather",
+__all__ = ["ZeroError", "Layout", "AdamW", "reduce_scatter", "adamw_shard_step", "allgather", "gather_unit",
            "step", "step_bucket", "step_overlapped", "step_dynamic", "LossScaler", "step_host",
            "step_noalloc", "get_error", "IMPL_AUTO", "IMPL_REGISTER", "IMPL_BULK"]
 
@@ -160,6 +160,12 @@ def adamw_shard_step(layout, shard, reduced, master, m, v, p16_out, hp, stream=N
 def allgather(layout, unit, p16_shard, p16_full, stream=None):
     _check(_abi.lib().zero_allgather(layout.handle, int(unit), _ptr(p16_shard), _ptr(p16_full),
                                      _stream(stream)), "zero_allgather")
+
+
+def gather_unit(layout, unit, p16_shard, dst, stream=None):
+    """Unit `unit`'s fp16 parameters, contiguous, into dst (zero_gather_unit)."""
+    _check(_abi.lib().zero_gather_unit(layout.handle, int(unit), _ptr(p16_shard), _ptr(dst), _stream(stream)),
+           "zero_gather_unit")
 
 
 def step(layout, grads, master, m, v, p16_shard, p16_full, hp, nonfinite=None, events=None,

@@ -59,6 +59,7 @@ SIGNATURES = {
     "zero_reduce_scatter": (_i32, [_vp, _i64, _vp, _i64, _vp, _vp, _vp]),
     "zero_adamw_shard_step": (_i32, [_vp, _i32, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(AdamWHparams), _vp]),
     "zero_allgather": (_i32, [_vp, _i64, _vp, _vp, _vp]),
+    "zero_gather_unit": (_i32, [_vp, _i64, _vp, _vp, _vp]),
     "zero_step": (_i32, [_vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(AdamWHparams), _vp,
                          ctypes.POINTER(StepEvents), _vp]),
     "zero_step_bucket": (_i32, [_vp, _i64, _vp, _i64, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(AdamWHparams),

@@ -255,6 +255,18 @@ extern "C" zero_status zero_allgather(const zero_layout *L, int64_t unit, const 
     return cuda_status(zero::launch_copy_range(*L, lo, hi, p16_shard, p16_full, (cudaStream_t)stream));
 }
 
+extern "C" zero_status zero_gather_unit(const zero_layout *L, int64_t unit, const uint16_t *p16_shard,
+                                        uint16_t *dst, void *stream)
+{
+    zero_status s = check_device(L);
+    if (s != ZERO_OK) return s;
+    if (unit < 0 || unit >= (int64_t)L->unit_lo.size() || !p16_shard || !dst) return ZERO_ERR_INVALID;
+    if (!aligned16(p16_shard) || !aligned16(dst)) return ZERO_ERR_ALIGN;
+    const int64_t lo = L->unit_lo[(size_t)unit];
+    return cuda_status(zero::launch_gather_unit(p16_shard, lo, L->unit_hi[(size_t)unit] - lo, dst,
+                                                (cudaStream_t)stream));
+}
+
 namespace {
 
 zero_status check_step(const zero_layout *L, const uint16_t *grads, int64_t rank_stride, float *master,

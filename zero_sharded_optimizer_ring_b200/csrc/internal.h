@@ -81,6 +81,7 @@ cudaError_t launch_adamw_range(const zero_layout &L, int64_t lo, int64_t hi, con
                                const AdamScalars &c, cudaStream_t s);
 cudaError_t launch_copy_range(const zero_layout &L, int64_t lo, int64_t hi, const uint16_t *src,
                               uint16_t *dst, cudaStream_t s);
+cudaError_t launch_gather_unit(const uint16_t *src, int64_t lo, int64_t n, uint16_t *dst, cudaStream_t s);
 cudaError_t launch_fused_step(const zero_layout &L, const TileWork &w, const uint16_t *grads,
                               int64_t stride, float *master, float *m, float *v, uint16_t *p16,
                               const AdamScalars &c, int32_t *nonfinite, cudaStream_t s);

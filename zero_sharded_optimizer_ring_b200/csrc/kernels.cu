@@ -254,6 +254,37 @@ copy_range_kernel(int64_t lo, int64_t hi, const uint16_t *__restrict__ src, uint
     }
 }
 
+// Gather of one unit into a buffer of its own: dst[j] = src[lo + j], j < n.  With lo a
+// multiple of 8 both sides are 16-byte aligned and each thread moves 4 vectors; otherwise
+// each thread moves 8 scalars (still coalesced).  A grid of short blocks, as for the copy.
+__global__ void __launch_bounds__(kThreads)
+gather_unit_kernel(const uint16_t *__restrict__ src, int64_t lo, int64_t n, uint16_t *__restrict__ dst)
+{
+    if ((lo & 7) == 0) {
+        const uint16_t *s = src + lo;
+        const int64_t nv = n / kVec;
+        const int64_t base = (int64_t)blockIdx.x * kThreads * kCopyUnroll;
+        uint4 x[kCopyUnroll];
+#pragma unroll
+        for (int u = 0; u < kCopyUnroll; ++u) {
+            const int64_t q = base + (int64_t)u * kThreads + threadIdx.x;
+            if (q < nv) x[u] = *reinterpret_cast<const uint4 *>(s + q * kVec);
+        }
+#pragma unroll
+        for (int u = 0; u < kCopyUnroll; ++u) {
+            const int64_t q = base + (int64_t)u * kThreads + threadIdx.x;
+            if (q < nv) *reinterpret_cast<uint4 *>(dst + q * kVec) = x[u];
+        }
+        if (blockIdx.x == 0 && threadIdx.x < n - nv * kVec) dst[nv * kVec + threadIdx.x] = s[nv * kVec + threadIdx.x];
+    } else {
+        const int64_t base = (int64_t)blockIdx.x * kThreads * kCopyUnroll * kVec;
+        for (int u = 0; u < kCopyUnroll * kVec; ++u) {
+            const int64_t j = base + (int64_t)u * kThreads + threadIdx.x;
+            if (j < n) dst[j] = src[lo + j];
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------------
 // Tile index: one warp scans the segments' tile counts (exclusive prefix sum with
 // __shfl_up_sync, 32 segments per pass, carried across passes).  Row n_seg receives
@@ -330,6 +361,14 @@ cudaError_t dispatch_tiles(const zero_layout &L, const TileWork &w, const uint16
 }
 
 }  // namespace
+
+cudaError_t launch_gather_unit(const uint16_t *src, int64_t lo, int64_t n, uint16_t *dst, cudaStream_t s)
+{
+    if (n <= 0) return cudaSuccess;
+    const int64_t per_block = (int64_t)kThreads * kCopyUnroll * kVec;
+    gather_unit_kernel<<<(unsigned)((n + per_block - 1) / per_block), kThreads, 0, s>>>(src, lo, n, dst);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_tile_index(Seg *segs, int64_t n_seg, cudaStream_t s)
 {
