@@ -32,8 +32,10 @@ UNIT = "params/s"
 DEFAULT_WORKLOAD = "flat1p3b_n4_zero1"
 FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "bulk_step_flat1p3b_n4.md")
-KERNEL_SOURCE = os.path.join(ROOT, "zero_sharded_optimizer_ring_b200", "csrc", "bulk_step.cu")
+PROFILE_DIR = os.path.join(ROOT, "profiles")
+# the sources the fused bulk kernel is compiled from: a profile taken on other sources is stale
+KERNEL_SOURCES = [os.path.join(ROOT, "zero_sharded_optimizer_ring_b200", "csrc", f)
+                  for f in ("bulk_step.cu", "device_common.cuh", "internal.h")]
 
 
 def parse():
@@ -105,17 +107,27 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
 def profiled_traffic(workload):
-    """dram bytes per parameter of the fused kernel from the committed ncu summary, if
-    it was taken on this workload with the current kernel source; else None."""
+    """DRAM bytes per parameter of the fused kernel from a committed ncu summary
+    (profiles/*.md) taken for this workload on the current kernel sources; else None."""
     try:
-        text = open(PROFILE_SUMMARY).read()
-        sha = hashlib.sha256(open(KERNEL_SOURCE, "rb").read()).hexdigest()[:16]
-        m_sha = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
-        m_wl = re.search(r"workload:\s*(\S+)", text)
-        m_tr = re.search(r"dram_bytes_per_param:\s*([0-9.]+)", text)
-        if m_sha and m_tr and m_wl and m_sha.group(1) == sha and m_wl.group(1) == workload:
-            return float(m_tr.group(1))
+        sha = kernel_source_hash()
+        for name in sorted(os.listdir(PROFILE_DIR)):
+            if not name.endswith(".md"):
+                continue
+            text = open(os.path.join(PROFILE_DIR, name)).read()
+            m_sha = re.search(r"kernel_sources_sha256_16:\s*([0-9a-f]+)", text)
+            m_wl = re.search(r"workload:\s*(\S+)", text)
+            m_tr = re.search(r"dram_bytes_per_param:\s*([0-9.]+)", text)
+            if m_sha and m_tr and m_wl and m_sha.group(1) == sha and m_wl.group(1) == workload:
+                return float(m_tr.group(1))
     except Exception:
         pass
     return None
@@ -595,12 +607,16 @@ def run_zero3_passes(a, wl):
         cs.wait_stream(gs)
 
     res = {"gathers_only_ms": timed(gathers_only)}
+    gs_hi = torch.cuda.Stream(priority=torch.cuda.Stream.priority_range()[1])
     for name, work, order in (("forward", fwd, order_f), ("backward", bwd, order_b)):
         res[f"{name}_compute_only_ms"] = timed(compute_only(work))
         for n in (1, 2, 3):
             res[f"{name}_{n}slot_ms"] = timed(lambda: zero3_pass(lay, shard, slots[:n], order, work, gs, cs))
-        res[f"{name}_exposed_gather_1slot_ms"] = res[f"{name}_1slot_ms"] - res[f"{name}_compute_only_ms"]
-        res[f"{name}_exposed_gather_2slot_ms"] = res[f"{name}_2slot_ms"] - res[f"{name}_compute_only_ms"]
+        res[f"{name}_2slot_highprio_ms"] = timed(lambda: zero3_pass(lay, shard, slots[:2], order, work, gs_hi, cs))
+        for n in (1, 2):
+            res[f"{name}_exposed_gather_{n}slot_ms"] = res[f"{name}_{n}slot_ms"] - res[f"{name}_compute_only_ms"]
+        res[f"{name}_exposed_gather_2slot_highprio_ms"] = (res[f"{name}_2slot_highprio_ms"] -
+                                                           res[f"{name}_compute_only_ms"])
     gather_bytes = 4 * P
     print(json.dumps({"metric": "ZeRO-3 per-layer gather passes with prefetch", "workload": wl.name,
                       "units": lay.n_units, "tokens": T, "gather_bytes_per_pass": gather_bytes,
