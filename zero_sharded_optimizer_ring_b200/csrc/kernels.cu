@@ -395,9 +395,11 @@ cudaError_t launch_adamw_range(const zero_layout &L, int64_t lo, int64_t hi, con
                                const AdamScalars &c, cudaStream_t s)
 {
     if (hi <= lo) return cudaSuccess;
-    const int grid = grid_for(adamw_range_kernel, (hi - lo + kThreads * kVec - 1) / (kThreads * kVec),
-                              L.dev.num_sms);
-    adamw_range_kernel<<<grid, kThreads, 0, s>>>(lo, hi, reduced, master, m, v, p16, c);
+    // one vector per thread: a grid of short blocks keeps the blocks in flight on a compact
+    // window of the buffers (see copy_range_kernel)
+    const int64_t blocks = (hi - lo + kThreads * kVec - 1) / (kThreads * kVec);
+    (void)L;
+    adamw_range_kernel<<<(unsigned)(blocks > 0 ? blocks : 1), kThreads, 0, s>>>(lo, hi, reduced, master, m, v, p16, c);
     return cudaGetLastError();
 }
 
