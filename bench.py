@@ -108,9 +108,14 @@ def hbm_peak():
 
 
 def kernel_source_hash():
+    """Hash of the kernel's sources with comments and blank space removed, so that a
+    profile stays valid across comment-only edits."""
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
-        h.update(open(f, "rb").read())
+        text = open(f).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

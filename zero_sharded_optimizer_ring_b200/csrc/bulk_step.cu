@@ -6,8 +6,8 @@
 //
 //   warp 0, lane 0 (producer): for each chunk (2048 or 4096 elements) of its tiles, waits for a free
 //     stage of a shared-memory ring, posts the stage's byte count on the stage's "full"
-//     mbarrier and issues one cp.async.bulk (global -> shared, no tensor map, no
-//     multicast) per gradient slice (ranks in ring order) and per state array;
+//     mbarrier and issues one plain cp.async.bulk (global -> this CTA's shared memory, no
+//     tensor map) per gradient slice (ranks in ring order) and per state array;
 //   warps 1..8 or 1..16 (consumers): wait for the stage to fill, fold / update from shared memory
 //     (16-byte vectors, conflict-free for the gradients), store results with 16-byte
 //     streaming stores, and release the stage on its "empty" mbarrier.
