@@ -284,8 +284,49 @@ zero_status zero_step_dynamic(const zero_layout *layout, const uint16_t *grads, 
                               uint16_t *p16_full, const zero_adamw_hparams *hp, zero_loss_scaler *scaler,
                               int32_t *nonfinite, int32_t *applied, void *stream);
 
+/* ---- one GPU per rank (the step over NVLink peers) --------------------------------- */
+
+/* zero_step with each rank's gradients in a buffer of its own: rank r's gradient of flat
+ * element i is rank_grads[r][i] (host array of N device pointers, each 16-byte aligned,
+ * each >= P elements; they may point into this GPU's memory or into other GPUs' memory
+ * mapped with zero_ipc_open).  Uses the bulk-copy pipeline; N <= 16.  Same result as
+ * zero_step on the same values. */
+zero_status zero_step_ranks(const zero_layout *layout, const uint16_t *const *rank_grads, float *master,
+                            float *m, float *v, uint16_t *p16_shard, uint16_t *p16_full,
+                            const zero_adamw_hparams *hp, int32_t *nonfinite, void *stream);
+
+/* The fused reduce-scatter + update of shard `shard` alone, with that shard's optimizer
+ * state only: what the GPU owning shard k runs when every rank sits on its own GPU (P1
+ * Deepspeed ZeRO-1: each GPU updates the optimizer state of its own part).  The shard's
+ * N gradient slices are read from rank_grads (peers' buffers mapped with zero_ipc_open,
+ * this GPU's own for its rank) and folded in the ring order k, k+1, ..., k+N-1, so the
+ * result equals the single-GPU simulation bit for bit.
+ *   master_k, m_k, v_k: fp32 [S], element i of the flat buffer at [i - kS];
+ *   p16_out: fp16, full [P] (stages 0-2: element i at [i]) or, for stage 3, the shard's
+ *   own [S] (element i at [i - kS]).  Requires S % 8 == 0 and N <= 16.
+ * The caller makes sure the peers' gradients are complete before the call (a host
+ * barrier between ranks): the kernel reads peer memory but never waits on another GPU. */
+zero_status zero_step_shard(const zero_layout *layout, int32_t shard, const uint16_t *const *rank_grads,
+                            float *master_k, float *m_k, float *v_k, uint16_t *p16_out,
+                            const zero_adamw_hparams *hp, int32_t *nonfinite, void *stream);
+
+/* dst[i] = src[i] for i in shard `shard`'s range [kS, (k+1)S): the all-gather of the
+ * fp16 parameters when src is the owning GPU's full buffer, mapped with zero_ipc_open
+ * (P1 ZeRO-1 broadcast step).  Both flat-indexed fp16 [P], 16-byte aligned. */
+zero_status zero_copy_shard(const zero_layout *layout, int32_t shard, const uint16_t *src, uint16_t *dst,
+                            void *stream);
+
+/* CUDA IPC.  zero_ipc_get_handle exports the allocation dev_ptr lies in as a 64-byte
+ * handle plus dev_ptr's byte offset within it (pointers from a caching allocator lie
+ * inside larger allocations).  zero_ipc_open maps such a handle into this process (peer
+ * access enabled) and returns the address of the same byte; zero_ipc_close unmaps it,
+ * given the same offset. */
+zero_status zero_ipc_get_handle(const void *dev_ptr, void *handle_out, int64_t *offset_out);
+zero_status zero_ipc_open(const void *handle, int64_t offset, void **dev_ptr_out);
+zero_status zero_ipc_close(void *dev_ptr, int64_t offset);
+
 /* Select the fused kernel's implementation: 0 = automatic (the bulk-copy pipeline for
- * N in 1..8 and 16, register streaming otherwise), 1 = register streaming (vectorised
+ * N in 1..16, register streaming above), 1 = register streaming (vectorised
  * 16-byte loads held in registers), 2 = bulk-copy pipeline (cp.async.bulk into a
  * shared-memory ring, warp-specialised).  Results are bit-identical. */
 zero_status zero_set_impl(zero_layout *layout, int32_t impl);

@@ -1,0 +1,155 @@
+"""One buffer per rank, one shard at a time, and the multi-process step over CUDA IPC.
+
+- zero_step_ranks on separately allocated per-rank gradient buffers equals zero_step;
+- zero_step_shard run for every shard, with shard-local optimizer state, equals zero_step;
+- zero_copy_shard copies exactly the shard's range;
+- two processes sharing this GPU, each holding one rank's gradients and one shard's
+  state, run the multi-GPU step (CUDA IPC mappings, host barriers over gloo; no kernel
+  waits on the other process) and end bit-identical to the oracle.
+"""
+import datetime
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch.multiprocessing as mp
+
+import oracle
+import seeded_inputs as si
+from seeded_inputs.workloads import Workload, reduced_workloads
+import zero_sharded_optimizer_ring_b200 as zs
+import support as S
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _hp(wl, t):
+    return zs.AdamW(wl.lr, wl.beta1, wl.beta2, wl.eps, wl.weight_decay, wl.loss_scale, t)
+
+
+def _np(t):
+    a = t.cpu().numpy()
+    return a.view(np.uint16) if a.dtype == np.int16 else a
+
+
+def _layout(wl, wire=False):
+    return zs.Layout(list(wl.tensors), wl.n_ranks, wl.stage, wl.bucket_elems, wl.pad_align, list(wl.units),
+                     wire_fp16=wire).to_device()
+
+
+@pytest.mark.parametrize("key", ["flat1p3b_n4_zero1", "gpt2_small_n8_zero2", "ragged2000_n16_zero2",
+                                 "llama3b_n8_zero3"])
+@pytest.mark.parametrize("wire", [False, True])
+def test_step_ranks_and_step_shard_equal_step(key, wire):
+    wl = reduced_workloads()[key]
+    lay = _layout(wl, wire)
+    P, S_, N = lay.padded, lay.shard, wl.n_ranks
+    g, master, m, v = S.device_inputs(wl, P)
+    ref = dict(master=master.clone(), m=m.clone(), v=v.clone(), p16s=torch.zeros(P, dtype=torch.int16, device="cuda"),
+               p16f=torch.zeros(P, dtype=torch.int16, device="cuda"))
+    ranks = [g[r].clone() for r in range(N)]                       # separate allocations
+    a = dict(master=master.clone(), m=m.clone(), v=v.clone(), p16s=torch.zeros_like(ref["p16s"]),
+             p16f=torch.zeros_like(ref["p16f"]))
+    shards = [[x[k * S_:(k + 1) * S_].clone() for x in (master, m, v)] for k in range(N)]
+    p16_sh = torch.zeros(P, dtype=torch.int16, device="cuda")
+    p16_k = [torch.zeros(S_, dtype=torch.int16, device="cuda") for _ in range(N)]
+    for t in (1, 2):
+        zs.step(lay, g, ref["master"], ref["m"], ref["v"], ref["p16s"], ref["p16f"], _hp(wl, t))
+        zs.step_ranks(lay, ranks, a["master"], a["m"], a["v"], a["p16s"], a["p16f"], _hp(wl, t))
+        for k in range(N):
+            out = p16_k[k] if wl.stage == 3 else p16_sh
+            zs.step_shard(lay, k, ranks, *shards[k], out, _hp(wl, t))
+    torch.cuda.synchronize()
+    for name in ("master", "m", "v"):
+        S.assert_bits_equal(_np(a[name]), _np(ref[name]), name)
+        whole = torch.cat([shards[k][("master", "m", "v").index(name)] for k in range(N)])
+        S.assert_bits_equal(_np(whole), _np(ref[name]), name + " by shard")
+    S.assert_bits_equal(_np(a["p16f"]), _np(ref["p16f"]), "p16_full")
+    if wl.stage == 3:
+        S.assert_bits_equal(_np(torch.cat(p16_k)), _np(ref["p16s"]), "p16 by shard")
+    else:
+        S.assert_bits_equal(_np(p16_sh), _np(ref["p16f"]), "p16 by shard")
+
+
+def test_copy_shard_copies_exactly_the_shard():
+    wl = reduced_workloads()["flat1p3b_n4_zero1"]
+    lay = _layout(wl)
+    src = torch.randint(-9999, 9999, (lay.padded,), dtype=torch.int16, device="cuda")
+    for k in range(lay.n_ranks):
+        dst = torch.zeros_like(src)
+        zs.copy_shard(lay, k, src, dst)
+        torch.cuda.synchronize()
+        lo, hi = k * lay.shard, (k + 1) * lay.shard
+        assert torch.equal(dst[lo:hi], src[lo:hi])
+        assert int(torch.count_nonzero(dst[:lo])) == 0 and int(torch.count_nonzero(dst[hi:])) == 0
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _ipc_worker(rank, world, port, wl, steps, out):
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import seeded_inputs as si
+    import zero_sharded_optimizer_ring_b200 as zs
+    from zero_sharded_optimizer_ring_b200.multigpu import RankStep
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(0)
+    lay = zs.Layout(list(wl.tensors), world, wl.stage, wl.bucket_elems, wl.pad_align).to_device()
+    P, S_ = lay.padded, lay.shard
+    g_all = si.fill_grads(world, P, wl.psi, wl.seed, wl.grad_sigma, wl.loss_scale)
+    master = si.fill_f32(P, wl.psi, wl.seed, si.STREAM_MASTER, wl.master_sigma)
+    m = si.fill_f32(P, wl.psi, wl.seed, si.STREAM_M, wl.m_sigma)
+    v = si.fill_f32(P, wl.psi, wl.seed, si.STREAM_V, wl.v_sigma, True)
+    g = torch.from_numpy(g_all[rank].view(np.int16).copy()).cuda()
+    sl = slice(rank * S_, (rank + 1) * S_)
+    mk, m1, v1 = (torch.from_numpy(x[sl].copy()).cuda() for x in (master, m, v))
+    p16 = torch.zeros(P, dtype=torch.int16, device="cuda")
+    torch.cuda.synchronize()
+    rs = RankStep(lay, rank, world, g, mk, m1, v1, p16)
+    for t in range(1, steps + 1):
+        rs.step(zs.AdamW(wl.lr, wl.beta1, wl.beta2, wl.eps, wl.weight_decay, wl.loss_scale, t))
+    rs.close()
+    out.put((rank, mk.cpu().numpy(), m1.cpu().numpy(), v1.cpu().numpy(), p16.cpu().numpy().view(np.uint16)))
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("stage", [1, 2])
+def test_two_process_step_over_ipc_matches_oracle(stage):
+    wl = Workload(name="ipc", description="ipc", tensors=(300_007,), units=(), n_ranks=2, stage=stage,
+                  bucket_elems=50_001, steps=3, loss_scale=1024.0, m_sigma=1e-4, v_sigma=1e-6)
+    olay = S.oracle_layout(wl)
+    g, master, m, v = S.host_inputs(wl, olay.padded)
+    ref = oracle.run_steps(olay, stage, g, master, m, v, S.hyper(wl), wl.steps)
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_ipc_worker, args=(r, 2, port, wl, wl.steps, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    try:
+        res = sorted([q.get(timeout=300) for _ in range(2)], key=lambda x: x[0])
+    finally:
+        for p in procs:
+            p.join(60)
+            if p.exitcode is None:
+                p.kill()
+    assert all(p.exitcode == 0 for p in procs)
+    S_ = olay.shard
+    for rank, mk, m1, v1, p16 in res:
+        sl = slice(rank * S_, (rank + 1) * S_)
+        S.assert_bits_equal(mk, ref.master[sl], f"master shard {rank}")
+        S.assert_bits_equal(m1, ref.m[sl], f"m shard {rank}")
+        S.assert_bits_equal(v1, ref.v[sl], f"v shard {rank}")
+        S.assert_bits_equal(p16, ref.p16_full, f"p16 on rank {rank}")

@@ -1,0 +1,108 @@
+"""The multi-GPU step's protocol on CPU (gloo, 2 and 3 ranks, no GPU): every shard is
+updated exactly once per step by its owner, every rank gathers every other shard from
+its owner, and every read of a peer's buffer happens after the barrier that makes that
+buffer complete."""
+import os
+import socket
+import sys
+import time
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+class FakeLayout:
+    def __init__(self, n, stage=1):
+        self.n_ranks, self.stage = n, stage
+
+
+class RecordingOps:
+    """Stands in for the device: records what would run, and when."""
+
+    def __init__(self, rank):
+        self.rank, self.log = rank, []
+
+    def _rec(self, *what):
+        self.log.append((time.monotonic(), self.rank) + what)
+
+    def export(self, t):
+        return f"{t}@{self.rank}".encode()
+
+    def open(self, handle):
+        self._rec("open", handle.decode())
+        return "mapped:" + handle.decode()
+
+    def close(self, ptr):
+        self._rec("close", ptr)
+
+    def step_shard(self, layout, shard, rank_grads, master_k, m_k, v_k, p16_full, hp, nonfinite):
+        self._rec("update", shard, tuple(rank_grads), hp)
+
+    def copy_shard(self, layout, shard, src, dst):
+        self._rec("gather", shard, src, dst)
+
+    def sync(self):
+        self._rec("barrier")
+
+
+def _worker(rank, world, port, steps, out):
+    import datetime
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from zero_sharded_optimizer_ring_b200.multigpu import RankStep
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    ops = RecordingOps(rank)
+    rs = RankStep(FakeLayout(world), rank, world, "grads", "m0", "m1", "m2", "p16", ops=ops)
+    for t in range(steps):
+        ops._rec("grads_written", t)
+        rs.step(hp=t)
+    rs.close()
+    out.put(ops.log)
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_multigpu_step_protocol(world):
+    steps = 3
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, steps, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    logs = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    ev = sorted(e for log in logs for e in log)
+
+    for t in range(steps):
+        updates = [e for e in ev if e[2] == "update" and e[5] == t]
+        assert sorted((e[1], e[3]) for e in updates) == [(r, r) for r in range(world)]   # owner updates own shard
+        for e in updates:                                   # reads the right buffers
+            assert e[4] == tuple("grads" if r == e[1] else f"mapped:grads@{r}" for r in range(world))
+        written = max(e[0] for e in ev if e[2] == "grads_written" and e[3] == t)
+        assert min(e[0] for e in updates) > written         # nobody reads gradients still being written
+        done = max(e[0] for e in updates)
+        step_gathers = [e for e in ev if e[2] == "gather"][t * world * (world - 1):(t + 1) * world * (world - 1)]
+        assert all(done < e[0] for e in step_gathers)       # nobody reads parameters before their update
+        assert sorted((e[1], e[3]) for e in step_gathers) == \
+            sorted((r, j) for r in range(world) for j in range(world) if j != r)
+        for e in step_gathers:
+            assert e[4] == f"mapped:p16@{e[3]}" and e[5] == "p16"
+        if t + 1 < steps:                                   # next step's gradients after this step's reads
+            nxt = min(e[0] for e in ev if e[2] == "grads_written" and e[3] == t + 1)
+            assert nxt > max(e[0] for e in step_gathers)
+    closes = [e for e in ev if e[2] == "close"]
+    assert len(closes) == world * 2 * (world - 1)

@@ -17,7 +17,8 @@ from . import _abi
 
 __all__ = ["ZeroError", "Layout", "AdamW", "reduce_scatter", "adamw_shard_step", "allgather", "gather_unit",
            "step", "step_bucket", "step_overlapped", "step_dynamic", "LossScaler", "step_host",
-           "step_noalloc", "get_error", "IMPL_AUTO", "IMPL_REGISTER", "IMPL_BULK"]
+           "step_noalloc", "step_ranks", "step_shard", "copy_shard", "ipc_handle", "ipc_open", "ipc_close",
+           "get_error", "IMPL_AUTO", "IMPL_REGISTER", "IMPL_BULK"]
 
 IMPL_AUTO, IMPL_REGISTER, IMPL_BULK = 0, 1, 2
 
@@ -255,6 +256,57 @@ def step_noalloc(layout, grads, master, m, v, p16_shard, p16_full, hp, nonfinite
     _check(_abi.lib().zero_step_noalloc(layout.handle, _ptr(grads), _stride(grads, layout, rank_stride),
                                         _ptr(master), _ptr(m), _ptr(v), _ptr(p16_shard), _ptr(p16_full),
                                         ctypes.byref(h), _ptr(nonfinite), _stream(stream)), "zero_step_noalloc")
+
+
+def _ptr_array(ptrs):
+    arr = (ctypes.c_void_p * max(1, len(ptrs)))()
+    for i, p in enumerate(ptrs):
+        arr[i] = _ptr(p)
+    return arr
+
+
+def step_ranks(layout, rank_grads, master, m, v, p16_shard, p16_full, hp, nonfinite=None, stream=None):
+    """zero_step with rank r's gradients in rank_grads[r] (tensors or device addresses)."""
+    h = hp.c()
+    _check(_abi.lib().zero_step_ranks(layout.handle, _ptr_array(rank_grads), _ptr(master), _ptr(m), _ptr(v),
+                                      _ptr(p16_shard), _ptr(p16_full), ctypes.byref(h), _ptr(nonfinite),
+                                      _stream(stream)), "zero_step_ranks")
+
+
+def step_shard(layout, shard, rank_grads, master_k, m_k, v_k, p16_out, hp, nonfinite=None, stream=None):
+    """The update of one shard with shard-local state (zero_step_shard)."""
+    h = hp.c()
+    _check(_abi.lib().zero_step_shard(layout.handle, int(shard), _ptr_array(rank_grads), _ptr(master_k), _ptr(m_k),
+                                      _ptr(v_k), _ptr(p16_out), ctypes.byref(h), _ptr(nonfinite), _stream(stream)),
+           "zero_step_shard")
+
+
+def copy_shard(layout, shard, src, dst, stream=None):
+    _check(_abi.lib().zero_copy_shard(layout.handle, int(shard), _ptr(src), _ptr(dst), _stream(stream)),
+           "zero_copy_shard")
+
+
+def ipc_handle(tensor_or_ptr):
+    """(64-byte CUDA IPC handle of the allocation holding the pointer, byte offset)."""
+    buf = ctypes.create_string_buffer(64)
+    off = ctypes.c_int64(0)
+    _check(_abi.lib().zero_ipc_get_handle(_ptr(tensor_or_ptr), buf, ctypes.byref(off)), "zero_ipc_get_handle")
+    return buf.raw, off.value
+
+
+def ipc_open(handle):
+    """Map another process's (handle, offset); returns the device address in this process."""
+    raw, off = handle
+    p = ctypes.c_void_p()
+    _check(_abi.lib().zero_ipc_open(ctypes.create_string_buffer(bytes(raw), 64), int(off), ctypes.byref(p)),
+           "zero_ipc_open")
+    return p.value, int(off)
+
+
+def ipc_close(mapped):
+    """Unmap what ipc_open returned."""
+    ptr, off = mapped
+    _check(_abi.lib().zero_ipc_close(ptr, off), "zero_ipc_close")
 
 
 def get_error(layout, stream=None):

@@ -71,6 +71,12 @@ SIGNATURES = {
     "zero_step_host": (_i32, [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp,
                               ctypes.POINTER(AdamWHparams), _vp, _vp]),
     "zero_step_noalloc": (_i32, [_vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(AdamWHparams), _vp, _vp]),
+    "zero_step_ranks": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(AdamWHparams), _vp, _vp]),
+    "zero_step_shard": (_i32, [_vp, _i32, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(AdamWHparams), _vp, _vp]),
+    "zero_copy_shard": (_i32, [_vp, _i32, _vp, _vp, _vp]),
+    "zero_ipc_get_handle": (_i32, [_vp, _vp, ctypes.POINTER(_i64)]),
+    "zero_ipc_open": (_i32, [_vp, _i64, ctypes.POINTER(_vp)]),
+    "zero_ipc_close": (_i32, [_vp, _i64]),
     "zero_set_impl": (_i32, [_vp, _i32]),
     "zero_debug_set_wait": (_i32, [_vp, _i64, _i32]),
     "zero_get_error": (_i32, [_vp, _vp]),

@@ -1,7 +1,9 @@
 // extern "C" entry points: argument checks, the AdamW step scalars, kernel launches.
 #include <math.h>
 #include <stdint.h>
+#include <string.h>
 
+#include <mutex>
 #include <vector>
 
 #include "internal.h"
@@ -106,6 +108,7 @@ void release_device(zero_layout *L)
     if (L->dev.copy_in) cudaStreamDestroy(L->dev.copy_in);
     if (L->dev.copy_out) cudaStreamDestroy(L->dev.copy_out);
     if (L->dev.segs) cudaFree(L->dev.segs);
+    if (L->dev.segs_by_shard) cudaFree(L->dev.segs_by_shard);
     if (L->dev.error) cudaFree(L->dev.error);
     if (cur >= 0 && cur != L->dev.device) cudaSetDevice(cur);
     L->dev = zero::DeviceState();
@@ -159,7 +162,11 @@ extern "C" zero_status zero_layout_to_device(zero_layout *L, void *stream)
     sentinel.tile_begin = -1;
     sentinel.shard = sentinel.bucket = -1;
     rows.push_back(sentinel);
+    std::vector<Seg> rows2(L->segs_by_shard);
+    for (Seg &s : rows2) s.tile_begin = -1;
+    rows2.push_back(sentinel);
     if (cudaMalloc(&d.segs, rows.size() * sizeof(Seg)) != cudaSuccess ||
+        cudaMalloc(&d.segs_by_shard, rows2.size() * sizeof(Seg)) != cudaSuccess ||
         cudaMalloc(&d.error, sizeof(int32_t)) != cudaSuccess) {
         cudaGetLastError();
         release_device(L);
@@ -168,6 +175,9 @@ extern "C" zero_status zero_layout_to_device(zero_layout *L, void *stream)
     cudaError_t e = cudaMemcpyAsync(d.segs, rows.data(), rows.size() * sizeof(Seg), cudaMemcpyHostToDevice, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(d.error, 0, sizeof(int32_t), st);
     if (e == cudaSuccess) e = zero::launch_tile_index(d.segs, (int64_t)L->segs.size(), st);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(d.segs_by_shard, rows2.data(), rows2.size() * sizeof(Seg), cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = zero::launch_tile_index(d.segs_by_shard, (int64_t)L->segs_by_shard.size(), st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&d.copy_in, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&d.copy_out, cudaStreamNonBlocking);
@@ -289,6 +299,14 @@ void record(void *ev, cudaStream_t st)
     if (ev) cudaEventRecord((cudaEvent_t)ev, st);
 }
 
+// Rank r's gradients at grads + r * stride.
+zero::GradSource strided(const zero_layout *L, const uint16_t *grads, int64_t stride)
+{
+    zero::GradSource src = {};
+    for (int r = 0; r < L->n_ranks && r < zero::kMaxBulkRanks; ++r) src.rank[r] = grads + (int64_t)r * stride;
+    return src;
+}
+
 // The fused reduce-scatter + update over the tiles of `w`, in the selected implementation.
 cudaError_t fused(const zero_layout *L, const TileWork &w, const uint16_t *grads, int64_t stride, float *master,
                   float *m, float *v, uint16_t *p16, const AdamScalars &c, int32_t *nonfinite, cudaStream_t st)
@@ -297,8 +315,8 @@ cudaError_t fused(const zero_layout *L, const TileWork &w, const uint16_t *grads
     // 1-3 % faster than register streaming on every measured workload)
     const bool bulk = (L->impl == 2 || L->impl == 0) && zero::bulk_supported(L->n_ranks);
     if (bulk)
-        return zero::launch_bulk_step(*L, w, grads, stride, master, m, v, p16, c, nonfinite, L->dev.wait_limit_ns,
-                                      L->dev.skip_first_fill, st);
+        return zero::launch_bulk_step(*L, w, strided(L, grads, stride), master, m, v, 0, p16, 0, c, nonfinite,
+                                      L->dev.wait_limit_ns, L->dev.skip_first_fill, st);
     return zero::launch_fused_step(*L, w, grads, stride, master, m, v, p16, c, nonfinite, st);
 }
 
@@ -408,6 +426,148 @@ extern "C" zero_status zero_step_dynamic(const zero_layout *L, const uint16_t *g
         sc->skipped += 1;
     }
     return ZERO_OK;
+}
+
+namespace {
+
+TileWork shard_tiles(const zero_layout *L, int64_t k)
+{
+    TileWork w;
+    w.segs = L->dev.segs_by_shard;
+    w.seg_first = L->shard_seg_begin[(size_t)k];
+    const int64_t seg_end = L->shard_seg_begin[(size_t)k + 1];
+    w.tile_first = w.seg_first < (int64_t)L->segs_by_shard.size() ? L->segs_by_shard[(size_t)w.seg_first].tile_begin
+                                                                    : L->n_tiles;
+    const int64_t tile_end =
+        seg_end < (int64_t)L->segs_by_shard.size() ? L->segs_by_shard[(size_t)seg_end].tile_begin : L->n_tiles;
+    w.n_tiles = tile_end - w.tile_first;
+    return w;
+}
+
+zero_status rank_source(const zero_layout *L, const uint16_t *const *rank_grads, zero::GradSource *src)
+{
+    if (!rank_grads) return ZERO_ERR_INVALID;
+    if (L->n_ranks > zero::kMaxBulkRanks) return ZERO_ERR_INVALID;
+    *src = {};
+    for (int r = 0; r < L->n_ranks; ++r) {
+        if (!rank_grads[r]) return ZERO_ERR_INVALID;
+        if (!aligned16(rank_grads[r])) return ZERO_ERR_ALIGN;
+        src->rank[r] = rank_grads[r];
+    }
+    return ZERO_OK;
+}
+
+}  // namespace
+
+extern "C" zero_status zero_step_ranks(const zero_layout *L, const uint16_t *const *rank_grads, float *master,
+                                       float *m, float *v, uint16_t *p16_shard, uint16_t *p16_full,
+                                       const zero_adamw_hparams *hp, int32_t *nonfinite, void *stream)
+{
+    zero_status s = check_device(L);
+    if (s != ZERO_OK) return s;
+    if ((s = check_hparams(hp)) != ZERO_OK) return s;
+    if (L->padded == 0) return ZERO_OK;
+    zero::GradSource src;
+    if ((s = rank_source(L, rank_grads, &src)) != ZERO_OK) return s;
+    if ((s = check_state(master, m, v)) != ZERO_OK) return s;
+    if (!p16_full || (L->stage == 3 && !p16_shard)) return ZERO_ERR_INVALID;
+    if (!aligned16(p16_full) || (p16_shard && !aligned16(p16_shard))) return ZERO_ERR_ALIGN;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint16_t *p16 = L->stage == 3 ? p16_shard : p16_full;
+    cudaError_t e = zero::launch_bulk_step(*L, all_tiles(L), src, master, m, v, 0, p16, 0,
+                                           step_scalars(L->n_ranks, *hp), nonfinite, L->dev.wait_limit_ns,
+                                           L->dev.skip_first_fill, st);
+    if (e == cudaSuccess && L->stage == 3) e = zero::launch_copy_range(*L, 0, L->padded, p16_shard, p16_full, st);
+    return cuda_status(e);
+}
+
+extern "C" zero_status zero_step_shard(const zero_layout *L, int32_t shard, const uint16_t *const *rank_grads,
+                                       float *master_k, float *m_k, float *v_k, uint16_t *p16_out,
+                                       const zero_adamw_hparams *hp, int32_t *nonfinite, void *stream)
+{
+    zero_status s = check_device(L);
+    if (s != ZERO_OK) return s;
+    if ((s = check_hparams(hp)) != ZERO_OK) return s;
+    if (shard < 0 || shard >= L->n_ranks) return ZERO_ERR_INVALID;
+    if (L->padded == 0) return ZERO_OK;
+    if (L->shard % 8 != 0) return ZERO_ERR_ALIGN;
+    zero::GradSource src;
+    if ((s = rank_source(L, rank_grads, &src)) != ZERO_OK) return s;
+    if ((s = check_state(master_k, m_k, v_k)) != ZERO_OK) return s;
+    if (!p16_out) return ZERO_ERR_INVALID;
+    if (!aligned16(p16_out)) return ZERO_ERR_ALIGN;
+    const int64_t off = (int64_t)shard * L->shard;
+    return cuda_status(zero::launch_bulk_step(*L, shard_tiles(L, shard), src, master_k, m_k, v_k, off, p16_out,
+                                              L->stage == 3 ? off : 0, step_scalars(L->n_ranks, *hp), nonfinite,
+                                              L->dev.wait_limit_ns, L->dev.skip_first_fill, (cudaStream_t)stream));
+}
+
+extern "C" zero_status zero_copy_shard(const zero_layout *L, int32_t shard, const uint16_t *src, uint16_t *dst,
+                                       void *stream)
+{
+    zero_status s = check_device(L);
+    if (s != ZERO_OK) return s;
+    if (shard < 0 || shard >= L->n_ranks || !src || !dst) return ZERO_ERR_INVALID;
+    if (!aligned16(src) || !aligned16(dst)) return ZERO_ERR_ALIGN;
+    const int64_t lo = (int64_t)shard * L->shard;
+    return cuda_status(zero::launch_copy_range(*L, lo, lo + L->shard, src, dst, (cudaStream_t)stream));
+}
+
+namespace {
+
+// cuMemGetAddressRange (driver API), fetched at run time so that the library does not
+// link against the driver library: it finds the allocation a device pointer lies in.
+typedef int (*MemRangeFn)(unsigned long long *base, size_t *size, unsigned long long ptr);
+
+MemRangeFn mem_range_fn()
+{
+    static MemRangeFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuMemGetAddressRange", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<MemRangeFn>(p);
+    });
+    return fn;
+}
+
+}  // namespace
+
+extern "C" zero_status zero_ipc_get_handle(const void *dev_ptr, void *handle_out, int64_t *offset_out)
+{
+    if (!dev_ptr || !handle_out || !offset_out) return ZERO_ERR_INVALID;
+    MemRangeFn range = mem_range_fn();
+    if (!range) return ZERO_ERR_CUDA;
+    unsigned long long base = 0;
+    size_t size = 0;
+    if (range(&base, &size, (unsigned long long)(uintptr_t)dev_ptr) != 0) return ZERO_ERR_CUDA;
+    cudaIpcMemHandle_t h;
+    if (cudaIpcGetMemHandle(&h, (void *)(uintptr_t)base) != cudaSuccess) return ZERO_ERR_CUDA;
+    static_assert(sizeof(h) == 64, "CUDA IPC handles are 64 bytes");
+    memcpy(handle_out, &h, sizeof h);
+    *offset_out = (int64_t)((uintptr_t)dev_ptr - (uintptr_t)base);
+    return ZERO_OK;
+}
+
+extern "C" zero_status zero_ipc_open(const void *handle, int64_t offset, void **dev_ptr_out)
+{
+    if (!handle || !dev_ptr_out || offset < 0) return ZERO_ERR_INVALID;
+    cudaIpcMemHandle_t h;
+    memcpy(&h, handle, sizeof h);
+    void *base = nullptr;
+    *dev_ptr_out = nullptr;
+    if (cudaIpcOpenMemHandle(&base, h, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) return ZERO_ERR_CUDA;
+    *dev_ptr_out = static_cast<char *>(base) + offset;
+    return ZERO_OK;
+}
+
+extern "C" zero_status zero_ipc_close(void *dev_ptr, int64_t offset)
+{
+    if (!dev_ptr || offset < 0) return ZERO_ERR_INVALID;
+    return cudaIpcCloseMemHandle(static_cast<char *>(dev_ptr) - offset) == cudaSuccess ? ZERO_OK : ZERO_ERR_CUDA;
 }
 
 extern "C" zero_status zero_step_host(const zero_layout *L, const uint16_t *grads_host, uint16_t *grads_dev,

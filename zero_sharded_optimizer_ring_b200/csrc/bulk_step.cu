@@ -110,10 +110,11 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volati
 
 struct BulkArgs {
     TileWork w;
-    const uint16_t *grads;
-    int64_t stride;
-    float *master, *mom1, *mom2;
-    uint16_t *p16;
+    GradSource src;              // rank r's gradient of flat element i: src.rank[r][i]
+    float *master, *mom1, *mom2;  // element i at [i - state_off]
+    int64_t state_off;
+    uint16_t *p16;                // element i at [i - p16_off]
+    int64_t p16_off;
     AdamScalars c;
     int32_t *nonfinite;
     int32_t *error;
@@ -125,7 +126,7 @@ struct BulkArgs {
 // Shared memory: [full[S], empty[S] mbarriers][abort flag] ... stage ring (128-B aligned):
 // stage s = N gradient slices of kChunk fp16, then master, m, v slices of kChunk fp32.
 template <int N, bool kWire>
-__global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(BulkArgs A)
+__global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(const __grid_constant__ BulkArgs A)
 {
     constexpr int kChunk = BulkShape<N>::kChunk;
     constexpr int kConsumerWarps = BulkShape<N>::kConsumerWarps;
@@ -172,11 +173,11 @@ __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(Bu
 #pragma unroll
                 for (int j = 0; j < N; ++j)
                     bulk_load(smem_addr(base + (size_t)j * kChunk * 2),
-                              A.grads + (int64_t)ring_rank(tr.shard, j, N) * A.stride + q0, n * 2u, bar);
+                              A.src.rank[ring_rank(tr.shard, j, N)] + q0, n * 2u, bar);
                 unsigned char *st_base = base + (size_t)N * kChunk * 2;
-                bulk_load(smem_addr(st_base), A.master + q0, n * 4u, bar);
-                bulk_load(smem_addr(st_base + kChunk * 4), A.mom1 + q0, n * 4u, bar);
-                bulk_load(smem_addr(st_base + kChunk * 8), A.mom2 + q0, n * 4u, bar);
+                bulk_load(smem_addr(st_base), A.master + (q0 - A.state_off), n * 4u, bar);
+                bulk_load(smem_addr(st_base + kChunk * 4), A.mom1 + (q0 - A.state_off), n * 4u, bar);
+                bulk_load(smem_addr(st_base + kChunk * 8), A.mom2 + (q0 - A.state_off), n * 4u, bar);
                 posted = it + 1;
             }
         }
@@ -239,13 +240,13 @@ __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(Bu
                     adamw_elem(acc[e], A.c, pf[e], mf[e], vf[e], h[e]);
                 }
                 const int64_t q = q0 + e0;
-                float4 *pp = reinterpret_cast<float4 *>(A.master + q);
-                float4 *mp = reinterpret_cast<float4 *>(A.mom1 + q);
-                float4 *vp = reinterpret_cast<float4 *>(A.mom2 + q);
+                float4 *pp = reinterpret_cast<float4 *>(A.master + (q - A.state_off));
+                float4 *mp = reinterpret_cast<float4 *>(A.mom1 + (q - A.state_off));
+                float4 *vp = reinterpret_cast<float4 *>(A.mom2 + (q - A.state_off));
                 __stcs(pp, p4[0]); __stcs(pp + 1, p4[1]);
                 __stcs(mp, m4[0]); __stcs(mp + 1, m4[1]);
                 __stcs(vp, v4[0]); __stcs(vp + 1, v4[1]);
-                __stcs(reinterpret_cast<uint4 *>(A.p16 + q),
+                __stcs(reinterpret_cast<uint4 *>(A.p16 + (q - A.p16_off)),
                        make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16)));
             }
             __syncwarp();
@@ -260,22 +261,22 @@ __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(Bu
             const int64_t i = ct < n_head ? tr.a + ct : tail_begin + (ct - n_head);
             float acc;
             if constexpr (kWire) {
-                uint32_t h = A.grads[(int64_t)tr.shard * A.stride + i];
-                for (int j = 1; j < N; ++j) h = hadd1(h, A.grads[(int64_t)ring_rank(tr.shard, j, N) * A.stride + i]);
+                uint32_t h = A.src.rank[tr.shard][i];
+                for (int j = 1; j < N; ++j) h = hadd1(h, A.src.rank[ring_rank(tr.shard, j, N)][i]);
                 acc = h2f(h);
             } else {
-                acc = h2f(A.grads[(int64_t)tr.shard * A.stride + i]);
-                for (int j = 1; j < N; ++j)
-                    acc = __fadd_rn(acc, h2f(A.grads[(int64_t)ring_rank(tr.shard, j, N) * A.stride + i]));
+                acc = h2f(A.src.rank[tr.shard][i]);
+                for (int j = 1; j < N; ++j) acc = __fadd_rn(acc, h2f(A.src.rank[ring_rank(tr.shard, j, N)][i]));
             }
             bad += !isfinite(acc);
-            float p = A.master[i], m = A.mom1[i], v = A.mom2[i];
+            const int64_t si = i - A.state_off;
+            float p = A.master[si], m = A.mom1[si], v = A.mom2[si];
             uint32_t h;
             adamw_elem(acc, A.c, p, m, v, h);
-            A.master[i] = p;
-            A.mom1[i] = m;
-            A.mom2[i] = v;
-            A.p16[i] = (uint16_t)h;
+            A.master[si] = p;
+            A.mom1[si] = m;
+            A.mom2[si] = v;
+            A.p16[i - A.p16_off] = (uint16_t)h;
         }
         if (A.nonfinite) {
             if (__any_sync(0xffffffffu, bad != 0)) {
@@ -307,27 +308,24 @@ cudaError_t launch_bulk_n(const zero_layout &L, BulkArgs &a, cudaStream_t st)
 
 }  // namespace
 
-bool bulk_supported(int n_ranks)
-{
-    switch (n_ranks) {
-        case 1: case 2: case 3: case 4: case 5: case 6: case 7: case 8: case 16: return true;
-        default: return false;
-    }
-}
+bool bulk_supported(int n_ranks) { return n_ranks >= 1 && n_ranks <= 16; }
 
-cudaError_t launch_bulk_step(const zero_layout &L, const TileWork &w, const uint16_t *grads, int64_t stride,
-                             float *master, float *m, float *v, uint16_t *p16, const AdamScalars &c,
-                             int32_t *nonfinite, uint64_t wait_limit_ns, int skip_first_fill, cudaStream_t st)
+cudaError_t launch_bulk_step(const zero_layout &L, const TileWork &w, const GradSource &src, float *master,
+                             float *m, float *v, int64_t state_off, uint16_t *p16, int64_t p16_off,
+                             const AdamScalars &c, int32_t *nonfinite, uint64_t wait_limit_ns,
+                             int skip_first_fill, cudaStream_t st)
 {
     if (w.n_tiles <= 0) return cudaSuccess;
+    if ((state_off & 7) != 0 || (p16_off & 7) != 0) return cudaErrorMisalignedAddress;
     BulkArgs a;
     a.w = w;
-    a.grads = grads;
-    a.stride = stride;
+    a.src = src;
     a.master = master;
     a.mom1 = m;
     a.mom2 = v;
+    a.state_off = state_off;
     a.p16 = p16;
+    a.p16_off = p16_off;
     a.c = c;
     a.nonfinite = nonfinite;
     a.error = L.dev.error;
@@ -343,6 +341,13 @@ cudaError_t launch_bulk_step(const zero_layout &L, const TileWork &w, const uint
         case 6: return launch_bulk_n<6>(L, a, st);
         case 7: return launch_bulk_n<7>(L, a, st);
         case 8: return launch_bulk_n<8>(L, a, st);
+        case 9: return launch_bulk_n<9>(L, a, st);
+        case 10: return launch_bulk_n<10>(L, a, st);
+        case 11: return launch_bulk_n<11>(L, a, st);
+        case 12: return launch_bulk_n<12>(L, a, st);
+        case 13: return launch_bulk_n<13>(L, a, st);
+        case 14: return launch_bulk_n<14>(L, a, st);
+        case 15: return launch_bulk_n<15>(L, a, st);
         case 16: return launch_bulk_n<16>(L, a, st);
         default: return cudaErrorInvalidValue;
     }

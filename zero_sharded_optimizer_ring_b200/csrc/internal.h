@@ -22,6 +22,14 @@ struct Seg {
 };
 static_assert(sizeof(Seg) == 32, "device table row is 32 bytes");
 
+// Where each rank's gradients live for the bulk pipeline: rank r's value of flat element i
+// is rank[r][i].  One strided buffer (rank[r] = grads + r * stride), separate buffers on
+// this GPU, or other GPUs' buffers mapped into this process.
+constexpr int kMaxBulkRanks = 16;
+struct GradSource {
+    const uint16_t *rank[kMaxBulkRanks];
+};
+
 // fp32 scalars of one AdamW step, each computed on the host in double and rounded once.
 struct AdamScalars {
     float inv_scale;   // 1 / (N * loss_scale)
@@ -44,6 +52,7 @@ struct TileWork {
 struct DeviceState {
     int device = -1;
     Seg *segs = nullptr;          // n_seg + 1 rows
+    Seg *segs_by_shard = nullptr; // the same rows ordered by shard, then bucket (+ closing row)
     int32_t *error = nullptr;     // device error word (timeouts)
     int num_sms = 0;
     size_t smem_optin = 0;
@@ -64,6 +73,8 @@ struct zero_layout {
     std::vector<int64_t> bucket_lo, bucket_hi;
     std::vector<int64_t> bucket_seg_begin;     // n_buckets + 1: first segment of each bucket
     std::vector<zero::Seg> segs;               // host copy, tile_begin filled on the host too
+    std::vector<zero::Seg> segs_by_shard;      // shard-major order, with its own tile numbering
+    std::vector<int64_t> shard_seg_begin;      // n_ranks + 1: first shard-major row of each shard
     std::vector<int64_t> unit_lo, unit_hi;
     int64_t n_tiles = 0;
     int32_t impl = 0;
@@ -88,8 +99,11 @@ cudaError_t launch_fused_step(const zero_layout &L, const TileWork &w, const uin
 
 // bulk_step.cu
 bool bulk_supported(int n_ranks);
-cudaError_t launch_bulk_step(const zero_layout &L, const TileWork &w, const uint16_t *grads, int64_t stride,
-                             float *master, float *m, float *v, uint16_t *p16, const AdamScalars &c,
-                             int32_t *nonfinite, uint64_t wait_limit_ns, int skip_first_fill, cudaStream_t st);
+// master / m / v hold flat elements [state_off, ...) and p16 [p16_off, ...): element i is
+// at index i - off (both offsets multiples of 8).
+cudaError_t launch_bulk_step(const zero_layout &L, const TileWork &w, const GradSource &src, float *master,
+                             float *m, float *v, int64_t state_off, uint16_t *p16, int64_t p16_off,
+                             const AdamScalars &c, int32_t *nonfinite, uint64_t wait_limit_ns,
+                             int skip_first_fill, cudaStream_t st);
 
 }  // namespace zero

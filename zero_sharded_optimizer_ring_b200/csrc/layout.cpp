@@ -91,6 +91,19 @@ extern "C" zero_status zero_layout_create(const zero_layout_desc *d, zero_layout
         L->bucket_seg_begin.push_back((int64_t)L->segs.size());
         L->n_tiles = tiles;
 
+        // the same segments shard-major (one shard's segments contiguous), renumbered
+        for (int64_t k = 0; k < N; ++k) {
+            L->shard_seg_begin.push_back((int64_t)L->segs_by_shard.size());
+            for (const zero::Seg &sg : L->segs)
+                if (sg.shard == k) L->segs_by_shard.push_back(sg);
+        }
+        L->shard_seg_begin.push_back((int64_t)L->segs_by_shard.size());
+        int64_t t2 = 0;
+        for (zero::Seg &sg : L->segs_by_shard) {
+            sg.tile_begin = t2;
+            t2 += ceil_div(sg.hi, zero::kTileElems) - sg.lo / zero::kTileElems;
+        }
+
         // gather units: tensor ranges; the last unit also takes the tail padding
         if (P > 0) {
             if (d->n_units == 0) {

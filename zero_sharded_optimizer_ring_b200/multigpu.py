@@ -1,0 +1,98 @@
+"""The step with one process per GPU (host orchestration only).
+
+Rank r holds its own fp16 gradients [P], the optimizer state of shard r (master, m, v:
+[S] each, rank r owning shard r as in rkmt.cn/news/44736 "Deepspeed ZeRO-1", where GPU0
+is responsible for the first third) and the full fp16 parameters [P] (ZeRO stages 0-2).
+Every rank maps the other ranks' gradient and parameter buffers with CUDA IPC once; a
+step then runs three phases, each closed by a host barrier:
+
+  1. every rank's gradients are complete (barrier);
+  2. rank r runs zero_step_shard for shard r: the fused kernel pulls the shard's slices
+     from all N gradient buffers over NVLink and folds them in the ring order r, r+1, ...,
+     r+N-1, which equals the single-GPU simulation bit for bit (barrier);
+  3. rank r copies every other shard's new fp16 parameters from its owner's buffer into
+     its own (the all-gather; barrier before anyone writes those buffers again).
+
+No kernel waits on another GPU: the barriers are host-side, after a device
+synchronisation, so each kernel only reads peer memory that is complete and stable.
+"""
+
+
+class CudaOps:
+    """The device operations of a step, through the library's C ABI."""
+
+    def __init__(self):
+        import zero_sharded_optimizer_ring_b200 as zs
+        self.zs = zs
+
+    def export(self, t):
+        return self.zs.ipc_handle(t)
+
+    def open(self, handle):
+        return self.zs.ipc_open(handle)             # (device address, offset)
+
+    def close(self, mapped):
+        self.zs.ipc_close(mapped)
+
+    @staticmethod
+    def _addr(x):
+        return x[0] if isinstance(x, tuple) else x
+
+    def step_shard(self, layout, shard, rank_grads, master_k, m_k, v_k, p16_full, hp, nonfinite):
+        self.zs.step_shard(layout, shard, [self._addr(g) for g in rank_grads], master_k, m_k, v_k, p16_full, hp,
+                           nonfinite)
+
+    def copy_shard(self, layout, shard, src, dst):
+        self.zs.copy_shard(layout, shard, self._addr(src), dst)
+
+    def sync(self):
+        import torch
+        torch.cuda.synchronize()
+
+
+class RankStep:
+    """One rank's share of the multi-GPU step (see the module docstring)."""
+
+    def __init__(self, layout, rank, world, grads, master_k, m_k, v_k, p16_full, group=None, ops=None):
+        import torch.distributed as dist
+        if layout.n_ranks != world:
+            raise ValueError("the layout's rank count must equal the world size")
+        if layout.stage == 3:
+            raise ValueError("stage 3 keeps no full parameter buffer per rank; use stages 0-2")
+        self.dist, self.group = dist, group
+        self.layout, self.rank, self.world = layout, rank, world
+        self.ops = ops or CudaOps()
+        self.grads, self.state, self.p16_full = grads, (master_k, m_k, v_k), p16_full
+        mine = (rank, self.ops.export(grads), self.ops.export(p16_full))
+        everyone = [None] * world
+        dist.all_gather_object(everyone, mine, group=group)
+        self.opened = []
+        self.peer_grads = [None] * world
+        self.peer_p16 = [None] * world
+        for r, hg, hp16 in everyone:
+            if r == rank:
+                self.peer_grads[r], self.peer_p16[r] = grads, p16_full
+            else:
+                self.peer_grads[r] = self.ops.open(hg)
+                self.peer_p16[r] = self.ops.open(hp16)
+                self.opened += [self.peer_grads[r], self.peer_p16[r]]
+
+    def _barrier(self):
+        self.ops.sync()
+        self.dist.barrier(group=self.group)
+
+    def step(self, hp, nonfinite=None):
+        self._barrier()                                     # 1: all gradients written
+        self.ops.step_shard(self.layout, self.rank, self.peer_grads, *self.state, self.p16_full, hp, nonfinite)
+        self._barrier()                                     # 2: every shard updated
+        for j in range(self.world):
+            if j != self.rank:
+                self.ops.copy_shard(self.layout, j, self.peer_p16[j], self.p16_full)
+        self._barrier()                                     # 3: parameters gathered everywhere
+
+    def close(self):
+        """Unmap the peers' buffers (before the process group or the buffers go away)."""
+        self._barrier()
+        for p in self.opened:
+            self.ops.close(p)
+        self.opened = []
