@@ -333,3 +333,30 @@ def test_bulk_pipeline_bounded_wait_reports_timeout():
     b = _bufs(lay, wl)
     _run(lay, wl, b, 1)
     _check_full(wl, lay, b, ref)
+
+
+@pytest.mark.parametrize("key", ["flat1p3b_n4_zero1", "llama3b_n8_zero3"])
+def test_checkpoint_resume_equals_uninterrupted(key):
+    """The optimizer state is the caller's buffers: copying them to host memory after two
+    steps, wiping the device buffers and a fresh layout, restoring, and running two more
+    steps gives exactly the four-step result (the library keeps no state of its own)."""
+    wl = reduced_workloads()[key]
+    lay = _layout(wl, zs.IMPL_BULK)
+    a = _bufs(lay, wl)
+    _run(lay, wl, a, 4)
+    b = _bufs(lay, wl)
+    for t in (1, 2):
+        zs.step(lay, b["g"], b["master"], b["m"], b["v"], b["p16_shard"], b["p16_full"], _hp(wl, t))
+    torch.cuda.synchronize()
+    saved = {k: b[k].cpu().clone() for k in ("master", "m", "v", "p16_shard", "p16_full")}
+    for k in saved:
+        b[k].fill_(7)
+    lay.close()
+    lay2 = _layout(wl, zs.IMPL_BULK)
+    for k, x in saved.items():
+        b[k].copy_(x)
+    for t in (3, 4):
+        zs.step(lay2, b["g"], b["master"], b["m"], b["v"], b["p16_shard"], b["p16_full"], _hp(wl, t))
+    torch.cuda.synchronize()
+    for k in ("master", "m", "v", "p16_full"):
+        S.assert_bits_equal(_np(b[k]), _np(a[k]), k)
