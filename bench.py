@@ -61,6 +61,9 @@ def parse():
     ap.add_argument("--overlap", action="store_true",
                     help="measure the bucket-pipelined step behind a simulated backward pass "
                          "(its own JSON line; not the headline)")
+    ap.add_argument("--shrink", type=int, default=0,
+                    help="divide every tensor of the workload by this factor (same structure, smaller: "
+                         "small cases for profiler captures; not a bench line)")
     ap.add_argument("--psi", type=int, default=0,
                     help="flat workloads only: run the same shape with this many parameters "
                          "(small cases for profiler captures; not a bench line)")
@@ -633,6 +636,8 @@ def main():
     a = parse()
     from seeded_inputs.workloads import full_workloads
     wl = full_workloads()[a.workload]
+    if a.shrink > 1:
+        wl = wl.with_(tensors=tuple(max(1, t // a.shrink) for t in wl.tensors), name=f"{wl.name}_shrink{a.shrink}")
     if a.psi:
         if len(wl.tensors) != 1:
             raise SystemExit("--psi applies to flat (single-tensor) workloads only")
