@@ -61,6 +61,14 @@ def parse():
     ap.add_argument("--overlap", action="store_true",
                     help="measure the bucket-pipelined step behind a simulated backward pass "
                          "(its own JSON line; not the headline)")
+    ap.add_argument("--backward", default="generator", choices=["generator", "gemm"],
+                    help="--overlap: the simulated backward. generator = the seeded generator's kernels "
+                         "rewrite each bucket's gradients (ALU-bound); gemm = two bf16 GEMMs per bucket "
+                         "(cuBLAS, 4 * tokens FLOPs per parameter; tensor-core bound)")
+    ap.add_argument("--bwd-tokens", type=int, default=4096, help="--overlap --backward gemm: tokens per rank")
+    ap.add_argument("--max-ctas", default="0",
+                    help="cap on the fused kernel's CTAs (zero_set_max_ctas; 0 = one per SM). With --overlap "
+                         "a comma-separated list, one JSON line each")
     ap.add_argument("--shrink", type=int, default=0,
                     help="divide every tensor of the workload by this factor (same structure, smaller: "
                          "small cases for profiler captures; not a bench line)")
@@ -213,7 +221,13 @@ def variant_config(a, wl, world):
         c["ring_partials"] = "fp16 wire"
     if a.dynamic:
         c["step"] = "zero_step_dynamic"
+    if first_cap(a):
+        c["max_ctas"] = first_cap(a)
     return c
+
+
+def first_cap(a):
+    return int(str(a.max_ctas).split(",")[0])
 
 
 # ---------------------------------------------------------------- CPU oracle sample
@@ -302,6 +316,8 @@ def run_ours(a, wl):
     lay.to_device()
     if a.kernel:
         lay.set_impl(a.kernel)
+    if first_cap(a):
+        lay.set_max_ctas(first_cap(a))
     P, psi, N = lay.padded, lay.psi, wl.n_ranks
     g = torch.empty((N, P), dtype=torch.int16, device="cuda")
     si.fill_grads_cuda(g, psi, wl.seed, wl.grad_sigma, wl.loss_scale, wl.heavy_frac, wl.heavy_mult)
@@ -461,8 +477,9 @@ def run_overlap(a, wl):
     _, buckets, _, _ = lay.tables()
     ev = lambda: torch.cuda.Event(enable_timing=True)
     hi_pri = torch.cuda.Stream.priority_range()[1]       # numerically lowest = highest priority
+    caps = [int(x) for x in str(a.max_ctas).split(",")]
 
-    def backward_fn(producer):
+    def generator_backward(producer):
         def backward(events=None):
             for b, (lo, hi) in enumerate(buckets):
                 si.fill_grads_range_cuda(g, int(lo), int(hi), psi, wl.seed, wl.grad_sigma, wl.loss_scale,
@@ -471,18 +488,46 @@ def run_overlap(a, wl):
                     events[b].record(producer)
         return backward
 
-    t = 0
+    def gemm_backward(producer):
+        # per bucket of n_b parameters, viewed as a [D, n_b / D] weight: the activation
+        # gradient [T, D] x [D, n] and the weight gradient [D, T] x [T, n], 4 T n_b FLOPs;
+        # the gradients themselves are generated once, here, and stay
+        si.fill_grads_cuda(g, psi, wl.seed, wl.grad_sigma, wl.loss_scale, wl.heavy_frac, wl.heavy_mult)
+        T, D = a.bwd_tokens, 4096
+        A = torch.randn(T, D, device="cuda", dtype=torch.bfloat16)
+        shapes = [max(128, (int(hi - lo) // D + 127) // 128 * 128) for lo, hi in buckets]
+        mats = {n: (torch.randn(D, n, device="cuda", dtype=torch.bfloat16),
+                    torch.empty(T, n, device="cuda", dtype=torch.bfloat16),
+                    torch.empty(D, n, device="cuda", dtype=torch.bfloat16)) for n in set(shapes)}
 
+        def backward(events=None):
+            with torch.cuda.stream(producer):
+                for b, n in enumerate(shapes):
+                    w, act, wgrad = mats[n]
+                    torch.mm(A, w, out=act)
+                    torch.mm(A.t(), act, out=wgrad)
+                    if events is not None:
+                        events[b].record(producer)
+        backward.tflop = sum(4.0 * T * D * n for n in shapes) / 1e12
+        return backward
+
+    t = 0
     reps = max(3, a.steps // 20)
-    for prio_name, prio in (("default", 0), ("high", hi_pri)):
+    if a.backward == "gemm":
+        runs = [("default", 0, cap) for cap in caps]
+    else:
+        runs = [("default", 0, caps[0]), ("high", hi_pri, caps[0])]
+    for prio_name, prio, cap in runs:
+        lay.set_max_ctas(cap)
         producer, compute = torch.cuda.Stream(), torch.cuda.Stream(priority=prio)
-        t = _overlap_reps(a, wl, lay, g, master, m, v, p16_shard, p16_full, backward_fn(producer), producer,
-                          compute, ev, reps, t, prio_name)
+        make = gemm_backward if a.backward == "gemm" else generator_backward
+        t = _overlap_reps(a, wl, lay, g, master, m, v, p16_shard, p16_full, make(producer), producer,
+                          compute, ev, reps, t, prio_name, cap)
     zs.get_error(lay)
 
 
 def _overlap_reps(a, wl, lay, g, master, m, v, p16_shard, p16_full, backward, producer, compute, ev, reps, t,
-                  prio_name):
+                  prio_name, cap):
     import torch
     import zero_sharded_optimizer_ring_b200 as zs
 
@@ -518,8 +563,10 @@ def _overlap_reps(a, wl, lay, g, master, m, v, p16_shard, p16_full, backward, pr
     tb, ts, tp = (statistics.median(res[k]) for k in ("bwd", "step", "pipe"))
     print(json.dumps({
         "metric": "bucket-pipelined step behind a simulated backward (overlap)", "workload": wl.name,
-        "compute_stream_priority": prio_name, "buckets": lay.n_buckets, "reps": reps, "t_backward_ms": tb,
-        "t_step_ms": ts, "t_pipelined_ms": tp, "exposed_step_ms": tp - tb, "overlap_efficiency": (tb + ts - tp) / ts,
+        "backward": a.backward, "compute_stream_priority": prio_name, "max_ctas": cap, "buckets": lay.n_buckets,
+        "reps": reps, "t_backward_ms": tb, "t_step_ms": ts, "t_pipelined_ms": tp, "exposed_step_ms": tp - tb,
+        "overlap_efficiency": (tb + ts - tp) / ts,
+        **({"backward_tflops": backward.tflop / (tb / 1e3)} if hasattr(backward, "tflop") else {}),
         "note": "overlap_efficiency = share of the step hidden behind the backward (1 = fully hidden)"}),
         flush=True)
     return t

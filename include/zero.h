@@ -331,6 +331,16 @@ zero_status zero_ipc_close(void *dev_ptr, int64_t offset);
  * shared-memory ring, warp-specialised).  Results are bit-identical. */
 zero_status zero_set_impl(zero_layout *layout, int32_t impl);
 
+/* Cap on the number of CTAs of the tile-walking kernels (the fused step in both
+ * implementations, and the reduce-scatter): 0 (the default) = as many as the GPU holds
+ * (one per SM for the pipeline), k > 0 = at most k.  Every grid size gives bit-identical
+ * results: tiles are dealt to CTAs by a fixed stride.  A capped step leaves the other
+ * SMs to concurrent work (a backward pass whose gradients the step consumes bucket by
+ * bucket, as in [P1] "DDP": the first finished group is synchronised while the next is
+ * computed); it is slower alone, since each SM moves at most ~60 GB/s through the
+ * step's arithmetic.  Negative k: ZERO_ERR_INVALID.  No counterpart on the pages. */
+zero_status zero_set_max_ctas(zero_layout *layout, int32_t max_ctas);
+
 /* Test hook of the bulk-copy pipeline's bounded waits: every in-kernel wait gives up
  * after wait_limit_ns nanoseconds (default 2e9) and records ZERO_ERR_TIMEOUT.  With
  * skip_first_fill = 1 the pipeline never posts its first chunk, so the consumers' wait

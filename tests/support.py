@@ -115,9 +115,17 @@ def assert_f16_ulp(got, want, what, ulps=F16_ULPS):
     assert d.max(initial=0) <= ulps, f"{what}: max {d.max()} ulp"
 
 
-def assert_bits_equal(got, want, what):
+def assert_bits_equal(got, want, what, any_nan=False):
+    """Bit for bit.  any_nan: a NaN matches any NaN (float32, or fp16 bits as uint16) —
+    IEEE 754 leaves the payload of an invalid operation's NaN open: x86 gives 0xFFC00000
+    for 0/0, CUDA 0x7FFFFFFF — while NaN positions must still agree."""
     got = np.ascontiguousarray(got)
     want = np.ascontiguousarray(want)
-    diff = got.view(np.uint8).reshape(got.size, -1) != want.view(np.uint8).reshape(want.size, -1)
-    n = int(diff.any(axis=1).sum())
+    diff = (got.view(np.uint8).reshape(got.size, -1) != want.view(np.uint8).reshape(want.size, -1)).any(axis=1)
+    if any_nan:
+        isnan = f16_isnan if got.dtype == np.uint16 else np.isnan
+        nan_g, nan_w = isnan(got).reshape(-1), isnan(want).reshape(-1)
+        assert np.array_equal(nan_g, nan_w), f"{what}: NaN positions differ"
+        diff &= ~(nan_g & nan_w)
+    n = int(diff.sum())
     assert n == 0, f"{what}: {n} elements differ bitwise"

@@ -106,3 +106,14 @@ def test_empty_layout():
     assert (lay.psi, lay.padded, lay.n_buckets, lay.n_segments, lay.n_units, lay.n_tiles) == (0, 0, 0, 0, 0, 0)
     lay = zs.Layout([0, 0], 3, 3, 0)
     assert lay.padded == 0
+
+
+def test_tuning_setters_validate_arguments():
+    lay = zs.Layout([1000], 2, 1, 100)
+    lay.set_max_ctas(0)
+    lay.set_max_ctas(37)
+    lay.set_impl(2)
+    for bad in (lambda: lay.set_max_ctas(-1), lambda: lay.set_impl(3), lambda: lay.set_impl(-1)):
+        with pytest.raises(zs.ZeroError) as e:
+            bad()
+        assert e.value.status == 1

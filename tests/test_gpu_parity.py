@@ -141,6 +141,24 @@ def test_deterministic_rerun():
         S.assert_bits_equal(outs[0][k], outs[1][k], k)
 
 
+@pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("key", ["flat1p3b_n4_zero1", "ragged2000_n16_zero2", "llama3b_n8_zero3"])
+def test_capped_grid_matches_oracle(key, impl):
+    """zero_set_max_ctas: any grid size deals the same tiles, so every cap gives the
+    oracle's result bit for bit (one CTA walks every tile)."""
+    wl = reduced_workloads()[key]
+    ref, _ = _oracle(wl)
+    lay = _layout(wl, impl)
+    for cap in (1, 7, 37):
+        lay.set_max_ctas(cap)
+        b = _bufs(lay, wl)
+        _run(lay, wl, b, wl.steps)
+        _check_full(wl, lay, b, ref)
+        red = torch.zeros(lay.padded, dtype=torch.float32, device="cuda")
+        zs.reduce_scatter(lay, -1, b["g"], red)
+        S.assert_bits_equal(_np(red), ref.reduced, "reduced")
+
+
 def test_device_tile_index_matches_host():
     for wl in list(reduced_workloads().values()) + list(full_workloads().values()):
         lay = _layout(wl)
@@ -236,6 +254,46 @@ def test_nonfinite_counts_per_bucket():
     assert list(_np(nf)) == list(ref.nonfinite)
     assert sum(ref.nonfinite) == len(marks)
     S.assert_f16_ulp(_np(p16), ref.p16_full, "p16")
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_zero_and_signed_zero_operands(impl):
+    """Exact zeros take the kernels' shortcut around the square root and the divisions:
+    zero gradients with zero moments (untouched rows), gradients of -0, moments of -0,
+    zero gradients with warm moments, and eps = 0 (where 0 / 0 must stay NaN), for every
+    step against the oracle bit for bit."""
+    wl = _edge([40_000, 9_001], 4, 2, 10_007, 8, steps=3, m_sigma=1e-4, v_sigma=1e-6)
+    olay = S.oracle_layout(wl)
+    P = olay.padded
+    g, master, m, v = S.host_inputs(wl, P)
+    g[:, :12_000] = 0                                   # untouched rows: zero gradient, zero moments
+    m[:12_000] = 0
+    v[:12_000] = 0
+    g[:, 12_000:14_000] = 0x8000                        # -0 gradients, warm moments
+    g[:, 14_000:16_000] = 0x8000                        # -0 gradients, -0 first moment, zero second
+    m[14_000:16_000] = -0.0
+    v[14_000:16_000] = 0
+    g[1, 16_000:18_000] = 0x8000                        # one rank's -0 among finite gradients
+    g[:, 18_000:20_000] = 0                             # zero gradient, warm moments
+    for eps in (1e-8, 0.0):
+        w = wl.with_(eps=eps)
+        ref = oracle.run_steps(olay, w.stage, g, master, m, v, S.hyper(w), w.steps)
+        lay = _layout(w, impl)
+        b = dict(g=torch.from_numpy(g.view(np.int16)).cuda(), master=torch.from_numpy(master).cuda(),
+                 m=torch.from_numpy(m).cuda(), v=torch.from_numpy(v).cuda(),
+                 p16_shard=torch.zeros(P, dtype=torch.int16, device="cuda"),
+                 p16_full=torch.zeros(P, dtype=torch.int16, device="cuda"),
+                 nonfinite=torch.zeros(lay.n_buckets, dtype=torch.int32, device="cuda"))
+        for t in range(1, w.steps + 1):
+            b["nonfinite"].zero_()
+            zs.step(lay, b["g"], b["master"], b["m"], b["v"], b["p16_shard"], b["p16_full"], _hp(w, t),
+                    nonfinite=b["nonfinite"])
+        zs.get_error(lay)
+        for k, want in (("master", ref.master), ("m", ref.m), ("v", ref.v), ("p16_full", ref.p16_full)):
+            S.assert_bits_equal(_np(b[k]), want, k, any_nan=True)
+        if eps == 0.0:
+            assert np.isnan(ref.master[:12_000]).all()     # 0 / (0 + 0): the shortcut must not hide it
+        assert np.signbit(ref.m[14_000:16_000]).all() and not ref.m[14_000:16_000].any()
 
 
 def test_bad_arguments_rejected():

@@ -132,6 +132,10 @@ class Layout:
     def set_impl(self, impl):
         _check(_abi.lib().zero_set_impl(self._h, int(impl)), "zero_set_impl")
 
+    def set_max_ctas(self, max_ctas):
+        """At most max_ctas CTAs per fused-step / reduce-scatter launch (0 = all SMs)."""
+        _check(_abi.lib().zero_set_max_ctas(self._h, int(max_ctas)), "zero_set_max_ctas")
+
     def debug_set_wait(self, wait_limit_ns, skip_first_fill=0):
         _check(_abi.lib().zero_debug_set_wait(self._h, int(wait_limit_ns), int(skip_first_fill)),
                "zero_debug_set_wait")

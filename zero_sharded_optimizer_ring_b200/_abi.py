@@ -78,6 +78,7 @@ SIGNATURES = {
     "zero_ipc_open": (_i32, [_vp, _i64, ctypes.POINTER(_vp)]),
     "zero_ipc_close": (_i32, [_vp, _i64]),
     "zero_set_impl": (_i32, [_vp, _i32]),
+    "zero_set_max_ctas": (_i32, [_vp, _i32]),
     "zero_debug_set_wait": (_i32, [_vp, _i64, _i32]),
     "zero_get_error": (_i32, [_vp, _vp]),
     "zero_status_string": (ctypes.c_char_p, [_i32]),

@@ -70,8 +70,15 @@ __device__ __forceinline__ void adamw_elem(float s, const AdamScalars &c, float 
     const float pd = __fmul_rn(p, c.decay);
     m = __fadd_rn(__fmul_rn(m, c.beta1), __fmul_rn(g, c.omb1));
     v = __fadd_rn(__fmul_rn(v, c.beta2), __fmul_rn(__fmul_rn(g, g), c.omb2));
-    const float denom = __fadd_rn(__fdiv_rn(__fsqrt_rn(v), c.sqrt_bc2), c.eps);
-    p = __fsub_rn(pd, __fmul_rn(c.step_size, __fdiv_rn(m, denom)));
+    // Zero operands skip the square root and the divisions, whose IEEE sequences leave
+    // their fast path on them (a parameter with zero gradient and zero moments, e.g. an
+    // embedding row no batch has touched, would otherwise cost about twice as much).
+    // Both shortcuts are exact: sqrt(+-0) = +-0 and +-0 / c = +-0 for the step's
+    // sqrt(1 - beta2^t) > 0; +-0 / denom = +-0 for denom > 0 (NaN and 0 divide as usual).
+    const float q = v == 0.0f ? v : __fdiv_rn(__fsqrt_rn(v), c.sqrt_bc2);
+    const float denom = __fadd_rn(q, c.eps);
+    const float ratio = (m == 0.0f && denom > 0.0f) ? m : __fdiv_rn(m, denom);
+    p = __fsub_rn(pd, __fmul_rn(c.step_size, ratio));
     h = f2h(p);
 }
 

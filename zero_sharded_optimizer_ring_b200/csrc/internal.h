@@ -78,6 +78,7 @@ struct zero_layout {
     std::vector<int64_t> unit_lo, unit_hi;
     int64_t n_tiles = 0;
     int32_t impl = 0;
+    int32_t max_ctas = 0;                      // > 0: cap on the grid of the tile-walking kernels
     zero::DeviceState dev;
 };
 

@@ -314,13 +314,14 @@ __global__ void tile_index_kernel(Seg *segs, int64_t n_seg)
 }
 
 template <class K>
-int grid_for(K kernel, int64_t work_items, int num_sms)
+int grid_for(K kernel, int64_t work_items, int num_sms, int max_ctas = 0)
 {
     int per_sm = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0) != cudaSuccess ||
         per_sm < 1)
         per_sm = 1;
     int64_t g = (int64_t)per_sm * (num_sms > 0 ? num_sms : 148);
+    if (max_ctas > 0 && g > max_ctas) g = max_ctas;
     if (g > work_items) g = work_items;
     return (int)(g < 1 ? 1 : g);
 }
@@ -331,7 +332,7 @@ cudaError_t launch_tiles(const zero_layout &L, const TileWork &w, const uint16_t
                          const AdamScalars &c, int32_t *nonfinite, cudaStream_t st)
 {
     auto kern = L.wire16 ? tile_kernel<NT, U, kFused, true> : tile_kernel<NT, U, kFused, false>;
-    const int grid = grid_for(kern, w.n_tiles, L.dev.num_sms);
+    const int grid = grid_for(kern, w.n_tiles, L.dev.num_sms, L.max_ctas);
     kern<<<grid, kThreads, 0, st>>>(w, L.n_ranks, grads, stride, reduced, master, m, v, p16, c, nonfinite);
     return cudaGetLastError();
 }
