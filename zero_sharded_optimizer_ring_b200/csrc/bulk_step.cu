@@ -235,10 +235,8 @@ __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(co
                 float *vf = reinterpret_cast<float *>(v4);
                 uint32_t h[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    bad += !isfinite(acc[e]);
-                    adamw_elem(acc[e], A.c, pf[e], mf[e], vf[e], h[e]);
-                }
+                for (int e = 0; e < 8; ++e) bad += !isfinite(acc[e]);
+                adamw8(acc, A.c, pf, mf, vf, h);
                 const int64_t q = q0 + e0;
                 float4 *pp = reinterpret_cast<float4 *>(A.master + (q - A.state_off));
                 float4 *mp = reinterpret_cast<float4 *>(A.mom1 + (q - A.state_off));

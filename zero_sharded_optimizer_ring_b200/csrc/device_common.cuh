@@ -62,24 +62,67 @@ __device__ __forceinline__ uint32_t hadd1(uint32_t a, uint32_t b)
     return (uint32_t)__half_as_ushort(__hadd(__ushort_as_half((unsigned short)a), __ushort_as_half((unsigned short)b)));
 }
 
-// One element of the shard update.  Order of operations as documented in zero.h.
-__device__ __forceinline__ void adamw_elem(float s, const AdamScalars &c, float &p, float &m,
-                                           float &v, uint32_t &h)
+// The shard update, order of operations as documented in zero.h, in two parts: the
+// moments (p becomes the decayed weight), then the step from the new moments.
+__device__ __forceinline__ void adamw_moments(float s, const AdamScalars &c, float &p, float &m, float &v)
 {
     const float g = __fmul_rn(s, c.inv_scale);
-    const float pd = __fmul_rn(p, c.decay);
+    p = __fmul_rn(p, c.decay);
     m = __fadd_rn(__fmul_rn(m, c.beta1), __fmul_rn(g, c.omb1));
     v = __fadd_rn(__fmul_rn(v, c.beta2), __fmul_rn(__fmul_rn(g, g), c.omb2));
-    // Zero operands skip the square root and the divisions, whose IEEE sequences leave
-    // their fast path on them (a parameter with zero gradient and zero moments, e.g. an
-    // embedding row no batch has touched, would otherwise cost about twice as much).
-    // Both shortcuts are exact: sqrt(+-0) = +-0 and +-0 / c = +-0 for the step's
-    // sqrt(1 - beta2^t) > 0; +-0 / denom = +-0 for denom > 0 (NaN and 0 divide as usual).
+}
+
+__device__ __forceinline__ void adamw_apply(const AdamScalars &c, float &p, float m, float v)
+{
+    const float denom = __fadd_rn(__fdiv_rn(__fsqrt_rn(v), c.sqrt_bc2), c.eps);
+    p = __fsub_rn(p, __fmul_rn(c.step_size, __fdiv_rn(m, denom)));
+}
+
+// The same step for moments that may be exactly zero.  Zero operands send the IEEE
+// square-root and divide sequences off their fast path (a parameter with zero gradient
+// and zero moments, e.g. an embedding row no batch has touched, then costs about twice
+// as much), so they are skipped by two exact identities: sqrt(+-0) / c = +-0 for the
+// step's c = sqrt(1 - beta2^t) > 0, and +-0 / denom = +-0 for denom > 0 (0 / 0 and NaN
+// still divide, and give NaN as before).
+__device__ __forceinline__ void adamw_apply_zeros(const AdamScalars &c, float &p, float m, float v)
+{
     const float q = v == 0.0f ? v : __fdiv_rn(__fsqrt_rn(v), c.sqrt_bc2);
     const float denom = __fadd_rn(q, c.eps);
     const float ratio = (m == 0.0f && denom > 0.0f) ? m : __fdiv_rn(m, denom);
-    p = __fsub_rn(pd, __fmul_rn(c.step_size, ratio));
+    p = __fsub_rn(p, __fmul_rn(c.step_size, ratio));
+}
+
+// One element (ragged edges).
+__device__ __forceinline__ void adamw_elem(float s, const AdamScalars &c, float &p, float &m,
+                                           float &v, uint32_t &h)
+{
+    adamw_moments(s, c, p, m, v);
+    adamw_apply_zeros(c, p, m, v);
     h = f2h(p);
+}
+
+// Eight elements.  The branch is decided on the incoming second moments, before any
+// arithmetic: a group where all are nonzero (dense training after its first step: every
+// group) runs the plain straight-line update; a group holding a zero (cold start,
+// untouched or frozen rows) takes the element-wise shortcuts.  Both give the same bits,
+// so the choice only decides speed.
+__device__ __forceinline__ void adamw8(const float *s, const AdamScalars &c, float *p, float *m, float *v,
+                                       uint32_t *h)
+{
+    bool zero = false;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) zero |= v[e] == 0.0f;
+    if (!zero) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            adamw_moments(s[e], c, p[e], m[e], v[e]);
+            adamw_apply(c, p[e], m[e], v[e]);
+            h[e] = f2h(p[e]);
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) adamw_elem(s[e], c, p[e], m[e], v[e], h[e]);
+    }
 }
 
 __device__ __forceinline__ int is_nonfinite(float x) { return !isfinite(x); }

@@ -132,8 +132,7 @@ tile_kernel(TileWork w, int n_ranks, const uint16_t *__restrict__ grads, int64_t
                     float *mf = reinterpret_cast<float *>(m4);
                     float *vf = reinterpret_cast<float *>(v4);
                     uint32_t h[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) adamw_elem(acc[u][e], c, pf[e], mf[e], vf[e], h[e]);
+                    adamw8(acc[u], c, pf, mf, vf, h);
                     __stcs(pp, p4[0]); __stcs(pp + 1, p4[1]);
                     __stcs(mp, m4[0]); __stcs(mp + 1, m4[1]);
                     __stcs(vp, v4[0]); __stcs(vp + 1, v4[1]);
@@ -196,8 +195,7 @@ adamw_range_kernel(int64_t lo, int64_t hi, const float *__restrict__ reduced, fl
         float *mf = reinterpret_cast<float *>(m4);
         float *vf = reinterpret_cast<float *>(v4);
         uint32_t h[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) adamw_elem(rf[e], c, pf[e], mf[e], vf[e], h[e]);
+        adamw8(rf, c, pf, mf, vf, h);
         __stcs(pp, p4[0]); __stcs(pp + 1, p4[1]);
         __stcs(mp, m4[0]); __stcs(mp + 1, m4[1]);
         __stcs(vp, v4[0]); __stcs(vp + 1, v4[1]);
