@@ -140,9 +140,9 @@ def profiled_traffic(workload):
                 continue
             text = open(os.path.join(PROFILE_DIR, name)).read()
             m_sha = re.search(r"kernel_sources_sha256_16:\s*([0-9a-f]+)", text)
-            m_wl = re.search(r"workload:\s*(\S+)", text)
+            m_wl = re.search(r"workload:[ \t]*(.+)", text)
             m_tr = re.search(r"dram_bytes_per_param:\s*([0-9.]+)", text)
-            if m_sha and m_tr and m_wl and m_sha.group(1) == sha and m_wl.group(1) == workload:
+            if m_sha and m_tr and m_wl and m_sha.group(1) == sha and workload in m_wl.group(1).split():
                 return float(m_tr.group(1))
     except Exception:
         pass
