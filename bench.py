@@ -54,6 +54,9 @@ def parse():
                     help="partial sums travel the ring as fp16 (its own line; not the headline)")
     ap.add_argument("--dynamic", action="store_true",
                     help="time zero_step_dynamic (reduce-scatter, overflow check, update) instead of the fused step")
+    ap.add_argument("--dynamic-commit", action="store_true",
+                    help="time zero_step_dynamic_commit (one fused pass into a second state set, overflow "
+                         "check, swap) instead of the fused step")
     ap.add_argument("--zero3-passes", action="store_true",
                     help="time ZeRO-3's per-layer forward and backward gathers with 1-3 prefetch slots "
                          "against a simulated layer compute (its own JSON line)")
@@ -221,6 +224,8 @@ def variant_config(a, wl, world):
         c["ring_partials"] = "fp16 wire"
     if a.dynamic:
         c["step"] = "zero_step_dynamic"
+    if a.dynamic_commit:
+        c["step"] = "zero_step_dynamic_commit"
     if first_cap(a):
         c["max_ctas"] = first_cap(a)
     return c
@@ -349,6 +354,23 @@ def run_ours(a, wl):
             zs.step_dynamic(lay, g, reduced, master, m, v, p16_shard, p16_full, hp(t), scaler, nonfinite)
             if events:
                 events["update_end"].record()
+    elif a.dynamic_commit:
+        # two state sets and two fp16 parameter buffers; an applied step swaps them (the
+        # scale never overflows here, so every step applies)
+        scaler = zs.LossScaler(wl.loss_scale, window=1 << 40)
+        sets = [[master, m, v], [torch.empty_like(master), torch.empty_like(m), torch.empty_like(v)]]
+        p16_sets = [p16_shard if wl.stage == 3 else p16_full, torch.empty_like(p16_full)]
+
+        def one_step(t, events=None):
+            if events:
+                events["update_begin"].record()
+            applied = zs.step_dynamic_commit(lay, g, sets[0], sets[1], p16_sets[1], p16_full, hp(t), scaler,
+                                             nonfinite)
+            if events:
+                events["update_end"].record()
+            if applied:
+                sets.reverse()
+                p16_sets.reverse()
     else:
         def one_step(t, events=None):
             zs.step(lay, g, master, m, v, p16_shard, p16_full, hp(t), nonfinite=nonfinite, events=events)
@@ -381,14 +403,15 @@ def run_ours(a, wl):
     ms = max_over_ranks(start.elapsed_time(end) / K, world, "cuda")
     upd_ms = max_over_ranks(sum(e["update_begin"].elapsed_time(e["update_end"]) for e in ev) / K, world, "cuda")
     gat_ms = None
-    if wl.stage == 3:
+    if wl.stage == 3 and not (a.dynamic or a.dynamic_commit):      # those modes time one bracket
         gat_ms = max_over_ranks(sum(e["gather_begin"].elapsed_time(e["gather_end"]) for e in ev) / K, world, "cuda")
-    launches_per_step = 2 if wl.stage == 3 else 1
+    # our kernels per step: the fused kernel (reduce + update for --dynamic), the gather
+    launches_per_step = (2 if a.dynamic else 1) + (1 if wl.stage == 3 else 0)
 
     # end to end through the host-buffer entry point: gradients from pinned host memory
     # in, fp16 parameters to pinned host memory out, every step
     e2e = None
-    if a.e2e_steps > 0 and not a.dynamic:
+    if a.e2e_steps > 0 and not (a.dynamic or a.dynamic_commit):
         del g
         torch.cuda.empty_cache()
         g_host = torch.empty((N, P), dtype=torch.int16).pin_memory()
@@ -422,10 +445,14 @@ def run_ours(a, wl):
         impl_name += ", fp16 wire"
     if a.dynamic:
         impl_name = "dynamic loss scaling: reduce-scatter + overflow check + update (two passes)"
+    if a.dynamic_commit:
+        impl_name = "dynamic loss scaling, two-phase commit: fused pass into a second state set + overflow check"
     peak, peak_kind = hbm_peak()
     fused_bytes = fused_bytes_per_param(wl) * P
     if a.dynamic:
         fused_bytes = (2 * wl.n_ranks + 4 + 4 + 24 + 2) * P     # reduce pass + update pass
+    if (a.dynamic or a.dynamic_commit) and wl.stage == 3:
+        fused_bytes += 4 * P                                    # the events bracket the gather too
     achieved = fused_bytes / (upd_ms / 1e3) / 1e9
     traffic_pp = profiled_traffic(wl.name)
     step_bytes = ideal_bytes_per_param(wl) * P

@@ -284,6 +284,30 @@ zero_status zero_step_dynamic(const zero_layout *layout, const uint16_t *grads, 
                               uint16_t *p16_full, const zero_adamw_hparams *hp, zero_loss_scaler *scaler,
                               int32_t *nonfinite, int32_t *applied, void *stream);
 
+/* The same step as a two-phase commit: one fused pass (each gradient and state byte
+ * crossing HBM once, as in zero_step) reads the optimizer state from the *_in buffers and
+ * writes the updated state to the *_out buffers and the fp16 parameters to p16_out; the
+ * per-bucket non-finite counts are copied back (the stream is synchronised) and decide:
+ *   *applied = 1: every count is zero; the *_out buffers and p16_out hold the step (for
+ *     stage 3, p16_out is the shard-written buffer and every unit has been gathered from
+ *     it into p16_full).  The caller makes the out set its current state.
+ *   *applied = 0: the *_out buffers and p16_out hold values of a discarded update; the
+ *     *_in buffers, the caller's current fp16 parameters and p16_full are untouched.
+ * The scaler advances as in zero_step_dynamic; loss_scale and step come from it.
+ * Stage 0-2: p16_out is a full fp16 parameter buffer [P] (p16_full unused, may be NULL);
+ * stage 3: p16_out [P] receives the owners' shards, p16_full [P] the gathered result.
+ * Costs the fused step's bytes instead of the reduce-then-update pair of
+ * zero_step_dynamic, for a second state set (12 bytes and 2 for fp16 per parameter).
+ * No in buffer may overlap an out buffer (ZERO_ERR_INVALID).  Bulk-copy pipeline only:
+ * N <= 16.  nonfinite: device int32 [n_buckets], required, zeroed here.  The pages name
+ * no overflow handling; this is the two-phase form of the skip described above. */
+zero_status zero_step_dynamic_commit(const zero_layout *layout, const uint16_t *grads, int64_t rank_stride,
+                                     const float *master_in, const float *m_in, const float *v_in,
+                                     float *master_out, float *m_out, float *v_out, uint16_t *p16_out,
+                                     uint16_t *p16_full, const zero_adamw_hparams *hp,
+                                     zero_loss_scaler *scaler, int32_t *nonfinite, int32_t *applied,
+                                     void *stream);
+
 /* ---- one GPU per rank (the step over NVLink peers) --------------------------------- */
 
 /* zero_step with each rank's gradients in a buffer of its own: rank r's gradient of flat

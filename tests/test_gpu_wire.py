@@ -124,6 +124,80 @@ def test_dynamic_loss_scaling_matches_oracle(wire):
         S.assert_bits_equal(_np(b[k]), want, k)
 
 
+@pytest.mark.parametrize("wire", [False, True])
+@pytest.mark.parametrize("key", ["flat1p3b_n4_zero1", "llama3b_n8_zero3", "ragged2000_n16_zero2"])
+def test_dynamic_commit_matches_oracle(key, wire):
+    """The two-phase commit: state read from one buffer set, written to the other, the
+    sets swapped only on applied steps.  Same skip / apply trace, scaler and final state
+    as the oracle's dynamic run; a skipped step leaves the current set and p16 untouched."""
+    wl = reduced_workloads()[key]
+    olay = S.oracle_layout(wl)
+    P, psi = olay.padded, wl.psi
+    _, master, m, v = S.host_inputs(wl, P)
+    start, steps = 2.0 ** 24, 10
+
+    def grads_at(scale, i):
+        return si.fill_grads(wl.n_ranks, P, psi, wl.seed + i, wl.grad_sigma, scale)
+
+    osc = oracle.LossScaler(start, window=3)
+    ref, trace = oracle.run_steps_dynamic(olay, wl.stage, grads_at, master, m, v, S.hyper(wl), steps, osc,
+                                          wire16=wire)
+    assert any(o for _, o, _ in trace) and not all(o for _, o, _ in trace)
+
+    lay = _layout(wl, zs.IMPL_BULK, wire)
+    b = _bufs(wl, P)
+    cur = (b["master"], b["m"], b["v"])
+    nxt = tuple(torch.full_like(x, float("nan")) for x in cur)
+    # stages 0-2: two full fp16 buffers take turns; stage 3: two shard-written buffers
+    # take turns and p16_full receives the gather of an applied step
+    p16_cur = b["p16_shard"] if wl.stage == 3 else b["p16_full"]
+    p16_nxt = torch.zeros_like(p16_cur)
+    gathered = b["p16_full"] if wl.stage == 3 else None
+    sc = zs.LossScaler(start, window=3)
+    got = []
+    for i in range(steps):
+        used = sc.scale
+        si.fill_grads_cuda(b["g"], psi, wl.seed + i, wl.grad_sigma, used)
+        kept = list(cur) + [p16_cur] + ([gathered] if gathered is not None else [])
+        before = [x.clone() for x in kept]
+        applied = zs.step_dynamic_commit(lay, b["g"], cur, nxt, p16_nxt, gathered, _hp(wl, 1), sc,
+                                         b["nonfinite"])
+        got.append((used, not applied, sc.step if applied else 0))
+        if applied:
+            cur, nxt = nxt, cur
+            p16_cur, p16_nxt = p16_nxt, p16_cur
+        else:
+            for x, y in zip(kept, before):
+                S.assert_bits_equal(_np(x), _np(y), "untouched on a skipped step")
+    torch.cuda.synchronize()
+    zs.get_error(lay)
+    assert got == trace
+    assert (sc.scale, sc.clean_steps, sc.step, sc.skipped) == (osc.scale, osc.clean_steps, osc.step, osc.skipped)
+    for name, x, want in (("master", cur[0], ref.master), ("m", cur[1], ref.m), ("v", cur[2], ref.v),
+                          ("p16_full", gathered if wl.stage == 3 else p16_cur, ref.p16_full)):
+        S.assert_bits_equal(_np(x), want, name)
+
+
+def test_dynamic_commit_rejects_overlap_and_large_n():
+    wl = reduced_workloads()["flat1p3b_n4_zero1"]
+    lay = _layout(wl, zs.IMPL_BULK, False)
+    b = _bufs(wl, lay.padded)
+    st = (b["master"], b["m"], b["v"])
+    sc = zs.LossScaler(1024.0)
+    for out in (st, (b["master"], torch.empty_like(b["m"]), torch.empty_like(b["v"]))):
+        with pytest.raises(zs.ZeroError) as e:
+            zs.step_dynamic_commit(lay, b["g"], st, out, b["p16_shard"], None, _hp(wl, 1), sc, b["nonfinite"])
+        assert e.value.status == 1
+    big = zs.Layout([10_000], 17, 1, 0, 8).to_device()
+    g17 = torch.zeros((17, big.padded), dtype=torch.int16, device="cuda")
+    s17 = [torch.zeros(big.padded, dtype=torch.float32, device="cuda") for _ in range(6)]
+    p17 = torch.zeros(big.padded, dtype=torch.int16, device="cuda")
+    with pytest.raises(zs.ZeroError) as e:
+        zs.step_dynamic_commit(big, g17, s17[:3], s17[3:], p17, None, _hp(wl, 1), sc, b["nonfinite"])
+    assert e.value.status == 1
+    assert (sc.step, sc.skipped) == (0, 0)
+
+
 def test_wire_full_size_sampled():
     wl = full_workloads()["flat1p3b_n4_zero1"]
     olay = S.oracle_layout(wl)

@@ -16,7 +16,7 @@ import numpy as np
 from . import _abi
 
 __all__ = ["ZeroError", "Layout", "AdamW", "reduce_scatter", "adamw_shard_step", "allgather", "gather_unit",
-           "step", "step_bucket", "step_overlapped", "step_dynamic", "LossScaler", "step_host",
+           "step", "step_bucket", "step_overlapped", "step_dynamic", "step_dynamic_commit", "LossScaler", "step_host",
            "step_noalloc", "step_ranks", "step_shard", "copy_shard", "ipc_handle", "ipc_open", "ipc_close",
            "get_error", "IMPL_AUTO", "IMPL_REGISTER", "IMPL_BULK"]
 
@@ -237,6 +237,21 @@ def step_dynamic(layout, grads, reduced, master, m, v, p16_shard, p16_full, hp, 
                                         _ptr(reduced), _ptr(master), _ptr(m), _ptr(v), _ptr(p16_shard),
                                         _ptr(p16_full), ctypes.byref(h), ctypes.byref(scaler.c), _ptr(nonfinite),
                                         ctypes.byref(applied), _stream(stream)), "zero_step_dynamic")
+    return bool(applied.value)
+
+
+def step_dynamic_commit(layout, grads, state_in, state_out, p16_out, p16_full, hp, scaler, nonfinite,
+                        rank_stride=None, stream=None):
+    """zero_step_dynamic_commit: state_in / state_out are (master, m, v) triples.  Returns
+    True if the step was applied (then state_out and p16_out are the new current set)."""
+    h = hp.c()
+    applied = ctypes.c_int32(0)
+    (mi, m_i, vi), (mo, m_o, vo) = state_in, state_out
+    _check(_abi.lib().zero_step_dynamic_commit(layout.handle, _ptr(grads), _stride(grads, layout, rank_stride),
+                                               _ptr(mi), _ptr(m_i), _ptr(vi), _ptr(mo), _ptr(m_o), _ptr(vo),
+                                               _ptr(p16_out), _ptr(p16_full), ctypes.byref(h),
+                                               ctypes.byref(scaler.c), _ptr(nonfinite), ctypes.byref(applied),
+                                               _stream(stream)), "zero_step_dynamic_commit")
     return bool(applied.value)
 
 

@@ -379,40 +379,18 @@ extern "C" zero_status zero_step_overlapped(const zero_layout *L, void *const *r
     return cuda_status(e);
 }
 
-extern "C" zero_status zero_step_dynamic(const zero_layout *L, const uint16_t *grads, int64_t rank_stride,
-                                         float *reduced, float *master, float *m, float *v, uint16_t *p16_shard,
-                                         uint16_t *p16_full, const zero_adamw_hparams *hp, zero_loss_scaler *sc,
-                                         int32_t *nonfinite, int32_t *applied, void *stream)
+namespace {
+
+bool scaler_valid(const zero_loss_scaler *sc)
 {
-    if (!L || !hp || !sc || !applied) return ZERO_ERR_INVALID;
-    if (!(sc->scale > 0.0) || !finite_d(sc->scale) || !(sc->factor > 1.0) || !finite_d(sc->factor) ||
-        sc->window < 1 || !(sc->min_scale > 0.0) || !finite_d(sc->min_scale) || sc->step < 0)
-        return ZERO_ERR_INVALID;
-    zero_adamw_hparams h = *hp;
-    h.loss_scale = sc->scale;
-    h.step = sc->step + 1;
-    zero_status s = check_step(L, grads, rank_stride, master, m, v, p16_shard, p16_full, &h);
-    if (s != ZERO_OK) return s;
-    *applied = 0;
-    if (L->padded == 0) return ZERO_OK;
-    if (!reduced || !nonfinite) return ZERO_ERR_INVALID;
-    if (!aligned16(reduced)) return ZERO_ERR_ALIGN;
-    cudaStream_t st = (cudaStream_t)stream;
-    const size_t nb = L->bucket_lo.size();
-    std::vector<int32_t> counts(nb, 0);
-    cudaError_t e = cudaMemsetAsync(nonfinite, 0, nb * sizeof(int32_t), st);
-    if (e == cudaSuccess) e = zero::launch_reduce_scatter(*L, all_tiles(L), grads, rank_stride, reduced, nonfinite, st);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(counts.data(), nonfinite, nb * sizeof(int32_t), cudaMemcpyDeviceToHost, st);
-    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
-    if (e != cudaSuccess) return ZERO_ERR_CUDA;
-    int64_t bad = 0;
-    for (int32_t c : counts) bad += c;
-    if (bad == 0) {
-        uint16_t *p16 = L->stage == 3 ? p16_shard : p16_full;
-        e = zero::launch_adamw_range(*L, 0, L->padded, reduced, master, m, v, p16, step_scalars(L->n_ranks, h), st);
-        if (e == cudaSuccess && L->stage == 3) e = zero::launch_copy_range(*L, 0, L->padded, p16_shard, p16_full, st);
-        if (e != cudaSuccess) return ZERO_ERR_CUDA;
-        *applied = 1;
+    return sc->scale > 0.0 && finite_d(sc->scale) && sc->factor > 1.0 && finite_d(sc->factor) && sc->window >= 1 &&
+           sc->min_scale > 0.0 && finite_d(sc->min_scale) && sc->step >= 0;
+}
+
+// After a step: an applied one counts towards the growth window; a skipped one backs off.
+void scaler_advance(zero_loss_scaler *sc, bool applied)
+{
+    if (applied) {
         sc->step += 1;
         sc->clean_steps += 1;
         if (sc->clean_steps == sc->window) {
@@ -425,6 +403,104 @@ extern "C" zero_status zero_step_dynamic(const zero_layout *L, const uint16_t *g
         sc->clean_steps = 0;
         sc->skipped += 1;
     }
+}
+
+// The per-bucket counts back on the host (synchronises the stream); their sum.
+cudaError_t total_nonfinite(const zero_layout *L, const int32_t *nonfinite, cudaStream_t st, int64_t *bad)
+{
+    std::vector<int32_t> counts(L->bucket_lo.size(), 0);
+    cudaError_t e = cudaMemcpyAsync(counts.data(), nonfinite, counts.size() * sizeof(int32_t),
+                                    cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    *bad = 0;
+    for (int32_t c : counts) *bad += c;
+    return e;
+}
+
+bool overlaps(const void *a, const void *b, int64_t bytes)
+{
+    const uintptr_t x = (uintptr_t)a, y = (uintptr_t)b;
+    return x < y + (uintptr_t)bytes && y < x + (uintptr_t)bytes;
+}
+
+}  // namespace
+
+extern "C" zero_status zero_step_dynamic(const zero_layout *L, const uint16_t *grads, int64_t rank_stride,
+                                         float *reduced, float *master, float *m, float *v, uint16_t *p16_shard,
+                                         uint16_t *p16_full, const zero_adamw_hparams *hp, zero_loss_scaler *sc,
+                                         int32_t *nonfinite, int32_t *applied, void *stream)
+{
+    if (!L || !hp || !sc || !applied) return ZERO_ERR_INVALID;
+    if (!scaler_valid(sc)) return ZERO_ERR_INVALID;
+    zero_adamw_hparams h = *hp;
+    h.loss_scale = sc->scale;
+    h.step = sc->step + 1;
+    zero_status s = check_step(L, grads, rank_stride, master, m, v, p16_shard, p16_full, &h);
+    if (s != ZERO_OK) return s;
+    *applied = 0;
+    if (L->padded == 0) return ZERO_OK;
+    if (!reduced || !nonfinite) return ZERO_ERR_INVALID;
+    if (!aligned16(reduced)) return ZERO_ERR_ALIGN;
+    cudaStream_t st = (cudaStream_t)stream;
+    const size_t nb = L->bucket_lo.size();
+    int64_t bad = 0;
+    cudaError_t e = cudaMemsetAsync(nonfinite, 0, nb * sizeof(int32_t), st);
+    if (e == cudaSuccess) e = zero::launch_reduce_scatter(*L, all_tiles(L), grads, rank_stride, reduced, nonfinite, st);
+    if (e == cudaSuccess) e = total_nonfinite(L, nonfinite, st, &bad);
+    if (e != cudaSuccess) return ZERO_ERR_CUDA;
+    if (bad == 0) {
+        uint16_t *p16 = L->stage == 3 ? p16_shard : p16_full;
+        e = zero::launch_adamw_range(*L, 0, L->padded, reduced, master, m, v, p16, step_scalars(L->n_ranks, h), st);
+        if (e == cudaSuccess && L->stage == 3) e = zero::launch_copy_range(*L, 0, L->padded, p16_shard, p16_full, st);
+        if (e != cudaSuccess) return ZERO_ERR_CUDA;
+        *applied = 1;
+    }
+    scaler_advance(sc, bad == 0);
+    return ZERO_OK;
+}
+
+extern "C" zero_status zero_step_dynamic_commit(const zero_layout *L, const uint16_t *grads, int64_t rank_stride,
+                                                const float *master_in, const float *m_in, const float *v_in,
+                                                float *master_out, float *m_out, float *v_out, uint16_t *p16_out,
+                                                uint16_t *p16_full, const zero_adamw_hparams *hp,
+                                                zero_loss_scaler *sc, int32_t *nonfinite, int32_t *applied,
+                                                void *stream)
+{
+    if (!L || !hp || !sc || !applied) return ZERO_ERR_INVALID;
+    if (!scaler_valid(sc)) return ZERO_ERR_INVALID;
+    zero_adamw_hparams h = *hp;
+    h.loss_scale = sc->scale;
+    h.step = sc->step + 1;
+    // the out set goes through the usual step checks; the in set is checked alike here
+    zero_status s = check_step(L, grads, rank_stride, master_out, m_out, v_out, p16_out,
+                               L->stage == 3 ? p16_full : p16_out, &h);
+    if (s != ZERO_OK) return s;
+    *applied = 0;
+    if (L->padded == 0) return ZERO_OK;
+    if ((s = check_state(master_in, m_in, v_in)) != ZERO_OK) return s;
+    if (!nonfinite) return ZERO_ERR_INVALID;
+    if (!zero::bulk_supported(L->n_ranks)) return ZERO_ERR_INVALID;
+    const int64_t fb = L->padded * 4;
+    const float *ins[3] = {master_in, m_in, v_in};
+    const float *outs[3] = {master_out, m_out, v_out};
+    for (const float *a : ins)
+        for (const float *b : outs)
+            if (overlaps(a, b, fb)) return ZERO_ERR_INVALID;
+    cudaStream_t st = (cudaStream_t)stream;
+    int64_t bad = 0;
+    cudaError_t e = cudaMemsetAsync(nonfinite, 0, L->bucket_lo.size() * sizeof(int32_t), st);
+    if (e == cudaSuccess)
+        e = zero::launch_bulk_step(*L, all_tiles(L), strided(L, grads, rank_stride), master_out, m_out, v_out, 0,
+                                   p16_out, 0, step_scalars(L->n_ranks, h), nonfinite, L->dev.wait_limit_ns,
+                                   L->dev.skip_first_fill, st, master_in, m_in, v_in);
+    if (e == cudaSuccess) e = total_nonfinite(L, nonfinite, st, &bad);
+    if (e != cudaSuccess) return ZERO_ERR_CUDA;
+    if (bad == 0) {
+        if (L->stage == 3 && zero::launch_copy_range(*L, 0, L->padded, p16_out, p16_full, st) != cudaSuccess)
+            return ZERO_ERR_CUDA;
+        *applied = 1;
+    }
+    scaler_advance(sc, bad == 0);
     return ZERO_OK;
 }
 

@@ -111,7 +111,8 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volati
 struct BulkArgs {
     TileWork w;
     GradSource src;              // rank r's gradient of flat element i: src.rank[r][i]
-    float *master, *mom1, *mom2;  // element i at [i - state_off]
+    const float *master_in, *mom1_in, *mom2_in;  // state read: element i at [i - state_off]
+    float *master, *mom1, *mom2;                 // state written (the same buffers, or a second set)
     int64_t state_off;
     uint16_t *p16;                // element i at [i - p16_off]
     int64_t p16_off;
@@ -175,9 +176,9 @@ __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(co
                     bulk_load(smem_addr(base + (size_t)j * kChunk * 2),
                               A.src.rank[ring_rank(tr.shard, j, N)] + q0, n * 2u, bar);
                 unsigned char *st_base = base + (size_t)N * kChunk * 2;
-                bulk_load(smem_addr(st_base), A.master + (q0 - A.state_off), n * 4u, bar);
-                bulk_load(smem_addr(st_base + kChunk * 4), A.mom1 + (q0 - A.state_off), n * 4u, bar);
-                bulk_load(smem_addr(st_base + kChunk * 8), A.mom2 + (q0 - A.state_off), n * 4u, bar);
+                bulk_load(smem_addr(st_base), A.master_in + (q0 - A.state_off), n * 4u, bar);
+                bulk_load(smem_addr(st_base + kChunk * 4), A.mom1_in + (q0 - A.state_off), n * 4u, bar);
+                bulk_load(smem_addr(st_base + kChunk * 8), A.mom2_in + (q0 - A.state_off), n * 4u, bar);
                 posted = it + 1;
             }
         }
@@ -268,7 +269,7 @@ __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(co
             }
             bad += !isfinite(acc);
             const int64_t si = i - A.state_off;
-            float p = A.master[si], m = A.mom1[si], v = A.mom2[si];
+            float p = A.master_in[si], m = A.mom1_in[si], v = A.mom2_in[si];
             uint32_t h;
             adamw_elem(acc, A.c, p, m, v, h);
             A.master[si] = p;
@@ -312,7 +313,8 @@ bool bulk_supported(int n_ranks) { return n_ranks >= 1 && n_ranks <= 16; }
 cudaError_t launch_bulk_step(const zero_layout &L, const TileWork &w, const GradSource &src, float *master,
                              float *m, float *v, int64_t state_off, uint16_t *p16, int64_t p16_off,
                              const AdamScalars &c, int32_t *nonfinite, uint64_t wait_limit_ns,
-                             int skip_first_fill, cudaStream_t st)
+                             int skip_first_fill, cudaStream_t st, const float *master_in,
+                             const float *m_in, const float *v_in)
 {
     if (w.n_tiles <= 0) return cudaSuccess;
     if ((state_off & 7) != 0 || (p16_off & 7) != 0) return cudaErrorMisalignedAddress;
@@ -322,6 +324,9 @@ cudaError_t launch_bulk_step(const zero_layout &L, const TileWork &w, const Grad
     a.master = master;
     a.mom1 = m;
     a.mom2 = v;
+    a.master_in = master_in ? master_in : master;
+    a.mom1_in = m_in ? m_in : m;
+    a.mom2_in = v_in ? v_in : v;
     a.state_off = state_off;
     a.p16 = p16;
     a.p16_off = p16_off;

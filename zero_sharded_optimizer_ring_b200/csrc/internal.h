@@ -101,10 +101,12 @@ cudaError_t launch_fused_step(const zero_layout &L, const TileWork &w, const uin
 // bulk_step.cu
 bool bulk_supported(int n_ranks);
 // master / m / v hold flat elements [state_off, ...) and p16 [p16_off, ...): element i is
-// at index i - off (both offsets multiples of 8).
+// at index i - off (both offsets multiples of 8).  The state is read from master_in /
+// m_in / v_in where given (same indexing; a second buffer set), else from master / m / v.
 cudaError_t launch_bulk_step(const zero_layout &L, const TileWork &w, const GradSource &src, float *master,
                              float *m, float *v, int64_t state_off, uint16_t *p16, int64_t p16_off,
                              const AdamScalars &c, int32_t *nonfinite, uint64_t wait_limit_ns,
-                             int skip_first_fill, cudaStream_t st);
+                             int skip_first_fill, cudaStream_t st, const float *master_in = nullptr,
+                             const float *m_in = nullptr, const float *v_in = nullptr);
 
 }  // namespace zero
