@@ -189,6 +189,17 @@ zero_status zero_allgather(const zero_layout *layout, int64_t unit, const uint16
 zero_status zero_gather_unit(const zero_layout *layout, int64_t unit, const uint16_t *p16_shard,
                              uint16_t *dst, void *stream);
 
+/* The same gather when every rank keeps only its own shard ([P1] "ZeRO-3" on N GPUs: a
+ * layer's parameters are fetched from the ranks that hold them before its forward and
+ * again before its backward).  rank_p16: host array of N device pointers (N <= 16), rank
+ * k's buffer holding flat elements [k*S, (k+1)*S) of the fp16 parameters (its shard, as
+ * zero_step_shard writes it for stage 3), each 16-byte aligned; they may point into this
+ * GPU's memory or into other GPUs' memory mapped with zero_ipc_open (plain loads over
+ * NVLink).  dst[j] = element unit_lo + j, j < unit_hi - unit_lo; dst 16-byte aligned.
+ * Bit-identical to zero_gather_unit on the concatenated shards. */
+zero_status zero_gather_unit_ranks(const zero_layout *layout, int64_t unit, const uint16_t *const *rank_p16,
+                                   uint16_t *dst, void *stream);
+
 /* One whole optimizer step of the layout's stage: the reduce-scatter of every bucket
  * fused with the shard update, each gradient and state byte crossing HBM once; the
  * reduced sums stay in registers.  Stages 0-2 write the fp16 parameters straight into

@@ -3,9 +3,12 @@
 - zero_step_ranks on separately allocated per-rank gradient buffers equals zero_step;
 - zero_step_shard run for every shard, with shard-local optimizer state, equals zero_step;
 - zero_copy_shard copies exactly the shard's range;
+- zero_gather_unit_ranks, reading each rank's own shard buffer, equals zero_gather_unit
+  (vector and element paths, units across shard edges, 16 ranks);
 - two processes sharing this GPU, each holding one rank's gradients and one shard's
   state, run the multi-GPU step (CUDA IPC mappings, host barriers over gloo; no kernel
-  waits on the other process) and end bit-identical to the oracle.
+  waits on the other process) and end bit-identical to the oracle; for ZeRO-3 each keeps
+  only its parameter shard and gathers every layer from both owners.
 """
 import datetime
 import os
@@ -88,6 +91,43 @@ def test_copy_shard_copies_exactly_the_shard():
         assert int(torch.count_nonzero(dst[:lo])) == 0 and int(torch.count_nonzero(dst[hi:])) == 0
 
 
+@pytest.mark.parametrize("tensors,N,A,units", [
+    ((13, 4099, 8190, 5), 3, 1, (0, 1, 3)),            # S not a multiple of 8: element path
+    ((13, 4099, 8190, 5), 3, 8, (0, 1, 3)),            # unit starts not 8-aligned: element path
+    ((4096, 8192, 40_960, 8), 4, 8, (0, 1, 2, 3)),     # vector path, units across shard edges
+    ((1000,) * 16, 16, 8, tuple(range(16))),
+])
+def test_gather_unit_ranks_equals_gather_unit(tensors, N, A, units):
+    lay = zs.Layout(list(tensors), N, 3, 0, A, list(units)).to_device()
+    P, S_ = lay.padded, lay.shard
+    whole = torch.randint(-30000, 30000, (P,), dtype=torch.int16, device="cuda")
+    shards = [whole[k * S_:(k + 1) * S_].clone() for k in range(N)]          # one allocation per rank
+    _, _, _, u = lay.tables()
+    for j, (lo, hi) in enumerate(u):
+        want = torch.zeros(int(hi - lo), dtype=torch.int16, device="cuda")
+        got = torch.full_like(want, -1)
+        zs.gather_unit(lay, j, whole, want)
+        zs.gather_unit_ranks(lay, j, shards, got)
+        torch.cuda.synchronize()
+        assert torch.equal(got, want) and torch.equal(want, whole[int(lo):int(hi)])
+
+
+def test_gather_unit_ranks_rejects_bad_arguments():
+    lay = zs.Layout([1000] * 17, 17, 3, 0, 8, list(range(17))).to_device()
+    shards = [torch.zeros(lay.shard, dtype=torch.int16, device="cuda") for _ in range(17)]
+    dst = torch.zeros(1000, dtype=torch.int16, device="cuda")
+    for call in (lambda: zs.gather_unit_ranks(lay, 0, shards, dst),          # N > 16
+                 lambda: zs.gather_unit_ranks(lay, 17, shards, dst)):         # no such unit
+        with pytest.raises(zs.ZeroError) as e:
+            call()
+        assert e.value.status == 1
+    lay4 = zs.Layout([1000] * 4, 4, 3, 0, 8, list(range(4))).to_device()
+    s4 = [torch.zeros(lay4.shard + 8, dtype=torch.int16, device="cuda") for _ in range(4)]
+    with pytest.raises(zs.ZeroError) as e:
+        zs.gather_unit_ranks(lay4, 0, [s4[0][1:]] + s4[1:], dst)              # misaligned shard
+    assert e.value.status == 2
+
+
 def _free_port():
     s = socket.socket()
     s.bind(("127.0.0.1", 0))
@@ -106,7 +146,7 @@ def _ipc_worker(rank, world, port, wl, steps, out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120))
     torch.cuda.set_device(0)
-    lay = zs.Layout(list(wl.tensors), world, wl.stage, wl.bucket_elems, wl.pad_align).to_device()
+    lay = zs.Layout(list(wl.tensors), world, wl.stage, wl.bucket_elems, wl.pad_align, list(wl.units)).to_device()
     P, S_ = lay.padded, lay.shard
     g_all = si.fill_grads(world, P, wl.psi, wl.seed, wl.grad_sigma, wl.loss_scale)
     master = si.fill_f32(P, wl.psi, wl.seed, si.STREAM_MASTER, wl.master_sigma)
@@ -115,20 +155,30 @@ def _ipc_worker(rank, world, port, wl, steps, out):
     g = torch.from_numpy(g_all[rank].view(np.int16).copy()).cuda()
     sl = slice(rank * S_, (rank + 1) * S_)
     mk, m1, v1 = (torch.from_numpy(x[sl].copy()).cuda() for x in (master, m, v))
-    p16 = torch.zeros(P, dtype=torch.int16, device="cuda")
+    p16 = torch.zeros(S_ if wl.stage == 3 else P, dtype=torch.int16, device="cuda")   # ZeRO-3: own shard
     torch.cuda.synchronize()
     rs = RankStep(lay, rank, world, g, mk, m1, v1, p16)
     for t in range(1, steps + 1):
         rs.step(zs.AdamW(wl.lr, wl.beta1, wl.beta2, wl.eps, wl.weight_decay, wl.loss_scale, t))
+    full = p16
+    if wl.stage == 3:                   # every layer from its owners, as a forward pass would
+        _, _, _, units = lay.tables()
+        full = torch.cat([torch.zeros(int(hi - lo), dtype=torch.int16, device="cuda") for lo, hi in units])
+        for j, (lo, hi) in enumerate(units):
+            buf = torch.zeros(int(hi - lo), dtype=torch.int16, device="cuda")
+            rs.gather_unit(j, buf)
+            full[int(lo):int(hi)] = buf
+        torch.cuda.synchronize()
     rs.close()
-    out.put((rank, mk.cpu().numpy(), m1.cpu().numpy(), v1.cpu().numpy(), p16.cpu().numpy().view(np.uint16)))
+    out.put((rank, mk.cpu().numpy(), m1.cpu().numpy(), v1.cpu().numpy(), full.cpu().numpy().view(np.uint16)))
     dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("stage", [1, 2])
+@pytest.mark.parametrize("stage", [1, 2, 3])
 def test_two_process_step_over_ipc_matches_oracle(stage):
-    wl = Workload(name="ipc", description="ipc", tensors=(300_007,), units=(), n_ranks=2, stage=stage,
-                  bucket_elems=50_001, steps=3, loss_scale=1024.0, m_sigma=1e-4, v_sigma=1e-6)
+    wl = Workload(name="ipc", description="ipc", tensors=(100_003, 77_777, 122_227), units=(0, 1, 2), n_ranks=2,
+                  stage=stage, bucket_elems=50_001, steps=3, loss_scale=1024.0, m_sigma=1e-4, v_sigma=1e-6,
+                  pad_align=8)
     olay = S.oracle_layout(wl)
     g, master, m, v = S.host_inputs(wl, olay.padded)
     ref = oracle.run_steps(olay, stage, g, master, m, v, S.hyper(wl), wl.steps)

@@ -22,8 +22,8 @@ def _free_port():
 
 
 class FakeLayout:
-    def __init__(self, n, stage=1):
-        self.n_ranks, self.stage = n, stage
+    def __init__(self, n, stage=1, n_units=3):
+        self.n_ranks, self.stage, self.n_units = n, stage, n_units
 
 
 class RecordingOps:
@@ -51,11 +51,14 @@ class RecordingOps:
     def copy_shard(self, layout, shard, src, dst):
         self._rec("gather", shard, src, dst)
 
+    def gather_unit_ranks(self, layout, unit, shards, dst, stream=None):
+        self._rec("unit", unit, tuple(shards), dst)
+
     def sync(self):
         self._rec("barrier")
 
 
-def _worker(rank, world, port, steps, out):
+def _worker(rank, world, port, steps, out, stage=1):
     import datetime
     import torch.distributed as dist
     sys.path.insert(0, ROOT)
@@ -63,10 +66,14 @@ def _worker(rank, world, port, steps, out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     ops = RecordingOps(rank)
-    rs = RankStep(FakeLayout(world), rank, world, "grads", "m0", "m1", "m2", "p16", ops=ops)
+    lay = FakeLayout(world, stage)
+    rs = RankStep(lay, rank, world, "grads", "m0", "m1", "m2", "p16", ops=ops)
     for t in range(steps):
         ops._rec("grads_written", t)
         rs.step(hp=t)
+        if stage == 3:                  # the next forward and backward fetch every layer twice
+            for u in list(range(lay.n_units)) + list(range(lay.n_units))[::-1]:
+                rs.gather_unit(u, f"slot{u % 2}")
     rs.close()
     out.put(ops.log)
     dist.destroy_process_group()
@@ -106,3 +113,34 @@ def test_multigpu_step_protocol(world):
             assert nxt > max(e[0] for e in step_gathers)
     closes = [e for e in ev if e[2] == "close"]
     assert len(closes) == world * 2 * (world - 1)
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_multigpu_zero3_protocol(world):
+    """ZeRO-3: no third phase; every layer is gathered from all owners' shards, after every
+    owner has written its shard for the step and before any owner writes it again."""
+    steps = 3
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, steps, q, 3)) for r in range(world)]
+    for p in procs:
+        p.start()
+    logs = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    ev = sorted(e for log in logs for e in log)
+    assert not [e for e in ev if e[2] == "gather"]                   # no full-buffer copies
+    units = [e for e in ev if e[2] == "unit"]
+    assert len(units) == steps * world * 2 * 3
+    for e in units:                                                   # every owner's shard, mapped
+        assert e[4] == tuple("p16" if r == e[1] else f"mapped:p16@{r}" for r in range(world))
+    for t in range(steps):
+        updates = [e for e in ev if e[2] == "update" and e[5] == t]
+        assert sorted((e[1], e[3]) for e in updates) == [(r, r) for r in range(world)]
+        step_units = units[t * world * 6:(t + 1) * world * 6]
+        assert min(e[0] for e in step_units) > max(e[0] for e in updates)   # after every shard is written
+        if t + 1 < steps:
+            nxt = [e for e in ev if e[2] == "update" and e[5] == t + 1]
+            assert max(e[0] for e in step_units) < min(e[0] for e in nxt)   # before any is rewritten

@@ -15,7 +15,7 @@ import numpy as np
 
 from . import _abi
 
-__all__ = ["ZeroError", "Layout", "AdamW", "reduce_scatter", "adamw_shard_step", "allgather", "gather_unit",
+__all__ = ["ZeroError", "Layout", "AdamW", "reduce_scatter", "adamw_shard_step", "allgather", "gather_unit", "gather_unit_ranks",
            "step", "step_bucket", "step_overlapped", "step_dynamic", "step_dynamic_commit", "LossScaler", "step_host",
            "step_noalloc", "step_ranks", "step_shard", "copy_shard", "ipc_handle", "ipc_open", "ipc_close",
            "get_error", "IMPL_AUTO", "IMPL_REGISTER", "IMPL_BULK"]
@@ -171,6 +171,13 @@ def gather_unit(layout, unit, p16_shard, dst, stream=None):
     """Unit `unit`'s fp16 parameters, contiguous, into dst (zero_gather_unit)."""
     _check(_abi.lib().zero_gather_unit(layout.handle, int(unit), _ptr(p16_shard), _ptr(dst), _stream(stream)),
            "zero_gather_unit")
+
+
+def gather_unit_ranks(layout, unit, rank_p16, dst, stream=None):
+    """Unit `unit`'s fp16 parameters into dst from the ranks' own shard buffers
+    (zero_gather_unit_ranks); rank_p16[k]: tensor or device address of rank k's shard."""
+    _check(_abi.lib().zero_gather_unit_ranks(layout.handle, int(unit), _ptr_array(rank_p16), _ptr(dst),
+                                             _stream(stream)), "zero_gather_unit_ranks")
 
 
 def step(layout, grads, master, m, v, p16_shard, p16_full, hp, nonfinite=None, events=None,

@@ -80,6 +80,7 @@ SIGNATURES = {
     "zero_ipc_get_handle": (_i32, [_vp, _vp, ctypes.POINTER(_i64)]),
     "zero_ipc_open": (_i32, [_vp, _i64, ctypes.POINTER(_vp)]),
     "zero_ipc_close": (_i32, [_vp, _i64]),
+    "zero_gather_unit_ranks": (_i32, [_vp, _i64, _vp, _vp, _vp]),
     "zero_set_impl": (_i32, [_vp, _i32]),
     "zero_set_max_ctas": (_i32, [_vp, _i32]),
     "zero_debug_set_wait": (_i32, [_vp, _i64, _i32]),

@@ -6,6 +6,7 @@
 #include <mutex>
 #include <vector>
 
+#include "gather_ranks.h"
 #include "internal.h"
 
 using zero::AdamScalars;
@@ -275,6 +276,25 @@ extern "C" zero_status zero_gather_unit(const zero_layout *L, int64_t unit, cons
     const int64_t lo = L->unit_lo[(size_t)unit];
     return cuda_status(zero::launch_gather_unit(p16_shard, lo, L->unit_hi[(size_t)unit] - lo, dst,
                                                 (cudaStream_t)stream));
+}
+
+extern "C" zero_status zero_gather_unit_ranks(const zero_layout *L, int64_t unit, const uint16_t *const *rank_p16,
+                                              uint16_t *dst, void *stream)
+{
+    zero_status s = check_device(L);
+    if (s != ZERO_OK) return s;
+    if (unit < 0 || unit >= (int64_t)L->unit_lo.size() || !rank_p16 || !dst) return ZERO_ERR_INVALID;
+    if (L->n_ranks > zero::kMaxBulkRanks) return ZERO_ERR_INVALID;
+    zero::ShardPtrs src = {};
+    for (int r = 0; r < L->n_ranks; ++r) {
+        if (!rank_p16[r]) return ZERO_ERR_INVALID;
+        if (!aligned16(rank_p16[r])) return ZERO_ERR_ALIGN;
+        src.rank[r] = rank_p16[r];
+    }
+    if (!aligned16(dst)) return ZERO_ERR_ALIGN;
+    const int64_t lo = L->unit_lo[(size_t)unit];
+    return cuda_status(zero::launch_gather_ranks(src, L->shard, lo, L->unit_hi[(size_t)unit] - lo, dst,
+                                                 (cudaStream_t)stream));
 }
 
 namespace {

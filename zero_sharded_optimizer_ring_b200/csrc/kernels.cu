@@ -18,6 +18,7 @@
 #include <stdint.h>
 
 #include "device_common.cuh"
+#include "gather_ranks.h"
 
 namespace zero {
 namespace {
@@ -283,6 +284,48 @@ gather_unit_kernel(const uint16_t *__restrict__ src, int64_t lo, int64_t n, uint
     }
 }
 
+// Gather of one unit from the ranks' shard buffers: dst[j] = shard k's element lo + j - kS,
+// k = (lo + j) / S, where rank k's buffer holds flat elements [kS, (k+1)S) (on this GPU or a
+// peer's).  With lo and S multiples of 8 no 16-byte vector straddles two shards, so each
+// thread moves 4 vectors, every source and destination 16-byte aligned; otherwise each
+// thread moves 8 scalars.  A grid of short blocks, as for the copy.
+__global__ void __launch_bounds__(kThreads)
+gather_ranks_kernel(const __grid_constant__ ShardPtrs src, int64_t S, int64_t lo, int64_t n,
+                    uint16_t *__restrict__ dst)
+{
+    if ((lo & 7) == 0 && (S & 7) == 0) {
+        const int64_t nv = n / kVec;
+        const int64_t base = (int64_t)blockIdx.x * kThreads * kCopyUnroll;
+        uint4 x[kCopyUnroll];
+#pragma unroll
+        for (int u = 0; u < kCopyUnroll; ++u) {
+            const int64_t q = base + (int64_t)u * kThreads + threadIdx.x;
+            if (q < nv) {
+                const int64_t i = lo + q * kVec, k = i / S;
+                x[u] = *reinterpret_cast<const uint4 *>(src.rank[k] + (i - k * S));
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kCopyUnroll; ++u) {
+            const int64_t q = base + (int64_t)u * kThreads + threadIdx.x;
+            if (q < nv) *reinterpret_cast<uint4 *>(dst + q * kVec) = x[u];
+        }
+        if (blockIdx.x == 0 && threadIdx.x < n - nv * kVec) {
+            const int64_t j = nv * kVec + threadIdx.x, i = lo + j, k = i / S;
+            dst[j] = src.rank[k][i - k * S];
+        }
+    } else {
+        const int64_t base = (int64_t)blockIdx.x * kThreads * kCopyUnroll * kVec;
+        for (int u = 0; u < kCopyUnroll * kVec; ++u) {
+            const int64_t j = base + (int64_t)u * kThreads + threadIdx.x;
+            if (j < n) {
+                const int64_t i = lo + j, k = i / S;
+                dst[j] = src.rank[k][i - k * S];
+            }
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------------
 // Tile index: one warp scans the segments' tile counts (exclusive prefix sum with
 // __shfl_up_sync, 32 segments per pass, carried across passes).  Row n_seg receives
@@ -366,6 +409,15 @@ cudaError_t launch_gather_unit(const uint16_t *src, int64_t lo, int64_t n, uint1
     if (n <= 0) return cudaSuccess;
     const int64_t per_block = (int64_t)kThreads * kCopyUnroll * kVec;
     gather_unit_kernel<<<(unsigned)((n + per_block - 1) / per_block), kThreads, 0, s>>>(src, lo, n, dst);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather_ranks(const ShardPtrs &src, int64_t S, int64_t lo, int64_t n, uint16_t *dst,
+                                cudaStream_t s)
+{
+    if (n <= 0) return cudaSuccess;
+    const int64_t per_block = (int64_t)kThreads * kCopyUnroll * kVec;
+    gather_ranks_kernel<<<(unsigned)((n + per_block - 1) / per_block), kThreads, 0, s>>>(src, S, lo, n, dst);
     return cudaGetLastError();
 }
 
