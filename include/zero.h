@@ -345,6 +345,28 @@ zero_status zero_step_shard(const zero_layout *layout, int32_t shard, const uint
                             float *master_k, float *m_k, float *v_k, uint16_t *p16_out,
                             const zero_adamw_hparams *hp, int32_t *nonfinite, void *stream);
 
+/* zero_step_shard as the first phase of a two-phase commit under dynamic loss scaling
+ * (see zero_step_dynamic_commit): the shard's state is read from *_in and the step
+ * written to *_out (each [S], no in buffer overlapping an out buffer) and the fp16
+ * parameters to p16_out (laid out as for zero_step_shard; the caller keeps a second
+ * parameter buffer for it); loss_scale and step come from the scaler, which is NOT
+ * advanced.  Clears and fills nonfinite (device int32 [n_buckets], required), synchronises
+ * the stream and stores the shard's count of non-finite reduced gradients in
+ * *nonfinite_total (host).  The step must be kept or dropped on every rank alike: the
+ * caller sums the ranks' counts (one all-reduce of an integer), then advances every
+ * rank's scaler with zero_loss_scaler_advance and, if the sum is zero, makes the out
+ * buffers current everywhere.  N <= 16, S % 8 == 0. */
+zero_status zero_step_shard_commit(const zero_layout *layout, int32_t shard, const uint16_t *const *rank_grads,
+                                   const float *master_in, const float *m_in, const float *v_in,
+                                   float *master_out, float *m_out, float *v_out, uint16_t *p16_out,
+                                   const zero_adamw_hparams *hp, const zero_loss_scaler *scaler,
+                                   int32_t *nonfinite, int64_t *nonfinite_total, void *stream);
+
+/* Advance the scaler after a step: applied = 1 counts towards the growth window, 0 backs
+ * the scale off (the rules of zero_loss_scaler).  For callers that decide the step
+ * themselves (zero_step_shard_commit on several ranks). */
+zero_status zero_loss_scaler_advance(zero_loss_scaler *scaler, int32_t applied);
+
 /* dst[i] = src[i] for i in shard `shard`'s range [kS, (k+1)S): the all-gather of the
  * fp16 parameters when src is the owning GPU's full buffer, mapped with zero_ipc_open
  * (P1 ZeRO-1 broadcast step).  Both flat-indexed fp16 [P], 16-byte aligned. */

@@ -203,3 +203,97 @@ def test_two_process_step_over_ipc_matches_oracle(stage):
         S.assert_bits_equal(m1, ref.m[sl], f"m shard {rank}")
         S.assert_bits_equal(v1, ref.v[sl], f"v shard {rank}")
         S.assert_bits_equal(p16, ref.p16_full, f"p16 on rank {rank}")
+
+
+def _ipc_dyn_worker(rank, world, port, wl, steps, start, out):
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import seeded_inputs as si
+    import zero_sharded_optimizer_ring_b200 as zs
+    from zero_sharded_optimizer_ring_b200.multigpu import RankStep
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(0)
+    lay = zs.Layout(list(wl.tensors), world, wl.stage, wl.bucket_elems, wl.pad_align, list(wl.units)).to_device()
+    P, S_ = lay.padded, lay.shard
+    master = si.fill_f32(P, wl.psi, wl.seed, si.STREAM_MASTER, wl.master_sigma)
+    m = si.fill_f32(P, wl.psi, wl.seed, si.STREAM_M, wl.m_sigma)
+    v = si.fill_f32(P, wl.psi, wl.seed, si.STREAM_V, wl.v_sigma, True)
+    sl = slice(rank * S_, (rank + 1) * S_)
+    state = [torch.from_numpy(x[sl].copy()).cuda() for x in (master, m, v)]
+    spare = [torch.full((S_,), float("nan"), device="cuda") for _ in range(3)]
+    n16 = S_ if wl.stage == 3 else P
+    p16 = torch.zeros(n16, dtype=torch.int16, device="cuda")
+    p16b = torch.zeros(n16, dtype=torch.int16, device="cuda")
+    g = torch.zeros(P, dtype=torch.int16, device="cuda")
+    nf = torch.zeros(lay.n_buckets, dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    rs = RankStep(lay, rank, world, g, *state, p16, spare=(*spare, p16b))
+    sc = zs.LossScaler(start, window=3)
+    trace = []
+    hp = zs.AdamW(wl.lr, wl.beta1, wl.beta2, wl.eps, wl.weight_decay, 1.0, 1)
+    for i in range(steps):
+        used = sc.scale
+        g_all = si.fill_grads(world, P, wl.psi, wl.seed + i, wl.grad_sigma, used)
+        g.copy_(torch.from_numpy(g_all[rank].view(np.int16).copy()).cuda())
+        torch.cuda.synchronize()
+        applied = rs.step_dynamic(hp, sc, nf)
+        trace.append((used, not applied, sc.step if applied else 0))
+    full = rs.p16
+    if wl.stage == 3:
+        _, _, _, units = lay.tables()
+        full = torch.zeros(P, dtype=torch.int16, device="cuda")
+        for j, (lo, hi) in enumerate(units):
+            buf = torch.zeros(int(hi - lo), dtype=torch.int16, device="cuda")
+            rs.gather_unit(j, buf)
+            full[int(lo):int(hi)] = buf
+    torch.cuda.synchronize()
+    out.put((rank, trace, (sc.scale, sc.clean_steps, sc.step, sc.skipped), [x.cpu().numpy() for x in rs.state],
+             full.cpu().numpy().view(np.uint16)))
+    rs.close()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("stage", [1, 2, 3])
+def test_two_process_dynamic_commit_matches_oracle(stage):
+    """Dynamic loss scaling with one process per rank: both processes take the oracle's
+    skip / apply sequence (one shard's overflow skips the step on both) and end with the
+    oracle's scaler, state shards and fp16 parameters."""
+    wl = Workload(name="ipcdyn", description="ipc dynamic", tensors=(100_003, 77_777, 122_227), units=(0, 1, 2),
+                  n_ranks=2, stage=stage, bucket_elems=50_001, steps=8, loss_scale=1.0, m_sigma=1e-4,
+                  v_sigma=1e-6, pad_align=8)
+    olay = S.oracle_layout(wl)
+    P, psi = olay.padded, wl.psi
+    _, master, m, v = S.host_inputs(wl, P)
+    start = 2.0 ** 24
+
+    def grads_at(scale, i):
+        return si.fill_grads(2, P, psi, wl.seed + i, wl.grad_sigma, scale)
+
+    osc = oracle.LossScaler(start, window=3)
+    ref, trace = oracle.run_steps_dynamic(olay, stage, grads_at, master, m, v, S.hyper(wl), wl.steps, osc)
+    assert any(o for _, o, _ in trace) and not all(o for _, o, _ in trace)
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_ipc_dyn_worker, args=(r, 2, port, wl, wl.steps, start, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    try:
+        res = sorted([q.get(timeout=300) for _ in range(2)], key=lambda x: x[0])
+    finally:
+        for p in procs:
+            p.join(60)
+            if p.exitcode is None:
+                p.kill()
+    assert all(p.exitcode == 0 for p in procs)
+    S_ = olay.shard
+    for rank, got_trace, scaler, (mk, m1, v1), p16 in res:
+        assert got_trace == trace
+        assert scaler == (osc.scale, osc.clean_steps, osc.step, osc.skipped)
+        sl = slice(rank * S_, (rank + 1) * S_)
+        S.assert_bits_equal(mk, ref.master[sl], f"master shard {rank}")
+        S.assert_bits_equal(m1, ref.m[sl], f"m shard {rank}")
+        S.assert_bits_equal(v1, ref.v[sl], f"v shard {rank}")
+        S.assert_bits_equal(p16, ref.p16_full, f"p16 on rank {rank}")

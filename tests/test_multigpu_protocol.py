@@ -144,3 +144,88 @@ def test_multigpu_zero3_protocol(world):
         if t + 1 < steps:
             nxt = [e for e in ev if e[2] == "update" and e[5] == t + 1]
             assert max(e[0] for e in step_units) < min(e[0] for e in nxt)   # before any is rewritten
+
+
+class DynamicOps(RecordingOps):
+    """RecordingOps plus the commit step: shard `bad_at[0]` reports an overflow at step
+    `bad_at[1]`; the all-reduce is a real one over the gloo group."""
+
+    def __init__(self, rank, bad_at):
+        super().__init__(rank)
+        self.bad_at = bad_at
+        self.t = 0
+
+    def step_shard_commit(self, layout, shard, rank_grads, state_in, state_out, p16_out, hp, scaler, nonfinite):
+        self._rec("commit", shard, state_in, state_out, p16_out)
+        return 5 if (shard, self.t) == self.bad_at else 0
+
+    def all_reduce_sum(self, x, group=None):
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([x], dtype=torch.int64)
+        dist.all_reduce(t, group=group)
+        self._rec("allreduce", int(t.item()))
+        return int(t.item())
+
+    def advance(self, scaler, applied):
+        scaler.append(applied)
+        self._rec("advance", applied)
+
+
+def _dyn_worker(rank, world, port, steps, bad_at, out):
+    import datetime
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from zero_sharded_optimizer_ring_b200.multigpu import RankStep
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    ops = DynamicOps(rank, bad_at)
+    rs = RankStep(FakeLayout(world), rank, world, "grads", "a0", "a1", "a2", "p16a", ops=ops,
+                  spare=("b0", "b1", "b2", "p16b"))
+    decisions = []
+    for t in range(steps):
+        ops.t = t
+        ops._rec("grads_written", t)
+        rs.step_dynamic(hp=t, scaler=decisions, nonfinite="nf")
+        ops._rec("current", rs.state, rs.p16)
+    rs.close()
+    out.put((rank, decisions, ops.log))
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_multigpu_dynamic_commit_protocol(world):
+    """One shard overflows at step 1: every rank skips that step (same decision, no
+    gathers, the current set unchanged); every applied step reads the current set, writes
+    the other one, swaps everywhere and gathers the owners' new buffers."""
+    steps, bad_at = 4, (world - 1, 1)
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_dyn_worker, args=(r, world, port, steps, bad_at, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted([q.get(timeout=120) for _ in range(world)], key=lambda x: x[0])
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    want = [True, False, True, True]
+    for rank, decisions, log in res:
+        assert decisions == want                                      # the same decision everywhere
+        commits = [e for e in log if e[2] == "commit"]
+        currents = [e for e in log if e[2] == "current"]
+        cur = ("a0", "a1", "a2"), "p16a"
+        other = {"a": (("b0", "b1", "b2"), "p16b"), "b": (("a0", "a1", "a2"), "p16a")}
+        for t, applied in enumerate(want):
+            c = commits[t]
+            assert c[3] == rank and c[4] == cur[0]                   # reads the current set
+            nxt = other[cur[1][-1]]
+            assert (c[5], c[6]) == nxt                                # writes the other one
+            if applied:
+                cur = nxt
+            assert (currents[t][3], currents[t][4]) == cur
+        gathers = [e for e in log if e[2] == "gather"]
+        assert len(gathers) == (world - 1) * sum(want)                # none for the skipped step
+        for e in gathers:
+            assert e[4].startswith("mapped:p16") and e[5] in ("p16a", "p16b") and e[4].endswith(f"@{e[3]}")
+            assert e[4][len("mapped:"):].split("@")[0] == e[5]        # from the owners' current buffer

@@ -17,7 +17,7 @@ from . import _abi
 
 __all__ = ["ZeroError", "Layout", "AdamW", "reduce_scatter", "adamw_shard_step", "allgather", "gather_unit", "gather_unit_ranks",
            "step", "step_bucket", "step_overlapped", "step_dynamic", "step_dynamic_commit", "LossScaler", "step_host",
-           "step_noalloc", "step_ranks", "step_shard", "copy_shard", "ipc_handle", "ipc_open", "ipc_close",
+           "step_noalloc", "step_ranks", "step_shard", "step_shard_commit", "copy_shard", "ipc_handle", "ipc_open", "ipc_close",
            "get_error", "IMPL_AUTO", "IMPL_REGISTER", "IMPL_BULK"]
 
 IMPL_AUTO, IMPL_REGISTER, IMPL_BULK = 0, 1, 2
@@ -226,13 +226,19 @@ def step_overlapped(layout, ready_events, grads, master, m, v, p16_shard, p16_fu
 
 
 class LossScaler:
-    """Dynamic loss scaling state (zero_loss_scaler); advanced by step_dynamic()."""
+    """Dynamic loss scaling state (zero_loss_scaler); advanced by step_dynamic() and
+    step_dynamic_commit(), or by advance() where the caller decides the step."""
 
     def __init__(self, scale, factor=2.0, window=1000, min_scale=1.0):
         self.c = _abi.LossScaler(float(scale), float(factor), int(window), float(min_scale), 0, 0, 0)
 
     def __getattr__(self, name):
         return getattr(self.__dict__["c"], name)
+
+    def advance(self, applied):
+        """zero_loss_scaler_advance: count an applied step, or back off after a skipped one."""
+        _check(_abi.lib().zero_loss_scaler_advance(ctypes.byref(self.c), int(bool(applied))),
+               "zero_loss_scaler_advance")
 
 
 def step_dynamic(layout, grads, reduced, master, m, v, p16_shard, p16_full, hp, scaler, nonfinite,
@@ -305,6 +311,22 @@ def step_shard(layout, shard, rank_grads, master_k, m_k, v_k, p16_out, hp, nonfi
     _check(_abi.lib().zero_step_shard(layout.handle, int(shard), _ptr_array(rank_grads), _ptr(master_k), _ptr(m_k),
                                       _ptr(v_k), _ptr(p16_out), ctypes.byref(h), _ptr(nonfinite), _stream(stream)),
            "zero_step_shard")
+
+
+def step_shard_commit(layout, shard, rank_grads, state_in, state_out, p16_out, hp, scaler, nonfinite,
+                      stream=None):
+    """zero_step_shard_commit: shard `shard`'s update from state_in into state_out ((master,
+    m, v) triples of [S] buffers) at the scaler's scale and step; returns the shard's count
+    of non-finite reduced gradients (the stream is synchronised).  The scaler is not
+    advanced: the ranks decide together."""
+    h = hp.c()
+    total = ctypes.c_int64(0)
+    (mi, m_i, vi), (mo, m_o, vo) = state_in, state_out
+    _check(_abi.lib().zero_step_shard_commit(layout.handle, int(shard), _ptr_array(rank_grads), _ptr(mi), _ptr(m_i),
+                                             _ptr(vi), _ptr(mo), _ptr(m_o), _ptr(vo), _ptr(p16_out), ctypes.byref(h),
+                                             ctypes.byref(scaler.c), _ptr(nonfinite), ctypes.byref(total),
+                                             _stream(stream)), "zero_step_shard_commit")
+    return int(total.value)
 
 
 def copy_shard(layout, shard, src, dst, stream=None):

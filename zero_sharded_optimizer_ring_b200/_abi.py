@@ -76,6 +76,10 @@ SIGNATURES = {
     "zero_step_noalloc": (_i32, [_vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(AdamWHparams), _vp, _vp]),
     "zero_step_ranks": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(AdamWHparams), _vp, _vp]),
     "zero_step_shard": (_i32, [_vp, _i32, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(AdamWHparams), _vp, _vp]),
+    "zero_step_shard_commit": (_i32, [_vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                      ctypes.POINTER(AdamWHparams), ctypes.POINTER(LossScaler), _vp,
+                                      ctypes.POINTER(_i64), _vp]),
+    "zero_loss_scaler_advance": (_i32, [ctypes.POINTER(LossScaler), _i32]),
     "zero_copy_shard": (_i32, [_vp, _i32, _vp, _vp, _vp]),
     "zero_ipc_get_handle": (_i32, [_vp, _vp, ctypes.POINTER(_i64)]),
     "zero_ipc_open": (_i32, [_vp, _i64, ctypes.POINTER(_vp)]),

@@ -598,6 +598,54 @@ extern "C" zero_status zero_step_shard(const zero_layout *L, int32_t shard, cons
                                               L->dev.wait_limit_ns, L->dev.skip_first_fill, (cudaStream_t)stream));
 }
 
+extern "C" zero_status zero_step_shard_commit(const zero_layout *L, int32_t shard, const uint16_t *const *rank_grads,
+                                              const float *master_in, const float *m_in, const float *v_in,
+                                              float *master_out, float *m_out, float *v_out, uint16_t *p16_out,
+                                              const zero_adamw_hparams *hp, const zero_loss_scaler *sc,
+                                              int32_t *nonfinite, int64_t *nonfinite_total, void *stream)
+{
+    if (!L || !hp || !sc || !nonfinite_total) return ZERO_ERR_INVALID;
+    if (!scaler_valid(sc)) return ZERO_ERR_INVALID;
+    zero_status s = check_device(L);
+    if (s != ZERO_OK) return s;
+    zero_adamw_hparams h = *hp;
+    h.loss_scale = sc->scale;
+    h.step = sc->step + 1;
+    if ((s = check_hparams(&h)) != ZERO_OK) return s;
+    if (shard < 0 || shard >= L->n_ranks) return ZERO_ERR_INVALID;
+    *nonfinite_total = 0;
+    if (L->padded == 0) return ZERO_OK;
+    if (L->shard % 8 != 0) return ZERO_ERR_ALIGN;
+    zero::GradSource src;
+    if ((s = rank_source(L, rank_grads, &src)) != ZERO_OK) return s;
+    if ((s = check_state(master_in, m_in, v_in)) != ZERO_OK) return s;
+    if ((s = check_state(master_out, m_out, v_out)) != ZERO_OK) return s;
+    if (!p16_out || !nonfinite) return ZERO_ERR_INVALID;
+    if (!aligned16(p16_out)) return ZERO_ERR_ALIGN;
+    const int64_t fb = L->shard * 4;
+    const float *ins[3] = {master_in, m_in, v_in};
+    const float *outs[3] = {master_out, m_out, v_out};
+    for (const float *a : ins)
+        for (const float *b : outs)
+            if (overlaps(a, b, fb)) return ZERO_ERR_INVALID;
+    cudaStream_t st = (cudaStream_t)stream;
+    const int64_t off = (int64_t)shard * L->shard;
+    cudaError_t e = cudaMemsetAsync(nonfinite, 0, L->bucket_lo.size() * sizeof(int32_t), st);
+    if (e == cudaSuccess)
+        e = zero::launch_bulk_step(*L, shard_tiles(L, shard), src, master_out, m_out, v_out, off, p16_out,
+                                   L->stage == 3 ? off : 0, step_scalars(L->n_ranks, h), nonfinite,
+                                   L->dev.wait_limit_ns, L->dev.skip_first_fill, st, master_in, m_in, v_in);
+    if (e == cudaSuccess) e = total_nonfinite(L, nonfinite, st, nonfinite_total);
+    return cuda_status(e);
+}
+
+extern "C" zero_status zero_loss_scaler_advance(zero_loss_scaler *sc, int32_t applied)
+{
+    if (!sc || !scaler_valid(sc) || applied < 0 || applied > 1) return ZERO_ERR_INVALID;
+    scaler_advance(sc, applied == 1);
+    return ZERO_OK;
+}
+
 extern "C" zero_status zero_copy_shard(const zero_layout *L, int32_t shard, const uint16_t *src, uint16_t *dst,
                                        void *stream)
 {

@@ -20,6 +20,13 @@ step then runs three phases, each closed by a host barrier:
 
 No kernel waits on another GPU: the barriers are host-side, after a device
 synchronisation, so each kernel only reads peer memory that is complete and stable.
+
+Under dynamic loss scaling (step_dynamic) every rank keeps a second state set and a
+second parameter buffer.  Phase 2 becomes the first half of a two-phase commit: the
+owner writes its shard's step into the spare set (zero_step_shard_commit) and counts the
+non-finite reduced gradients; one all-reduce of that integer (the only exchange this
+adds) gives every rank the same decision, after which all scalers advance alike and,
+if no shard overflowed, every rank makes the spare set current and phase 3 follows.
 """
 
 
@@ -53,6 +60,21 @@ class CudaOps:
     def gather_unit_ranks(self, layout, unit, shards, dst, stream=None):
         self.zs.gather_unit_ranks(layout, unit, [self._addr(p) for p in shards], dst, stream=stream)
 
+    def step_shard_commit(self, layout, shard, rank_grads, state_in, state_out, p16_out, hp, scaler, nonfinite):
+        return self.zs.step_shard_commit(layout, shard, [self._addr(g) for g in rank_grads], state_in, state_out,
+                                         p16_out, hp, scaler, nonfinite)
+
+    def all_reduce_sum(self, x, group=None):
+        import torch
+        import torch.distributed as dist
+        dev = "cuda" if dist.get_backend(group) == "nccl" else "cpu"
+        t = torch.tensor([int(x)], dtype=torch.int64, device=dev)
+        dist.all_reduce(t, group=group)
+        return int(t.item())
+
+    def advance(self, scaler, applied):
+        scaler.advance(applied)
+
     def sync(self):
         import torch
         torch.cuda.synchronize()
@@ -61,29 +83,48 @@ class CudaOps:
 class RankStep:
     """One rank's share of the multi-GPU step (see the module docstring)."""
 
-    def __init__(self, layout, rank, world, grads, master_k, m_k, v_k, p16, group=None, ops=None):
+    def __init__(self, layout, rank, world, grads, master_k, m_k, v_k, p16, group=None, ops=None, spare=None):
         """p16: the full fp16 parameters [P] (stages 0-2) or this rank's shard of them [S]
-        (stage 3)."""
+        (stage 3).  spare: (master_k, m_k, v_k, p16) of the same shapes, the second set
+        that step_dynamic() needs."""
         import torch.distributed as dist
         if layout.n_ranks != world:
             raise ValueError("the layout's rank count must equal the world size")
         self.dist, self.group = dist, group
         self.layout, self.rank, self.world = layout, rank, world
         self.ops = ops or CudaOps()
-        self.grads, self.state, self.p16 = grads, (master_k, m_k, v_k), p16
-        mine = (rank, self.ops.export(grads), self.ops.export(p16))
+        self.grads = grads
+        self.sets = [((master_k, m_k, v_k), p16)]
+        if spare is not None:
+            self.sets.append((tuple(spare[:3]), spare[3]))
+        self.cur = 0
+        mine = (rank, self.ops.export(grads), [self.ops.export(p) for _, p in self.sets])
         everyone = [None] * world
         dist.all_gather_object(everyone, mine, group=group)
         self.opened = []
         self.peer_grads = [None] * world
-        self.peer_p16 = [None] * world
-        for r, hg, hp16 in everyone:
+        self.peer_p16 = [[None] * world for _ in self.sets]       # [set][rank]
+        for r, hg, hps in everyone:
             if r == rank:
-                self.peer_grads[r], self.peer_p16[r] = grads, p16
+                self.peer_grads[r] = grads
+                for s, (_, p) in enumerate(self.sets):
+                    self.peer_p16[s][r] = p
             else:
                 self.peer_grads[r] = self.ops.open(hg)
-                self.peer_p16[r] = self.ops.open(hp16)
-                self.opened += [self.peer_grads[r], self.peer_p16[r]]
+                self.opened.append(self.peer_grads[r])
+                for s, h in enumerate(hps):
+                    self.peer_p16[s][r] = self.ops.open(h)
+                    self.opened.append(self.peer_p16[s][r])
+
+    @property
+    def state(self):
+        """The current (master, m, v) of this rank's shard."""
+        return self.sets[self.cur][0]
+
+    @property
+    def p16(self):
+        """The current fp16 parameters (full, or this rank's shard for stage 3)."""
+        return self.sets[self.cur][1]
 
     def _barrier(self):
         self.ops.sync()
@@ -93,11 +134,31 @@ class RankStep:
         self._barrier()                                     # 1: all gradients written
         self.ops.step_shard(self.layout, self.rank, self.peer_grads, *self.state, self.p16, hp, nonfinite)
         self._barrier()                                     # 2: every shard updated
+        self._gather_all()
+
+    def step_dynamic(self, hp, scaler, nonfinite):
+        """One step under dynamic loss scaling (the gradients carry scaler.scale); returns
+        True if it was applied on every rank, False if some shard overflowed and every
+        rank skipped it.  nonfinite: device int32 [n_buckets] scratch."""
+        if len(self.sets) < 2:
+            raise ValueError("step_dynamic needs the spare buffer set")
+        self._barrier()                                     # 1: all gradients written
+        nxt = 1 - self.cur
+        bad = self.ops.step_shard_commit(self.layout, self.rank, self.peer_grads, self.sets[self.cur][0],
+                                         self.sets[nxt][0], self.sets[nxt][1], hp, scaler, nonfinite)
+        applied = self.ops.all_reduce_sum(bad, self.group) == 0   # 2: every rank's shard counted
+        self.ops.advance(scaler, applied)
+        if applied:
+            self.cur = nxt
+            self._gather_all()
+        return applied
+
+    def _gather_all(self):
         if self.layout.stage == 3:
             return                                          # layers are gathered when used
         for j in range(self.world):
             if j != self.rank:
-                self.ops.copy_shard(self.layout, j, self.peer_p16[j], self.p16)
+                self.ops.copy_shard(self.layout, j, self.peer_p16[self.cur][j], self.p16)
         self._barrier()                                     # 3: parameters gathered everywhere
 
     def gather_unit(self, unit, dst, stream=None):
@@ -106,7 +167,7 @@ class RankStep:
         before its backward)."""
         if self.layout.stage != 3:
             raise ValueError("stages 0-2 keep the full parameters in p16")
-        self.ops.gather_unit_ranks(self.layout, unit, self.peer_p16, dst, stream)
+        self.ops.gather_unit_ranks(self.layout, unit, self.peer_p16[self.cur], dst, stream)
 
     def close(self):
         """Unmap the peers' buffers (before the process group or the buffers go away)."""
