@@ -72,6 +72,9 @@ def parse():
     ap.add_argument("--max-ctas", default="0",
                     help="cap on the fused kernel's CTAs (zero_set_max_ctas; 0 = one per SM). With --overlap "
                          "a comma-separated list, one JSON line each")
+    ap.add_argument("--bucket-group", default="1",
+                    help="--overlap: buckets per launch (zero_step_overlapped_grouped); a comma-separated list, "
+                         "one JSON line each")
     ap.add_argument("--shrink", type=int, default=0,
                     help="divide every tensor of the workload by this factor (same structure, smaller: "
                          "small cases for profiler captures; not a bench line)")
@@ -540,21 +543,22 @@ def run_overlap(a, wl):
 
     t = 0
     reps = max(3, a.steps // 20)
+    groups = [int(x) for x in str(a.bucket_group).split(",")]
     if a.backward == "gemm":
-        runs = [("default", 0, cap) for cap in caps]
+        runs = [("default", 0, cap, grp) for cap in caps for grp in groups]
     else:
-        runs = [("default", 0, caps[0]), ("high", hi_pri, caps[0])]
-    for prio_name, prio, cap in runs:
+        runs = [("default", 0, caps[0], grp) for grp in groups] + [("high", hi_pri, caps[0], groups[0])]
+    for prio_name, prio, cap, grp in runs:
         lay.set_max_ctas(cap)
         producer, compute = torch.cuda.Stream(), torch.cuda.Stream(priority=prio)
         make = gemm_backward if a.backward == "gemm" else generator_backward
         t = _overlap_reps(a, wl, lay, g, master, m, v, p16_shard, p16_full, make(producer), producer,
-                          compute, ev, reps, t, prio_name, cap)
+                          compute, ev, reps, t, prio_name, cap, grp)
     zs.get_error(lay)
 
 
 def _overlap_reps(a, wl, lay, g, master, m, v, p16_shard, p16_full, backward, producer, compute, ev, reps, t,
-                  prio_name, cap):
+                  prio_name, cap, group):
     import torch
     import zero_sharded_optimizer_ring_b200 as zs
 
@@ -580,7 +584,7 @@ def _overlap_reps(a, wl, lay, g, master, m, v, p16_shard, p16_full, backward, pr
         s2, e2 = ev(), ev()
         s2.record(producer)
         backward(ready)
-        zs.step_overlapped(lay, ready, g, master, m, v, p16_shard, p16_full, hp(), stream=compute)
+        zs.step_overlapped(lay, ready, g, master, m, v, p16_shard, p16_full, hp(), stream=compute, group=group)
         e2.record(compute)
         torch.cuda.synchronize()
         if rep >= a.warmup:
@@ -590,7 +594,8 @@ def _overlap_reps(a, wl, lay, g, master, m, v, p16_shard, p16_full, backward, pr
     tb, ts, tp = (statistics.median(res[k]) for k in ("bwd", "step", "pipe"))
     print(json.dumps({
         "metric": "bucket-pipelined step behind a simulated backward (overlap)", "workload": wl.name,
-        "backward": a.backward, "compute_stream_priority": prio_name, "max_ctas": cap, "buckets": lay.n_buckets,
+        "backward": a.backward, "compute_stream_priority": prio_name, "max_ctas": cap, "bucket_group": group,
+        "buckets": lay.n_buckets,
         "reps": reps, "t_backward_ms": tb, "t_step_ms": ts, "t_pipelined_ms": tp, "exposed_step_ms": tp - tb,
         "overlap_efficiency": (tb + ts - tp) / ts,
         **({"backward_tflops": backward.tflop / (tb / 1e3)} if hasattr(backward, "tflop") else {}),

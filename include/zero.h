@@ -236,6 +236,18 @@ zero_status zero_step_overlapped(const zero_layout *layout, void *const *ready_e
                                  float *v, uint16_t *p16_shard, uint16_t *p16_full,
                                  const zero_adamw_hparams *hp, int32_t *nonfinite, void *stream);
 
+/* zero_step_overlapped with one launch per `group` consecutive buckets (group >= 1; the
+ * last group may be shorter): `stream` waits for the ready events of all the group's
+ * buckets, then runs their fused update as one kernel.  With many small buckets (a
+ * bucket of 10^6 parameters is ~9 us of work at full bandwidth) this trades a later
+ * start for fewer launches interleaved with the backward pass.  group = 1 is
+ * zero_step_overlapped.  Same results.  No counterpart on the pages (their buckets are
+ * the launch unit). */
+zero_status zero_step_overlapped_grouped(const zero_layout *layout, void *const *ready_events, int64_t group,
+                                         const uint16_t *grads, int64_t rank_stride, float *master, float *m,
+                                         float *v, uint16_t *p16_shard, uint16_t *p16_full,
+                                         const zero_adamw_hparams *hp, int32_t *nonfinite, void *stream);
+
 /* zero_step for gradients that live in HOST memory (page-locked), with the fp16
  * parameters returned to host memory: per bucket, the N gradient slices are copied to
  * the device staging buffer grads_dev on an internal copy stream, the bucket's fused

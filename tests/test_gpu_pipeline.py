@@ -62,8 +62,9 @@ def test_step_bucket_equals_step(key, order):
     _same(a, b)
 
 
+@pytest.mark.parametrize("group", [1, 3, 1000])
 @pytest.mark.parametrize("key", ["flat1p3b_n4_zero1", "llama3b_n8_zero3", "ragged2000_n16_zero2"])
-def test_overlapped_step_with_simulated_backward(key):
+def test_overlapped_step_with_simulated_backward(key, group):
     wl = reduced_workloads()[key]
     lay, bufs = _setup(wl)
     a, b = bufs(), bufs()
@@ -81,7 +82,7 @@ def test_overlapped_step_with_simulated_backward(key):
                                      wl.heavy_frac, wl.heavy_mult, cuda_stream=producer.cuda_stream)
             ready[bk].record(producer)
         zs.step_overlapped(lay, ready, b["g"], b["master"], b["m"], b["v"], b["p16_shard"], b["p16_full"],
-                           _hp(wl, t), nonfinite=b["nonfinite"], stream=consumer)
+                           _hp(wl, t), nonfinite=b["nonfinite"], stream=consumer, group=group)
     zs.get_error(lay)
     _same(a, b)
 
@@ -95,3 +96,9 @@ def test_overlapped_rejects_unrecorded_events():
                            b["v"], None, b["p16_full"], _hp(wl, 1))
     with pytest.raises(zs.ZeroError):
         zs.step_bucket(lay, lay.n_buckets, b["g"], b["master"], b["m"], b["v"], None, b["p16_full"], _hp(wl, 1))
+    ready = [torch.cuda.Event() for _ in range(lay.n_buckets)]
+    for e in ready:
+        e.record()
+    with pytest.raises(zs.ZeroError) as err:
+        zs.step_overlapped(lay, ready, b["g"], b["master"], b["m"], b["v"], None, b["p16_full"], _hp(wl, 1), group=0)
+    assert err.value.status == 1

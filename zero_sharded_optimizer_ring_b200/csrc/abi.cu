@@ -67,17 +67,21 @@ TileWork all_tiles(const zero_layout *L)
     return w;
 }
 
-TileWork bucket_tiles(const zero_layout *L, int64_t b)
+// The tiles of buckets [b0, b1): consecutive buckets' segments, and so their tiles, are
+// contiguous in the bucket-major table.
+TileWork bucket_range_tiles(const zero_layout *L, int64_t b0, int64_t b1)
 {
     TileWork w;
     w.segs = L->dev.segs;
-    w.seg_first = L->bucket_seg_begin[(size_t)b];
-    const int64_t seg_end = L->bucket_seg_begin[(size_t)b + 1];
+    w.seg_first = L->bucket_seg_begin[(size_t)b0];
+    const int64_t seg_end = L->bucket_seg_begin[(size_t)b1];
     w.tile_first = L->segs[(size_t)w.seg_first].tile_begin;
     const int64_t tile_end = seg_end < (int64_t)L->segs.size() ? L->segs[(size_t)seg_end].tile_begin : L->n_tiles;
     w.n_tiles = tile_end - w.tile_first;
     return w;
 }
+
+TileWork bucket_tiles(const zero_layout *L, int64_t b) { return bucket_range_tiles(L, b, b + 1); }
 
 zero_status check_grads(const zero_layout *L, const void *grads, int64_t rank_stride)
 {
@@ -376,27 +380,40 @@ extern "C" zero_status zero_step_bucket(const zero_layout *L, int64_t bucket, co
                              step_scalars(L->n_ranks, *hp), nonfinite, (cudaStream_t)stream));
 }
 
-extern "C" zero_status zero_step_overlapped(const zero_layout *L, void *const *ready_events, const uint16_t *grads,
-                                            int64_t rank_stride, float *master, float *m, float *v,
-                                            uint16_t *p16_shard, uint16_t *p16_full, const zero_adamw_hparams *hp,
-                                            int32_t *nonfinite, void *stream)
+extern "C" zero_status zero_step_overlapped_grouped(const zero_layout *L, void *const *ready_events, int64_t group,
+                                                    const uint16_t *grads, int64_t rank_stride, float *master, float *m,
+                                                    float *v, uint16_t *p16_shard, uint16_t *p16_full,
+                                                    const zero_adamw_hparams *hp, int32_t *nonfinite, void *stream)
 {
     zero_status s = check_step(L, grads, rank_stride, master, m, v, p16_shard, p16_full, hp);
-    if (s != ZERO_OK || L->padded == 0) return s;
+    if (s != ZERO_OK) return s;
+    if (group < 1) return ZERO_ERR_INVALID;
+    if (L->padded == 0) return ZERO_OK;
     if (!ready_events) return ZERO_ERR_INVALID;
-    for (size_t b = 0; b < L->bucket_lo.size(); ++b)
+    const int64_t nb = (int64_t)L->bucket_lo.size();
+    for (int64_t b = 0; b < nb; ++b)
         if (!ready_events[b]) return ZERO_ERR_INVALID;
     cudaStream_t st = (cudaStream_t)stream;
     const AdamScalars c = step_scalars(L->n_ranks, *hp);
     uint16_t *p16 = L->stage == 3 ? p16_shard : p16_full;
     cudaError_t e = cudaSuccess;
-    for (size_t b = 0; e == cudaSuccess && b < L->bucket_lo.size(); ++b) {
-        e = cudaStreamWaitEvent(st, (cudaEvent_t)ready_events[b], 0);
+    for (int64_t b0 = 0; e == cudaSuccess && b0 < nb; b0 += group) {
+        const int64_t b1 = b0 + group < nb ? b0 + group : nb;
+        for (int64_t b = b0; e == cudaSuccess && b < b1; ++b) e = cudaStreamWaitEvent(st, (cudaEvent_t)ready_events[b], 0);
         if (e == cudaSuccess)
-            e = fused(L, bucket_tiles(L, (int64_t)b), grads, rank_stride, master, m, v, p16, c, nonfinite, st);
+            e = fused(L, bucket_range_tiles(L, b0, b1), grads, rank_stride, master, m, v, p16, c, nonfinite, st);
     }
     if (e == cudaSuccess && L->stage == 3) e = zero::launch_copy_range(*L, 0, L->padded, p16_shard, p16_full, st);
     return cuda_status(e);
+}
+
+extern "C" zero_status zero_step_overlapped(const zero_layout *L, void *const *ready_events, const uint16_t *grads,
+                                            int64_t rank_stride, float *master, float *m, float *v,
+                                            uint16_t *p16_shard, uint16_t *p16_full, const zero_adamw_hparams *hp,
+                                            int32_t *nonfinite, void *stream)
+{
+    return zero_step_overlapped_grouped(L, ready_events, 1, grads, rank_stride, master, m, v, p16_shard, p16_full,
+                                        hp, nonfinite, stream);
 }
 
 namespace {
