@@ -6,7 +6,8 @@
   oracle's per-element path;
 - edge cases: one rank, unaligned segment edges (shard rounding 1), one-element
   buckets, a rank count without a compiled specialisation, empty layouts, non-finite
-  gradients, per-bucket / per-shard / per-unit calls, the host-buffer step.
+  gradients, zero and -0 operands, capped grids, a flat buffer of more than 2^32
+  elements, per-bucket / per-shard / per-unit calls, the host-buffer step.
 """
 import numpy as np
 import pytest
@@ -371,6 +372,32 @@ def test_full_size_sampled(key, impl):
     # the padding stayed zero
     assert int(torch.count_nonzero(b["p16_full"][lay.psi:])) == 0
     assert int(torch.count_nonzero(b["master"][lay.psi:])) == 0
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_flat_buffer_beyond_2_32_elements(impl):
+    """ψ just above 2^32 (N=2, full fp32 state: 86 GB on the device): element indices,
+    byte offsets and tile numbers past 32 bits, sampled against the oracle, including
+    every element around 2^31 and 2^32 and the shard edge."""
+    wl = Workload(name="beyond32", description="beyond 2^32", tensors=((1 << 32) + 4097,), units=(), n_ranks=2,
+                  stage=1, bucket_elems=1_000_000_007, steps=2, loss_scale=1024.0, m_sigma=1e-4, v_sigma=1e-6)
+    olay = S.oracle_layout(wl)
+    lay = _layout(wl, impl)
+    assert lay.padded > (1 << 32) and lay.n_tiles > (1 << 20)
+    b = _bufs(lay, wl)
+    _run(lay, wl, b, wl.steps)
+    near = [c + d for c in (1 << 31, 1 << 32, olay.shard) for d in range(-9, 10)]
+    idx = np.unique(np.concatenate([S.sample_indices(olay), np.array(near, np.int64)]))
+    it = torch.from_numpy(idx).cuda()
+    red_ref, master, m, v, p16 = S.sampled_oracle(wl, olay, idx, wl.steps)
+    for k, want in (("master", master), ("m", m), ("v", v), ("p16_full", p16)):
+        S.assert_bits_equal(_np(b[k][it]), want, k)
+    assert int(b["nonfinite"].sum()) == 0
+    del b["m"], b["v"], b["p16_shard"]
+    red = torch.empty(lay.padded, dtype=torch.float32, device="cuda")
+    zs.reduce_scatter(lay, -1, b["g"], red)
+    S.assert_bits_equal(_np(red[it]), red_ref, "reduced")
+    assert int(torch.count_nonzero(b["p16_full"][lay.psi:])) == 0
 
 
 def test_bulk_pipeline_bounded_wait_reports_timeout():
