@@ -117,3 +117,37 @@ def test_tuning_setters_validate_arguments():
         with pytest.raises(zs.ZeroError) as e:
             bad()
         assert e.value.status == 1
+
+
+DEVICE_CALLS = ["zero_reduce_scatter", "zero_adamw_shard_step", "zero_allgather", "zero_gather_unit",
+                "zero_gather_unit_ranks", "zero_step", "zero_step_bucket", "zero_step_overlapped",
+                "zero_step_overlapped_grouped", "zero_step_dynamic", "zero_step_dynamic_commit", "zero_step_host",
+                "zero_step_ranks", "zero_step_shard", "zero_step_shard_commit", "zero_copy_shard",
+                "zero_layout_device_segments", "zero_get_error", "zero_debug_set_wait"]
+
+
+@pytest.mark.parametrize("name", DEVICE_CALLS)
+def test_device_calls_refuse_a_layout_not_on_the_device(name):
+    """Every device entry point checks its layout (and arguments) before any CUDA call:
+    with a layout never uploaded it returns INVALID or STATE here, where no GPU exists
+    (a CUDA call would have answered ZERO_ERR_CUDA).  zero_step_noalloc is the one entry
+    that needs no upload, so it is not in the list."""
+    lay = zs.Layout([1000, 24], 2, 1, 100)
+    fn = getattr(_abi.lib(), name)
+    hp = _abi.AdamWHparams(1e-3, 0.9, 0.999, 1e-8, 0.0, 1.0, 1)
+    sc = _abi.LossScaler(1024.0, 2.0, 10, 1.0, 0, 0, 0)
+    args = []
+    for t in fn.argtypes:
+        if t is _abi.ctypes.POINTER(_abi.AdamWHparams):
+            args.append(ctypes.byref(hp))
+        elif t is _abi.ctypes.POINTER(_abi.LossScaler):
+            args.append(ctypes.byref(sc))
+        elif t in (ctypes.c_int32, ctypes.c_int64):
+            args.append(0)
+        elif t is ctypes.c_void_p:
+            args.append(None)
+        else:
+            args.append(t())                                # a NULL pointer of that type
+    args[0] = lay.handle
+    assert fn(*args) in (1, 6), name                       # ZERO_ERR_INVALID or ZERO_ERR_STATE
+    assert (sc.step, sc.skipped) == (0, 0)
