@@ -321,8 +321,9 @@ zero_status zero_step_dynamic(const zero_layout *layout, const uint16_t *grads, 
  * stage 3: p16_out [P] receives the owners' shards, p16_full [P] the gathered result.
  * Costs the fused step's bytes instead of the reduce-then-update pair of
  * zero_step_dynamic, for a second state set (12 bytes and 2 for fp16 per parameter).
- * No in buffer may overlap an out buffer (ZERO_ERR_INVALID).  Bulk-copy pipeline only:
- * N <= 16.  nonfinite: device int32 [n_buckets], required, zeroed here.  The pages name
+ * No in buffer may overlap an out buffer (ZERO_ERR_INVALID).  Either implementation
+ * (zero_set_impl; register streaming for N > 16).  nonfinite: device int32 [n_buckets],
+ * required, zeroed here.  The pages name
  * no overflow handling; this is the two-phase form of the skip described above. */
 zero_status zero_step_dynamic_commit(const zero_layout *layout, const uint16_t *grads, int64_t rank_stride,
                                      const float *master_in, const float *m_in, const float *v_in,

@@ -124,13 +124,25 @@ def test_dynamic_loss_scaling_matches_oracle(wire):
         S.assert_bits_equal(_np(b[k]), want, k)
 
 
-@pytest.mark.parametrize("wire", [False, True])
-@pytest.mark.parametrize("key", ["flat1p3b_n4_zero1", "llama3b_n8_zero3", "ragged2000_n16_zero2"])
-def test_dynamic_commit_matches_oracle(key, wire):
+def _commit_cases():
+    red = reduced_workloads()
+    cases = [(k, w, impl) for k in ("flat1p3b_n4_zero1", "llama3b_n8_zero3", "ragged2000_n16_zero2")
+             for w in (False, True) for impl in (zs.IMPL_BULK, zs.IMPL_REGISTER)]
+    return cases + [("ragged_n17", w, zs.IMPL_AUTO) for w in (False, True)]
+
+
+def _commit_workload(key):
+    if key == "ragged_n17":                 # no pipeline specialisation: register streaming
+        return reduced_workloads()["ragged2000_n16_zero2"].with_(n_ranks=17)
+    return reduced_workloads()[key]
+
+
+@pytest.mark.parametrize("key,wire,impl", _commit_cases())
+def test_dynamic_commit_matches_oracle(key, wire, impl):
     """The two-phase commit: state read from one buffer set, written to the other, the
     sets swapped only on applied steps.  Same skip / apply trace, scaler and final state
     as the oracle's dynamic run; a skipped step leaves the current set and p16 untouched."""
-    wl = reduced_workloads()[key]
+    wl = _commit_workload(key)
     olay = S.oracle_layout(wl)
     P, psi = olay.padded, wl.psi
     _, master, m, v = S.host_inputs(wl, P)
@@ -144,7 +156,7 @@ def test_dynamic_commit_matches_oracle(key, wire):
                                           wire16=wire)
     assert any(o for _, o, _ in trace) and not all(o for _, o, _ in trace)
 
-    lay = _layout(wl, zs.IMPL_BULK, wire)
+    lay = _layout(wl, impl, wire)
     b = _bufs(wl, P)
     cur = (b["master"], b["m"], b["v"])
     nxt = tuple(torch.full_like(x, float("nan")) for x in cur)
@@ -178,7 +190,7 @@ def test_dynamic_commit_matches_oracle(key, wire):
         S.assert_bits_equal(_np(x), want, name)
 
 
-def test_dynamic_commit_rejects_overlap_and_large_n():
+def test_dynamic_commit_rejects_overlapping_sets():
     wl = reduced_workloads()["flat1p3b_n4_zero1"]
     lay = _layout(wl, zs.IMPL_BULK, False)
     b = _bufs(wl, lay.padded)
@@ -188,13 +200,6 @@ def test_dynamic_commit_rejects_overlap_and_large_n():
         with pytest.raises(zs.ZeroError) as e:
             zs.step_dynamic_commit(lay, b["g"], st, out, b["p16_shard"], None, _hp(wl, 1), sc, b["nonfinite"])
         assert e.value.status == 1
-    big = zs.Layout([10_000], 17, 1, 0, 8).to_device()
-    g17 = torch.zeros((17, big.padded), dtype=torch.int16, device="cuda")
-    s17 = [torch.zeros(big.padded, dtype=torch.float32, device="cuda") for _ in range(6)]
-    p17 = torch.zeros(big.padded, dtype=torch.int16, device="cuda")
-    with pytest.raises(zs.ZeroError) as e:
-        zs.step_dynamic_commit(big, g17, s17[:3], s17[3:], p17, None, _hp(wl, 1), sc, b["nonfinite"])
-    assert e.value.status == 1
     assert (sc.step, sc.skipped) == (0, 0)
 
 

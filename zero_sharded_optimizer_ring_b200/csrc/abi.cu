@@ -516,7 +516,6 @@ extern "C" zero_status zero_step_dynamic_commit(const zero_layout *L, const uint
     if (L->padded == 0) return ZERO_OK;
     if ((s = check_state(master_in, m_in, v_in)) != ZERO_OK) return s;
     if (!nonfinite) return ZERO_ERR_INVALID;
-    if (!zero::bulk_supported(L->n_ranks)) return ZERO_ERR_INVALID;
     const int64_t fb = L->padded * 4;
     const float *ins[3] = {master_in, m_in, v_in};
     const float *outs[3] = {master_out, m_out, v_out};
@@ -526,10 +525,14 @@ extern "C" zero_status zero_step_dynamic_commit(const zero_layout *L, const uint
     cudaStream_t st = (cudaStream_t)stream;
     int64_t bad = 0;
     cudaError_t e = cudaMemsetAsync(nonfinite, 0, L->bucket_lo.size() * sizeof(int32_t), st);
-    if (e == cudaSuccess)
+    const bool bulk = (L->impl == 2 || L->impl == 0) && zero::bulk_supported(L->n_ranks);
+    if (e == cudaSuccess && bulk)
         e = zero::launch_bulk_step(*L, all_tiles(L), strided(L, grads, rank_stride), master_out, m_out, v_out, 0,
                                    p16_out, 0, step_scalars(L->n_ranks, h), nonfinite, L->dev.wait_limit_ns,
                                    L->dev.skip_first_fill, st, master_in, m_in, v_in);
+    else if (e == cudaSuccess)
+        e = zero::launch_fused_step_to(*L, all_tiles(L), grads, rank_stride, master_in, m_in, v_in, master_out,
+                                       m_out, v_out, p16_out, step_scalars(L->n_ranks, h), nonfinite, st);
     if (e == cudaSuccess) e = total_nonfinite(L, nonfinite, st, &bad);
     if (e != cudaSuccess) return ZERO_ERR_CUDA;
     if (bad == 0) {

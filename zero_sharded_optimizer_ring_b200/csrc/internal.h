@@ -97,6 +97,12 @@ cudaError_t launch_gather_unit(const uint16_t *src, int64_t lo, int64_t n, uint1
 cudaError_t launch_fused_step(const zero_layout &L, const TileWork &w, const uint16_t *grads,
                               int64_t stride, float *master, float *m, float *v, uint16_t *p16,
                               const AdamScalars &c, int32_t *nonfinite, cudaStream_t s);
+// The same update out of place (register streaming, any N): state read from *_in,
+// written to master / m / v (buffers that do not overlap the in set).
+cudaError_t launch_fused_step_to(const zero_layout &L, const TileWork &w, const uint16_t *grads,
+                                 int64_t stride, const float *master_in, const float *m_in, const float *v_in,
+                                 float *master, float *m, float *v, uint16_t *p16, const AdamScalars &c,
+                                 int32_t *nonfinite, cudaStream_t s);
 
 // bulk_step.cu
 bool bulk_supported(int n_ranks);

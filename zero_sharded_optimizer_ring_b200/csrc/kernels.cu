@@ -46,14 +46,23 @@ __device__ __forceinline__ float fold_scalar(const uint16_t *__restrict__ grads,
 // Tile kernel: ring reduce-scatter of every tile of the launch, then either the
 // fused shard update (kFused) or a store of the fp32 sums.
 //   NT = compile-time rank count (0 = runtime n_ranks), U = vectors per thread whose
-//   loads are in flight together, kWire = fp16 wire (partials rounded to fp16 per hop).
-template <int NT, int U, bool kFused, bool kWire>
+//   loads are in flight together, kWire = fp16 wire (partials rounded to fp16 per hop),
+//   kOut = the fused update reads the state from `in` and writes it to master / mom1 /
+//   mom2 (two buffer sets that do not overlap); otherwise it updates them in place.
+struct StateIn {
+    const float *master, *mom1, *mom2;
+};
+
+template <int NT, int U, bool kFused, bool kWire, bool kOut = false>
 __global__ void __launch_bounds__(kThreads)
 tile_kernel(TileWork w, int n_ranks, const uint16_t *__restrict__ grads, int64_t stride,
             float *__restrict__ reduced, float *__restrict__ master, float *__restrict__ mom1,
             float *__restrict__ mom2, uint16_t *__restrict__ p16, AdamScalars c,
-            int32_t *__restrict__ nonfinite)
+            int32_t *__restrict__ nonfinite, StateIn in)
 {
+    const float *__restrict__ master_in = kOut ? in.master : master;
+    const float *__restrict__ mom1_in = kOut ? in.mom1 : mom1;
+    const float *__restrict__ mom2_in = kOut ? in.mom2 : mom2;
     const int n = NT > 0 ? NT : n_ranks;
     int64_t s = w.seg_first;
     const int64_t t_end = w.tile_first + w.n_tiles;
@@ -126,9 +135,12 @@ tile_kernel(TileWork w, int n_ranks, const uint16_t *__restrict__ grads, int64_t
                     float4 *pp = reinterpret_cast<float4 *>(master + q);
                     float4 *mp = reinterpret_cast<float4 *>(mom1 + q);
                     float4 *vp = reinterpret_cast<float4 *>(mom2 + q);
-                    float4 p4[2] = {__ldcs(pp), __ldcs(pp + 1)};
-                    float4 m4[2] = {__ldcs(mp), __ldcs(mp + 1)};
-                    float4 v4[2] = {__ldcs(vp), __ldcs(vp + 1)};
+                    const float4 *pi = reinterpret_cast<const float4 *>(master_in + q);
+                    const float4 *mi = reinterpret_cast<const float4 *>(mom1_in + q);
+                    const float4 *vi = reinterpret_cast<const float4 *>(mom2_in + q);
+                    float4 p4[2] = {__ldcs(pi), __ldcs(pi + 1)};
+                    float4 m4[2] = {__ldcs(mi), __ldcs(mi + 1)};
+                    float4 v4[2] = {__ldcs(vi), __ldcs(vi + 1)};
                     float *pf = reinterpret_cast<float *>(p4);
                     float *mf = reinterpret_cast<float *>(m4);
                     float *vf = reinterpret_cast<float *>(v4);
@@ -157,7 +169,7 @@ tile_kernel(TileWork w, int n_ranks, const uint16_t *__restrict__ grads, int64_t
             const float acc = fold_scalar<kWire>(grads, stride, k, n, i);
             bad += is_nonfinite(acc);
             if constexpr (kFused) {
-                float p = master[i], m = mom1[i], v = mom2[i];
+                float p = master_in[i], m = mom1_in[i], v = mom2_in[i];
                 uint32_t h;
                 adamw_elem(acc, c, p, m, v, h);
                 master[i] = p;
@@ -374,7 +386,8 @@ cudaError_t launch_tiles(const zero_layout &L, const TileWork &w, const uint16_t
 {
     auto kern = L.wire16 ? tile_kernel<NT, U, kFused, true> : tile_kernel<NT, U, kFused, false>;
     const int grid = grid_for(kern, w.n_tiles, L.dev.num_sms, L.max_ctas);
-    kern<<<grid, kThreads, 0, st>>>(w, L.n_ranks, grads, stride, reduced, master, m, v, p16, c, nonfinite);
+    kern<<<grid, kThreads, 0, st>>>(w, L.n_ranks, grads, stride, reduced, master, m, v, p16, c, nonfinite,
+                                    StateIn{nullptr, nullptr, nullptr});
     return cudaGetLastError();
 }
 
@@ -439,6 +452,19 @@ cudaError_t launch_fused_step(const zero_layout &L, const TileWork &w, const uin
                               const AdamScalars &c, int32_t *nonfinite, cudaStream_t s)
 {
     return dispatch_tiles<true>(L, w, grads, stride, nullptr, master, m, v, p16, c, nonfinite, s);
+}
+
+cudaError_t launch_fused_step_to(const zero_layout &L, const TileWork &w, const uint16_t *grads,
+                                 int64_t stride, const float *master_in, const float *m_in, const float *v_in,
+                                 float *master, float *m, float *v, uint16_t *p16, const AdamScalars &c,
+                                 int32_t *nonfinite, cudaStream_t s)
+{
+    if (w.n_tiles <= 0) return cudaSuccess;
+    auto kern = L.wire16 ? tile_kernel<0, 1, true, true, true> : tile_kernel<0, 1, true, false, true>;
+    const int grid = grid_for(kern, w.n_tiles, L.dev.num_sms, L.max_ctas);
+    kern<<<grid, kThreads, 0, s>>>(w, L.n_ranks, grads, stride, nullptr, master, m, v, p16, c, nonfinite,
+                                   StateIn{master_in, m_in, v_in});
+    return cudaGetLastError();
 }
 
 cudaError_t launch_adamw_range(const zero_layout &L, int64_t lo, int64_t hi, const float *reduced,
