@@ -229,3 +229,44 @@ def test_multigpu_dynamic_commit_protocol(world):
         for e in gathers:
             assert e[4].startswith("mapped:p16") and e[5] in ("p16a", "p16b") and e[4].endswith(f"@{e[3]}")
             assert e[4][len("mapped:"):].split("@")[0] == e[5]        # from the owners' current buffer
+
+
+def _dying_worker(rank, world, port, out):
+    import datetime
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from zero_sharded_optimizer_ring_b200.multigpu import RankStep
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=10))
+    ops = RecordingOps(rank)
+    rs = RankStep(FakeLayout(world), rank, world, "grads", "m0", "m1", "m2", "p16", ops=ops)
+    rs.step(hp=0)                                       # one good step on every rank
+    if rank == world - 1:
+        os._exit(3)                                     # this rank dies between steps
+    t0 = time.monotonic()
+    try:
+        rs.step(hp=1)
+        out.put((rank, "no error", time.monotonic() - t0, ops.log))
+    except Exception as e:                              # the barrier reports the dead peer
+        out.put((rank, type(e).__name__, time.monotonic() - t0, ops.log))
+
+
+def test_dead_rank_stops_the_others_at_the_first_barrier():
+    """A rank that dies between steps is noticed by the others at their next host barrier
+    (the process group ends it with an error within its timeout): no surviving rank starts
+    the update that would read the dead rank's gradients."""
+    world = 3
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_dying_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in range(world - 1)]
+    for p in procs:
+        p.join(60)
+    assert procs[-1].exitcode == 3
+    for rank, what, seconds, log in res:
+        assert what != "no error" and seconds < 60, (rank, what, seconds)
+        updates = [e for e in log if e[2] == "update"]
+        assert [e[5] for e in updates] == [0]           # step 1's update never started
