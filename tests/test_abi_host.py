@@ -151,3 +151,27 @@ def test_device_calls_refuse_a_layout_not_on_the_device(name):
     args[0] = lay.handle
     assert fn(*args) in (1, 6), name                       # ZERO_ERR_INVALID or ZERO_ERR_STATE
     assert (sc.step, sc.skipped) == (0, 0)
+
+
+def test_scaler_advance_follows_the_oracle_scaler():
+    """zero_loss_scaler_advance (the library's scaler rules, also used inside the dynamic
+    steps) against the oracle's LossScaler, over a long random skip / apply sequence that
+    reaches the floor and several growths; invalid arguments are refused."""
+    rng = np.random.default_rng(5)
+    lib_sc = zs.LossScaler(2.0 ** 10, factor=2.0, window=4, min_scale=0.5)
+    ref = oracle.LossScaler(2.0 ** 10, factor=2.0, window=4, min_scale=0.5)
+    seen_floor = grew = 0
+    for i in range(2000):
+        overflow = bool(rng.random() < (0.6 if i < 300 else 0.1))
+        before = ref.scale
+        lib_sc.advance(not overflow)
+        ref.update(overflow)
+        seen_floor += ref.scale == 0.5
+        grew += ref.scale > before
+        assert (lib_sc.scale, lib_sc.clean_steps, lib_sc.step, lib_sc.skipped) == \
+            (ref.scale, ref.clean_steps, ref.step, ref.skipped), i
+    assert seen_floor and grew > 5
+    with pytest.raises(zs.ZeroError):
+        zs.LossScaler(0.0).advance(True)                    # scale must be > 0
+    with pytest.raises(zs.ZeroError):
+        zs.LossScaler(8.0, factor=1.0).advance(False)       # factor must be > 1
