@@ -259,6 +259,33 @@ def oracle_sample_run(wl, psi_s, steps=1):
     return time.perf_counter() - t0
 
 
+class one_core:
+    """Run the oracle pinned to one CPU of this process's allowed set (restored after)."""
+
+    def __enter__(self):
+        self.saved = None
+        if hasattr(os, "sched_getaffinity"):
+            self.saved = os.sched_getaffinity(0)
+            os.sched_setaffinity(0, {min(self.saved)})
+        return self
+
+    def __exit__(self, *exc):
+        if self.saved is not None:
+            os.sched_setaffinity(0, self.saved)
+
+
+def host_info():
+    model = ""
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count(), "cpu_model": model, "pinned_to_one_core": hasattr(os, "sched_setaffinity")}
+
+
 def size_sample(wl, seconds):
     """Largest power-of-two sample whose one-step oracle run fits `seconds`."""
     psi_s = 1 << 16
@@ -270,9 +297,10 @@ def size_sample(wl, seconds):
 
 
 def cpu_baseline(wl, seconds):
-    psi_s = size_sample(wl, seconds)
-    t = oracle_sample_run(wl, psi_s)
-    return {"value": psi_s / t, "unit": UNIT, "cores": 1, "kind": "oracle",
+    with one_core():
+        psi_s = size_sample(wl, seconds)
+        t = oracle_sample_run(wl, psi_s)
+    return {"value": psi_s / t, "unit": UNIT, "cores": 1, "kind": "oracle", "host": host_info(),
             "sample": f"first {psi_s} parameters of {wl.name} (same N={wl.n_ranks}, stage {wl.stage}, "
                       f"inputs, AdamW), one step, single-threaded C oracle, {t:.1f} s"}
 
@@ -282,10 +310,11 @@ def run_reference(a, wl):
     if rank != 0:
         return
     per_step = a.ref_seconds / (a.steps + a.warmup)
-    psi_s = size_sample(wl, per_step)
-    for _ in range(a.warmup):
-        oracle_sample_run(wl, psi_s)
-    ts = [oracle_sample_run(wl, psi_s) for _ in range(a.steps)]
+    with one_core():
+        psi_s = size_sample(wl, per_step)
+        for _ in range(a.warmup):
+            oracle_sample_run(wl, psi_s)
+        ts = [oracle_sample_run(wl, psi_s) for _ in range(a.steps)]
     t = sum(ts) / len(ts)
     value = psi_s / t
     sample = (f"each step: first {psi_s} parameters of {wl.name} (same N={wl.n_ranks}, stage {wl.stage}, inputs, "
@@ -294,7 +323,8 @@ def run_reference(a, wl):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": a.gpus, "steps": a.steps,
         "warmup": a.warmup, "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": workload_config(wl, 1),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample,
+                         "host": host_info()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 
