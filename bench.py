@@ -78,6 +78,16 @@ def parse():
     ap.add_argument("--shrink", type=int, default=0,
                     help="divide every tensor of the workload by this factor (same structure, smaller: "
                          "small cases for profiler captures; not a bench line)")
+    ap.add_argument("--also", default="auto",
+                    help="workloads timed after the headline in the same run (comma-separated, or none); "
+                         "auto = the Llama-shaped ZeRO-3 list after the default flat list")
+    ap.add_argument("--record-traffic", default="",
+                    help="host-only: read this ncu CSV (dram__bytes_read.sum, dram__bytes_write.sum, "
+                         "gpu__time_duration.sum per launch) and write the per-launch traffic record of "
+                         "--record-tag for --workload under profiles/")
+    ap.add_argument("--record-kernel", default="bulk_step_kernel", help="--record-traffic: kernel name regex")
+    ap.add_argument("--record-tag", default="bulk_step", help="--record-traffic: record name prefix")
+    ap.add_argument("--record-note", default="", help="--record-traffic: how the capture was taken")
     ap.add_argument("--psi", type=int, default=0,
                     help="flat workloads only: run the same shape with this many parameters "
                          "(small cases for profiler captures; not a bench line)")
@@ -126,7 +136,7 @@ def hbm_peak():
 
 def kernel_source_hash():
     """Hash of the kernel's sources with comments and blank space removed, so that a
-    profile stays valid across comment-only edits."""
+    traffic record stays valid across comment-only edits."""
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
         text = open(f).read()
@@ -136,23 +146,60 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload):
-    """DRAM bytes per parameter of the fused kernel from a committed ncu summary
-    (profiles/*.md) taken for this workload on the current kernel sources; else None."""
+def traffic_record_name(kernel_tag, workload):
+    return os.path.join(PROFILE_DIR, f"{kernel_tag}_{workload}.json")
+
+
+def profiled_traffic(kernel_tag, workload, padded):
+    """DRAM bytes (read + write) per launch of a kernel on a workload, from the record
+    `--record-traffic` wrote for a full-size capture of the same launch configuration
+    on the current kernel sources; None when there is no such record."""
     try:
-        sha = kernel_source_hash()
-        for name in sorted(os.listdir(PROFILE_DIR)):
-            if not name.endswith(".md"):
-                continue
-            text = open(os.path.join(PROFILE_DIR, name)).read()
-            m_sha = re.search(r"kernel_sources_sha256_16:\s*([0-9a-f]+)", text)
-            m_wl = re.search(r"workload:[ \t]*(.+)", text)
-            m_tr = re.search(r"dram_bytes_per_param:\s*([0-9.]+)", text)
-            if m_sha and m_tr and m_wl and m_sha.group(1) == sha and workload in m_wl.group(1).split():
-                return float(m_tr.group(1))
-    except Exception:
-        pass
-    return None
+        rec = json.load(open(traffic_record_name(kernel_tag, workload)))
+    except (OSError, ValueError):
+        return None
+    if rec.get("kernel_sources_sha256_16") != kernel_source_hash() or rec.get("padded_params") != padded:
+        return None
+    return rec["dram_bytes_read_per_launch"] + rec["dram_bytes_write_per_launch"]
+
+
+_NCU_UNITS = {"byte": 1.0, "kbyte": 1e3, "mbyte": 1e6, "gbyte": 1e9, "tbyte": 1e12,
+              "nsecond": 1e-9, "usecond": 1e-6, "msecond": 1e-3, "second": 1.0}
+
+
+def record_traffic(a, wl):
+    """Turn an ncu CSV capture (metrics dram__bytes_read.sum, dram__bytes_write.sum,
+    gpu__time_duration.sum of the launches of one kernel) into the per-launch record
+    profiled_traffic() reads.  Host-only; no GPU needed."""
+    import csv
+    rows = list(csv.reader(l for l in open(a.record_traffic) if l.startswith('"')))
+    head, body = rows[0], rows[1:]
+    col = {k: head.index(k) for k in ("ID", "Kernel Name", "Metric Name", "Metric Unit", "Metric Value")}
+    launches = {}
+    for r in body:
+        if not re.search(a.record_kernel, r[col["Kernel Name"]]):
+            continue
+        unit = _NCU_UNITS.get(r[col["Metric Unit"]].strip().lower(), 1.0)
+        val = float(r[col["Metric Value"]].replace(",", "")) * unit
+        d = launches.setdefault(r[col["ID"]], {"kernel": r[col["Kernel Name"]]})
+        d[r[col["Metric Name"]]] = val
+    got = [d for d in launches.values() if "dram__bytes_read.sum" in d and "dram__bytes_write.sum" in d]
+    if not got:
+        raise SystemExit(f"no launch of {a.record_kernel!r} with both DRAM metrics in {a.record_traffic}")
+    import zero_sharded_optimizer_ring_b200 as zs      # host-only partitioner: the padded size
+    P = zs.Layout(list(wl.tensors), wl.n_ranks, wl.stage, wl.bucket_elems, wl.pad_align, list(wl.units)).padded
+    n = len(got)
+    rec = {"kernel": got[0]["kernel"], "workload": wl.name, "padded_params": P,
+           "kernel_sources_sha256_16": kernel_source_hash(), "launches": n,
+           "dram_bytes_read_per_launch": sum(d["dram__bytes_read.sum"] for d in got) / n,
+           "dram_bytes_write_per_launch": sum(d["dram__bytes_write.sum"] for d in got) / n,
+           "gpu_time_ms_per_launch": sum(d.get("gpu__time_duration.sum", 0.0) for d in got) / n * 1e3,
+           "capture": a.record_note}
+    out = traffic_record_name(a.record_tag, wl.name)
+    with open(out, "w") as f:
+        json.dump(rec, f, indent=1)
+        f.write("\n")
+    print(json.dumps(rec))
 
 
 class ClockSampler:
@@ -169,7 +216,7 @@ class ClockSampler:
         self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
         try:
             self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                       "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+                                       "-lms", "10"], stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.p = None
 
@@ -332,10 +379,11 @@ def run_reference(a, wl):
 # ---------------------------------------------------------------- the GPU arm
 
 def run_ours(a, wl):
+    """The GPU arm: the headline workload, then (default run) the second roofline target
+    in the same process, its buffers allocated only after the first's are freed."""
     import torch
     import torch.distributed as dist
-    import seeded_inputs as si
-    import zero_sharded_optimizer_ring_b200 as zs
+    from seeded_inputs.workloads import full_workloads
 
     rank, local, world = dist_env()
     torch.cuda.set_device(local)
@@ -349,8 +397,46 @@ def run_ours(a, wl):
             dist.barrier(device_ids=[local])
         torch.cuda.synchronize()
 
+    out = _measure(a, wl, world, rank, barrier, headline=True)
+    extra = {}
+    for name in also_workloads(a):
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        extra[name] = _measure(a, full_workloads()[name], world, rank, barrier, headline=False)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    if extra:
+        out["configs"] = extra
+    if world == 1 and a.cpu_seconds > 0:
+        out["cpu_baseline"] = cpu_baseline(wl, a.cpu_seconds)
+    print(json.dumps(out), flush=True)
+
+
+def also_workloads(a):
+    """Workloads timed after the headline in the same run.  By default the plain run of
+    the flat 1.3e9 list adds the Llama-shaped ZeRO-3 list: the two fused-step roofline
+    targets, both on the clock of one bench invocation."""
+    if a.also == "none":
+        return []
+    if a.also != "auto":
+        return [x for x in a.also.split(",") if x]
+    variant = a.wire_fp16 or a.dynamic or a.dynamic_commit or a.shrink > 1 or a.psi or a.kernel
+    return ["llama3b_n8_zero3"] if a.workload == DEFAULT_WORKLOAD and not variant else []
+
+
+def _measure(a, wl, world, rank, barrier, headline):
+    """Time K fused steps of one workload (after W warm-up steps) with CUDA events, max
+    over ranks; the headline also runs the end-to-end host-buffer leg and the requested
+    variant (fp16 wire, dynamic scaling).  Returns the JSON fields (rank 0's view)."""
+    import torch
+    import seeded_inputs as si
+    import zero_sharded_optimizer_ring_b200 as zs
+
+    plain = not headline
     lay = zs.Layout(list(wl.tensors), wl.n_ranks, wl.stage, wl.bucket_elems, wl.pad_align, list(wl.units),
-                    wire_fp16=a.wire_fp16)
+                    wire_fp16=a.wire_fp16 and not plain)
     lay.to_device()
     if a.kernel:
         lay.set_impl(a.kernel)
@@ -370,11 +456,13 @@ def run_ours(a, wl):
     p16_full = torch.zeros(P, dtype=torch.int16, device="cuda")
     p16_shard = torch.zeros(P, dtype=torch.int16, device="cuda") if wl.stage == 3 else None
     nonfinite = torch.zeros(max(1, lay.n_buckets), dtype=torch.int32, device="cuda")
+    dynamic = a.dynamic and not plain
+    dynamic_commit = a.dynamic_commit and not plain
 
     def hp(t):
         return zs.AdamW(wl.lr, wl.beta1, wl.beta2, wl.eps, wl.weight_decay, wl.loss_scale, t)
 
-    if a.dynamic:
+    if dynamic:
         # the scale the gradients carry never overflows here, so every step applies; the
         # timed work is the reduce-scatter pass, the overflow check (a host round trip)
         # and the update pass
@@ -387,7 +475,7 @@ def run_ours(a, wl):
             zs.step_dynamic(lay, g, reduced, master, m, v, p16_shard, p16_full, hp(t), scaler, nonfinite)
             if events:
                 events["update_end"].record()
-    elif a.dynamic_commit:
+    elif dynamic_commit:
         # two state sets and two fp16 parameter buffers; an applied step swaps them (the
         # scale never overflows here, so every step applies)
         scaler = zs.LossScaler(wl.loss_scale, window=1 << 40)
@@ -436,15 +524,15 @@ def run_ours(a, wl):
     ms = max_over_ranks(start.elapsed_time(end) / K, world, "cuda")
     upd_ms = max_over_ranks(sum(e["update_begin"].elapsed_time(e["update_end"]) for e in ev) / K, world, "cuda")
     gat_ms = None
-    if wl.stage == 3 and not (a.dynamic or a.dynamic_commit):      # those modes time one bracket
+    if wl.stage == 3 and not (dynamic or dynamic_commit):      # those modes time one bracket
         gat_ms = max_over_ranks(sum(e["gather_begin"].elapsed_time(e["gather_end"]) for e in ev) / K, world, "cuda")
     # our kernels per step: the fused kernel (reduce + update for --dynamic), the gather
-    launches_per_step = (2 if a.dynamic else 1) + (1 if wl.stage == 3 else 0)
+    launches_per_step = (2 if dynamic else 1) + (1 if wl.stage == 3 else 0)
 
     # end to end through the host-buffer entry point: gradients from pinned host memory
     # in, fp16 parameters to pinned host memory out, every step
     e2e = None
-    if a.e2e_steps > 0 and not (a.dynamic or a.dynamic_commit):
+    if headline and a.e2e_steps > 0 and not (dynamic or dynamic_commit):
         del g
         torch.cuda.empty_cache()
         g_host = torch.empty((N, P), dtype=torch.int16).pin_memory()
@@ -466,33 +554,35 @@ def run_ours(a, wl):
         e2e = {"value": throughput(psi, world, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": 2 * N * P, "d2h_bytes_per_step": 2 * P,
                "steps": a.e2e_steps, "path": "zero_step_host (pinned host grads in, fp16 params out)"}
-
-    if world > 1:
-        dist.destroy_process_group()
+        del g_host, p16_host, ge
+    lay.close()
     if rank != 0:
-        return
+        return None
 
     impl_name = {0: "bulk-copy pipeline (bulk_step_kernel, automatic choice)", 1: "register streaming (tile_kernel)",
                  2: "bulk-copy pipeline (bulk_step_kernel)"}[a.kernel]
-    if a.wire_fp16:
+    if a.wire_fp16 and not plain:
         impl_name += ", fp16 wire"
-    if a.dynamic:
+    if dynamic:
         impl_name = "dynamic loss scaling: reduce-scatter + overflow check + update (two passes)"
-    if a.dynamic_commit:
+    if dynamic_commit:
         impl_name = "dynamic loss scaling, two-phase commit: fused pass into a second state set + overflow check"
     peak, peak_kind = hbm_peak()
     fused_bytes = fused_bytes_per_param(wl) * P
-    if a.dynamic:
+    if dynamic:
         fused_bytes = (2 * wl.n_ranks + 4 + 4 + 24 + 2) * P     # reduce pass + update pass
-    if (a.dynamic or a.dynamic_commit) and wl.stage == 3:
+    if (dynamic or dynamic_commit) and wl.stage == 3:
         fused_bytes += 4 * P                                    # the events bracket the gather too
     achieved = fused_bytes / (upd_ms / 1e3) / 1e9
-    traffic_pp = profiled_traffic(wl.name)
+    plain_fused = not (dynamic or dynamic_commit or (a.wire_fp16 and not plain))
+    kernel_tag = {0: "bulk_step", 1: "tile_kernel", 2: "bulk_step"}[a.kernel]
+    traffic = profiled_traffic(kernel_tag, wl.name, P) if plain_fused else None
     step_bytes = ideal_bytes_per_param(wl) * P
     out = {
         "metric": METRIC, "value": throughput(psi, world, ms), "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": variant_config(a, wl, world),
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": variant_config(a, wl, world) if headline else workload_config(wl, world),
         "hbm": {"achieved_gbs_step": step_bytes / (ms / 1e3) / 1e9, "ideal_bytes_per_param": ideal_bytes_per_param(wl),
                 "frac_of_measured_peak": step_bytes / (ms / 1e3) / 1e9 / peak,
                 "frac_of_nominal_8tbs": step_bytes / (ms / 1e3) / 1e9 / NOMINAL_HBM_GBS},
@@ -500,17 +590,23 @@ def run_ours(a, wl):
                      "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": achieved / peak, "kernel_ms": upd_ms,
                      "algorithmic_bytes_per_launch": fused_bytes,
-                     "traffic": traffic_pp * P if traffic_pp else None},
+                     "traffic": traffic},
         "gpu_launches": K * launches_per_step,
-        "e2e": e2e,
         "clocks": clocks,
     }
+    if headline:
+        out["e2e"] = e2e
     if gat_ms is not None:
+        gather_bytes = 4 * P
         out["gather_kernel_ms"] = gat_ms
-        out["gather_gbs"] = 4 * P / (gat_ms / 1e3) / 1e9
-    if world == 1 and a.cpu_seconds > 0:
-        out["cpu_baseline"] = cpu_baseline(wl, a.cpu_seconds)
-    print(json.dumps(out), flush=True)
+        out["gather_gbs"] = gather_bytes / (gat_ms / 1e3) / 1e9
+        out["gather_roofline"] = {
+            "bound": "hbm", "kernel": "all-gather copy (copy_range_kernel)",
+            "achieved": gather_bytes / (gat_ms / 1e3) / 1e9, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+            "frac": gather_bytes / (gat_ms / 1e3) / 1e9 / peak, "kernel_ms": gat_ms,
+            "algorithmic_bytes_per_launch": gather_bytes,
+            "traffic": profiled_traffic("copy_range", wl.name, P) if plain_fused else None}
+    return out
 
 
 def run_overlap(a, wl):
@@ -751,7 +847,9 @@ def main():
         if len(wl.tensors) != 1:
             raise SystemExit("--psi applies to flat (single-tensor) workloads only")
         wl = wl.with_(tensors=(a.psi,), name=f"{wl.name}_psi{a.psi}")
-    if a.impl == "reference":
+    if a.record_traffic:
+        record_traffic(a, wl)
+    elif a.impl == "reference":
         run_reference(a, wl)
     elif a.overlap:
         run_overlap(a, wl)

@@ -278,8 +278,9 @@ zero_status zero_step_host(const zero_layout *layout, const uint16_t *grads_host
  *     takes (ZERO_NOALLOC_MAX_SEGMENTS + 1) x 32 bytes = 256 KiB on every GPU that
  *     loads the library, until the process exits.
  *   - The first call on each device looks up the array's device address (which can load
- *     the library's device code onto that device); make that first call before any
- *     stream capture begins.
+ *     the library's device code onto that device) and keeps it; make that first call
+ *     before any stream capture begins.  A cudaDeviceReset invalidates the kept address:
+ *     do not call this entry point on a device after resetting it.
  *   - All calls on a device share the one array, and it keeps whatever the last call
  *     wrote.  Each call rewrites every row it reads (the rows are copied from the
  *     layout's host table, which waits for earlier work on `stream` to finish, and the

@@ -129,3 +129,31 @@ def assert_bits_equal(got, want, what, any_nan=False):
         diff &= ~(nan_g & nan_w)
     n = int(diff.sum())
     assert n == 0, f"{what}: {n} elements differ bitwise"
+
+
+def oracle_run(wl, steps=None):
+    """The oracle's result after `steps` (default: the workload's) optimizer steps on the
+    workload's seeded inputs, and the oracle's layout."""
+    lay = oracle_layout(wl)
+    g, master, m, v = host_inputs(wl, lay.padded)
+    return oracle.run_steps(lay, wl.stage, g, master, m, v, hyper(wl), steps or wl.steps), lay
+
+
+def to_np(t):
+    """A device tensor as a host array; int16 tensors (fp16 bit patterns) as uint16."""
+    a = t.cpu().numpy()
+    return a.view(np.uint16) if a.dtype == np.int16 else a
+
+
+def assert_state_matches_oracle(wl, got, ref, what=""):
+    """got: dict with device tensors master, m, v, p16_full (and p16_shard for stage 3).
+    Within the parity tolerance first (fp32 1e-6 relative, fp16 1 ulp), then bit for bit:
+    both sides run the same sequence of correctly rounded operations."""
+    S_f32 = (("master", ref.master), ("m", ref.m), ("v", ref.v))
+    for name, want in S_f32:
+        assert_f32_close(to_np(got[name]), want, what + name)
+    f16 = [("p16_full", ref.p16_full)] + ([("p16_shard", ref.p16_shard)] if wl.stage == 3 else [])
+    for name, want in f16:
+        assert_f16_ulp(to_np(got[name]), want, what + name)
+    for name, want in S_f32 + tuple(f16):
+        assert_bits_equal(to_np(got[name]), want, what + name + " (bits)")

@@ -108,17 +108,20 @@ def test_reduced_workload_all_elements(key, impl):
 
 
 @pytest.mark.parametrize("key", list(reduced_workloads()))
-def test_unfused_path_equals_fused(key):
+def test_unfused_path_matches_oracle(key):
+    """The three standalone boundary calls, one bucket / shard / unit at a time:
+    zero_reduce_scatter per bucket, zero_adamw_shard_step per shard, zero_allgather per
+    unit (stage 3), against the oracle's whole steps, bit for bit."""
     wl = reduced_workloads()[key]
+    steps = 2
+    ref, _ = _oracle(wl, steps)
     lay = _layout(wl)
-    a = _bufs(lay, wl)
     b = _bufs(lay, wl)
     red = torch.zeros(lay.padded, dtype=torch.float32, device="cuda")
-    for t in range(1, 3):
-        zs.step(lay, a["g"], a["master"], a["m"], a["v"], a["p16_shard"], a["p16_full"], _hp(wl, t))
-        # per bucket, per shard, per unit
+    for t in range(1, steps + 1):
+        b["nonfinite"].zero_()
         for bk in range(lay.n_buckets):
-            zs.reduce_scatter(lay, bk, b["g"], red)
+            zs.reduce_scatter(lay, bk, b["g"], red, nonfinite=b["nonfinite"])
         for k in range(lay.n_ranks):
             out = b["p16_shard"] if wl.stage == 3 else b["p16_full"]
             zs.adamw_shard_step(lay, k, red, b["master"], b["m"], b["v"], out, _hp(wl, t))
@@ -126,8 +129,10 @@ def test_unfused_path_equals_fused(key):
             for u in range(lay.n_units):
                 zs.allgather(lay, u, b["p16_shard"], b["p16_full"])
     torch.cuda.synchronize()
-    for name in ("master", "m", "v", "p16_full"):
-        S.assert_bits_equal(_np(a[name]), _np(b[name]), name)
+    S.assert_bits_equal(_np(red), ref.reduced, "reduced (last step)")
+    _check_full(wl, lay, b, ref)
+    if wl.stage == 3:
+        S.assert_bits_equal(_np(b["p16_shard"]), ref.p16_shard, "p16_shard")
 
 
 def test_deterministic_rerun():
@@ -320,23 +325,25 @@ def test_bad_arguments_rejected():
                 zs.AdamW(loss_scale=0.0, step=1))
 
 
-def test_host_buffer_step_equals_device_step():
+def test_host_buffer_step_matches_oracle():
+    """zero_step_host: gradients from pinned host memory, fp16 parameters back to pinned
+    host memory; the device state and the host parameters equal the oracle's."""
     for key in ("flat1p3b_n4_zero1", "llama3b_n8_zero3", "ragged2000_n16_zero2"):
         wl = reduced_workloads()[key]
+        ref, olay = _oracle(wl, 2)
         lay = _layout(wl)
-        a = _bufs(lay, wl)
         b = _bufs(lay, wl)
-        g_host = a["g"].cpu().pin_memory()
+        g_host = torch.from_numpy(S.host_inputs(wl, olay.padded)[0].view(np.int16))
+        pad = b["g"].shape[1] - g_host.shape[1]
+        g_host = torch.nn.functional.pad(g_host, (0, pad)).contiguous().pin_memory()
         b["g"].zero_()
         p16_host = torch.zeros(lay.padded, dtype=torch.int16).pin_memory()
         for t in range(1, 3):
-            zs.step(lay, a["g"], a["master"], a["m"], a["v"], a["p16_shard"], a["p16_full"], _hp(wl, t))
             zs.step_host(lay, g_host, b["g"], b["master"], b["m"], b["v"], b["p16_shard"], b["p16_full"],
                          p16_host, _hp(wl, t))
         torch.cuda.synchronize()
-        for name in ("master", "m", "v", "p16_full"):
-            S.assert_bits_equal(_np(a[name]), _np(b[name]), name)
-        S.assert_bits_equal(p16_host.numpy().view(np.uint16), _np(a["p16_full"]), "p16_host")
+        S.assert_state_matches_oracle(wl, b, ref, key + ": ")
+        S.assert_bits_equal(p16_host.numpy().view(np.uint16), ref.p16_full, key + ": p16_host")
 
 
 # ------------------------------------------------------------- full size, sampled
@@ -421,14 +428,14 @@ def test_bulk_pipeline_bounded_wait_reports_timeout():
 
 
 @pytest.mark.parametrize("key", ["flat1p3b_n4_zero1", "llama3b_n8_zero3"])
-def test_checkpoint_resume_equals_uninterrupted(key):
+def test_checkpoint_resume_matches_oracle(key):
     """The optimizer state is the caller's buffers: copying them to host memory after two
     steps, wiping the device buffers and a fresh layout, restoring, and running two more
-    steps gives exactly the four-step result (the library keeps no state of its own)."""
+    steps gives the oracle's uninterrupted four-step result (the library keeps no state
+    of its own)."""
     wl = reduced_workloads()[key]
+    ref, _ = _oracle(wl, 4)
     lay = _layout(wl, zs.IMPL_BULK)
-    a = _bufs(lay, wl)
-    _run(lay, wl, a, 4)
     b = _bufs(lay, wl)
     for t in (1, 2):
         zs.step(lay, b["g"], b["master"], b["m"], b["v"], b["p16_shard"], b["p16_full"], _hp(wl, t))
@@ -443,5 +450,4 @@ def test_checkpoint_resume_equals_uninterrupted(key):
     for t in (3, 4):
         zs.step(lay2, b["g"], b["master"], b["m"], b["v"], b["p16_shard"], b["p16_full"], _hp(wl, t))
     torch.cuda.synchronize()
-    for k in ("master", "m", "v", "p16_full"):
-        S.assert_bits_equal(_np(b[k]), _np(a[k]), k)
+    S.assert_state_matches_oracle(wl, b, ref)

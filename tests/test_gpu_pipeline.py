@@ -1,11 +1,12 @@
-"""Bucket pipelining: the per-bucket step and the event-gated step against zero_step.
+"""Bucket pipelining: the per-bucket step and the event-gated step against the oracle.
 
 A simulated backward pass writes one bucket of gradients at a time, last bucket of the
-flat buffer first (the order a backward pass completes them), on its own stream and
-records an event per bucket; zero_step_overlapped runs each bucket's fused update on
-another stream as soon as its event fires.  Results must equal zero_step's bit for bit.
+flat buffer first (the order a backward pass completes them: rkmt.cn/news/44736 "DDP",
+en.pswp.cn/web/84187 "DDP" buckets), on its own stream and records an event per bucket;
+zero_step_overlapped runs each bucket's fused update on another stream as soon as its
+event fires.  Every state buffer, the fp16 parameters and the per-bucket non-finite
+counts must equal the CPU oracle's (oracle.run_steps) bit for bit.
 """
-import numpy as np
 import pytest
 
 from seeded_inputs.workloads import reduced_workloads
@@ -35,46 +36,48 @@ def _setup(wl):
     return lay, bufs
 
 
-def _same(a, b):
+def _check(wl, lay, b, ref):
     torch.cuda.synchronize()
-    for k in ("master", "m", "v", "p16_full", "p16_shard", "nonfinite"):
-        S.assert_bits_equal(a[k].cpu().numpy(), b[k].cpu().numpy(), k)
+    S.assert_state_matches_oracle(wl, b, ref)
+    assert list(S.to_np(b["nonfinite"])[:lay.n_buckets]) == list(ref.nonfinite)
+
+
+STEPS = 2
 
 
 @pytest.mark.parametrize("key", list(reduced_workloads()))
 @pytest.mark.parametrize("order", ["bucket", "reverse"])
-def test_step_bucket_equals_step(key, order):
+def test_step_bucket_matches_oracle(key, order):
     wl = reduced_workloads()[key]
+    ref, _ = S.oracle_run(wl, STEPS)
     lay, bufs = _setup(wl)
-    a, b = bufs(), bufs()
-    _, buckets, _, _ = lay.tables()
+    b = bufs()
     seq = list(range(lay.n_buckets))
     if order == "reverse":
         seq.reverse()
-    for t in (1, 2):
-        zs.step(lay, a["g"], a["master"], a["m"], a["v"], a["p16_shard"], a["p16_full"], _hp(wl, t),
-                nonfinite=a["nonfinite"])
+    for t in range(1, STEPS + 1):
+        b["nonfinite"].zero_()
         for bk in seq:
             zs.step_bucket(lay, bk, b["g"], b["master"], b["m"], b["v"], b["p16_shard"], b["p16_full"], _hp(wl, t),
                            nonfinite=b["nonfinite"])
         if wl.stage == 3:
             zs.allgather(lay, -1, b["p16_shard"], b["p16_full"])
-    _same(a, b)
+    _check(wl, lay, b, ref)
 
 
 @pytest.mark.parametrize("group", [1, 3, 1000])
 @pytest.mark.parametrize("key", ["flat1p3b_n4_zero1", "llama3b_n8_zero3", "ragged2000_n16_zero2"])
 def test_overlapped_step_with_simulated_backward(key, group):
     wl = reduced_workloads()[key]
+    ref, _ = S.oracle_run(wl, STEPS)
     lay, bufs = _setup(wl)
-    a, b = bufs(), bufs()
+    b = bufs()
     _, buckets, _, _ = lay.tables()
     producer, consumer = torch.cuda.Stream(), torch.cuda.Stream()
-    for t in (1, 2):
-        zs.step(lay, a["g"], a["master"], a["m"], a["v"], a["p16_shard"], a["p16_full"], _hp(wl, t),
-                nonfinite=a["nonfinite"])
+    for t in range(1, STEPS + 1):
         torch.cuda.synchronize()
         b["g"].zero_()
+        b["nonfinite"].zero_()
         torch.cuda.synchronize()
         ready = [torch.cuda.Event() for _ in range(lay.n_buckets)]
         for bk, (lo, hi) in enumerate(buckets):            # the backward: bucket 0 (the tail) first
@@ -84,7 +87,7 @@ def test_overlapped_step_with_simulated_backward(key, group):
         zs.step_overlapped(lay, ready, b["g"], b["master"], b["m"], b["v"], b["p16_shard"], b["p16_full"],
                            _hp(wl, t), nonfinite=b["nonfinite"], stream=consumer, group=group)
     zs.get_error(lay)
-    _same(a, b)
+    _check(wl, lay, b, ref)
 
 
 def test_overlapped_rejects_unrecorded_events():

@@ -1,10 +1,12 @@
 """One buffer per rank, one shard at a time, and the multi-process step over CUDA IPC.
 
-- zero_step_ranks on separately allocated per-rank gradient buffers equals zero_step;
-- zero_step_shard run for every shard, with shard-local optimizer state, equals zero_step;
-- zero_copy_shard copies exactly the shard's range;
-- zero_gather_unit_ranks, reading each rank's own shard buffer, equals zero_gather_unit
-  (vector and element paths, units across shard edges, 16 ranks);
+- zero_step_ranks on separately allocated per-rank gradient buffers, and zero_step_shard
+  run for every shard with shard-local optimizer state, equal the oracle;
+- zero_copy_shard copies exactly the shard's range of the stepped parameters, which
+  equals the oracle's;
+- zero_gather_unit_ranks, reading each rank's own shard buffer as the CUDA step wrote
+  it, gives the oracle's gathered layer (vector and element paths, units across shard
+  edges, 16 ranks);
 - two processes sharing this GPU, each holding one rank's gradients and one shard's
   state, run the multi-GPU step (CUDA IPC mappings, host barriers over gloo; no kernel
   waits on the other process) and end bit-identical to the oracle; for ZeRO-3 each keeps
@@ -44,51 +46,72 @@ def _layout(wl, wire=False):
                      wire_fp16=wire).to_device()
 
 
+def _oracle_ref(wl, steps, wire=False):
+    olay = S.oracle_layout(wl)
+    g, master, m, v = S.host_inputs(wl, olay.padded)
+    return oracle.run_steps(olay, wl.stage, g, master, m, v, S.hyper(wl), steps, wire16=wire)
+
+
 @pytest.mark.parametrize("key", ["flat1p3b_n4_zero1", "gpt2_small_n8_zero2", "ragged2000_n16_zero2",
                                  "llama3b_n8_zero3"])
 @pytest.mark.parametrize("wire", [False, True])
-def test_step_ranks_and_step_shard_equal_step(key, wire):
+def test_step_ranks_and_step_shard_match_oracle(key, wire):
     wl = reduced_workloads()[key]
+    steps = 2
+    ref = _oracle_ref(wl, steps, wire)
     lay = _layout(wl, wire)
     P, S_, N = lay.padded, lay.shard, wl.n_ranks
     g, master, m, v = S.device_inputs(wl, P)
-    ref = dict(master=master.clone(), m=m.clone(), v=v.clone(), p16s=torch.zeros(P, dtype=torch.int16, device="cuda"),
-               p16f=torch.zeros(P, dtype=torch.int16, device="cuda"))
     ranks = [g[r].clone() for r in range(N)]                       # separate allocations
-    a = dict(master=master.clone(), m=m.clone(), v=v.clone(), p16s=torch.zeros_like(ref["p16s"]),
-             p16f=torch.zeros_like(ref["p16f"]))
+    a = dict(master=master.clone(), m=m.clone(), v=v.clone(), p16s=torch.zeros(P, dtype=torch.int16, device="cuda"),
+             p16f=torch.zeros(P, dtype=torch.int16, device="cuda"))
     shards = [[x[k * S_:(k + 1) * S_].clone() for x in (master, m, v)] for k in range(N)]
     p16_sh = torch.zeros(P, dtype=torch.int16, device="cuda")
     p16_k = [torch.zeros(S_, dtype=torch.int16, device="cuda") for _ in range(N)]
-    for t in (1, 2):
-        zs.step(lay, g, ref["master"], ref["m"], ref["v"], ref["p16s"], ref["p16f"], _hp(wl, t))
+    for t in range(1, steps + 1):
         zs.step_ranks(lay, ranks, a["master"], a["m"], a["v"], a["p16s"], a["p16f"], _hp(wl, t))
         for k in range(N):
             out = p16_k[k] if wl.stage == 3 else p16_sh
             zs.step_shard(lay, k, ranks, *shards[k], out, _hp(wl, t))
     torch.cuda.synchronize()
-    for name in ("master", "m", "v"):
-        S.assert_bits_equal(_np(a[name]), _np(ref[name]), name)
+    for name, want in (("master", ref.master), ("m", ref.m), ("v", ref.v)):
+        S.assert_bits_equal(_np(a[name]), want, name)
         whole = torch.cat([shards[k][("master", "m", "v").index(name)] for k in range(N)])
-        S.assert_bits_equal(_np(whole), _np(ref[name]), name + " by shard")
-    S.assert_bits_equal(_np(a["p16f"]), _np(ref["p16f"]), "p16_full")
+        S.assert_bits_equal(_np(whole), want, name + " by shard")
+    S.assert_bits_equal(_np(a["p16f"]), ref.p16_full, "p16_full")
     if wl.stage == 3:
-        S.assert_bits_equal(_np(torch.cat(p16_k)), _np(ref["p16s"]), "p16 by shard")
+        S.assert_bits_equal(_np(a["p16s"]), ref.p16_shard, "p16_shard")
+        S.assert_bits_equal(_np(torch.cat(p16_k)), ref.p16_shard, "p16 by shard")
     else:
-        S.assert_bits_equal(_np(p16_sh), _np(ref["p16f"]), "p16 by shard")
+        S.assert_bits_equal(_np(p16_sh), ref.p16_full, "p16 by shard")
+
+
+def _stepped(wl, steps=2):
+    """The CUDA step's fp16 output (stage 3: the shard buffer; else the full buffer) after
+    `steps` steps, and the oracle's result on the same inputs."""
+    ref = _oracle_ref(wl, steps)
+    lay = _layout(wl)
+    P = lay.padded
+    g, master, m, v = S.device_inputs(wl, P)
+    p16s = torch.zeros(P, dtype=torch.int16, device="cuda")
+    p16f = torch.zeros(P, dtype=torch.int16, device="cuda")
+    for t in range(1, steps + 1):
+        zs.step(lay, g, master, m, v, p16s, p16f, _hp(wl, t))
+    torch.cuda.synchronize()
+    return lay, (p16s if wl.stage == 3 else p16f), ref
 
 
 def test_copy_shard_copies_exactly_the_shard():
     wl = reduced_workloads()["flat1p3b_n4_zero1"]
-    lay = _layout(wl)
-    src = torch.randint(-9999, 9999, (lay.padded,), dtype=torch.int16, device="cuda")
+    lay, src, ref = _stepped(wl)
     for k in range(lay.n_ranks):
         dst = torch.zeros_like(src)
         zs.copy_shard(lay, k, src, dst)
         torch.cuda.synchronize()
         lo, hi = k * lay.shard, (k + 1) * lay.shard
-        assert torch.equal(dst[lo:hi], src[lo:hi])
-        assert int(torch.count_nonzero(dst[:lo])) == 0 and int(torch.count_nonzero(dst[hi:])) == 0
+        got = _np(dst)
+        S.assert_bits_equal(got[lo:hi], ref.p16_full[lo:hi], f"shard {k}")
+        assert not got[:lo].any() and not got[hi:].any(), f"shard {k}: written outside its range"
 
 
 @pytest.mark.parametrize("tensors,N,A,units", [
@@ -97,19 +120,20 @@ def test_copy_shard_copies_exactly_the_shard():
     ((4096, 8192, 40_960, 8), 4, 8, (0, 1, 2, 3)),     # vector path, units across shard edges
     ((1000,) * 16, 16, 8, tuple(range(16))),
 ])
-def test_gather_unit_ranks_equals_gather_unit(tensors, N, A, units):
-    lay = zs.Layout(list(tensors), N, 3, 0, A, list(units)).to_device()
-    P, S_ = lay.padded, lay.shard
-    whole = torch.randint(-30000, 30000, (P,), dtype=torch.int16, device="cuda")
+def test_gather_unit_ranks_matches_oracle(tensors, N, A, units):
+    wl = Workload(name="gather_ranks", description="stage-3 gather from per-rank shards", tensors=tuple(tensors),
+                  units=tuple(units), n_ranks=N, stage=3, bucket_elems=0, steps=2, loss_scale=1024.0, pad_align=A)
+    lay, whole, ref = _stepped(wl)
+    S_ = lay.shard
     shards = [whole[k * S_:(k + 1) * S_].clone() for k in range(N)]          # one allocation per rank
     _, _, _, u = lay.tables()
     for j, (lo, hi) in enumerate(u):
-        want = torch.zeros(int(hi - lo), dtype=torch.int16, device="cuda")
-        got = torch.full_like(want, -1)
-        zs.gather_unit(lay, j, whole, want)
+        got = torch.full((int(hi - lo) + 16,), -1, dtype=torch.int16, device="cuda")
         zs.gather_unit_ranks(lay, j, shards, got)
         torch.cuda.synchronize()
-        assert torch.equal(got, want) and torch.equal(want, whole[int(lo):int(hi)])
+        g = _np(got)
+        S.assert_bits_equal(g[:hi - lo], ref.p16_full[lo:hi], f"unit {j}")
+        assert (g[hi - lo:] == 0xFFFF).all(), f"unit {j}: write past the unit"
 
 
 def test_gather_unit_ranks_rejects_bad_arguments():

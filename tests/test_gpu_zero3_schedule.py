@@ -1,50 +1,74 @@
-"""ZeRO-3 per-layer gathers: zero_gather_unit and the prefetching schedule.
+"""ZeRO-3 per-layer gathers: zero_gather_unit and the prefetching schedule, against the
+oracle.
 
-Every unit gathered into its own buffer equals its range of the shard buffer, bit for bit
-(aligned and unaligned unit starts).  Under the prefetching schedule, each layer's
-"compute" (a deliberate delay, then a copy of the gathered buffer to the unit's place in
-an output buffer) must see its own unit's parameters: a slot overwritten before its
-layer finished would show up as a mismatch.
+rkmt.cn/news/44736 "Deepspeed ZeRO-3": each layer's parameters are gathered from the
+ranks that hold them before the layer's forward pass, and again before its backward
+pass.  Here the shards are those the CUDA step wrote for stage 3, and every gathered
+unit must equal the oracle's fully gathered parameters (oracle.run_steps, which gathers
+unit by unit from its own shards) over the unit's range, bit for bit, for aligned and
+unaligned unit starts.  Under the prefetching schedule each layer's "compute" (a
+deliberate delay, then a copy of the gathered buffer to the unit's place in an output
+buffer) must see its own unit's parameters: a slot overwritten before its layer
+finished would show up as a mismatch against the oracle.
 """
-import numpy as np
 import pytest
 
 from seeded_inputs.workloads import reduced_workloads
 import zero_sharded_optimizer_ring_b200 as zs
 from zero_sharded_optimizer_ring_b200.schedule import zero3_pass
+import support as S
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
 
-def _setup(tensors, units, N=8):
-    lay = zs.Layout(list(tensors), N, 3, 50_000, 1, list(units)).to_device()
+def _workload(aligned=True):
+    wl = reduced_workloads()["llama3b_n8_zero3"]
+    if not aligned:     # a 3-element first tensor moves every later unit start off the 8-grid
+        wl = wl.with_(name=wl.name + "_unaligned", tensors=(3,) + tuple(wl.tensors)[1:])
+    return wl
+
+
+def _stepped_shards(wl):
+    """Run the CUDA step for the workload's steps; returns the layout, the stage-3 shard
+    buffer it wrote, and the oracle's result on the same seeded inputs."""
+    ref, _ = S.oracle_run(wl)
+    lay = zs.Layout(list(wl.tensors), wl.n_ranks, wl.stage, wl.bucket_elems, wl.pad_align,
+                    list(wl.units)).to_device()
     P = lay.padded
-    shard = torch.randint(-30000, 30000, (P,), dtype=torch.int16, device="cuda")
-    _, _, _, u = lay.tables()
-    return lay, shard, u
+    g, master, m, v = S.device_inputs(wl, P)
+    p16_shard = torch.zeros(P, dtype=torch.int16, device="cuda")
+    p16_full = torch.zeros(P, dtype=torch.int16, device="cuda")
+    for t in range(1, wl.steps + 1):
+        zs.step(lay, g, master, m, v, p16_shard, p16_full,
+                zs.AdamW(wl.lr, wl.beta1, wl.beta2, wl.eps, wl.weight_decay, wl.loss_scale, t))
+    zs.get_error(lay)
+    torch.cuda.synchronize()
+    S.assert_bits_equal(S.to_np(p16_shard), ref.p16_shard, "p16_shard")
+    return lay, p16_shard, ref
 
 
 @pytest.mark.parametrize("aligned", [True, False])
-def test_gather_unit_equals_its_range(aligned):
-    wl = reduced_workloads()["llama3b_n8_zero3"]
-    tensors = list(wl.tensors) if aligned else [3] + list(wl.tensors)[1:]
-    units = list(wl.units)
-    lay, shard, u = _setup(tensors, units)
+def test_gather_unit_matches_oracle(aligned):
+    wl = _workload(aligned)
+    lay, shard, ref = _stepped_shards(wl)
+    _, _, _, u = lay.tables()
     assert aligned == all(lo % 8 == 0 for lo, _ in u)
     for k, (lo, hi) in enumerate(u):
         dst = torch.full((hi - lo + 16,), 7, dtype=torch.int16, device="cuda")
         zs.gather_unit(lay, k, shard, dst)
         torch.cuda.synchronize()
-        assert torch.equal(dst[:hi - lo], shard[lo:hi])
-        assert torch.all(dst[hi - lo:] == 7)
+        got = S.to_np(dst)
+        S.assert_bits_equal(got[:hi - lo], ref.p16_full[lo:hi], f"unit {k}")
+        assert (got[hi - lo:] == 7).all(), f"unit {k}: write past the unit"
 
 
 @pytest.mark.parametrize("n_slots", [1, 2, 3])
 @pytest.mark.parametrize("backward", [False, True])
 def test_prefetch_schedule_gives_each_layer_its_parameters(n_slots, backward):
-    wl = reduced_workloads()["llama3b_n8_zero3"]
-    lay, shard, u = _setup(wl.tensors, wl.units)
+    wl = _workload()
+    lay, shard, ref = _stepped_shards(wl)
+    _, _, _, u = lay.tables()
     width = int(max(hi - lo for lo, hi in u))
     slots = [torch.zeros(width, dtype=torch.int16, device="cuda") for _ in range(n_slots)]
     out = torch.zeros(lay.padded, dtype=torch.int16, device="cuda")
@@ -61,4 +85,4 @@ def test_prefetch_schedule_gives_each_layer_its_parameters(n_slots, backward):
     torch.cuda.synchronize()                        # inputs written on the default stream
     zero3_pass(lay, shard, slots, order, compute, gs, cs)
     torch.cuda.synchronize()
-    assert torch.equal(out, shard)
+    S.assert_bits_equal(S.to_np(out), ref.p16_full, "layers as the compute saw them")

@@ -6,7 +6,8 @@ allocation may cause); zero_step_noalloc serves them by keeping the step's scrat
 segment table and its tile index) in a static device array.  These tests call it through
 the C ABI on a layout that was never uploaded (so no library allocation exists at all)
 and check its outputs against zero_step's, within the tolerance of the other parity
-tests, on two calls in a row (the second call runs on the array the first one left).
+tests and then bit for bit (both kernels follow the same rounded operations), on two
+calls in a row (the second call runs on the array the first one left).
 
 This file is collected last on purpose: if it fails, every other test has already run.
 """
@@ -62,6 +63,10 @@ def test_noalloc_matches_step_on_two_calls(key):
         if wl.stage == 3:
             S.assert_f16_ulp(_np(b["p16_shard"]), _np(a["p16_shard"]), f"p16_shard after call {t}")
         assert np.array_equal(_np(b["nonfinite"]), _np(a["nonfinite"]))
+        # the header promises more than the tolerance: the same bits as zero_step
+        names = ("master", "m", "v", "p16_full") + (("p16_shard",) if wl.stage == 3 else ())
+        for name in names:
+            S.assert_bits_equal(_np(b[name]), _np(a[name]), f"{name} after call {t} (bits)")
 
 
 def test_noalloc_rejects_layouts_beyond_its_table():

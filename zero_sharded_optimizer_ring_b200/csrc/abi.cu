@@ -12,10 +12,14 @@
 using zero::AdamScalars;
 using zero::Seg;
 using zero::TileWork;
+using zero::check_hparams;
+using zero::step_scalars;
 
 namespace {
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+bool finite_d(double x) { return isfinite(x) != 0; }
 
 zero_status check_device(const zero_layout *L)
 {
@@ -27,35 +31,6 @@ zero_status check_device(const zero_layout *L)
 }
 
 zero_status cuda_status(cudaError_t e) { return e == cudaSuccess ? ZERO_OK : ZERO_ERR_CUDA; }
-
-bool finite_d(double x) { return isfinite(x) != 0; }
-
-zero_status check_hparams(const zero_adamw_hparams *h)
-{
-    if (!h) return ZERO_ERR_INVALID;
-    if (h->step < 1 || !finite_d(h->lr) || !finite_d(h->eps) || !finite_d(h->weight_decay) ||
-        !finite_d(h->loss_scale) || !(h->loss_scale > 0.0) || !(h->beta1 >= 0.0 && h->beta1 < 1.0) ||
-        !(h->beta2 >= 0.0 && h->beta2 < 1.0))
-        return ZERO_ERR_INVALID;
-    return ZERO_OK;
-}
-
-// The step's fp32 scalars, each evaluated in double and rounded once.
-AdamScalars step_scalars(int32_t n_ranks, const zero_adamw_hparams &h)
-{
-    AdamScalars c;
-    const double t = (double)h.step;
-    c.inv_scale = (float)(1.0 / ((double)n_ranks * h.loss_scale));
-    c.decay = (float)(1.0 - h.lr * h.weight_decay);
-    c.beta1 = (float)h.beta1;
-    c.omb1 = (float)(1.0 - h.beta1);
-    c.beta2 = (float)h.beta2;
-    c.omb2 = (float)(1.0 - h.beta2);
-    c.step_size = (float)(h.lr / (1.0 - pow(h.beta1, t)));
-    c.sqrt_bc2 = (float)sqrt(1.0 - pow(h.beta2, t));
-    c.eps = (float)h.eps;
-    return c;
-}
 
 TileWork all_tiles(const zero_layout *L)
 {
@@ -120,6 +95,37 @@ void release_device(zero_layout *L)
 }
 
 }  // namespace
+
+namespace zero {
+
+zero_status check_hparams(const zero_adamw_hparams *h)
+{
+    if (!h) return ZERO_ERR_INVALID;
+    if (h->step < 1 || !finite_d(h->lr) || !finite_d(h->eps) || !finite_d(h->weight_decay) ||
+        !finite_d(h->loss_scale) || !(h->loss_scale > 0.0) || !(h->beta1 >= 0.0 && h->beta1 < 1.0) ||
+        !(h->beta2 >= 0.0 && h->beta2 < 1.0))
+        return ZERO_ERR_INVALID;
+    return ZERO_OK;
+}
+
+// The step's fp32 scalars, each evaluated in double and rounded once.
+AdamScalars step_scalars(int32_t n_ranks, const zero_adamw_hparams &h)
+{
+    AdamScalars c;
+    const double t = (double)h.step;
+    c.inv_scale = (float)(1.0 / ((double)n_ranks * h.loss_scale));
+    c.decay = (float)(1.0 - h.lr * h.weight_decay);
+    c.beta1 = (float)h.beta1;
+    c.omb1 = (float)(1.0 - h.beta1);
+    c.beta2 = (float)h.beta2;
+    c.omb2 = (float)(1.0 - h.beta2);
+    c.step_size = (float)(h.lr / (1.0 - pow(h.beta1, t)));
+    c.sqrt_bc2 = (float)sqrt(1.0 - pow(h.beta2, t));
+    c.eps = (float)h.eps;
+    return c;
+}
+
+}  // namespace zero
 
 extern "C" void zero_layout_destroy(zero_layout *L)
 {

@@ -73,6 +73,7 @@ struct zero_layout {
     std::vector<int64_t> bucket_lo, bucket_hi;
     std::vector<int64_t> bucket_seg_begin;     // n_buckets + 1: first segment of each bucket
     std::vector<zero::Seg> segs;               // host copy, tile_begin filled on the host too
+    zero::Seg closing{};                       // the table's closing row: lo = hi = P, shard = bucket = -1
     std::vector<zero::Seg> segs_by_shard;      // shard-major order, with its own tile numbering
     std::vector<int64_t> shard_seg_begin;      // n_ranks + 1: first shard-major row of each shard
     std::vector<int64_t> unit_lo, unit_hi;
@@ -83,6 +84,11 @@ struct zero_layout {
 };
 
 namespace zero {
+
+// abi.cu: hyper-parameter rules shared by every step entry point, and the step's fp32
+// scalars (each evaluated in double and rounded once).
+zero_status check_hparams(const zero_adamw_hparams *h);
+AdamScalars step_scalars(int32_t n_ranks, const zero_adamw_hparams &h);
 
 // kernels.cu
 cudaError_t launch_tile_index(Seg *segs, int64_t n_seg, cudaStream_t s);

@@ -366,6 +366,18 @@ __global__ void tile_index_kernel(Seg *segs, int64_t n_seg)
     if (lane == 0) segs[n_seg].tile_begin = carry;
 }
 
+// The SM count a layout recorded on upload; a layout that was never uploaded (the
+// allocation-free step) asks the current device.
+int sm_count(int recorded)
+{
+    if (recorded > 0) return recorded;
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
+        return n;
+    return 148;
+}
+
 template <class K>
 int grid_for(K kernel, int64_t work_items, int num_sms, int max_ctas = 0)
 {
@@ -373,7 +385,7 @@ int grid_for(K kernel, int64_t work_items, int num_sms, int max_ctas = 0)
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0) != cudaSuccess ||
         per_sm < 1)
         per_sm = 1;
-    int64_t g = (int64_t)per_sm * (num_sms > 0 ? num_sms : 148);
+    int64_t g = (int64_t)per_sm * sm_count(num_sms);
     if (max_ctas > 0 && g > max_ctas) g = max_ctas;
     if (g > work_items) g = work_items;
     return (int)(g < 1 ? 1 : g);

@@ -90,6 +90,9 @@ extern "C" zero_status zero_layout_create(const zero_layout_desc *d, zero_layout
         }
         L->bucket_seg_begin.push_back((int64_t)L->segs.size());
         L->n_tiles = tiles;
+        L->closing.lo = L->closing.hi = P;
+        L->closing.tile_begin = -1;
+        L->closing.shard = L->closing.bucket = -1;
 
         // the same segments shard-major (one shard's segments contiguous), renumbered
         for (int64_t k = 0; k < N; ++k) {

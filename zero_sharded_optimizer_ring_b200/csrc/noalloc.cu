@@ -9,7 +9,6 @@
 // below, a file-scope static device array that exists on every GPU that loads the
 // library, from load until the process exits, so a call allocates nothing.
 #include <cuda_runtime.h>
-#include <math.h>
 #include <stdint.h>
 
 #include <mutex>
@@ -26,8 +25,11 @@ static __device__ __align__(256) zero::Seg g_step_scratch[ZERO_NOALLOC_MAX_SEGME
 std::mutex g_lock;
 zero::Seg *g_scratch_addr[kMaxDevices] = {};
 
-// Device address of g_step_scratch on the current device, looked up once per device.
-// (In host code the array's name is only a host-side handle; the kernels need this.)
+// Device address of g_step_scratch on the current device, looked up on the first call on
+// each device and kept for the life of the process.  (In host code the array's name is
+// only a host-side handle; the kernels need this.)  A cudaDeviceReset tears down the
+// device's context and with it the array's mapping, so the kept address is stale after
+// one: a process that resets a device must not call this entry point on it again.
 zero_status scratch_address(zero::Seg **out)
 {
     int dev = -1;
@@ -46,13 +48,6 @@ zero_status scratch_address(zero::Seg **out)
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
-bool hparams_ok(const zero_adamw_hparams *h)
-{
-    return h && h->step >= 1 && isfinite(h->lr) && isfinite(h->eps) && isfinite(h->weight_decay) &&
-           isfinite(h->loss_scale) && h->loss_scale > 0.0 && h->beta1 >= 0.0 && h->beta1 < 1.0 &&
-           h->beta2 >= 0.0 && h->beta2 < 1.0;
-}
-
 }  // namespace
 
 extern "C" zero_status zero_step_noalloc(const zero_layout *L, const uint16_t *grads, int64_t rank_stride,
@@ -60,7 +55,7 @@ extern "C" zero_status zero_step_noalloc(const zero_layout *L, const uint16_t *g
                                          uint16_t *p16_full, const zero_adamw_hparams *hp,
                                          int32_t *nonfinite, void *stream)
 {
-    if (!L || !hparams_ok(hp)) return ZERO_ERR_INVALID;
+    if (!L || zero::check_hparams(hp) != ZERO_OK) return ZERO_ERR_INVALID;
     if (L->padded == 0) return ZERO_OK;
     const int64_t n_seg = (int64_t)L->segs.size();
     if (n_seg > ZERO_NOALLOC_MAX_SEGMENTS) return ZERO_ERR_INVALID;   // table would not fit
@@ -77,30 +72,15 @@ extern "C" zero_status zero_step_noalloc(const zero_layout *L, const uint16_t *g
     cudaStream_t st = (cudaStream_t)stream;
 
     // Every call rewrites rows 0..n_seg before any kernel reads them (the row contents
-    // from the host, then the first-tile column from the device scan), so nothing left
-    // over from an earlier call is ever read.  The host rows are pageable memory: the
-    // copy has taken them by the time cudaMemcpyAsync returns.
-    zero::Seg closing;
-    closing.lo = closing.hi = L->padded;
-    closing.tile_begin = -1;
-    closing.shard = closing.bucket = -1;
+    // from the layout's host table and closing row, then the first-tile column from the
+    // device scan), so nothing left over from an earlier call is ever read.  Both host
+    // sources belong to the layout and live as long as it does.
     cudaError_t e = cudaMemcpyAsync(table, L->segs.data(), (size_t)n_seg * sizeof(zero::Seg),
                                     cudaMemcpyHostToDevice, st);
     if (e == cudaSuccess)
-        e = cudaMemcpyAsync(table + n_seg, &closing, sizeof closing, cudaMemcpyHostToDevice, st);
+        e = cudaMemcpyAsync(table + n_seg, &L->closing, sizeof(zero::Seg), cudaMemcpyHostToDevice, st);
     if (e == cudaSuccess) e = zero::launch_tile_index(table, n_seg, st);
-
-    zero::AdamScalars c;
-    const double t = (double)hp->step;
-    c.inv_scale = (float)(1.0 / ((double)L->n_ranks * hp->loss_scale));
-    c.decay = (float)(1.0 - hp->lr * hp->weight_decay);
-    c.beta1 = (float)hp->beta1;
-    c.omb1 = (float)(1.0 - hp->beta1);
-    c.beta2 = (float)hp->beta2;
-    c.omb2 = (float)(1.0 - hp->beta2);
-    c.step_size = (float)(hp->lr / (1.0 - pow(hp->beta1, t)));
-    c.sqrt_bc2 = (float)sqrt(1.0 - pow(hp->beta2, t));
-    c.eps = (float)hp->eps;
+    const zero::AdamScalars c = zero::step_scalars(L->n_ranks, *hp);
 
     zero::TileWork w;
     w.segs = table;
