@@ -33,9 +33,9 @@ DEFAULT_WORKLOAD = "flat1p3b_n4_zero1"
 FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0
 PROFILE_DIR = os.path.join(ROOT, "profiles")
-# the sources the fused bulk kernel is compiled from: a profile taken on other sources is stale
-KERNEL_SOURCES = [os.path.join(ROOT, "zero_sharded_optimizer_ring_b200", "csrc", f)
-                  for f in ("bulk_step.cu", "device_common.cuh", "internal.h")]
+# the library's device sources: a traffic record taken on other sources is stale
+_CSRC = os.path.join(ROOT, "zero_sharded_optimizer_ring_b200", "csrc")
+KERNEL_SOURCES = sorted(os.path.join(_CSRC, f) for f in os.listdir(_CSRC) if f.endswith((".cu", ".cuh", ".h")))
 
 
 def parse():
@@ -61,6 +61,11 @@ def parse():
                     help="time ZeRO-3's per-layer forward and backward gathers with 1-3 prefetch slots "
                          "against a simulated layer compute (its own JSON line)")
     ap.add_argument("--tokens", type=int, default=2048, help="--zero3-passes: tokens per rank")
+    ap.add_argument("--carveout", default="0",
+                    help="--zero3-passes: comma-separated SM counts the layer GEMMs leave free (cuBLAS SM-count "
+                         "target through torch's matmul carveout), one sweep row set each")
+    ap.add_argument("--gather-ctas", default="0",
+                    help="--zero3-passes: comma-separated gather CTA caps (zero_set_gather_ctas; 0 = default grid)")
     ap.add_argument("--overlap", action="store_true",
                     help="measure the bucket-pipelined step behind a simulated backward pass "
                          "(its own JSON line; not the headline)")
@@ -739,7 +744,7 @@ def run_zero3_passes(a, wl):
     compute alone (parameters already in place) and the gathers alone."""
     import torch
     import zero_sharded_optimizer_ring_b200 as zs
-    from zero_sharded_optimizer_ring_b200.schedule import zero3_pass
+    from zero_sharded_optimizer_ring_b200.schedule import layer_breakdown, zero3_pass
     from seeded_inputs.workloads import llama_tensors
 
     torch.cuda.set_device(dist_env()[1])
@@ -791,20 +796,24 @@ def run_zero3_passes(a, wl):
     order_f = list(range(lay.n_units))
     order_b = order_f[::-1]
 
-    def timed(fn):
-        best = None
+    def timed(fn, breakdown=False):
+        """Best of 3 repetitions after the warm-up; with breakdown, fn returns the pass's
+        events and the per-layer breakdown of the best repetition comes back too."""
+        best, best_bd = None, None
         for rep in range(a.warmup + 3):
             torch.cuda.synchronize()
             s0, e0 = ev(), ev()
             s0.record(gs)
             cs.wait_event(s0)
-            fn()
+            marks = fn()
             e0.record(cs)
             torch.cuda.synchronize()
             if rep >= a.warmup:
                 t = s0.elapsed_time(e0)
-                best = t if best is None else min(best, t)
-        return best
+                if best is None or t < best:
+                    best = t
+                    best_bd = layer_breakdown(marks, s0) if breakdown else None
+        return (best, best_bd) if breakdown else best
 
     def compute_only(work):
         def run():
@@ -819,22 +828,47 @@ def run_zero3_passes(a, wl):
             zs.gather_unit(lay, k, shard, slots[k % 3], stream=gs)
         cs.wait_stream(gs)
 
+    def short(bd):
+        return {k: round(v, 4) for k, v in bd.items() if k.startswith("sum_")} | {
+            "max_wait_ms": round(max(bd["wait_ms"]), 4),
+            "layers_waiting": sum(1 for w in bd["wait_ms"] if w > 0.005)}
+
+    set_carveout = torch._C._set_sm_carveout_experimental
+    passes = (("forward", fwd, order_f), ("backward", bwd, order_b))
     res = {"gathers_only_ms": timed(gathers_only)}
-    gs_hi = torch.cuda.Stream(priority=torch.cuda.Stream.priority_range()[1])
-    for name, work, order in (("forward", fwd, order_f), ("backward", bwd, order_b)):
+    for name, work, order in passes:
         res[f"{name}_compute_only_ms"] = timed(compute_only(work))
         for n in (1, 2, 3):
-            res[f"{name}_{n}slot_ms"] = timed(lambda: zero3_pass(lay, shard, slots[:n], order, work, gs, cs))
-        res[f"{name}_2slot_highprio_ms"] = timed(lambda: zero3_pass(lay, shard, slots[:2], order, work, gs_hi, cs))
+            t, bd = timed(lambda: zero3_pass(lay, shard, slots[:n], order, work, gs, cs), breakdown=True)
+            res[f"{name}_{n}slot_ms"] = t
+            res[f"{name}_{n}slot_breakdown"] = short(bd)
         for n in (1, 2):
             res[f"{name}_exposed_gather_{n}slot_ms"] = res[f"{name}_{n}slot_ms"] - res[f"{name}_compute_only_ms"]
-        res[f"{name}_exposed_gather_2slot_highprio_ms"] = (res[f"{name}_2slot_highprio_ms"] -
-                                                           res[f"{name}_compute_only_ms"])
+
+    # gathers on a capped grid beside GEMMs that leave SMs free: the matmul SM carveout
+    # (cuBLAS's SM-count target) x the gather kernels' CTA cap (zero_set_gather_ctas)
+    sweep = []
+    for c in [int(x) for x in a.carveout.split(",")]:
+        set_carveout(c if c > 0 else None)
+        comp = {name: timed(compute_only(work)) for name, work, _ in passes}
+        for gcap in [int(x) for x in a.gather_ctas.split(",")]:
+            lay.set_gather_ctas(gcap)
+            row = {"carveout_sms": c, "gather_ctas": gcap, "gathers_only_ms": round(timed(gathers_only), 4)}
+            for name, work, order in passes:
+                t, bd = timed(lambda: zero3_pass(lay, shard, slots[:2], order, work, gs, cs), breakdown=True)
+                row[f"{name}_compute_only_ms"] = round(comp[name], 4)
+                row[f"{name}_2slot_ms"] = round(t, 4)
+                row[f"{name}_exposed_vs_full_gpu_compute_ms"] = round(t - res[f"{name}_compute_only_ms"], 4)
+                row[f"{name}_breakdown"] = short(bd)
+            sweep.append(row)
+    set_carveout(None)
+    lay.set_gather_ctas(0)
     gather_bytes = 4 * P
     print(json.dumps({"metric": "ZeRO-3 per-layer gather passes with prefetch", "workload": wl.name,
                       "units": lay.n_units, "tokens": T, "gather_bytes_per_pass": gather_bytes,
                       "gather_gbs": gather_bytes / (res["gathers_only_ms"] / 1e3) / 1e9,
-                      **{k: round(v, 4) for k, v in res.items()}}), flush=True)
+                      **{k: (round(v, 4) if isinstance(v, float) else v) for k, v in res.items()},
+                      "sweep": sweep}), flush=True)
 
 
 def main():

@@ -46,7 +46,10 @@ typedef enum {
     ZERO_ERR_CUDA = 3,      /* a CUDA runtime call or kernel launch failed */
     ZERO_ERR_OOM = 4,       /* allocation of the layout's own tables failed */
     ZERO_ERR_TIMEOUT = 5,   /* a bounded wait inside a kernel gave up (see zero_get_error) */
-    ZERO_ERR_STATE = 6      /* layout not uploaded, or uploaded to another device */
+    ZERO_ERR_STATE = 6,     /* layout not uploaded, or uploaded to another device */
+    ZERO_ERR_BOUNDS = 7     /* debug build only (ZERO_DEBUG): a kernel found a segment or tile
+                               index outside the layout's table or buffers, skipped that tile
+                               and recorded this code (see zero_get_error) */
 } zero_status;
 
 typedef struct zero_layout zero_layout;   /* opaque; owned by the library */
@@ -411,6 +414,15 @@ zero_status zero_set_impl(zero_layout *layout, int32_t impl);
  * computed); it is slower alone, since each SM moves at most ~60 GB/s through the
  * step's arithmetic.  Negative k: ZERO_ERR_INVALID.  No counterpart on the pages. */
 zero_status zero_set_max_ctas(zero_layout *layout, int32_t max_ctas);
+
+/* Grid of the all-gather copies (zero_allgather, zero_gather_unit, and the gather inside
+ * the stage-3 steps): 0 (the default) = a grid of short blocks over the whole range, the
+ * fastest when a gather has the GPU to itself; k > 0 = k persistent CTAs of 1024 threads,
+ * each with 128 KB of loads in flight, so that a gather occupies at most k SMs and can run
+ * beside a layer's compute that leaves those SMs free (P1 ZeRO-3: the next layer's
+ * parameters are gathered while the current layer computes).  Results are identical for
+ * every k.  Negative k: ZERO_ERR_INVALID.  No counterpart on the pages. */
+zero_status zero_set_gather_ctas(zero_layout *layout, int32_t max_ctas);
 
 /* Test hook of the bulk-copy pipeline's bounded waits: every in-kernel wait gives up
  * after wait_limit_ns nanoseconds (default 2e9) and records ZERO_ERR_TIMEOUT.  With

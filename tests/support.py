@@ -157,3 +157,51 @@ def assert_state_matches_oracle(wl, got, ref, what=""):
         assert_f16_ulp(to_np(got[name]), want, what + name)
     for name, want in S_f32 + tuple(f16):
         assert_bits_equal(to_np(got[name]), want, what + name + " (bits)")
+
+
+# ---------------------------------------------------------------- guard regions
+# compute-sanitizer is not available to these tests, so writes past a buffer are caught
+# the old way: every output buffer sits between two guard regions of a fixed byte
+# pattern, and the guards are compared after each step.
+
+GUARD_BYTES = 4096          # a multiple of 16, so the guarded buffer keeps 16-byte alignment
+GUARD_BYTE = 0x5A
+
+
+class Guarded:
+    """A device tensor of `n` elements with a guard region before and after it."""
+
+    def __init__(self, n, dtype, fill=None):
+        import torch
+        item = torch.empty((), dtype=dtype).element_size()
+        self.g = GUARD_BYTES // item
+        self.raw = torch.empty(n + 2 * self.g, dtype=dtype, device="cuda")
+        self.raw.view(torch.uint8).fill_(GUARD_BYTE)
+        self.t = self.raw[self.g:self.g + n]
+        if fill is not None:
+            self.t.copy_(fill)
+
+    def intact(self):
+        import torch
+        b = self.raw.view(torch.uint8)
+        return bool((b[:GUARD_BYTES] == GUARD_BYTE).all()) and bool((b[-GUARD_BYTES:] == GUARD_BYTE).all())
+
+
+def guard_outputs(bufs, names=("master", "m", "v", "p16_shard", "p16_full", "nonfinite")):
+    """Move the named tensors of a buffer dict into guarded allocations (same values);
+    returns the guards."""
+    guards = {}
+    for k in names:
+        if bufs.get(k) is None:
+            continue
+        gd = Guarded(bufs[k].numel(), bufs[k].dtype, fill=bufs[k])
+        bufs[k] = gd.t
+        guards[k] = gd
+    return guards
+
+
+def assert_guards_intact(guards, what=""):
+    import torch
+    torch.cuda.synchronize()
+    broken = [k for k, gd in guards.items() if not gd.intact()]
+    assert not broken, f"{what}: guard regions overwritten around {broken}"

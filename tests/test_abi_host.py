@@ -19,7 +19,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module", autouse=True)
 def _built():
-    build.build()
+    build.build_all()
 
 
 def _declared():
@@ -31,10 +31,20 @@ def _declared():
 def test_exports_every_declared_function():
     names = _declared()
     assert len(names) >= 15
-    lib = ctypes.CDLL(_abi.LIB_PATH)
-    for n in names:
-        assert hasattr(lib, n), n
+    for path in (build.LIB, build.LIB_DEBUG):      # the release library and its bounds-checking twin
+        lib = ctypes.CDLL(path)
+        for n in names:
+            assert hasattr(lib, n), (path, n)
     assert set(names) == set(_abi.SIGNATURES)
+
+
+def test_status_codes_named_in_the_binding_and_the_library():
+    src = open(os.path.join(ROOT, "include", "zero.h")).read()
+    codes = {int(v): k for k, v in re.findall(r"\b(ZERO_(?:OK|ERR_[A-Z]+))\s*=\s*(\d+)", src)}
+    assert codes == _abi.STATUS_NAMES
+    lib = _abi.lib()
+    for c in codes:
+        assert lib.zero_status_string(c).decode() != "unknown status", codes[c]
 
 
 def _compare(tensors, N, stage, B, A, units):
@@ -113,7 +123,10 @@ def test_tuning_setters_validate_arguments():
     lay.set_max_ctas(0)
     lay.set_max_ctas(37)
     lay.set_impl(2)
-    for bad in (lambda: lay.set_max_ctas(-1), lambda: lay.set_impl(3), lambda: lay.set_impl(-1)):
+    lay.set_gather_ctas(0)
+    lay.set_gather_ctas(16)
+    for bad in (lambda: lay.set_max_ctas(-1), lambda: lay.set_impl(3), lambda: lay.set_impl(-1),
+                lambda: lay.set_gather_ctas(-1)):
         with pytest.raises(zs.ZeroError) as e:
             bad()
         assert e.value.status == 1

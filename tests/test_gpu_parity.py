@@ -36,12 +36,16 @@ def _layout(wl, impl=zs.IMPL_REGISTER):
 IMPLS = [zs.IMPL_REGISTER, zs.IMPL_BULK]
 
 
-def _bufs(lay, wl, rank_stride=None):
+def _bufs(lay, wl, rank_stride=None, guard=False):
+    """Device inputs and zeroed outputs; with guard=True every written buffer sits between
+    guard regions (S.Guarded), checked by _run after each step."""
     g, master, m, v = S.device_inputs(wl, lay.padded, rank_stride)
     p16_shard = torch.zeros(lay.padded, dtype=torch.int16, device="cuda")
     p16_full = torch.zeros(lay.padded, dtype=torch.int16, device="cuda")
     nonfinite = torch.zeros(max(1, lay.n_buckets), dtype=torch.int32, device="cuda")
-    return dict(g=g, master=master, m=m, v=v, p16_shard=p16_shard, p16_full=p16_full, nonfinite=nonfinite)
+    b = dict(g=g, master=master, m=m, v=v, p16_shard=p16_shard, p16_full=p16_full, nonfinite=nonfinite)
+    b["_guards"] = S.guard_outputs(b) if guard else {}
+    return b
 
 
 def _run(lay, wl, b, steps):
@@ -49,6 +53,8 @@ def _run(lay, wl, b, steps):
         b["nonfinite"].zero_()
         zs.step(lay, b["g"], b["master"], b["m"], b["v"], b["p16_shard"], b["p16_full"], _hp(wl, t),
                 nonfinite=b["nonfinite"])
+        if b["_guards"]:
+            S.assert_guards_intact(b["_guards"], f"step {t}")
     zs.get_error(lay)
     torch.cuda.synchronize()
 
@@ -95,7 +101,7 @@ def test_reduced_workload_all_elements(key, impl):
     ref, olay = _oracle(wl)
     lay = _layout(wl, impl)
     assert lay.n_tiles >= 8 and lay.n_buckets >= 1     # several tiles, ragged edges
-    b = _bufs(lay, wl)
+    b = _bufs(lay, wl, guard=True)
     _run(lay, wl, b, wl.steps)
     _check_full(wl, lay, b, ref)
 
@@ -142,7 +148,7 @@ def test_deterministic_rerun():
     for _ in range(2):
         b = _bufs(lay, wl)
         _run(lay, wl, b, 2)
-        outs.append({k: _np(v) for k, v in b.items() if k != "g"})
+        outs.append({k: _np(v) for k, v in b.items() if k not in ("g", "_guards")})
     for k in outs[0]:
         S.assert_bits_equal(outs[0][k], outs[1][k], k)
 
@@ -203,7 +209,7 @@ def test_edge_cases(key, impl):
     wl = EDGES[key]
     ref, _ = _oracle(wl)
     lay = _layout(wl, impl)
-    b = _bufs(lay, wl)
+    b = _bufs(lay, wl, guard=True)
     _run(lay, wl, b, wl.steps)
     _check_full(wl, lay, b, ref)
 

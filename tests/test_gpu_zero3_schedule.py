@@ -48,10 +48,12 @@ def _stepped_shards(wl):
     return lay, p16_shard, ref
 
 
+@pytest.mark.parametrize("gather_ctas", [0, 1, 3, 16])
 @pytest.mark.parametrize("aligned", [True, False])
-def test_gather_unit_matches_oracle(aligned):
+def test_gather_unit_matches_oracle(aligned, gather_ctas):
     wl = _workload(aligned)
     lay, shard, ref = _stepped_shards(wl)
+    lay.set_gather_ctas(gather_ctas)            # the grid is the caller's choice; results are not
     _, _, _, u = lay.tables()
     assert aligned == all(lo % 8 == 0 for lo, _ in u)
     for k, (lo, hi) in enumerate(u):
@@ -61,6 +63,28 @@ def test_gather_unit_matches_oracle(aligned):
         got = S.to_np(dst)
         S.assert_bits_equal(got[:hi - lo], ref.p16_full[lo:hi], f"unit {k}")
         assert (got[hi - lo:] == 7).all(), f"unit {k}: write past the unit"
+
+
+@pytest.mark.parametrize("gather_ctas", [1, 5, 148])
+@pytest.mark.parametrize("aligned", [True, False])
+def test_capped_allgather_matches_oracle(aligned, gather_ctas):
+    """zero_allgather (whole buffer and unit by unit, unaligned unit edges included) on a
+    capped grid writes exactly the oracle's gathered parameters and nothing else."""
+    wl = _workload(aligned)
+    lay, shard, ref = _stepped_shards(wl)
+    lay.set_gather_ctas(gather_ctas)
+    _, _, _, u = lay.tables()
+    full = torch.full((lay.padded + 64,), 7, dtype=torch.int16, device="cuda")
+    zs.allgather(lay, -1, shard, full[:lay.padded])
+    torch.cuda.synchronize()
+    S.assert_bits_equal(S.to_np(full)[:lay.padded], ref.p16_full, "whole buffer")
+    assert (S.to_np(full)[lay.padded:] == 7).all()
+    full.fill_(7)
+    for k in range(lay.n_units):
+        zs.allgather(lay, k, shard, full[:lay.padded])
+    torch.cuda.synchronize()
+    S.assert_bits_equal(S.to_np(full)[:lay.padded], ref.p16_full, "unit by unit")
+    assert (S.to_np(full)[lay.padded:] == 7).all()
 
 
 @pytest.mark.parametrize("n_slots", [1, 2, 3])

@@ -50,12 +50,14 @@ def test_noalloc_matches_step_on_two_calls(key):
     assert host_only.n_segments <= _abi.NOALLOC_MAX_SEGMENTS
     a = _bufs(uploaded.padded, wl)
     b = _bufs(uploaded.padded, wl)
+    guards = S.guard_outputs(b)            # a write past any output buffer shows up here
     for t in (1, 2):
         zs.step(uploaded, a["g"], a["master"], a["m"], a["v"], a["p16_shard"], a["p16_full"], _hp(wl, t),
                 nonfinite=a["nonfinite"])
         zs.step_noalloc(host_only, b["g"], b["master"], b["m"], b["v"], b["p16_shard"], b["p16_full"],
                         _hp(wl, t), nonfinite=b["nonfinite"])
         torch.cuda.synchronize()
+        S.assert_guards_intact(guards, f"call {t}")
         S.assert_f32_close(_np(b["master"]), _np(a["master"]), f"master after call {t}")
         S.assert_f32_close(_np(b["m"]), _np(a["m"]), f"m after call {t}")
         S.assert_f32_close(_np(b["v"]), _np(a["v"]), f"v after call {t}")

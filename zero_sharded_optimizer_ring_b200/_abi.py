@@ -3,7 +3,9 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libzero_b200.so")
+# ZERO_B200_DEBUG=1 selects the bounds-checking build (libzero_b200_debug.so, same ABI)
+DEBUG = os.environ.get("ZERO_B200_DEBUG", "") == "1"
+LIB_PATH = os.path.join(_HERE, "libzero_b200_debug.so" if DEBUG else "libzero_b200.so")
 
 _vp = ctypes.c_void_p
 _i64 = ctypes.c_int64
@@ -13,7 +15,7 @@ _p_i64 = ctypes.POINTER(ctypes.c_int64)
 ZERO_OK = 0
 NOALLOC_MAX_SEGMENTS = 8191   # ZERO_NOALLOC_MAX_SEGMENTS in include/zero.h
 STATUS_NAMES = {0: "ZERO_OK", 1: "ZERO_ERR_INVALID", 2: "ZERO_ERR_ALIGN", 3: "ZERO_ERR_CUDA",
-                4: "ZERO_ERR_OOM", 5: "ZERO_ERR_TIMEOUT", 6: "ZERO_ERR_STATE"}
+                4: "ZERO_ERR_OOM", 5: "ZERO_ERR_TIMEOUT", 6: "ZERO_ERR_STATE", 7: "ZERO_ERR_BOUNDS"}
 
 
 class LayoutDesc(ctypes.Structure):
@@ -89,6 +91,7 @@ SIGNATURES = {
     "zero_gather_unit_ranks": (_i32, [_vp, _i64, _vp, _vp, _vp]),
     "zero_set_impl": (_i32, [_vp, _i32]),
     "zero_set_max_ctas": (_i32, [_vp, _i32]),
+    "zero_set_gather_ctas": (_i32, [_vp, _i32]),
     "zero_debug_set_wait": (_i32, [_vp, _i64, _i32]),
     "zero_get_error": (_i32, [_vp, _vp]),
     "zero_status_string": (ctypes.c_char_p, [_i32]),
@@ -103,7 +106,8 @@ def lib():
     if _LIB is None:
         if not os.path.exists(LIB_PATH):
             raise ImportError(f"{LIB_PATH} is missing: build it with "
-                              "`python -m zero_sharded_optimizer_ring_b200.build` (nvcc, sm_100a)")
+                              "`python -m zero_sharded_optimizer_ring_b200.build"
+                              f"{' --debug' if DEBUG else ''}` (nvcc, sm_100a)")
         L = ctypes.CDLL(LIB_PATH)
         for name, (res, args) in SIGNATURES.items():
             fn = getattr(L, name)

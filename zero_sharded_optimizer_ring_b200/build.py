@@ -13,6 +13,9 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libzero_b200.so")
+# the same sources with ZERO_DEBUG: every located segment and tile is bounds-checked in the
+# kernels (a failed check skips the tile and records ZERO_ERR_BOUNDS; nothing traps)
+LIB_DEBUG = os.path.join(HERE, "libzero_b200_debug.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
@@ -29,23 +32,32 @@ def _deps():
     return files
 
 
-def build(force=False, verbose_ptxas=False):
-    if not force and os.path.exists(LIB):
-        t = os.path.getmtime(LIB)
+def build(force=False, verbose_ptxas=False, debug=False):
+    lib = LIB_DEBUG if debug else LIB
+    if not force and os.path.exists(lib):
+        t = os.path.getmtime(lib)
         if all(os.path.getmtime(f) <= t for f in _deps()):
-            return LIB
-    os.makedirs(BUILD_DIR, exist_ok=True)
+            return lib
+    out_dir = os.path.join(BUILD_DIR, "debug" if debug else "release")
+    os.makedirs(out_dir, exist_ok=True)
     objs = []
     for src in SOURCES:
-        obj = os.path.join(BUILD_DIR, src + ".o")
+        obj = os.path.join(out_dir, src + ".o")
         extra = ["-Xptxas", "-v"] if verbose_ptxas and src.endswith(".cu") else []
+        if debug:
+            extra.append("-DZERO_DEBUG")
         subprocess.run([NVCC, *ARCH, *FLAGS, *extra, "-c", os.path.join(CSRC, src), "-o", obj], check=True)
         objs.append(obj)
-    tmp = LIB + ".tmp"
-    subprocess.run([NVCC, *ARCH, "-shared", "-o", tmp, *objs], check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    tmp = lib + ".tmp"
+    subprocess.run([NVCC, *ARCH, "-shared", "-o", tmp, *objs, "-ldl"], check=True)
+    os.replace(tmp, lib)
+    return lib
+
+
+def build_all(force=False):
+    """The release library and its bounds-checking debug twin."""
+    return build(force=force), build(force=force, debug=True)
 
 
 if __name__ == "__main__":
-    build(force=True, verbose_ptxas="-v" in sys.argv)
+    build(force=True, verbose_ptxas="-v" in sys.argv, debug="--debug" in sys.argv)

@@ -39,6 +39,7 @@ TileWork all_tiles(const zero_layout *L)
     w.seg_first = 0;
     w.tile_first = 0;
     w.n_tiles = L->n_tiles;
+    w.bounds = zero::tile_bounds(*L, 0, L->padded);
     return w;
 }
 
@@ -53,6 +54,7 @@ TileWork bucket_range_tiles(const zero_layout *L, int64_t b0, int64_t b1)
     w.tile_first = L->segs[(size_t)w.seg_first].tile_begin;
     const int64_t tile_end = seg_end < (int64_t)L->segs.size() ? L->segs[(size_t)seg_end].tile_begin : L->n_tiles;
     w.n_tiles = tile_end - w.tile_first;
+    w.bounds = zero::tile_bounds(*L, 0, L->padded);
     return w;
 }
 
@@ -144,12 +146,14 @@ extern "C" const char *zero_status_string(zero_status s)
         case ZERO_ERR_OOM: return "out of memory";
         case ZERO_ERR_TIMEOUT: return "a bounded wait in a kernel timed out";
         case ZERO_ERR_STATE: return "layout not uploaded to the current device";
+        case ZERO_ERR_BOUNDS: return "a kernel found a segment or tile index out of bounds (debug build)";
     }
     return "unknown status";
 }
 
 extern "C" zero_status zero_layout_to_device(zero_layout *L, void *stream)
 {
+    ZERO_RANGE("zero_layout_to_device");
     if (!L) return ZERO_ERR_INVALID;
     int cur = -1;
     if (cudaGetDevice(&cur) != cudaSuccess) return ZERO_ERR_CUDA;
@@ -210,6 +214,7 @@ extern "C" zero_status zero_layout_to_device(zero_layout *L, void *stream)
 
 extern "C" zero_status zero_layout_device_segments(const zero_layout *L, int64_t *out, void *stream)
 {
+    ZERO_RANGE("zero_layout_device_segments");
     zero_status s = check_device(L);
     if (s != ZERO_OK) return s;
     if (!out) return ZERO_ERR_INVALID;
@@ -232,6 +237,7 @@ extern "C" zero_status zero_reduce_scatter(const zero_layout *L, int64_t bucket,
                                            int64_t rank_stride, float *reduced, int32_t *nonfinite,
                                            void *stream)
 {
+    ZERO_RANGE("zero_reduce_scatter");
     zero_status s = check_device(L);
     if (s != ZERO_OK) return s;
     if (bucket < -1 || bucket >= (int64_t)L->bucket_lo.size()) return ZERO_ERR_INVALID;
@@ -248,6 +254,7 @@ extern "C" zero_status zero_adamw_shard_step(const zero_layout *L, int32_t shard
                                              float *master, float *m, float *v, uint16_t *p16_out,
                                              const zero_adamw_hparams *hp, void *stream)
 {
+    ZERO_RANGE("zero_adamw_shard_step");
     zero_status s = check_device(L);
     if (s != ZERO_OK) return s;
     if (shard < -1 || shard >= L->n_ranks) return ZERO_ERR_INVALID;
@@ -265,6 +272,7 @@ extern "C" zero_status zero_adamw_shard_step(const zero_layout *L, int32_t shard
 extern "C" zero_status zero_allgather(const zero_layout *L, int64_t unit, const uint16_t *p16_shard,
                                       uint16_t *p16_full, void *stream)
 {
+    ZERO_RANGE("zero_allgather");
     zero_status s = check_device(L);
     if (s != ZERO_OK) return s;
     if (unit < -1 || unit >= (int64_t)L->unit_lo.size()) return ZERO_ERR_INVALID;
@@ -279,18 +287,20 @@ extern "C" zero_status zero_allgather(const zero_layout *L, int64_t unit, const 
 extern "C" zero_status zero_gather_unit(const zero_layout *L, int64_t unit, const uint16_t *p16_shard,
                                         uint16_t *dst, void *stream)
 {
+    ZERO_RANGE("zero_gather_unit");
     zero_status s = check_device(L);
     if (s != ZERO_OK) return s;
     if (unit < 0 || unit >= (int64_t)L->unit_lo.size() || !p16_shard || !dst) return ZERO_ERR_INVALID;
     if (!aligned16(p16_shard) || !aligned16(dst)) return ZERO_ERR_ALIGN;
     const int64_t lo = L->unit_lo[(size_t)unit];
-    return cuda_status(zero::launch_gather_unit(p16_shard, lo, L->unit_hi[(size_t)unit] - lo, dst,
+    return cuda_status(zero::launch_gather_unit(p16_shard, lo, L->unit_hi[(size_t)unit] - lo, dst, L->gather_ctas,
                                                 (cudaStream_t)stream));
 }
 
 extern "C" zero_status zero_gather_unit_ranks(const zero_layout *L, int64_t unit, const uint16_t *const *rank_p16,
                                               uint16_t *dst, void *stream)
 {
+    ZERO_RANGE("zero_gather_unit_ranks");
     zero_status s = check_device(L);
     if (s != ZERO_OK) return s;
     if (unit < 0 || unit >= (int64_t)L->unit_lo.size() || !rank_p16 || !dst) return ZERO_ERR_INVALID;
@@ -358,6 +368,7 @@ extern "C" zero_status zero_step(const zero_layout *L, const uint16_t *grads, in
                                  uint16_t *p16_full, const zero_adamw_hparams *hp,
                                  int32_t *nonfinite, const zero_step_events *ev, void *stream)
 {
+    ZERO_RANGE("zero_step");
     zero_status s = check_step(L, grads, rank_stride, master, m, v, p16_shard, p16_full, hp);
     if (s != ZERO_OK || L->padded == 0) return s;
     cudaStream_t st = (cudaStream_t)stream;
@@ -379,6 +390,7 @@ extern "C" zero_status zero_step_bucket(const zero_layout *L, int64_t bucket, co
                                         uint16_t *p16_shard, uint16_t *p16_full, const zero_adamw_hparams *hp,
                                         int32_t *nonfinite, void *stream)
 {
+    ZERO_RANGE("zero_step_bucket");
     zero_status s = check_step(L, grads, rank_stride, master, m, v, p16_shard, p16_full, hp);
     if (s != ZERO_OK || L->padded == 0) return s;
     if (bucket < 0 || bucket >= (int64_t)L->bucket_lo.size()) return ZERO_ERR_INVALID;
@@ -392,6 +404,7 @@ extern "C" zero_status zero_step_overlapped_grouped(const zero_layout *L, void *
                                                     float *v, uint16_t *p16_shard, uint16_t *p16_full,
                                                     const zero_adamw_hparams *hp, int32_t *nonfinite, void *stream)
 {
+    ZERO_RANGE("zero_step_overlapped_grouped");
     zero_status s = check_step(L, grads, rank_stride, master, m, v, p16_shard, p16_full, hp);
     if (s != ZERO_OK) return s;
     if (group < 1) return ZERO_ERR_INVALID;
@@ -419,6 +432,7 @@ extern "C" zero_status zero_step_overlapped(const zero_layout *L, void *const *r
                                             uint16_t *p16_shard, uint16_t *p16_full, const zero_adamw_hparams *hp,
                                             int32_t *nonfinite, void *stream)
 {
+    ZERO_RANGE("zero_step_overlapped");
     return zero_step_overlapped_grouped(L, ready_events, 1, grads, rank_stride, master, m, v, p16_shard, p16_full,
                                         hp, nonfinite, stream);
 }
@@ -474,6 +488,7 @@ extern "C" zero_status zero_step_dynamic(const zero_layout *L, const uint16_t *g
                                          uint16_t *p16_full, const zero_adamw_hparams *hp, zero_loss_scaler *sc,
                                          int32_t *nonfinite, int32_t *applied, void *stream)
 {
+    ZERO_RANGE("zero_step_dynamic");
     if (!L || !hp || !sc || !applied) return ZERO_ERR_INVALID;
     if (!scaler_valid(sc)) return ZERO_ERR_INVALID;
     zero_adamw_hparams h = *hp;
@@ -510,6 +525,7 @@ extern "C" zero_status zero_step_dynamic_commit(const zero_layout *L, const uint
                                                 zero_loss_scaler *sc, int32_t *nonfinite, int32_t *applied,
                                                 void *stream)
 {
+    ZERO_RANGE("zero_step_dynamic_commit");
     if (!L || !hp || !sc || !applied) return ZERO_ERR_INVALID;
     if (!scaler_valid(sc)) return ZERO_ERR_INVALID;
     zero_adamw_hparams h = *hp;
@@ -564,6 +580,7 @@ TileWork shard_tiles(const zero_layout *L, int64_t k)
     const int64_t tile_end =
         seg_end < (int64_t)L->segs_by_shard.size() ? L->segs_by_shard[(size_t)seg_end].tile_begin : L->n_tiles;
     w.n_tiles = tile_end - w.tile_first;
+    w.bounds = zero::tile_bounds(*L, k * L->shard, (k + 1) * L->shard);   // shard-local state
     return w;
 }
 
@@ -586,6 +603,7 @@ extern "C" zero_status zero_step_ranks(const zero_layout *L, const uint16_t *con
                                        float *m, float *v, uint16_t *p16_shard, uint16_t *p16_full,
                                        const zero_adamw_hparams *hp, int32_t *nonfinite, void *stream)
 {
+    ZERO_RANGE("zero_step_ranks");
     zero_status s = check_device(L);
     if (s != ZERO_OK) return s;
     if ((s = check_hparams(hp)) != ZERO_OK) return s;
@@ -608,6 +626,7 @@ extern "C" zero_status zero_step_shard(const zero_layout *L, int32_t shard, cons
                                        float *master_k, float *m_k, float *v_k, uint16_t *p16_out,
                                        const zero_adamw_hparams *hp, int32_t *nonfinite, void *stream)
 {
+    ZERO_RANGE("zero_step_shard");
     zero_status s = check_device(L);
     if (s != ZERO_OK) return s;
     if ((s = check_hparams(hp)) != ZERO_OK) return s;
@@ -631,6 +650,7 @@ extern "C" zero_status zero_step_shard_commit(const zero_layout *L, int32_t shar
                                               const zero_adamw_hparams *hp, const zero_loss_scaler *sc,
                                               int32_t *nonfinite, int64_t *nonfinite_total, void *stream)
 {
+    ZERO_RANGE("zero_step_shard_commit");
     if (!L || !hp || !sc || !nonfinite_total) return ZERO_ERR_INVALID;
     if (!scaler_valid(sc)) return ZERO_ERR_INVALID;
     zero_status s = check_device(L);
@@ -668,6 +688,7 @@ extern "C" zero_status zero_step_shard_commit(const zero_layout *L, int32_t shar
 
 extern "C" zero_status zero_loss_scaler_advance(zero_loss_scaler *sc, int32_t applied)
 {
+    ZERO_RANGE("zero_loss_scaler_advance");
     if (!sc || !scaler_valid(sc) || applied < 0 || applied > 1) return ZERO_ERR_INVALID;
     scaler_advance(sc, applied == 1);
     return ZERO_OK;
@@ -676,6 +697,7 @@ extern "C" zero_status zero_loss_scaler_advance(zero_loss_scaler *sc, int32_t ap
 extern "C" zero_status zero_copy_shard(const zero_layout *L, int32_t shard, const uint16_t *src, uint16_t *dst,
                                        void *stream)
 {
+    ZERO_RANGE("zero_copy_shard");
     zero_status s = check_device(L);
     if (s != ZERO_OK) return s;
     if (shard < 0 || shard >= L->n_ranks || !src || !dst) return ZERO_ERR_INVALID;
@@ -709,6 +731,7 @@ MemRangeFn mem_range_fn()
 
 extern "C" zero_status zero_ipc_get_handle(const void *dev_ptr, void *handle_out, int64_t *offset_out)
 {
+    ZERO_RANGE("zero_ipc_get_handle");
     if (!dev_ptr || !handle_out || !offset_out) return ZERO_ERR_INVALID;
     MemRangeFn range = mem_range_fn();
     if (!range) return ZERO_ERR_CUDA;
@@ -725,6 +748,7 @@ extern "C" zero_status zero_ipc_get_handle(const void *dev_ptr, void *handle_out
 
 extern "C" zero_status zero_ipc_open(const void *handle, int64_t offset, void **dev_ptr_out)
 {
+    ZERO_RANGE("zero_ipc_open");
     if (!handle || !dev_ptr_out || offset < 0) return ZERO_ERR_INVALID;
     cudaIpcMemHandle_t h;
     memcpy(&h, handle, sizeof h);
@@ -737,6 +761,7 @@ extern "C" zero_status zero_ipc_open(const void *handle, int64_t offset, void **
 
 extern "C" zero_status zero_ipc_close(void *dev_ptr, int64_t offset)
 {
+    ZERO_RANGE("zero_ipc_close");
     if (!dev_ptr || offset < 0) return ZERO_ERR_INVALID;
     return cudaIpcCloseMemHandle(static_cast<char *>(dev_ptr) - offset) == cudaSuccess ? ZERO_OK : ZERO_ERR_CUDA;
 }
@@ -746,6 +771,7 @@ extern "C" zero_status zero_step_host(const zero_layout *L, const uint16_t *grad
                                       uint16_t *p16_shard, uint16_t *p16_full, uint16_t *p16_host,
                                       const zero_adamw_hparams *hp, int32_t *nonfinite, void *stream)
 {
+    ZERO_RANGE("zero_step_host");
     zero_status s = check_step(L, grads_dev, rank_stride, master, m, v, p16_shard, p16_full, hp);
     if (s != ZERO_OK || L->padded == 0) return s;
     if (!grads_host || !p16_host) return ZERO_ERR_INVALID;
@@ -794,6 +820,7 @@ extern "C" zero_status zero_step_host(const zero_layout *L, const uint16_t *grad
 
 extern "C" zero_status zero_get_error(const zero_layout *L, void *stream)
 {
+    ZERO_RANGE("zero_get_error");
     zero_status s = check_device(L);
     if (s != ZERO_OK) return s;
     cudaStream_t st = (cudaStream_t)stream;
@@ -807,6 +834,7 @@ extern "C" zero_status zero_get_error(const zero_layout *L, void *stream)
 
 extern "C" zero_status zero_debug_set_wait(zero_layout *L, int64_t wait_limit_ns, int32_t skip_first_fill)
 {
+    ZERO_RANGE("zero_debug_set_wait");
     if (!L || wait_limit_ns <= 0 || skip_first_fill < 0 || skip_first_fill > 1) return ZERO_ERR_INVALID;
     if (L->dev.device < 0) return ZERO_ERR_STATE;
     L->dev.wait_limit_ns = (uint64_t)wait_limit_ns;

@@ -158,7 +158,8 @@ __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(co
         uint32_t posted = 0;      // chunks whose copies were issued
         bool ok = true;
         for (int64_t t = A.w.tile_first + blockIdx.x; ok && t < t_end; t += gridDim.x) {
-            const TileRange tr = locate_tile(A.w.segs, s, t);
+            const TileRange tr = locate_tile(A.w, s, t);
+            if (!tile_in_bounds(A.w, s, tr)) continue;     // debug builds; the consumers skip it too
             const int64_t va = (tr.a + kVec - 1) / kVec * kVec, vb = tr.b / kVec * kVec;
             for (int64_t q0 = va; ok && q0 < vb; q0 += kChunk, ++it) {
                 const uint32_t st = it % (uint32_t)A.stages, ph = (it / (uint32_t)A.stages) & 1u;
@@ -200,7 +201,8 @@ __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(co
     int64_t s = A.w.seg_first;
     uint32_t it = 0;
     for (int64_t t = A.w.tile_first + blockIdx.x; t < t_end; t += gridDim.x) {
-        const TileRange tr = locate_tile(A.w.segs, s, t);
+        const TileRange tr = locate_tile(A.w, s, t);
+        if (!tile_in_bounds(A.w, s, tr)) continue;
         const int64_t va = (tr.a + kVec - 1) / kVec * kVec, vb = tr.b / kVec * kVec;
         int bad = 0;
         for (int64_t q0 = va; q0 < vb; q0 += kChunk, ++it) {

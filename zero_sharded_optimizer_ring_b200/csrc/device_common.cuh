@@ -145,10 +145,16 @@ struct TileRange {
 
 // Locate tile t: advance the segment cursor s (tiles are visited in increasing order
 // by each CTA, so the cursor only moves forward), then clip the tile's cell of the
-// global kTileElems grid to the segment.
-__device__ __forceinline__ TileRange locate_tile(const Seg *__restrict__ segs, int64_t &s, int64_t t)
+// global kTileElems grid to the segment.  A debug build never lets the cursor pass the
+// closing row.
+__device__ __forceinline__ TileRange locate_tile(const TileWork &w, int64_t &s, int64_t t)
 {
+    const Seg *__restrict__ segs = w.segs;
+#ifdef ZERO_DEBUG
+    while (s < w.bounds.n_seg && __ldg(&segs[s + 1].tile_begin) <= t) ++s;
+#else
     while (__ldg(&segs[s + 1].tile_begin) <= t) ++s;
+#endif
     const int64_t lo = __ldg(&segs[s].lo), hi = __ldg(&segs[s].hi);
     const int64_t cell = lo / kTileElems + (t - __ldg(&segs[s].tile_begin));
     TileRange r;
@@ -157,6 +163,27 @@ __device__ __forceinline__ TileRange locate_tile(const Seg *__restrict__ segs, i
     r.shard = __ldg(&segs[s].shard);
     r.bucket = __ldg(&segs[s].bucket);
     return r;
+}
+
+// Debug builds: does the located tile lie inside the table, its shard, the padded buffer
+// and the launch's state buffers?  If not, record ZERO_ERR_BOUNDS (first error wins) and
+// tell the caller to skip it.  Release builds: always true, compiled away.
+__device__ __forceinline__ bool tile_in_bounds(const TileWork &w, int64_t s, const TileRange &r)
+{
+#ifdef ZERO_DEBUG
+    const TileBounds &B = w.bounds;
+    const bool ok = s >= w.seg_first && s < B.n_seg && r.a >= 0 && r.a < r.b && r.b <= B.padded &&
+                    r.b - r.a <= kTileElems && r.shard >= 0 && r.shard < B.n_ranks && r.bucket >= 0 &&
+                    r.bucket < B.n_buckets && r.a >= (int64_t)r.shard * B.shard &&
+                    r.b <= ((int64_t)r.shard + 1) * B.shard && r.a >= B.state_lo && r.b <= B.state_hi;
+    if (!ok && B.error) atomicCAS(B.error, 0, (int32_t)ZERO_ERR_BOUNDS);
+    return ok;
+#else
+    (void)w;
+    (void)s;
+    (void)r;
+    return true;
+#endif
 }
 
 // Rank at position j of the ring fold that starts at rank k.

@@ -2,13 +2,26 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
 #include <vector>
 
 #include "zero.h"
 
+// One named NVTX range per ABI call, so that a profiler's timeline (or an ncu --nvtx
+// filter) shows which entry point launched which kernels.  Without an attached tool the
+// push and pop are a test of a null pointer each.
+#define ZERO_RANGE(name) zero::CallRange zero_call_range_(name)
+
 namespace zero {
+
+struct CallRange {
+    explicit CallRange(const char *name) { nvtxRangePushA(name); }
+    ~CallRange() { nvtxRangePop(); }
+    CallRange(const CallRange &) = delete;
+    CallRange &operator=(const CallRange &) = delete;
+};
 
 // Elements per tile: the unit of work one CTA picks up.  A multiple of 8 so that
 // tile boundaries fall on 16-byte fp16 vectors.
@@ -41,12 +54,25 @@ struct AdamScalars {
     float eps;
 };
 
+// What a debug build (ZERO_DEBUG) checks every located tile against; filled by the
+// launch wrappers, read by no release kernel.  A tile that fails the check is skipped and
+// ZERO_ERR_BOUNDS is recorded in `error` (when non-null); nothing is read or written out
+// of bounds and nothing traps.
+struct TileBounds {
+    int64_t n_seg = 0;                   // table rows before the closing row
+    int64_t padded = 0, shard = 0;       // P, S
+    int64_t state_lo = 0, state_hi = 0;  // flat range the state buffers of the launch cover
+    int32_t n_ranks = 0, n_buckets = 0;
+    int32_t *error = nullptr;            // device error word
+};
+
 // Launch arguments of the tile-walking kernels (reduce-scatter, fused step).
 struct TileWork {
     const Seg *segs;       // device segment table (n_seg + 1 rows, last = sentinel)
     int64_t seg_first;     // first row of the launch's range
     int64_t tile_first;    // first global tile of the launch
     int64_t n_tiles;       // tiles in the launch
+    TileBounds bounds;     // debug builds only
 };
 
 struct DeviceState {
@@ -80,6 +106,7 @@ struct zero_layout {
     int64_t n_tiles = 0;
     int32_t impl = 0;
     int32_t max_ctas = 0;                      // > 0: cap on the grid of the tile-walking kernels
+    int32_t gather_ctas = 0;                   // > 0: the gathers run as that many persistent CTAs
     zero::DeviceState dev;
 };
 
@@ -91,6 +118,8 @@ zero_status check_hparams(const zero_adamw_hparams *h);
 AdamScalars step_scalars(int32_t n_ranks, const zero_adamw_hparams &h);
 
 // kernels.cu
+// The bounds of a launch over layout L whose state buffers cover flat [state_lo, state_hi).
+TileBounds tile_bounds(const zero_layout &L, int64_t state_lo, int64_t state_hi);
 cudaError_t launch_tile_index(Seg *segs, int64_t n_seg, cudaStream_t s);
 cudaError_t launch_reduce_scatter(const zero_layout &L, const TileWork &w, const uint16_t *grads,
                                   int64_t stride, float *reduced, int32_t *nonfinite, cudaStream_t s);
@@ -99,7 +128,8 @@ cudaError_t launch_adamw_range(const zero_layout &L, int64_t lo, int64_t hi, con
                                const AdamScalars &c, cudaStream_t s);
 cudaError_t launch_copy_range(const zero_layout &L, int64_t lo, int64_t hi, const uint16_t *src,
                               uint16_t *dst, cudaStream_t s);
-cudaError_t launch_gather_unit(const uint16_t *src, int64_t lo, int64_t n, uint16_t *dst, cudaStream_t s);
+cudaError_t launch_gather_unit(const uint16_t *src, int64_t lo, int64_t n, uint16_t *dst, int32_t max_ctas,
+                               cudaStream_t s);
 cudaError_t launch_fused_step(const zero_layout &L, const TileWork &w, const uint16_t *grads,
                               int64_t stride, float *master, float *m, float *v, uint16_t *p16,
                               const AdamScalars &c, int32_t *nonfinite, cudaStream_t s);

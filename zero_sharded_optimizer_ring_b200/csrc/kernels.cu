@@ -67,7 +67,8 @@ tile_kernel(TileWork w, int n_ranks, const uint16_t *__restrict__ grads, int64_t
     int64_t s = w.seg_first;
     const int64_t t_end = w.tile_first + w.n_tiles;
     for (int64_t t = w.tile_first + blockIdx.x; t < t_end; t += gridDim.x) {
-        const TileRange tr = locate_tile(w.segs, s, t);
+        const TileRange tr = locate_tile(w, s, t);
+        if (!tile_in_bounds(w, s, tr)) continue;
         const int k = tr.shard;
         int bad = 0;
         const int64_t va = (tr.a + kVec - 1) / kVec * kVec;
@@ -265,6 +266,51 @@ copy_range_kernel(int64_t lo, int64_t hi, const uint16_t *__restrict__ src, uint
     }
 }
 
+// Copy on a capped grid of persistent CTAs: d[j] = s[j] for j < n (s and d 16-byte
+// aligned), plus hn < 8 head elements hd[j] = hs[j].  Each thread keeps kCapUnroll 16-byte
+// vectors in flight, so one CTA of 1024 threads has 128 KB of loads outstanding: enough to
+// draw a large share of HBM bandwidth from a few SMs while the rest of the GPU computes
+// (the gathers of a ZeRO-3 forward pass beside its GEMMs).
+constexpr int kCapThreads = 1024;
+constexpr int kCapUnroll = 8;
+
+__global__ void __launch_bounds__(kCapThreads)
+copy_capped_kernel(const uint16_t *__restrict__ s, uint16_t *__restrict__ d, int64_t n,
+                   const uint16_t *__restrict__ hs, uint16_t *__restrict__ hd, int hn)
+{
+    const int64_t nv = n / kVec;
+    const int64_t step = (int64_t)gridDim.x * kCapThreads * kCapUnroll;
+    for (int64_t base = (int64_t)blockIdx.x * kCapThreads * kCapUnroll; base < nv; base += step) {
+        uint4 x[kCapUnroll];
+#pragma unroll
+        for (int u = 0; u < kCapUnroll; ++u) {
+            const int64_t q = base + (int64_t)u * kCapThreads + threadIdx.x;
+            if (q < nv) x[u] = __ldcs(reinterpret_cast<const uint4 *>(s + q * kVec));
+        }
+#pragma unroll
+        for (int u = 0; u < kCapUnroll; ++u) {
+            const int64_t q = base + (int64_t)u * kCapThreads + threadIdx.x;
+            if (q < nv) __stcs(reinterpret_cast<uint4 *>(d + q * kVec), x[u]);
+        }
+    }
+    if (blockIdx.x == 0) {
+        if (threadIdx.x < n - nv * kVec) d[nv * kVec + threadIdx.x] = s[nv * kVec + threadIdx.x];
+        if (threadIdx.x < hn) hd[threadIdx.x] = hs[threadIdx.x];
+    }
+}
+
+cudaError_t launch_copy_capped(const uint16_t *s, uint16_t *d, int64_t n, const uint16_t *hs, uint16_t *hd, int hn,
+                               int32_t max_ctas, cudaStream_t st)
+{
+    if (n <= 0 && hn <= 0) return cudaSuccess;
+    const int64_t per_cta = (int64_t)kCapThreads * kCapUnroll * kVec;
+    int64_t grid = (n + per_cta - 1) / per_cta;
+    if (grid > max_ctas) grid = max_ctas;
+    if (grid < 1) grid = 1;
+    copy_capped_kernel<<<(unsigned)grid, kCapThreads, 0, st>>>(s, d, n > 0 ? n : 0, hs, hd, hn);
+    return cudaGetLastError();
+}
+
 // Gather of one unit into a buffer of its own: dst[j] = src[lo + j], j < n.  With lo a
 // multiple of 8 both sides are 16-byte aligned and each thread moves 4 vectors; otherwise
 // each thread moves 8 scalars (still coalesced).  A grid of short blocks, as for the copy.
@@ -429,9 +475,25 @@ cudaError_t dispatch_tiles(const zero_layout &L, const TileWork &w, const uint16
 
 }  // namespace
 
-cudaError_t launch_gather_unit(const uint16_t *src, int64_t lo, int64_t n, uint16_t *dst, cudaStream_t s)
+TileBounds tile_bounds(const zero_layout &L, int64_t state_lo, int64_t state_hi)
+{
+    TileBounds b;
+    b.n_seg = (int64_t)L.segs.size();
+    b.padded = L.padded;
+    b.shard = L.shard;
+    b.state_lo = state_lo;
+    b.state_hi = state_hi;
+    b.n_ranks = L.n_ranks;
+    b.n_buckets = (int32_t)L.bucket_lo.size();
+    b.error = L.dev.error;
+    return b;
+}
+
+cudaError_t launch_gather_unit(const uint16_t *src, int64_t lo, int64_t n, uint16_t *dst, int32_t max_ctas,
+                               cudaStream_t s)
 {
     if (n <= 0) return cudaSuccess;
+    if (max_ctas > 0 && (lo & 7) == 0) return launch_copy_capped(src + lo, dst, n, nullptr, nullptr, 0, max_ctas, s);
     const int64_t per_block = (int64_t)kThreads * kCopyUnroll * kVec;
     gather_unit_kernel<<<(unsigned)((n + per_block - 1) / per_block), kThreads, 0, s>>>(src, lo, n, dst);
     return cudaGetLastError();
@@ -498,8 +560,13 @@ cudaError_t launch_copy_range(const zero_layout &L, int64_t lo, int64_t hi, cons
     if (hi <= lo) return cudaSuccess;
     const int64_t per_block = (int64_t)kThreads * kVec * kCopyUnroll;
     const int64_t va = (lo + kVec - 1) / kVec * kVec, vb = hi / kVec * kVec;
+    if (L.gather_ctas > 0) {
+        // head [lo, min(va, hi)) by one block's scalar pass, then [va, hi) vectorised
+        const int64_t head_end = va < hi ? va : hi;
+        return launch_copy_capped(src + head_end, dst + head_end, hi - head_end, src + lo, dst + lo,
+                                  (int)(head_end - lo), L.gather_ctas, s);
+    }
     const int64_t blocks = vb > va ? (vb - va + per_block - 1) / per_block : 1;
-    (void)L;
     copy_range_kernel<<<(unsigned)blocks, kThreads, 0, s>>>(lo, hi, src, dst);
     return cudaGetLastError();
 }

@@ -206,3 +206,10 @@ extern "C" zero_status zero_set_max_ctas(zero_layout *L, int32_t max_ctas)
     L->max_ctas = max_ctas;
     return ZERO_OK;
 }
+
+extern "C" zero_status zero_set_gather_ctas(zero_layout *L, int32_t max_ctas)
+{
+    if (!L || max_ctas < 0) return ZERO_ERR_INVALID;
+    L->gather_ctas = max_ctas;
+    return ZERO_OK;
+}

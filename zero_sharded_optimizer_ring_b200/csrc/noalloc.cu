@@ -55,6 +55,7 @@ extern "C" zero_status zero_step_noalloc(const zero_layout *L, const uint16_t *g
                                          uint16_t *p16_full, const zero_adamw_hparams *hp,
                                          int32_t *nonfinite, void *stream)
 {
+    ZERO_RANGE("zero_step_noalloc");
     if (!L || zero::check_hparams(hp) != ZERO_OK) return ZERO_ERR_INVALID;
     if (L->padded == 0) return ZERO_OK;
     const int64_t n_seg = (int64_t)L->segs.size();
@@ -87,6 +88,7 @@ extern "C" zero_status zero_step_noalloc(const zero_layout *L, const uint16_t *g
     w.seg_first = 0;
     w.tile_first = 0;
     w.n_tiles = L->n_tiles;
+    w.bounds = zero::tile_bounds(*L, 0, L->padded);   // no error word: a failed check only skips
     uint16_t *p16 = L->stage == 3 ? p16_shard : p16_full;
     if (e == cudaSuccess)
         e = zero::launch_fused_step(*L, w, grads, rank_stride, master, m, v, p16, c, nonfinite, st);
