@@ -61,11 +61,12 @@ def parse():
                     help="time ZeRO-3's per-layer forward and backward gathers with 1-3 prefetch slots "
                          "against a simulated layer compute (its own JSON line)")
     ap.add_argument("--tokens", type=int, default=2048, help="--zero3-passes: tokens per rank")
-    ap.add_argument("--carveout", default="0",
-                    help="--zero3-passes: comma-separated SM counts the layer GEMMs leave free (cuBLAS SM-count "
-                         "target through torch's matmul carveout), one sweep row set each")
-    ap.add_argument("--gather-ctas", default="0",
-                    help="--zero3-passes: comma-separated gather CTA caps (zero_set_gather_ctas; 0 = default grid)")
+    ap.add_argument("--zero3-configs", default="0:0:0,0:0:1,0:0:2,0:16:2,0:16:3",
+                    help="--zero3-passes sweep: comma-separated carveout:gather_ctas:slots (carveout = SMs the "
+                         "layer GEMMs leave free through cuBLAS's SM-count target; gather_ctas = "
+                         "zero_set_gather_ctas, 0 = default grid; slots 0 = the compute alone)")
+    ap.add_argument("--zero3-rounds", type=int, default=5, help="--zero3-passes: interleaved rounds of the sweep")
+    ap.add_argument("--blas", default="", help="--zero3-passes: torch preferred BLAS library (cublas, cublaslt)")
     ap.add_argument("--overlap", action="store_true",
                     help="measure the bucket-pipelined step behind a simulated backward pass "
                          "(its own JSON line; not the headline)")
@@ -75,11 +76,12 @@ def parse():
                          "(cuBLAS, 4 * tokens FLOPs per parameter; tensor-core bound)")
     ap.add_argument("--bwd-tokens", type=int, default=4096, help="--overlap --backward gemm: tokens per rank")
     ap.add_argument("--max-ctas", default="0",
-                    help="cap on the fused kernel's CTAs (zero_set_max_ctas; 0 = one per SM). With --overlap "
-                         "a comma-separated list, one JSON line each")
-    ap.add_argument("--bucket-group", default="1",
-                    help="--overlap: buckets per launch (zero_step_overlapped_grouped); a comma-separated list, "
+                    help="cap on the fused kernel's CTAs (zero_set_max_ctas; 0 = one per SM, and for the "
+                         "overlapped step the library's measured choice). With --overlap a comma-separated list, "
                          "one JSON line each")
+    ap.add_argument("--bucket-group", default="auto",
+                    help="--overlap: buckets per launch (zero_step_overlapped_grouped); auto = zero_step_overlapped "
+                         "(small buckets coalesced); a comma-separated list, one JSON line each")
     ap.add_argument("--shrink", type=int, default=0,
                     help="divide every tensor of the workload by this factor (same structure, smaller: "
                          "small cases for profiler captures; not a bench line)")
@@ -674,12 +676,16 @@ def run_overlap(a, wl):
 
     t = 0
     reps = max(3, a.steps // 20)
-    groups = [int(x) for x in str(a.bucket_group).split(",")]
+    groups = [None if x == "auto" else int(x) for x in str(a.bucket_group).split(",")]
     if a.backward == "gemm":
         runs = [("default", 0, cap, grp) for cap in caps for grp in groups]
     else:
         runs = [("default", 0, caps[0], grp) for grp in groups] + [("high", hi_pri, caps[0], groups[0])]
     for prio_name, prio, cap, grp in runs:
+        if cap == 0:       # a fresh layout: the overlapped step's grid tuner starts from scratch
+            lay.close()
+            lay = zs.Layout(list(wl.tensors), wl.n_ranks, wl.stage, wl.bucket_elems, wl.pad_align, list(wl.units))
+            lay.to_device()
         lay.set_max_ctas(cap)
         producer, compute = torch.cuda.Stream(), torch.cuda.Stream(priority=prio)
         make = gemm_backward if a.backward == "gemm" else generator_backward
@@ -696,8 +702,9 @@ def _overlap_reps(a, wl, lay, g, master, m, v, p16_shard, p16_full, backward, pr
     def hp():
         return zs.AdamW(wl.lr, wl.beta1, wl.beta2, wl.eps, wl.weight_decay, wl.loss_scale, t)
 
-    res = {"bwd": [], "step": [], "pipe": []}
-    for rep in range(a.warmup + reps):
+    res = {"bwd": [], "step": [], "pipe": [], "pipe_all": []}
+    warmup = a.warmup if cap else max(a.warmup, 2 * 4 + 2)     # the grid tuner times 4 caps twice
+    for rep in range(warmup + reps):
         torch.cuda.synchronize()
         s0, e0 = ev(), ev()
         s0.record(producer)
@@ -718,14 +725,18 @@ def _overlap_reps(a, wl, lay, g, master, m, v, p16_shard, p16_full, backward, pr
         zs.step_overlapped(lay, ready, g, master, m, v, p16_shard, p16_full, hp(), stream=compute, group=group)
         e2.record(compute)
         torch.cuda.synchronize()
-        if rep >= a.warmup:
+        res["pipe_all"].append(round(s2.elapsed_time(e2), 3))
+        if rep >= warmup:
             res["bwd"].append(s0.elapsed_time(e0))
             res["step"].append(s1.elapsed_time(e1))
             res["pipe"].append(s2.elapsed_time(e2))
     tb, ts, tp = (statistics.median(res[k]) for k in ("bwd", "step", "pipe"))
     print(json.dumps({
         "metric": "bucket-pipelined step behind a simulated backward (overlap)", "workload": wl.name,
-        "backward": a.backward, "compute_stream_priority": prio_name, "max_ctas": cap, "bucket_group": group,
+        "backward": a.backward, "compute_stream_priority": prio_name,
+        "max_ctas": cap if cap else "auto (measured by the library)",
+        "bucket_group": group if group else "auto (zero_step_overlapped: launches of >= 2^24 elements)",
+        "t_back_to_back_ms": tb + ts, "pipelined_every_call_ms": res["pipe_all"],
         "buckets": lay.n_buckets,
         "reps": reps, "t_backward_ms": tb, "t_step_ms": ts, "t_pipelined_ms": tp, "exposed_step_ms": tp - tb,
         "overlap_efficiency": (tb + ts - tp) / ts,
@@ -845,24 +856,52 @@ def run_zero3_passes(a, wl):
         for n in (1, 2):
             res[f"{name}_exposed_gather_{n}slot_ms"] = res[f"{name}_{n}slot_ms"] - res[f"{name}_compute_only_ms"]
 
-    # gathers on a capped grid beside GEMMs that leave SMs free: the matmul SM carveout
-    # (cuBLAS's SM-count target) x the gather kernels' CTA cap (zero_set_gather_ctas)
+    # gathers on a capped grid beside GEMMs that leave SMs free: configurations
+    # "carveout:gather_ctas:slots" (carveout = SMs the matmuls leave free through cuBLAS's
+    # SM-count target; gather_ctas = zero_set_gather_ctas; slots 0 = compute alone), each
+    # measured once per round, rounds interleaved so that clock drift hits all alike;
+    # reported: the median over rounds
     sweep = []
-    for c in [int(x) for x in a.carveout.split(",")]:
-        set_carveout(c if c > 0 else None)
-        comp = {name: timed(compute_only(work)) for name, work, _ in passes}
-        for gcap in [int(x) for x in a.gather_ctas.split(",")]:
-            lay.set_gather_ctas(gcap)
-            row = {"carveout_sms": c, "gather_ctas": gcap, "gathers_only_ms": round(timed(gathers_only), 4)}
-            for name, work, order in passes:
-                t, bd = timed(lambda: zero3_pass(lay, shard, slots[:2], order, work, gs, cs), breakdown=True)
-                row[f"{name}_compute_only_ms"] = round(comp[name], 4)
-                row[f"{name}_2slot_ms"] = round(t, 4)
-                row[f"{name}_exposed_vs_full_gpu_compute_ms"] = round(t - res[f"{name}_compute_only_ms"], 4)
-                row[f"{name}_breakdown"] = short(bd)
+    configs = [tuple(int(x) for x in c.split(":")) for c in a.zero3_configs.split(",") if c]
+    if configs:
+        if a.blas:
+            torch.backends.cuda.preferred_blas_library(a.blas)
+        rounds = {}
+        for rnd in range(a.zero3_rounds):
+            for c, gcap, n in configs:
+                set_carveout(c if c > 0 else None)
+                lay.set_gather_ctas(gcap)
+                for name, work, order in passes:
+                    if n == 0:
+                        fn = compute_only(work)
+                    else:
+                        fn = (lambda o=order, w=work, k=n: zero3_pass(lay, shard, slots[:k], o, w, gs, cs))
+                    torch.cuda.synchronize()
+                    s0, e0 = ev(), ev()
+                    s0.record(gs)
+                    cs.wait_event(s0)
+                    marks = fn()
+                    e0.record(cs)
+                    torch.cuda.synchronize()
+                    bd = layer_breakdown(marks, s0) if n else None
+                    rounds.setdefault((c, gcap, n, name), []).append((s0.elapsed_time(e0), bd))
+        set_carveout(None)
+        lay.set_gather_ctas(0)
+        for c, gcap, n in configs:
+            row = {"carveout_sms": c, "gather_ctas": gcap, "slots": n}
+            for name, _, _ in passes:
+                runs = sorted(rounds[(c, gcap, n, name)], key=lambda x: x[0])
+                t_med, bd = runs[len(runs) // 2]
+                row[f"{name}_ms"] = round(t_med, 4)
+                if bd:
+                    row[f"{name}_breakdown"] = short(bd)
             sweep.append(row)
-    set_carveout(None)
-    lay.set_gather_ctas(0)
+        base = {name: statistics.median(t for t, _ in rounds[(0, 0, 0, name)]) for name, _, _ in passes
+                } if (0, 0, 0) in configs else None
+        if base:
+            for row in sweep:
+                for name in base:
+                    row[f"{name}_exposed_ms"] = round(row[f"{name}_ms"] - base[name], 4)
     gather_bytes = 4 * P
     print(json.dumps({"metric": "ZeRO-3 per-layer gather passes with prefetch", "workload": wl.name,
                       "units": lay.n_units, "tokens": T, "gather_bytes_per_pass": gather_bytes,

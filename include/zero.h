@@ -229,23 +229,35 @@ zero_status zero_step_bucket(const zero_layout *layout, int64_t bucket, const ui
 /* zero_step overlapped with the backward pass that produces the gradients: for each
  * bucket b in bucket order (the order a backward pass completes them), `stream` waits
  * for ready_events[b] (a cudaEvent_t the caller records once bucket b's gradients are
- * written, typically on another stream), then runs bucket b's fused update.  Stage 3
- * then runs the all-gather.  ready_events: host array [n_buckets], none NULL.  As for
- * any cudaStreamWaitEvent, each wait takes the event's most recent record at the time of
+ * written, typically on another stream), then runs bucket b's fused update.  Consecutive
+ * buckets smaller than 2^24 elements share one launch, which waits for all of them,
+ * until the launch holds at least 2^24 elements (many small buckets otherwise interleave
+ * hundreds of short launches with the backward pass).  Stage 3 then runs the
+ * all-gather.  ready_events: host array [n_buckets], none NULL.  As for any
+ * cudaStreamWaitEvent, each wait takes the event's most recent record at the time of
  * this call: enqueue the producer's records first (the producer's work itself may still
- * be running).  Result identical to zero_step. */
+ * be running).  Result identical to zero_step.
+ *
+ * Grid: the update shares the GPU with the backward pass, and the best split of the SMs
+ * depends on the two workloads.  Unless zero_set_max_ctas fixed a cap, the library
+ * chooses one by measurement: over the layout's first overlapped calls it times whole
+ * calls (CUDA events on `stream`, from the first wait to the last launch) with the
+ * update capped at 1, 2/3, 1/2 and 1/3 of the SMs, two calls each, then keeps the
+ * fastest for every later call.  It never waits for these events: a call issued before
+ * the previous timed call has finished on the GPU is not timed.  The cap never changes
+ * a result. */
 zero_status zero_step_overlapped(const zero_layout *layout, void *const *ready_events,
                                  const uint16_t *grads, int64_t rank_stride, float *master, float *m,
                                  float *v, uint16_t *p16_shard, uint16_t *p16_full,
                                  const zero_adamw_hparams *hp, int32_t *nonfinite, void *stream);
 
 /* zero_step_overlapped with one launch per `group` consecutive buckets (group >= 1; the
- * last group may be shorter): `stream` waits for the ready events of all the group's
- * buckets, then runs their fused update as one kernel.  With many small buckets (a
- * bucket of 10^6 parameters is ~9 us of work at full bandwidth) this trades a later
- * start for fewer launches interleaved with the backward pass.  group = 1 is
- * zero_step_overlapped.  Same results.  No counterpart on the pages (their buckets are
- * the launch unit). */
+ * last group may be shorter; no other coalescing): `stream` waits for the ready events
+ * of all the group's buckets, then runs their fused update as one kernel.  With many
+ * small buckets (a bucket of 10^6 parameters is ~9 us of work at full bandwidth) this
+ * trades a later start for fewer launches interleaved with the backward pass.  The grid
+ * is chosen as for zero_step_overlapped.  Same results.  No counterpart on the pages
+ * (their buckets are the launch unit). */
 zero_status zero_step_overlapped_grouped(const zero_layout *layout, void *const *ready_events, int64_t group,
                                          const uint16_t *grads, int64_t rank_stride, float *master, float *m,
                                          float *v, uint16_t *p16_shard, uint16_t *p16_full,
@@ -412,7 +424,9 @@ zero_status zero_set_impl(zero_layout *layout, int32_t impl);
  * SMs to concurrent work (a backward pass whose gradients the step consumes bucket by
  * bucket, as in [P1] "DDP": the first finished group is synchronised while the next is
  * computed); it is slower alone, since each SM moves at most ~60 GB/s through the
- * step's arithmetic.  Negative k: ZERO_ERR_INVALID.  No counterpart on the pages. */
+ * step's arithmetic.  A cap set here also replaces the overlapped steps' own choice
+ * (see zero_step_overlapped).  Negative k: ZERO_ERR_INVALID.  No counterpart on the
+ * pages. */
 zero_status zero_set_max_ctas(zero_layout *layout, int32_t max_ctas);
 
 /* Grid of the all-gather copies (zero_allgather, zero_gather_unit, and the gather inside

@@ -65,7 +65,7 @@ def test_step_bucket_matches_oracle(key, order):
     _check(wl, lay, b, ref)
 
 
-@pytest.mark.parametrize("group", [1, 3, 1000])
+@pytest.mark.parametrize("group", [None, 1, 3, 1000])
 @pytest.mark.parametrize("key", ["flat1p3b_n4_zero1", "llama3b_n8_zero3", "ragged2000_n16_zero2"])
 def test_overlapped_step_with_simulated_backward(key, group):
     wl = reduced_workloads()[key]
@@ -86,6 +86,31 @@ def test_overlapped_step_with_simulated_backward(key, group):
             ready[bk].record(producer)
         zs.step_overlapped(lay, ready, b["g"], b["master"], b["m"], b["v"], b["p16_shard"], b["p16_full"],
                            _hp(wl, t), nonfinite=b["nonfinite"], stream=consumer, group=group)
+    zs.get_error(lay)
+    _check(wl, lay, b, ref)
+
+
+@pytest.mark.parametrize("key", ["flat1p3b_n4_zero1", "ragged2000_n16_zero2"])
+def test_overlapped_grid_tuner_keeps_results(key):
+    """With no cap set, the overlapped step times several grid caps over its first calls
+    and then keeps the fastest; every call, whatever its grid, must give the oracle's
+    result (12 steps: each candidate timed twice, then the chosen one)."""
+    wl = reduced_workloads()[key]
+    steps = 12
+    ref, _ = S.oracle_run(wl, steps)
+    lay, bufs = _setup(wl)
+    b = bufs()
+    _, buckets, _, _ = lay.tables()
+    producer, consumer = torch.cuda.Stream(), torch.cuda.Stream()
+    for t in range(1, steps + 1):
+        ready = [torch.cuda.Event() for _ in range(lay.n_buckets)]
+        for bk in range(lay.n_buckets):
+            ready[bk].record(producer)
+        b["nonfinite"].zero_()
+        torch.cuda.synchronize()
+        zs.step_overlapped(lay, ready, b["g"], b["master"], b["m"], b["v"], b["p16_shard"], b["p16_full"],
+                           _hp(wl, t), nonfinite=b["nonfinite"], stream=consumer, group=None if t % 2 else 2)
+        torch.cuda.synchronize()                  # the tuner reads the call's events next time
     zs.get_error(lay)
     _check(wl, lay, b, ref)
 

@@ -214,10 +214,12 @@ def step_bucket(layout, bucket, grads, master, m, v, p16_shard, p16_full, hp, no
 
 
 def step_overlapped(layout, ready_events, grads, master, m, v, p16_shard, p16_full, hp, nonfinite=None,
-                    rank_stride=None, stream=None, group=1):
+                    rank_stride=None, stream=None, group=None):
     """zero_step with bucket b gated on ready_events[b] (torch.cuda.Event, recorded by the
-    producer of bucket b's gradients); group > 1: one launch per `group` consecutive
-    buckets (zero_step_overlapped_grouped)."""
+    producer of bucket b's gradients).  group=None: zero_step_overlapped (small buckets
+    coalesced into launches of >= 2^24 elements); an integer: one launch per `group`
+    consecutive buckets (zero_step_overlapped_grouped).  Either way the grid cap is the
+    layout's (set_max_ctas) or, if none, the library's measured choice."""
     assert len(ready_events) == layout.n_buckets
     handles = (ctypes.c_void_p * max(1, layout.n_buckets))()
     for b, e in enumerate(ready_events):
@@ -225,7 +227,7 @@ def step_overlapped(layout, ready_events, grads, master, m, v, p16_shard, p16_fu
             raise ValueError(f"ready event of bucket {b} was never recorded")
         handles[b] = e.cuda_event
     h = hp.c()
-    if group == 1:
+    if group is None:
         _check(_abi.lib().zero_step_overlapped(layout.handle, handles, _ptr(grads),
                                                _stride(grads, layout, rank_stride), _ptr(master), _ptr(m), _ptr(v),
                                                _ptr(p16_shard), _ptr(p16_full), ctypes.byref(h), _ptr(nonfinite),

@@ -85,6 +85,8 @@ void release_device(zero_layout *L)
     for (cudaEvent_t e : L->dev.updated) cudaEventDestroy(e);
     L->dev.landed.clear();
     L->dev.updated.clear();
+    if (L->dev.tuner.begin) cudaEventDestroy(L->dev.tuner.begin);
+    if (L->dev.tuner.end) cudaEventDestroy(L->dev.tuner.end);
     if (L->dev.begin) cudaEventDestroy(L->dev.begin);
     if (L->dev.done) cudaEventDestroy(L->dev.done);
     if (L->dev.copy_in) cudaStreamDestroy(L->dev.copy_in);
@@ -198,6 +200,8 @@ extern "C" zero_status zero_layout_to_device(zero_layout *L, void *stream)
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&d.copy_out, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&d.begin, cudaEventDisableTiming);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&d.done, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreate(&d.tuner.begin);     // timing events
+    if (e == cudaSuccess) e = cudaEventCreate(&d.tuner.end);
     for (size_t b = 0; e == cudaSuccess && b < L->bucket_lo.size(); ++b) {
         cudaEvent_t a = nullptr, u = nullptr;
         e = cudaEventCreateWithFlags(&a, cudaEventDisableTiming);
@@ -399,32 +403,104 @@ extern "C" zero_status zero_step_bucket(const zero_layout *L, int64_t bucket, co
                              step_scalars(L->n_ranks, *hp), nonfinite, (cudaStream_t)stream));
 }
 
+namespace {
+
+// Launches of at least this many elements when zero_step_overlapped coalesces small
+// buckets (~0.5-1 GB of traffic, 80-150 us at full bandwidth: launch gaps stay negligible).
+constexpr int64_t kMinOverlapLaunch = int64_t(1) << 24;
+
+// The grid cap of candidate i of the overlapped step's tuner: SMs x {1, 2/3, 1/2, 1/3}.
+int32_t tuner_cap(const zero_layout *L, int i)
+{
+    static const int kSixths[zero::OverlapTuner::kCands] = {6, 4, 3, 2};
+    const int sms = L->dev.num_sms > 0 ? L->dev.num_sms : 148;
+    return i == 0 ? 0 : sms * kSixths[i] / 6;
+}
+
+// Grid cap of this overlapped call: the caller's (zero_set_max_ctas) if set; otherwise the
+// tuner's.  Harvests the previous timed call if its end event has completed (never waits),
+// then times the next candidate that still lacks trials, or settles on the fastest.
+// *timed: record the tuner's events around this call.
+int32_t overlap_cap(const zero_layout *L, bool *timed)
+{
+    *timed = false;
+    zero::OverlapTuner &T = L->dev.tuner;
+    if (L->max_ctas > 0 || !T.begin || !T.end) return L->max_ctas;
+    if (T.pending >= 0) {
+        if (cudaEventQuery(T.end) != cudaSuccess) return tuner_cap(L, T.pending);   // still running: untimed
+        float ms = 0.f;
+        if (cudaEventElapsedTime(&ms, T.begin, T.end) == cudaSuccess) {
+            float &b = T.best_ms[T.pending];
+            if (T.trials[T.pending] == 0 || ms < b) b = ms;
+            ++T.trials[T.pending];
+        }
+        T.pending = -1;
+    }
+    for (int i = 0; i < zero::OverlapTuner::kCands; ++i)
+        if (T.trials[i] < zero::OverlapTuner::kTrials) {
+            T.pending = i;
+            *timed = true;
+            return tuner_cap(L, i);
+        }
+    int best = 0;
+    for (int i = 1; i < zero::OverlapTuner::kCands; ++i)
+        if (T.best_ms[i] < T.best_ms[best]) best = i;
+    return tuner_cap(L, best);
+}
+
+// The overlapped step over launch groups: launch j covers buckets [first[j], first[j+1]).
+zero_status overlapped(const zero_layout *L, void *const *ready_events, const std::vector<int64_t> &first,
+                       const uint16_t *grads, int64_t rank_stride, float *master, float *m, float *v,
+                       uint16_t *p16_shard, uint16_t *p16_full, const zero_adamw_hparams *hp, int32_t *nonfinite,
+                       cudaStream_t st)
+{
+    const AdamScalars c = step_scalars(L->n_ranks, *hp);
+    uint16_t *p16 = L->stage == 3 ? p16_shard : p16_full;
+    bool timed = false;
+    const int32_t cap = overlap_cap(L, &timed);
+    cudaError_t e = timed ? cudaEventRecord(L->dev.tuner.begin, st) : cudaSuccess;
+    for (size_t j = 0; e == cudaSuccess && j + 1 < first.size(); ++j) {
+        for (int64_t b = first[j]; e == cudaSuccess && b < first[j + 1]; ++b)
+            e = cudaStreamWaitEvent(st, (cudaEvent_t)ready_events[b], 0);
+        TileWork w = bucket_range_tiles(L, first[j], first[j + 1]);
+        w.max_ctas = cap;
+        if (e == cudaSuccess) e = fused(L, w, grads, rank_stride, master, m, v, p16, c, nonfinite, st);
+    }
+    if (e == cudaSuccess && L->stage == 3) e = zero::launch_copy_range(*L, 0, L->padded, p16_shard, p16_full, st);
+    if (e == cudaSuccess && timed) e = cudaEventRecord(L->dev.tuner.end, st);
+    if (e != cudaSuccess && timed) L->dev.tuner.pending = -1;
+    return cuda_status(e);
+}
+
+zero_status check_overlapped(const zero_layout *L, void *const *ready_events, const uint16_t *grads,
+                             int64_t rank_stride, float *master, float *m, float *v, uint16_t *p16_shard,
+                             uint16_t *p16_full, const zero_adamw_hparams *hp)
+{
+    zero_status s = check_step(L, grads, rank_stride, master, m, v, p16_shard, p16_full, hp);
+    if (s != ZERO_OK || L->padded == 0) return s;
+    if (!ready_events) return ZERO_ERR_INVALID;
+    for (size_t b = 0; b < L->bucket_lo.size(); ++b)
+        if (!ready_events[b]) return ZERO_ERR_INVALID;
+    return ZERO_OK;
+}
+
+}  // namespace
+
 extern "C" zero_status zero_step_overlapped_grouped(const zero_layout *L, void *const *ready_events, int64_t group,
                                                     const uint16_t *grads, int64_t rank_stride, float *master, float *m,
                                                     float *v, uint16_t *p16_shard, uint16_t *p16_full,
                                                     const zero_adamw_hparams *hp, int32_t *nonfinite, void *stream)
 {
     ZERO_RANGE("zero_step_overlapped_grouped");
-    zero_status s = check_step(L, grads, rank_stride, master, m, v, p16_shard, p16_full, hp);
-    if (s != ZERO_OK) return s;
     if (group < 1) return ZERO_ERR_INVALID;
-    if (L->padded == 0) return ZERO_OK;
-    if (!ready_events) return ZERO_ERR_INVALID;
+    zero_status s = check_overlapped(L, ready_events, grads, rank_stride, master, m, v, p16_shard, p16_full, hp);
+    if (s != ZERO_OK || L->padded == 0) return s;
     const int64_t nb = (int64_t)L->bucket_lo.size();
-    for (int64_t b = 0; b < nb; ++b)
-        if (!ready_events[b]) return ZERO_ERR_INVALID;
-    cudaStream_t st = (cudaStream_t)stream;
-    const AdamScalars c = step_scalars(L->n_ranks, *hp);
-    uint16_t *p16 = L->stage == 3 ? p16_shard : p16_full;
-    cudaError_t e = cudaSuccess;
-    for (int64_t b0 = 0; e == cudaSuccess && b0 < nb; b0 += group) {
-        const int64_t b1 = b0 + group < nb ? b0 + group : nb;
-        for (int64_t b = b0; e == cudaSuccess && b < b1; ++b) e = cudaStreamWaitEvent(st, (cudaEvent_t)ready_events[b], 0);
-        if (e == cudaSuccess)
-            e = fused(L, bucket_range_tiles(L, b0, b1), grads, rank_stride, master, m, v, p16, c, nonfinite, st);
-    }
-    if (e == cudaSuccess && L->stage == 3) e = zero::launch_copy_range(*L, 0, L->padded, p16_shard, p16_full, st);
-    return cuda_status(e);
+    std::vector<int64_t> first;
+    for (int64_t b = 0; b < nb; b += group) first.push_back(b);
+    first.push_back(nb);
+    return overlapped(L, ready_events, first, grads, rank_stride, master, m, v, p16_shard, p16_full, hp, nonfinite,
+                      (cudaStream_t)stream);
 }
 
 extern "C" zero_status zero_step_overlapped(const zero_layout *L, void *const *ready_events, const uint16_t *grads,
@@ -433,8 +509,21 @@ extern "C" zero_status zero_step_overlapped(const zero_layout *L, void *const *r
                                             int32_t *nonfinite, void *stream)
 {
     ZERO_RANGE("zero_step_overlapped");
-    return zero_step_overlapped_grouped(L, ready_events, 1, grads, rank_stride, master, m, v, p16_shard, p16_full,
-                                        hp, nonfinite, stream);
+    zero_status s = check_overlapped(L, ready_events, grads, rank_stride, master, m, v, p16_shard, p16_full, hp);
+    if (s != ZERO_OK || L->padded == 0) return s;
+    // one launch per bucket, except that consecutive buckets smaller than kMinOverlapLaunch
+    // share a launch until they reach it (a launch waits for all of its buckets)
+    const int64_t nb = (int64_t)L->bucket_lo.size();
+    std::vector<int64_t> first;
+    int64_t acc = 0;
+    for (int64_t b = 0; b < nb; ++b) {
+        if (acc == 0) first.push_back(b);
+        acc += L->bucket_hi[(size_t)b] - L->bucket_lo[(size_t)b];
+        if (acc >= kMinOverlapLaunch) acc = 0;
+    }
+    first.push_back(nb);
+    return overlapped(L, ready_events, first, grads, rank_stride, master, m, v, p16_shard, p16_full, hp, nonfinite,
+                      (cudaStream_t)stream);
 }
 
 namespace {

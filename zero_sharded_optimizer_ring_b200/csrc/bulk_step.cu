@@ -302,7 +302,8 @@ cudaError_t launch_bulk_n(const zero_layout &L, BulkArgs &a, cudaStream_t st)
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int64_t grid = L.dev.num_sms > 0 ? L.dev.num_sms : 148;
-    if (L.max_ctas > 0 && grid > L.max_ctas) grid = L.max_ctas;
+    const int32_t cap = a.w.max_ctas > 0 ? a.w.max_ctas : L.max_ctas;
+    if (cap > 0 && grid > cap) grid = cap;
     if (grid > a.w.n_tiles) grid = a.w.n_tiles;
     kern<<<(unsigned)grid, BulkShape<N>::kThreads, smem, st>>>(a);
     return cudaGetLastError();

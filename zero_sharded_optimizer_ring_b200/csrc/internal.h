@@ -73,6 +73,19 @@ struct TileWork {
     int64_t tile_first;    // first global tile of the launch
     int64_t n_tiles;       // tiles in the launch
     TileBounds bounds;     // debug builds only
+    int32_t max_ctas = 0;  // > 0: this launch's grid cap (overrides the layout's)
+};
+
+// Grid-cap tuning of the overlapped step: each candidate cap (a fraction of the SMs) is
+// timed over whole calls (first wait to last launch, CUDA events on the caller's stream)
+// kTrials times, then the fastest is kept.  Nothing ever waits on these events: a call
+// whose predecessor has not finished yet is simply not timed.
+struct OverlapTuner {
+    static constexpr int kCands = 4, kTrials = 2;
+    float best_ms[kCands] = {0.f, 0.f, 0.f, 0.f};
+    int32_t trials[kCands] = {0, 0, 0, 0};
+    int32_t pending = -1;                 // candidate whose timed call is in flight
+    cudaEvent_t begin = nullptr, end = nullptr;
 };
 
 struct DeviceState {
@@ -85,6 +98,7 @@ struct DeviceState {
     cudaStream_t copy_in = nullptr, copy_out = nullptr;   // zero_step_host
     std::vector<cudaEvent_t> landed, updated;              // per bucket
     cudaEvent_t begin = nullptr, done = nullptr;           // per zero_step_host call
+    mutable OverlapTuner tuner;               // zero_step_overlapped's default grid choice
     uint64_t wait_limit_ns = 2000000000ull;   // bound of every in-kernel wait (2 s)
     int32_t skip_first_fill = 0;              // test hook of the bulk pipeline (see zero.h)
 };

@@ -443,7 +443,7 @@ cudaError_t launch_tiles(const zero_layout &L, const TileWork &w, const uint16_t
                          const AdamScalars &c, int32_t *nonfinite, cudaStream_t st)
 {
     auto kern = L.wire16 ? tile_kernel<NT, U, kFused, true> : tile_kernel<NT, U, kFused, false>;
-    const int grid = grid_for(kern, w.n_tiles, L.dev.num_sms, L.max_ctas);
+    const int grid = grid_for(kern, w.n_tiles, L.dev.num_sms, w.max_ctas > 0 ? w.max_ctas : L.max_ctas);
     kern<<<grid, kThreads, 0, st>>>(w, L.n_ranks, grads, stride, reduced, master, m, v, p16, c, nonfinite,
                                     StateIn{nullptr, nullptr, nullptr});
     return cudaGetLastError();
@@ -535,7 +535,7 @@ cudaError_t launch_fused_step_to(const zero_layout &L, const TileWork &w, const 
 {
     if (w.n_tiles <= 0) return cudaSuccess;
     auto kern = L.wire16 ? tile_kernel<0, 1, true, true, true> : tile_kernel<0, 1, true, false, true>;
-    const int grid = grid_for(kern, w.n_tiles, L.dev.num_sms, L.max_ctas);
+    const int grid = grid_for(kern, w.n_tiles, L.dev.num_sms, w.max_ctas > 0 ? w.max_ctas : L.max_ctas);
     kern<<<grid, kThreads, 0, s>>>(w, L.n_ranks, grads, stride, nullptr, master, m, v, p16, c, nonfinite,
                                    StateIn{master_in, m_in, v_in});
     return cudaGetLastError();
