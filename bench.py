@@ -95,6 +95,8 @@ def parse():
     ap.add_argument("--record-kernel", default="bulk_step_kernel", help="--record-traffic: kernel name regex")
     ap.add_argument("--record-tag", default="bulk_step", help="--record-traffic: record name prefix")
     ap.add_argument("--record-note", default="", help="--record-traffic: how the capture was taken")
+    ap.add_argument("--ranks", type=int, default=0,
+                    help="run the workload with this many simulated ranks (rank-count studies; not a bench line)")
     ap.add_argument("--psi", type=int, default=0,
                     help="flat workloads only: run the same shape with this many parameters "
                          "(small cases for profiler captures; not a bench line)")
@@ -429,7 +431,7 @@ def also_workloads(a):
         return []
     if a.also != "auto":
         return [x for x in a.also.split(",") if x]
-    variant = a.wire_fp16 or a.dynamic or a.dynamic_commit or a.shrink > 1 or a.psi or a.kernel
+    variant = a.wire_fp16 or a.dynamic or a.dynamic_commit or a.shrink > 1 or a.psi or a.kernel or a.ranks
     return ["llama3b_n8_zero3"] if a.workload == DEFAULT_WORKLOAD and not variant else []
 
 
@@ -916,6 +918,8 @@ def main():
     wl = full_workloads()[a.workload]
     if a.shrink > 1:
         wl = wl.with_(tensors=tuple(max(1, t // a.shrink) for t in wl.tensors), name=f"{wl.name}_shrink{a.shrink}")
+    if a.ranks:
+        wl = wl.with_(n_ranks=a.ranks, name=f"{wl.name}_ranks{a.ranks}")
     if a.psi:
         if len(wl.tensors) != 1:
             raise SystemExit("--psi applies to flat (single-tensor) workloads only")

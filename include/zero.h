@@ -194,7 +194,7 @@ zero_status zero_gather_unit(const zero_layout *layout, int64_t unit, const uint
 
 /* The same gather when every rank keeps only its own shard ([P1] "ZeRO-3" on N GPUs: a
  * layer's parameters are fetched from the ranks that hold them before its forward and
- * again before its backward).  rank_p16: host array of N device pointers (N <= 16), rank
+ * again before its backward).  rank_p16: host array of N device pointers (N <= 64), rank
  * k's buffer holding flat elements [k*S, (k+1)*S) of the fp16 parameters (its shard, as
  * zero_step_shard writes it for stage 3), each 16-byte aligned; they may point into this
  * GPU's memory or into other GPUs' memory mapped with zero_ipc_open (plain loads over
@@ -338,7 +338,7 @@ zero_status zero_step_dynamic(const zero_layout *layout, const uint16_t *grads, 
  * Costs the fused step's bytes instead of the reduce-then-update pair of
  * zero_step_dynamic, for a second state set (12 bytes and 2 for fp16 per parameter).
  * No in buffer may overlap an out buffer (ZERO_ERR_INVALID).  Either implementation
- * (zero_set_impl; register streaming for N > 16).  nonfinite: device int32 [n_buckets],
+ * (zero_set_impl; both serve every N).  nonfinite: device int32 [n_buckets],
  * required, zeroed here.  The pages name
  * no overflow handling; this is the two-phase form of the skip described above. */
 zero_status zero_step_dynamic_commit(const zero_layout *layout, const uint16_t *grads, int64_t rank_stride,
@@ -353,7 +353,7 @@ zero_status zero_step_dynamic_commit(const zero_layout *layout, const uint16_t *
 /* zero_step with each rank's gradients in a buffer of its own: rank r's gradient of flat
  * element i is rank_grads[r][i] (host array of N device pointers, each 16-byte aligned,
  * each >= P elements; they may point into this GPU's memory or into other GPUs' memory
- * mapped with zero_ipc_open).  Uses the bulk-copy pipeline; N <= 16.  Same result as
+ * mapped with zero_ipc_open).  Uses the bulk-copy pipeline; N <= 64.  Same result as
  * zero_step on the same values. */
 zero_status zero_step_ranks(const zero_layout *layout, const uint16_t *const *rank_grads, float *master,
                             float *m, float *v, uint16_t *p16_shard, uint16_t *p16_full,
@@ -367,7 +367,7 @@ zero_status zero_step_ranks(const zero_layout *layout, const uint16_t *const *ra
  * result equals the single-GPU simulation bit for bit.
  *   master_k, m_k, v_k: fp32 [S], element i of the flat buffer at [i - kS];
  *   p16_out: fp16, full [P] (stages 0-2: element i at [i]) or, for stage 3, the shard's
- *   own [S] (element i at [i - kS]).  Requires S % 8 == 0 and N <= 16.
+ *   own [S] (element i at [i - kS]).  Requires S % 8 == 0 and N <= 64.
  * The caller makes sure the peers' gradients are complete before the call (a host
  * barrier between ranks): the kernel reads peer memory but never waits on another GPU. */
 zero_status zero_step_shard(const zero_layout *layout, int32_t shard, const uint16_t *const *rank_grads,
@@ -384,7 +384,7 @@ zero_status zero_step_shard(const zero_layout *layout, int32_t shard, const uint
  * *nonfinite_total (host).  The step must be kept or dropped on every rank alike: the
  * caller sums the ranks' counts (one all-reduce of an integer), then advances every
  * rank's scaler with zero_loss_scaler_advance and, if the sum is zero, makes the out
- * buffers current everywhere.  N <= 16, S % 8 == 0. */
+ * buffers current everywhere.  N <= 64, S % 8 == 0. */
 zero_status zero_step_shard_commit(const zero_layout *layout, int32_t shard, const uint16_t *const *rank_grads,
                                    const float *master_in, const float *m_in, const float *v_in,
                                    float *master_out, float *m_out, float *v_out, uint16_t *p16_out,
@@ -411,10 +411,12 @@ zero_status zero_ipc_get_handle(const void *dev_ptr, void *handle_out, int64_t *
 zero_status zero_ipc_open(const void *handle, int64_t offset, void **dev_ptr_out);
 zero_status zero_ipc_close(void *dev_ptr, int64_t offset);
 
-/* Select the fused kernel's implementation: 0 = automatic (the bulk-copy pipeline for
- * N in 1..16, register streaming above), 1 = register streaming (vectorised
- * 16-byte loads held in registers), 2 = bulk-copy pipeline (cp.async.bulk into a
- * shared-memory ring, warp-specialised).  Results are bit-identical. */
+/* Select the fused kernel's implementation: 0 = automatic (the bulk-copy pipeline, which
+ * serves every N up to 64: compiled per rank count for N <= 16, one runtime-N instance
+ * above; register streaming beyond 64), 1 = register streaming (vectorised 16-byte loads
+ * held in registers; any N), 2 = bulk-copy pipeline (cp.async.bulk into a shared-memory
+ * ring, warp-specialised; N <= 64, register streaming above).  Results are
+ * bit-identical. */
 zero_status zero_set_impl(zero_layout *layout, int32_t impl);
 
 /* Cap on the number of CTAs of the tile-walking kernels (the fused step in both

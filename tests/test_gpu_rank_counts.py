@@ -1,11 +1,12 @@
 """GPU parity for every rank count the kernels specialise, and for counts they do not.
 
 The fused step has one compiled variant per rank count: the bulk-copy pipeline for
-N = 1..16, the register-streaming kernel for N = 1..8 and 16, and a runtime-N register
-kernel for all others. Each N runs a small ragged layout (several tiles per shard, bucket
-and shard edges that are not 8-aligned for odd N) for two steps, in both implementations
-and with fp32 and fp16 partials on the wire, and must equal the oracle bit for bit.
-zero_step_ranks (one gradient buffer per rank) is checked for every N the pipeline takes.
+N = 1..16 and one runtime-N pipeline instance for N = 17..64, the register-streaming
+kernel for N = 1..8 and 16, and a runtime-N register kernel for all others. Each N runs a
+small ragged layout (several tiles per shard, bucket and shard edges that are not
+8-aligned for odd N) for two steps, in both implementations and with fp32 and fp16
+partials on the wire, and must equal the oracle bit for bit. zero_step_ranks (one
+gradient buffer per rank) is checked for N = 1..16 and for runtime-N counts up to 64.
 """
 import numpy as np
 import pytest
@@ -18,7 +19,7 @@ import support as S
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
-RANK_COUNTS = list(range(1, 21)) + [24, 32, 64]
+RANK_COUNTS = list(range(1, 21)) + [24, 32, 50, 51, 64, 65]
 
 
 def _workload(N):
@@ -85,7 +86,7 @@ def test_every_rank_count_both_kernels(N, wire):
         _check(wl, b, ref, lay.n_buckets)
 
 
-@pytest.mark.parametrize("N", list(range(1, 17)))
+@pytest.mark.parametrize("N", list(range(1, 18)) + [24, 33, 51, 64])
 def test_step_ranks_every_pipeline_rank_count(N):
     wl = _workload(N)
     ref = _reference(wl, False)

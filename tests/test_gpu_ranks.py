@@ -137,11 +137,11 @@ def test_gather_unit_ranks_matches_oracle(tensors, N, A, units):
 
 
 def test_gather_unit_ranks_rejects_bad_arguments():
-    lay = zs.Layout([1000] * 17, 17, 3, 0, 8, list(range(17))).to_device()
-    shards = [torch.zeros(lay.shard, dtype=torch.int16, device="cuda") for _ in range(17)]
+    lay = zs.Layout([1000] * 65, 65, 3, 0, 8, list(range(65))).to_device()
+    shards = [torch.zeros(lay.shard, dtype=torch.int16, device="cuda") for _ in range(65)]
     dst = torch.zeros(1000, dtype=torch.int16, device="cuda")
-    for call in (lambda: zs.gather_unit_ranks(lay, 0, shards, dst),          # N > 16
-                 lambda: zs.gather_unit_ranks(lay, 17, shards, dst)):         # no such unit
+    for call in (lambda: zs.gather_unit_ranks(lay, 0, shards, dst),          # N > 64
+                 lambda: zs.gather_unit_ranks(lay, 65, shards, dst)):         # no such unit
         with pytest.raises(zs.ZeroError) as e:
             call()
         assert e.value.status == 1

@@ -32,6 +32,11 @@ namespace {
 // but more than about 120-170 KB in flight per SM costs DRAM efficiency.  Few ranks:
 // 4096-element chunks (one tile), 16 consumer warps, 2-3 stages.  More ranks: 2048-element
 // chunks, 8 consumer warps, at most 3 stages.
+//
+// N = 0 is the runtime rank count (17..kMaxBulkRanks): a stage of (2n + 12) bytes per
+// element grows with n, so the chunk is 1024 elements while two stages of it fit in
+// shared memory and 512 above; 4 consumer warps (one 16-byte vector per thread for a
+// 1024-element chunk).
 template <int N>
 struct BulkShape {
     static constexpr int kChunk = N <= 4 ? 4096 : 2048;        // elements per stage
@@ -39,6 +44,13 @@ struct BulkShape {
     static constexpr int kThreads = 32 * (1 + kConsumerWarps);
     static constexpr int kMaxStages = 3;
     static constexpr uint32_t kStageBytes = (uint32_t)kChunk * (2 * N + 12);
+};
+
+template <>
+struct BulkShape<0> {
+    static constexpr int kConsumerWarps = 4;
+    static constexpr int kThreads = 32 * (1 + kConsumerWarps);
+    static constexpr int kMaxStages = 3;
 };
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p)
@@ -122,21 +134,59 @@ struct BulkArgs {
     uint64_t wait_limit_ns;
     int32_t stages;
     int32_t skip_first_fill;   // test hook: never post chunk 0, so its consumers' wait expires
+    int32_t n_ranks, chunk;    // the runtime-N instance's rank count and elements per stage
 };
 
 // Shared memory: [full[S], empty[S] mbarriers][abort flag] ... stage ring (128-B aligned):
 // stage s = N gradient slices of kChunk fp16, then master, m, v slices of kChunk fp32.
+// The ring fold of one 16-byte vector (8 elements) from a stage: rank slices j = 0..n-1
+// (already in ring order) at base + j * chunk elements.
+template <int N, bool kWire>
+__device__ __forceinline__ void fold8(const unsigned char *base, int64_t e0, int n, int chunk, float (&acc)[8])
+{
+    if constexpr (kWire) {
+        uint4 h = *reinterpret_cast<const uint4 *>(base + e0 * 2);
+        if constexpr (N > 0) {
+#pragma unroll
+            for (int j = 1; j < N; ++j)
+                h = hadd8(h, *reinterpret_cast<const uint4 *>(base + ((size_t)j * chunk + e0) * 2));
+        } else {
+#pragma unroll 4
+            for (int j = 1; j < n; ++j)
+                h = hadd8(h, *reinterpret_cast<const uint4 *>(base + ((size_t)j * chunk + e0) * 2));
+        }
+        unpack8(h, acc);
+    } else {
+        unpack8(*reinterpret_cast<const uint4 *>(base + e0 * 2), acc);
+        if constexpr (N > 0) {
+#pragma unroll
+            for (int j = 1; j < N; ++j) add8(acc, *reinterpret_cast<const uint4 *>(base + ((size_t)j * chunk + e0) * 2));
+        } else {
+#pragma unroll 4
+            for (int j = 1; j < n; ++j) add8(acc, *reinterpret_cast<const uint4 *>(base + ((size_t)j * chunk + e0) * 2));
+        }
+    }
+}
+
 template <int N, bool kWire>
 __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(const __grid_constant__ BulkArgs A)
 {
-    constexpr int kChunk = BulkShape<N>::kChunk;
     constexpr int kConsumerWarps = BulkShape<N>::kConsumerWarps;
+    // compile-time for N > 0, from the launch for the runtime-N instance
+    int kChunk, n_r;
+    if constexpr (N > 0) {
+        kChunk = BulkShape<N>::kChunk;
+        n_r = N;
+    } else {
+        kChunk = A.chunk;
+        n_r = A.n_ranks;
+    }
+    const uint32_t kStageBytes = (uint32_t)kChunk * (2u * (uint32_t)n_r + 12u);
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem);
     uint64_t *empty = full + A.stages;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + A.stages);
     unsigned char *ring = smem + ((16 * A.stages + 4 + 127) / 128) * 128;
-    constexpr uint32_t kStageBytes = BulkShape<N>::kStageBytes;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -171,12 +221,18 @@ __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(co
                 const uint32_t n = (uint32_t)((vb - q0) < kChunk ? (vb - q0) : kChunk);
                 const uint32_t bar = smem_addr(&full[st]);
                 unsigned char *base = ring + (size_t)st * kStageBytes;
-                mbar_arrive_expect_tx(bar, n * (2u * N + 12u));
+                mbar_arrive_expect_tx(bar, n * (2u * (uint32_t)n_r + 12u));
+                if constexpr (N > 0) {
 #pragma unroll
-                for (int j = 0; j < N; ++j)
-                    bulk_load(smem_addr(base + (size_t)j * kChunk * 2),
-                              A.src.rank[ring_rank(tr.shard, j, N)] + q0, n * 2u, bar);
-                unsigned char *st_base = base + (size_t)N * kChunk * 2;
+                    for (int j = 0; j < N; ++j)
+                        bulk_load(smem_addr(base + (size_t)j * kChunk * 2),
+                                  A.src.rank[ring_rank(tr.shard, j, N)] + q0, n * 2u, bar);
+                } else {
+                    for (int j = 0; j < n_r; ++j)
+                        bulk_load(smem_addr(base + (size_t)j * kChunk * 2),
+                                  A.src.rank[ring_rank(tr.shard, j, n_r)] + q0, n * 2u, bar);
+                }
+                unsigned char *st_base = base + (size_t)n_r * kChunk * 2;
                 bulk_load(smem_addr(st_base), A.master_in + (q0 - A.state_off), n * 4u, bar);
                 bulk_load(smem_addr(st_base + kChunk * 4), A.mom1_in + (q0 - A.state_off), n * 4u, bar);
                 bulk_load(smem_addr(st_base + kChunk * 8), A.mom2_in + (q0 - A.state_off), n * 4u, bar);
@@ -215,19 +271,8 @@ __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(co
             for (int64_t vi = ct; vi * kVec < n; vi += 32 * kConsumerWarps) {
                 const int64_t e0 = vi * kVec;
                 float acc[8];
-                if constexpr (kWire) {
-                    uint4 h = *reinterpret_cast<const uint4 *>(base + e0 * 2);
-#pragma unroll
-                    for (int j = 1; j < N; ++j)
-                        h = hadd8(h, *reinterpret_cast<const uint4 *>(base + ((size_t)j * kChunk + e0) * 2));
-                    unpack8(h, acc);
-                } else {
-                    unpack8(*reinterpret_cast<const uint4 *>(base + e0 * 2), acc);
-#pragma unroll
-                    for (int j = 1; j < N; ++j)
-                        add8(acc, *reinterpret_cast<const uint4 *>(base + ((size_t)j * kChunk + e0) * 2));
-                }
-                const float *sp = reinterpret_cast<const float *>(base + (size_t)N * kChunk * 2);
+                fold8<N, kWire>(base, e0, n_r, kChunk, acc);
+                const float *sp = reinterpret_cast<const float *>(base + (size_t)n_r * kChunk * 2);
                 float4 p4[2] = {*reinterpret_cast<const float4 *>(sp + e0), *reinterpret_cast<const float4 *>(sp + e0 + 4)};
                 float4 m4[2] = {*reinterpret_cast<const float4 *>(sp + kChunk + e0),
                                 *reinterpret_cast<const float4 *>(sp + kChunk + e0 + 4)};
@@ -263,11 +308,11 @@ __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(co
             float acc;
             if constexpr (kWire) {
                 uint32_t h = A.src.rank[tr.shard][i];
-                for (int j = 1; j < N; ++j) h = hadd1(h, A.src.rank[ring_rank(tr.shard, j, N)][i]);
+                for (int j = 1; j < n_r; ++j) h = hadd1(h, A.src.rank[ring_rank(tr.shard, j, n_r)][i]);
                 acc = h2f(h);
             } else {
                 acc = h2f(A.src.rank[tr.shard][i]);
-                for (int j = 1; j < N; ++j) acc = __fadd_rn(acc, h2f(A.src.rank[ring_rank(tr.shard, j, N)][i]));
+                for (int j = 1; j < n_r; ++j) acc = __fadd_rn(acc, h2f(A.src.rank[ring_rank(tr.shard, j, n_r)][i]));
             }
             bad += !isfinite(acc);
             const int64_t si = i - A.state_off;
@@ -291,8 +336,16 @@ __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(co
 template <int N>
 cudaError_t launch_bulk_n(const zero_layout &L, BulkArgs &a, cudaStream_t st)
 {
-    constexpr size_t stage_bytes = BulkShape<N>::kStageBytes;
     const size_t budget = L.dev.smem_optin > 0 ? L.dev.smem_optin : 227 * 1024;
+    size_t stage_bytes;
+    if constexpr (N > 0) {
+        stage_bytes = BulkShape<N>::kStageBytes;
+    } else {
+        const size_t per_elem = 2 * (size_t)L.n_ranks + 12;
+        a.n_ranks = L.n_ranks;
+        a.chunk = 2 * 1024 * per_elem + 256 <= budget ? 1024 : 512;
+        stage_bytes = (size_t)a.chunk * per_elem;
+    }
     int stages = (int)((budget - 256) / stage_bytes);
     if (stages > BulkShape<N>::kMaxStages) stages = BulkShape<N>::kMaxStages;
     if (stages < 2) return cudaErrorInvalidConfiguration;
@@ -311,7 +364,7 @@ cudaError_t launch_bulk_n(const zero_layout &L, BulkArgs &a, cudaStream_t st)
 
 }  // namespace
 
-bool bulk_supported(int n_ranks) { return n_ranks >= 1 && n_ranks <= 16; }
+bool bulk_supported(int n_ranks) { return n_ranks >= 1 && n_ranks <= kMaxBulkRanks; }
 
 cudaError_t launch_bulk_step(const zero_layout &L, const TileWork &w, const GradSource &src, float *master,
                              float *m, float *v, int64_t state_off, uint16_t *p16, int64_t p16_off,
@@ -339,6 +392,8 @@ cudaError_t launch_bulk_step(const zero_layout &L, const TileWork &w, const Grad
     a.wait_limit_ns = wait_limit_ns;
     a.stages = 0;
     a.skip_first_fill = skip_first_fill;
+    a.n_ranks = L.n_ranks;
+    a.chunk = 0;
     switch (L.n_ranks) {
         case 1: return launch_bulk_n<1>(L, a, st);
         case 2: return launch_bulk_n<2>(L, a, st);
@@ -356,7 +411,9 @@ cudaError_t launch_bulk_step(const zero_layout &L, const TileWork &w, const Grad
         case 14: return launch_bulk_n<14>(L, a, st);
         case 15: return launch_bulk_n<15>(L, a, st);
         case 16: return launch_bulk_n<16>(L, a, st);
-        default: return cudaErrorInvalidValue;
+        default:
+            if (L.n_ranks > kMaxBulkRanks || L.n_ranks < 1) return cudaErrorInvalidValue;
+            return launch_bulk_n<0>(L, a, st);
     }
 }
 

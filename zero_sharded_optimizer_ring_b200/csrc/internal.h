@@ -38,7 +38,7 @@ static_assert(sizeof(Seg) == 32, "device table row is 32 bytes");
 // Where each rank's gradients live for the bulk pipeline: rank r's value of flat element i
 // is rank[r][i].  One strided buffer (rank[r] = grads + r * stride), separate buffers on
 // this GPU, or other GPUs' buffers mapped into this process.
-constexpr int kMaxBulkRanks = 16;
+constexpr int kMaxBulkRanks = 64;
 struct GradSource {
     const uint16_t *rank[kMaxBulkRanks];
 };
