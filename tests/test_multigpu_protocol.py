@@ -1,7 +1,8 @@
 """The multi-GPU step's protocol on CPU (gloo, 2 and 3 ranks, no GPU): every shard is
 updated exactly once per step by its owner, every rank gathers every other shard from
-its owner, and every read of a peer's buffer happens after the barrier that makes that
-buffer complete."""
+its owner, every read of a peer's buffer is enqueued after the host barrier that makes
+that buffer complete, and, in each rank's own stream order, after a wait on that peer's
+event for the phase that completed the buffer."""
 import os
 import socket
 import sys
@@ -56,6 +57,48 @@ class RecordingOps:
 
     def sync(self):
         self._rec("barrier")
+
+    def new_fence(self):
+        self.n_fences = getattr(self, "n_fences", 0) + 1
+        return f"fence{self.n_fences}@{self.rank}"
+
+    def fence_handle(self, ev):
+        return ev.encode()
+
+    def open_fence(self, handle):
+        return "mapped:" + handle.decode()
+
+    def record(self, ev, name):
+        self._rec("record", name)
+
+    def wait(self, ev, name, stream=None):
+        self._rec("wait", name[0], name[1])
+
+
+def _check_stream_order(log, world, stage=1):
+    """In one rank's log (its stream order): every device op that reads a peer's buffer
+    comes after a wait on that peer's event of the phase that completed the buffer, and a
+    rank rewrites its own parameters only after waiting for every peer to finish reading
+    them."""
+    rank = log[0][1]
+    peers = [r for r in range(world) if r != rank]
+    waited = set()                      # (phase, peer) waited on since that phase's last record
+    n_updates = 0
+    for e in log:
+        what = e[2]
+        if what == "record":
+            waited = {w for w in waited if w[0] != e[3]}
+        elif what == "wait":
+            waited.add((e[3], e[4]))
+        elif what == "update":
+            assert all(("grads", j) in waited for j in peers), (rank, "update before every peer's grads")
+            if n_updates and stage != 3:
+                assert all(("gathered", j) in waited for j in peers), (rank, "rewrites p16 still being read")
+            n_updates += 1
+        elif what == "gather":
+            assert ("updated", e[3]) in waited, (rank, "copies a shard before its owner's update")
+        elif what == "unit":
+            assert all(("updated", j) in waited for j in peers), (rank, "gathers a layer before its owners' update")
 
 
 def _worker(rank, world, port, steps, out, stage=1):
@@ -113,6 +156,8 @@ def test_multigpu_step_protocol(world):
             assert nxt > max(e[0] for e in step_gathers)
     closes = [e for e in ev if e[2] == "close"]
     assert len(closes) == world * 2 * (world - 1)
+    for log in logs:
+        _check_stream_order(log, world)
 
 
 @pytest.mark.parametrize("world", [2, 3])
@@ -144,6 +189,8 @@ def test_multigpu_zero3_protocol(world):
         if t + 1 < steps:
             nxt = [e for e in ev if e[2] == "update" and e[5] == t + 1]
             assert max(e[0] for e in step_units) < min(e[0] for e in nxt)   # before any is rewritten
+    for log in logs:
+        _check_stream_order(log, world, stage=3)
 
 
 class DynamicOps(RecordingOps):
