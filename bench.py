@@ -33,9 +33,14 @@ DEFAULT_WORKLOAD = "flat1p3b_n4_zero1"
 FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0
 PROFILE_DIR = os.path.join(ROOT, "profiles")
-# the library's device sources: a traffic record taken on other sources is stale
+# the sources each recorded kernel is compiled from: a traffic record taken on other
+# sources is stale
 _CSRC = os.path.join(ROOT, "zero_sharded_optimizer_ring_b200", "csrc")
-KERNEL_SOURCES = sorted(os.path.join(_CSRC, f) for f in os.listdir(_CSRC) if f.endswith((".cu", ".cuh", ".h")))
+KERNEL_SOURCES = {tag: [os.path.join(_CSRC, f) for f in files] for tag, files in {
+    "bulk_step": ("bulk_step.cu", "device_common.cuh", "internal.h"),
+    "tile_kernel": ("kernels.cu", "device_common.cuh", "internal.h"),
+    "copy_range": ("kernels.cu", "device_common.cuh", "internal.h"),
+}.items()}
 
 
 def parse():
@@ -143,11 +148,11 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash():
+def kernel_source_hash(kernel_tag):
     """Hash of the kernel's sources with comments and blank space removed, so that a
     traffic record stays valid across comment-only edits."""
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in KERNEL_SOURCES[kernel_tag]:
         text = open(f).read()
         text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
         text = re.sub(r"//[^\n]*", "", text)
@@ -167,7 +172,7 @@ def profiled_traffic(kernel_tag, workload, padded):
         rec = json.load(open(traffic_record_name(kernel_tag, workload)))
     except (OSError, ValueError):
         return None
-    if rec.get("kernel_sources_sha256_16") != kernel_source_hash() or rec.get("padded_params") != padded:
+    if rec.get("kernel_sources_sha256_16") != kernel_source_hash(kernel_tag) or rec.get("padded_params") != padded:
         return None
     return rec["dram_bytes_read_per_launch"] + rec["dram_bytes_write_per_launch"]
 
@@ -199,7 +204,7 @@ def record_traffic(a, wl):
     P = zs.Layout(list(wl.tensors), wl.n_ranks, wl.stage, wl.bucket_elems, wl.pad_align, list(wl.units)).padded
     n = len(got)
     rec = {"kernel": got[0]["kernel"], "workload": wl.name, "padded_params": P,
-           "kernel_sources_sha256_16": kernel_source_hash(), "launches": n,
+           "kernel_sources_sha256_16": kernel_source_hash(a.record_tag), "launches": n,
            "dram_bytes_read_per_launch": sum(d["dram__bytes_read.sum"] for d in got) / n,
            "dram_bytes_write_per_launch": sum(d["dram__bytes_write.sum"] for d in got) / n,
            "gpu_time_ms_per_launch": sum(d.get("gpu__time_duration.sum", 0.0) for d in got) / n * 1e3,
@@ -705,7 +710,7 @@ def _overlap_reps(a, wl, lay, g, master, m, v, p16_shard, p16_full, backward, pr
         return zs.AdamW(wl.lr, wl.beta1, wl.beta2, wl.eps, wl.weight_decay, wl.loss_scale, t)
 
     res = {"bwd": [], "step": [], "pipe": [], "pipe_all": []}
-    warmup = a.warmup if cap else max(a.warmup, 2 * 4 + 2)     # the grid tuner times 4 caps twice
+    warmup = a.warmup if cap else max(a.warmup, 1 + 5 * 2 + 1)   # the plan tuner: a warm-up, 5 plans twice
     for rep in range(warmup + reps):
         torch.cuda.synchronize()
         s0, e0 = ev(), ev()
@@ -852,7 +857,8 @@ def run_zero3_passes(a, wl):
     for name, work, order in passes:
         res[f"{name}_compute_only_ms"] = timed(compute_only(work))
         for n in (1, 2, 3):
-            t, bd = timed(lambda: zero3_pass(lay, shard, slots[:n], order, work, gs, cs), breakdown=True)
+            t, bd = timed(lambda: zero3_pass(lay, shard, slots[:n], order, work, gs, cs, gather_ctas=0,
+                                             matmul_sm_carveout=None, blas=None), breakdown=True)
             res[f"{name}_{n}slot_ms"] = t
             res[f"{name}_{n}slot_breakdown"] = short(bd)
         for n in (1, 2):
@@ -864,20 +870,28 @@ def run_zero3_passes(a, wl):
     # measured once per round, rounds interleaved so that clock drift hits all alike;
     # reported: the median over rounds
     sweep = []
-    configs = [tuple(int(x) for x in c.split(":")) for c in a.zero3_configs.split(",") if c]
+    # "default" = zero3_pass with its own defaults (capped gathers, matmul SM carveout,
+    # cuBLASLt), two slots
+    configs = [("default", "default", 2) if c == "default" else tuple(int(x) for x in c.split(":"))
+               for c in a.zero3_configs.split(",") if c]
     if configs:
         if a.blas:
             torch.backends.cuda.preferred_blas_library(a.blas)
         rounds = {}
         for rnd in range(a.zero3_rounds):
             for c, gcap, n in configs:
-                set_carveout(c if c > 0 else None)
-                lay.set_gather_ctas(gcap)
+                dflt = c == "default"
+                set_carveout(None if dflt or c == 0 else c)
+                lay.set_gather_ctas(0 if dflt else gcap)
                 for name, work, order in passes:
                     if n == 0:
                         fn = compute_only(work)
-                    else:
+                    elif dflt:
                         fn = (lambda o=order, w=work, k=n: zero3_pass(lay, shard, slots[:k], o, w, gs, cs))
+                    else:
+                        fn = (lambda o=order, w=work, k=n: zero3_pass(lay, shard, slots[:k], o, w, gs, cs,
+                                                                      gather_ctas=None, matmul_sm_carveout=None,
+                                                                      blas=None))
                     torch.cuda.synchronize()
                     s0, e0 = ev(), ev()
                     s0.record(gs)

@@ -238,14 +238,17 @@ zero_status zero_step_bucket(const zero_layout *layout, int64_t bucket, const ui
  * this call: enqueue the producer's records first (the producer's work itself may still
  * be running).  Result identical to zero_step.
  *
- * Grid: the update shares the GPU with the backward pass, and the best split of the SMs
- * depends on the two workloads.  Unless zero_set_max_ctas fixed a cap, the library
- * chooses one by measurement: over the layout's first overlapped calls it times whole
- * calls (CUDA events on `stream`, from the first wait to the last launch) with the
- * update capped at 1, 2/3, 1/2 and 1/3 of the SMs, two calls each, then keeps the
- * fastest for every later call.  It never waits for these events: a call issued before
- * the previous timed call has finished on the GPU is not timed.  The cap never changes
- * a result. */
+ * Launch plan: the update shares the GPU with the backward pass, and whether and how to
+ * split the SMs depends on the two workloads (and on the power budget they share).
+ * Unless zero_set_max_ctas fixed a cap, the library chooses a plan by measurement: after
+ * one untimed warm-up call it times whole calls (CUDA events on `stream`, from the first
+ * wait to the last launch) under five plans, round-robin, two calls each: the update
+ * following the backward bucket by bucket with its grid capped at 1, 2/3, 1/2 or 1/3 of
+ * the SMs, or deferred to one full-grid launch after the last bucket's event (the
+ * back-to-back order, for workloads where sharing the GPU does not pay); it then keeps
+ * the plan with the lowest mean for every later call.  It never waits for these
+ * events: a call issued before the previous timed call has finished on the GPU is not
+ * timed.  The plan never changes a result. */
 zero_status zero_step_overlapped(const zero_layout *layout, void *const *ready_events,
                                  const uint16_t *grads, int64_t rank_stride, float *master, float *m,
                                  float *v, uint16_t *p16_shard, uint16_t *p16_full,
@@ -338,7 +341,7 @@ zero_status zero_step_dynamic(const zero_layout *layout, const uint16_t *grads, 
  * Costs the fused step's bytes instead of the reduce-then-update pair of
  * zero_step_dynamic, for a second state set (12 bytes and 2 for fp16 per parameter).
  * No in buffer may overlap an out buffer (ZERO_ERR_INVALID).  Either implementation
- * (zero_set_impl; both serve every N).  nonfinite: device int32 [n_buckets],
+ * (zero_set_impl).  nonfinite: device int32 [n_buckets],
  * required, zeroed here.  The pages name
  * no overflow handling; this is the two-phase form of the skip described above. */
 zero_status zero_step_dynamic_commit(const zero_layout *layout, const uint16_t *grads, int64_t rank_stride,
@@ -411,12 +414,13 @@ zero_status zero_ipc_get_handle(const void *dev_ptr, void *handle_out, int64_t *
 zero_status zero_ipc_open(const void *handle, int64_t offset, void **dev_ptr_out);
 zero_status zero_ipc_close(void *dev_ptr, int64_t offset);
 
-/* Select the fused kernel's implementation: 0 = automatic (the bulk-copy pipeline, which
- * serves every N up to 64: compiled per rank count for N <= 16, one runtime-N instance
- * above; register streaming beyond 64), 1 = register streaming (vectorised 16-byte loads
- * held in registers; any N), 2 = bulk-copy pipeline (cp.async.bulk into a shared-memory
- * ring, warp-specialised; N <= 64, register streaming above).  Results are
- * bit-identical. */
+/* Select the fused kernel's implementation: 0 = automatic (the bulk-copy pipeline for
+ * N <= 16, where it has an instance per rank count; register streaming above, where it
+ * runs at the copy bandwidth), 1 = register streaming (vectorised 16-byte loads held in
+ * registers; any N), 2 = bulk-copy pipeline (cp.async.bulk into a shared-memory ring,
+ * warp-specialised; one runtime-N instance serves 17 <= N <= 64; register streaming
+ * above).  The per-rank-pointer calls (zero_step_ranks, zero_step_shard*) always use the
+ * pipeline.  Results are bit-identical. */
 zero_status zero_set_impl(zero_layout *layout, int32_t impl);
 
 /* Cap on the number of CTAs of the tile-walking kernels (the fused step in both

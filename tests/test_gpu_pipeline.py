@@ -92,11 +92,11 @@ def test_overlapped_step_with_simulated_backward(key, group):
 
 @pytest.mark.parametrize("key", ["flat1p3b_n4_zero1", "ragged2000_n16_zero2"])
 def test_overlapped_grid_tuner_keeps_results(key):
-    """With no cap set, the overlapped step times several grid caps over its first calls
-    and then keeps the fastest; every call, whatever its grid, must give the oracle's
-    result (12 steps: each candidate timed twice, then the chosen one)."""
+    """With no cap set, the overlapped step times several launch plans over its first calls
+    and then keeps the fastest; every call, whatever its plan, must give the oracle's
+    result (14 steps: a warm-up, each of five plans timed twice, then the chosen one)."""
     wl = reduced_workloads()[key]
-    steps = 12
+    steps = 14
     ref, _ = S.oracle_run(wl, steps)
     lay, bufs = _setup(wl)
     b = bufs()

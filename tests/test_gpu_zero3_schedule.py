@@ -87,9 +87,11 @@ def test_capped_allgather_matches_oracle(aligned, gather_ctas):
     assert (S.to_np(full)[lay.padded:] == 7).all()
 
 
+@pytest.mark.parametrize("gather_ctas", [0, None])
 @pytest.mark.parametrize("n_slots", [1, 2, 3])
 @pytest.mark.parametrize("backward", [False, True])
-def test_prefetch_schedule_gives_each_layer_its_parameters(n_slots, backward):
+def test_prefetch_schedule_gives_each_layer_its_parameters(n_slots, backward, gather_ctas):
+    """gather_ctas 0: the gathers' default grid; None: the schedule's own setting."""
     wl = _workload()
     lay, shard, ref = _stepped_shards(wl)
     _, _, _, u = lay.tables()
@@ -107,6 +109,8 @@ def test_prefetch_schedule_gives_each_layer_its_parameters(n_slots, backward):
 
     gs, cs = torch.cuda.Stream(), torch.cuda.Stream()
     torch.cuda.synchronize()                        # inputs written on the default stream
-    zero3_pass(lay, shard, slots, order, compute, gs, cs)
+    kw = {} if gather_ctas is None else {"gather_ctas": gather_ctas}
+    zero3_pass(lay, shard, slots, order, compute, gs, cs, **kw)
     torch.cuda.synchronize()
+    assert lay.gather_ctas == 0                     # the layout's setting is restored
     S.assert_bits_equal(S.to_np(out), ref.p16_full, "layers as the compute saw them")

@@ -139,6 +139,11 @@ class Layout:
     def set_gather_ctas(self, max_ctas):
         """All-gather copies as max_ctas persistent CTAs (0 = the default grid of short blocks)."""
         _check(_abi.lib().zero_set_gather_ctas(self._h, int(max_ctas)), "zero_set_gather_ctas")
+        self._gather_ctas = int(max_ctas)
+
+    @property
+    def gather_ctas(self):
+        return getattr(self, "_gather_ctas", 0)
 
     def debug_set_wait(self, wait_limit_ns, skip_first_fill=0):
         _check(_abi.lib().zero_debug_set_wait(self._h, int(wait_limit_ns), int(skip_first_fill)),

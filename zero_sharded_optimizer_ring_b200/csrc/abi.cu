@@ -355,10 +355,7 @@ zero::GradSource strided(const zero_layout *L, const uint16_t *grads, int64_t st
 cudaError_t fused(const zero_layout *L, const TileWork &w, const uint16_t *grads, int64_t stride, float *master,
                   float *m, float *v, uint16_t *p16, const AdamScalars &c, int32_t *nonfinite, cudaStream_t st)
 {
-    // automatic choice: the bulk-copy pipeline wherever it has a specialisation (it is
-    // faster than register streaming on every measured workload, by ~12 % on the flat
-    // N=4 list under the power cap)
-    const bool bulk = (L->impl == 2 || L->impl == 0) && zero::bulk_supported(L->n_ranks);
+    const bool bulk = zero::use_bulk(*L);
     if (bulk)
         return zero::launch_bulk_step(*L, w, strided(L, grads, stride), master, m, v, 0, p16, 0, c, nonfinite,
                                       L->dev.wait_limit_ns, L->dev.skip_first_fill, st);
@@ -409,43 +406,70 @@ namespace {
 // buckets (~0.5-1 GB of traffic, 80-150 us at full bandwidth: launch gaps stay negligible).
 constexpr int64_t kMinOverlapLaunch = int64_t(1) << 24;
 
-// The grid cap of candidate i of the overlapped step's tuner: SMs x {1, 2/3, 1/2, 1/3}.
+// Candidate plan i of the overlapped step's tuner: i < 4 follows the backward with the
+// update's grid capped at SMs x {1, 2/3, 1/2, 1/3} (0 = no cap); i == 4 defers the whole
+// update to one full-grid launch after the last bucket's event.
+constexpr int kDeferred = 4;
+
 int32_t tuner_cap(const zero_layout *L, int i)
 {
-    static const int kSixths[zero::OverlapTuner::kCands] = {6, 4, 3, 2};
+    static const int kSixths[4] = {6, 4, 3, 2};
     const int sms = L->dev.num_sms > 0 ? L->dev.num_sms : 148;
-    return i == 0 ? 0 : sms * kSixths[i] / 6;
+    return (i == 0 || i == kDeferred) ? 0 : sms * kSixths[i] / 6;
 }
 
-// Grid cap of this overlapped call: the caller's (zero_set_max_ctas) if set; otherwise the
-// tuner's.  Harvests the previous timed call if its end event has completed (never waits),
-// then times the next candidate that still lacks trials, or settles on the fastest.
-// *timed: record the tuner's events around this call.
-int32_t overlap_cap(const zero_layout *L, bool *timed)
+struct OverlapPlan {
+    int32_t cap = 0;          // grid cap of every launch (0 = full grid)
+    bool deferred = false;    // one launch after every bucket's event
+    bool timed = false;       // record the tuner's events around this call
+};
+
+// The plan of this overlapped call: the caller's cap (zero_set_max_ctas) if set;
+// otherwise the tuner's.  Harvests the previous timed call if its end event has
+// completed (never waits), then times the next candidate in round-robin order that
+// still lacks trials, or keeps the one with the lowest mean.
+OverlapPlan overlap_plan(const zero_layout *L)
 {
-    *timed = false;
+    OverlapPlan p;
     zero::OverlapTuner &T = L->dev.tuner;
-    if (L->max_ctas > 0 || !T.begin || !T.end) return L->max_ctas;
+    if (L->max_ctas > 0 || !T.begin || !T.end) {
+        p.cap = L->max_ctas;
+        return p;
+    }
+    const int K = zero::OverlapTuner::kCands;
     if (T.pending >= 0) {
-        if (cudaEventQuery(T.end) != cudaSuccess) return tuner_cap(L, T.pending);   // still running: untimed
+        if (cudaEventQuery(T.end) != cudaSuccess) {            // still running: same plan, untimed
+            p.cap = tuner_cap(L, T.pending);
+            p.deferred = T.pending == kDeferred;
+            return p;
+        }
         float ms = 0.f;
         if (cudaEventElapsedTime(&ms, T.begin, T.end) == cudaSuccess) {
-            float &b = T.best_ms[T.pending];
-            if (T.trials[T.pending] == 0 || ms < b) b = ms;
+            T.sum_ms[T.pending] += ms;
             ++T.trials[T.pending];
         }
         T.pending = -1;
     }
-    for (int i = 0; i < zero::OverlapTuner::kCands; ++i)
-        if (T.trials[i] < zero::OverlapTuner::kTrials) {
-            T.pending = i;
-            *timed = true;
-            return tuner_cap(L, i);
+    int pick = T.chosen;
+    if (pick < 0 && T.calls++ > 0) {                           // the first call is a warm-up
+        int fewest = 0;
+        for (int i = 1; i < K; ++i)
+            if (T.trials[i] < T.trials[fewest]) fewest = i;
+        if (T.trials[fewest] < zero::OverlapTuner::kTrials) {
+            T.pending = fewest;
+            p.timed = true;
+            pick = fewest;
+        } else {
+            int best = 0;
+            for (int i = 1; i < K; ++i)
+                if (T.sum_ms[i] < T.sum_ms[best]) best = i;
+            T.chosen = pick = best;
         }
-    int best = 0;
-    for (int i = 1; i < zero::OverlapTuner::kCands; ++i)
-        if (T.best_ms[i] < T.best_ms[best]) best = i;
-    return tuner_cap(L, best);
+    }
+    if (pick < 0) pick = 0;
+    p.cap = tuner_cap(L, pick);
+    p.deferred = pick == kDeferred;
+    return p;
 }
 
 // The overlapped step over launch groups: launch j covers buckets [first[j], first[j+1]).
@@ -456,19 +480,20 @@ zero_status overlapped(const zero_layout *L, void *const *ready_events, const st
 {
     const AdamScalars c = step_scalars(L->n_ranks, *hp);
     uint16_t *p16 = L->stage == 3 ? p16_shard : p16_full;
-    bool timed = false;
-    const int32_t cap = overlap_cap(L, &timed);
-    cudaError_t e = timed ? cudaEventRecord(L->dev.tuner.begin, st) : cudaSuccess;
-    for (size_t j = 0; e == cudaSuccess && j + 1 < first.size(); ++j) {
-        for (int64_t b = first[j]; e == cudaSuccess && b < first[j + 1]; ++b)
+    const OverlapPlan plan = overlap_plan(L);
+    const std::vector<int64_t> all = {0, (int64_t)L->bucket_lo.size()};
+    const std::vector<int64_t> &launches = plan.deferred ? all : first;
+    cudaError_t e = plan.timed ? cudaEventRecord(L->dev.tuner.begin, st) : cudaSuccess;
+    for (size_t j = 0; e == cudaSuccess && j + 1 < launches.size(); ++j) {
+        for (int64_t b = launches[j]; e == cudaSuccess && b < launches[j + 1]; ++b)
             e = cudaStreamWaitEvent(st, (cudaEvent_t)ready_events[b], 0);
-        TileWork w = bucket_range_tiles(L, first[j], first[j + 1]);
-        w.max_ctas = cap;
+        TileWork w = bucket_range_tiles(L, launches[j], launches[j + 1]);
+        w.max_ctas = plan.cap;
         if (e == cudaSuccess) e = fused(L, w, grads, rank_stride, master, m, v, p16, c, nonfinite, st);
     }
     if (e == cudaSuccess && L->stage == 3) e = zero::launch_copy_range(*L, 0, L->padded, p16_shard, p16_full, st);
-    if (e == cudaSuccess && timed) e = cudaEventRecord(L->dev.tuner.end, st);
-    if (e != cudaSuccess && timed) L->dev.tuner.pending = -1;
+    if (e == cudaSuccess && plan.timed) e = cudaEventRecord(L->dev.tuner.end, st);
+    if (e != cudaSuccess && plan.timed) L->dev.tuner.pending = -1;
     return cuda_status(e);
 }
 
@@ -637,7 +662,7 @@ extern "C" zero_status zero_step_dynamic_commit(const zero_layout *L, const uint
     cudaStream_t st = (cudaStream_t)stream;
     int64_t bad = 0;
     cudaError_t e = cudaMemsetAsync(nonfinite, 0, L->bucket_lo.size() * sizeof(int32_t), st);
-    const bool bulk = (L->impl == 2 || L->impl == 0) && zero::bulk_supported(L->n_ranks);
+    const bool bulk = zero::use_bulk(*L);
     if (e == cudaSuccess && bulk)
         e = zero::launch_bulk_step(*L, all_tiles(L), strided(L, grads, rank_stride), master_out, m_out, v_out, 0,
                                    p16_out, 0, step_scalars(L->n_ranks, h), nonfinite, L->dev.wait_limit_ns,

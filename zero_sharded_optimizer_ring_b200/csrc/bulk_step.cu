@@ -366,6 +366,18 @@ cudaError_t launch_bulk_n(const zero_layout &L, BulkArgs &a, cudaStream_t st)
 
 bool bulk_supported(int n_ranks) { return n_ranks >= 1 && n_ranks <= kMaxBulkRanks; }
 
+// The automatic choice (impl 0) for a strided gradient buffer, from B200 measurements of
+// both kernels: the pipeline where it has a compiled instance (N <= 16; ~12 % ahead of
+// register streaming on the flat N=4 list), register streaming above (0.99-1.01 of the
+// measured copy bandwidth at N = 24-64, where the runtime-N pipeline instance reaches
+// 0.48-0.87: its few consumer warps cannot fold that many ranks fast enough).
+bool use_bulk(const zero_layout &L)
+{
+    if (L.impl == 1) return false;
+    if (L.impl == 2) return bulk_supported(L.n_ranks);
+    return L.n_ranks >= 1 && L.n_ranks <= 16;
+}
+
 cudaError_t launch_bulk_step(const zero_layout &L, const TileWork &w, const GradSource &src, float *master,
                              float *m, float *v, int64_t state_off, uint16_t *p16, int64_t p16_off,
                              const AdamScalars &c, int32_t *nonfinite, uint64_t wait_limit_ns,

@@ -76,15 +76,20 @@ struct TileWork {
     int32_t max_ctas = 0;  // > 0: this launch's grid cap (overrides the layout's)
 };
 
-// Grid-cap tuning of the overlapped step: each candidate cap (a fraction of the SMs) is
-// timed over whole calls (first wait to last launch, CUDA events on the caller's stream)
-// kTrials times, then the fastest is kept.  Nothing ever waits on these events: a call
-// whose predecessor has not finished yet is simply not timed.
+// Launch-plan tuning of the overlapped step: candidate plans (the update's grid capped at
+// 1, 2/3, 1/2 or 1/3 of the SMs while it follows the backward bucket by bucket, or the
+// whole update deferred to one full-grid launch after the last bucket) are each timed
+// over whole calls (CUDA events on the caller's stream, first wait to last launch),
+// round-robin after one untimed warm-up call, kTrials times each; then the plan with the
+// lowest mean is kept.  Nothing ever waits on these events: a call issued before the
+// previous timed call has finished on the GPU is not timed.
 struct OverlapTuner {
-    static constexpr int kCands = 4, kTrials = 2;
-    float best_ms[kCands] = {0.f, 0.f, 0.f, 0.f};
-    int32_t trials[kCands] = {0, 0, 0, 0};
+    static constexpr int kCands = 5, kTrials = 2;
+    float sum_ms[kCands] = {0.f, 0.f, 0.f, 0.f, 0.f};
+    int32_t trials[kCands] = {0, 0, 0, 0, 0};
+    int32_t calls = 0;                    // calls seen (the first is a warm-up)
     int32_t pending = -1;                 // candidate whose timed call is in flight
+    int32_t chosen = -1;                  // the kept plan, once every candidate is timed
     cudaEvent_t begin = nullptr, end = nullptr;
 };
 
@@ -156,6 +161,7 @@ cudaError_t launch_fused_step_to(const zero_layout &L, const TileWork &w, const 
 
 // bulk_step.cu
 bool bulk_supported(int n_ranks);
+bool use_bulk(const zero_layout &L);   // the fused step's implementation for a strided buffer
 // master / m / v hold flat elements [state_off, ...) and p16 [p16_off, ...): element i is
 // at index i - off (both offsets multiples of 8).  The state is read from master_in /
 // m_in / v_in where given (same indexing; a second buffer set), else from master / m / v.

@@ -12,29 +12,77 @@ library kernel; the schedule is CUDA stream waits and events.
 from . import gather_unit
 
 
-def zero3_pass(layout, p16_shard, slots, units, compute, gather_stream, compute_stream):
+# How the gathers share the GPU with the layers' GEMMs during a pass (measured on the
+# Llama-shaped list, 2048 tokens, two slots): the gathers run as 16 persistent CTAs
+# (zero_set_gather_ctas) instead of a grid that floods every SM between GEMM waves, and
+# the layer GEMMs leave 16 SMs to them (cuBLAS's SM-count target, honoured on the cuBLASLt
+# path): the compute alone is no slower with 132 SMs, and the gathers then run beside it
+# instead of in its waves' way.
+GATHER_CTAS = 16
+MATMUL_SM_CARVEOUT = 16
+MATMUL_BLAS = "cublaslt"
+
+
+class _MatmulShare:
+    """Within the block, torch's matmuls leave `carveout` SMs free and prefer `blas`
+    (either None: unchanged); both restored on exit."""
+
+    def __init__(self, carveout, blas):
+        self.carveout, self.blas = carveout, blas
+
+    def __enter__(self):
+        import torch
+        self.saved_carveout = self.saved_blas = None
+        if self.carveout is not None and hasattr(torch._C, "_set_sm_carveout_experimental"):
+            self.saved_carveout = (torch._C._get_sm_carveout_experimental(),)
+            torch._C._set_sm_carveout_experimental(self.carveout or None)
+        if self.blas is not None:
+            self.saved_blas = (torch.backends.cuda.preferred_blas_library(),)
+            torch.backends.cuda.preferred_blas_library(self.blas)
+        return self
+
+    def __exit__(self, *exc):
+        import torch
+        if self.saved_carveout is not None:
+            torch._C._set_sm_carveout_experimental(self.saved_carveout[0])
+        if self.saved_blas is not None:
+            torch.backends.cuda.preferred_blas_library(self.saved_blas[0])
+
+
+def zero3_pass(layout, p16_shard, slots, units, compute, gather_stream, compute_stream,
+               gather_ctas=GATHER_CTAS, matmul_sm_carveout=MATMUL_SM_CARVEOUT, blas=MATMUL_BLAS):
     """Run one pass over `units` (a forward pass: ascending; a backward pass: descending).
 
     Unit units[j] is gathered into slots[j % len(slots)] on gather_stream, once the slot's
     previous occupant units[j - len(slots)] has been computed; compute(unit, buffer) is
     then called with compute_stream current and must enqueue the layer's work there.
-    Returns the list of (gather started, gathered, computed) torch.cuda.Event triples,
-    one per unit (timing events: layer_breakdown reads them)."""
+    During the pass the gathers run on gather_ctas persistent CTAs (None: the layout's
+    setting) and torch's matmuls leave matmul_sm_carveout SMs free and prefer `blas`
+    (None: unchanged); every setting is restored afterwards.  Returns the list of (gather
+    started, gathered, computed) torch.cuda.Event triples, one per unit (timing events:
+    layer_breakdown reads them)."""
     import torch
     n = len(slots)
     marks = []
-    for j, u in enumerate(units):
-        started, gathered, computed = (torch.cuda.Event(enable_timing=True) for _ in range(3))
-        if j >= n:
-            gather_stream.wait_event(marks[j - n][2])
-        started.record(gather_stream)
-        gather_unit(layout, u, p16_shard, slots[j % n], stream=gather_stream)
-        gathered.record(gather_stream)
-        compute_stream.wait_event(gathered)
-        with torch.cuda.stream(compute_stream):
-            compute(u, slots[j % n])
-        computed.record(compute_stream)
-        marks.append((started, gathered, computed))
+    saved_ctas = layout.gather_ctas
+    if gather_ctas is not None:
+        layout.set_gather_ctas(gather_ctas)
+    try:
+        with _MatmulShare(matmul_sm_carveout, blas):
+            for j, u in enumerate(units):
+                started, gathered, computed = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+                if j >= n:
+                    gather_stream.wait_event(marks[j - n][2])
+                started.record(gather_stream)
+                gather_unit(layout, u, p16_shard, slots[j % n], stream=gather_stream)
+                gathered.record(gather_stream)
+                compute_stream.wait_event(gathered)
+                with torch.cuda.stream(compute_stream):
+                    compute(u, slots[j % n])
+                computed.record(compute_stream)
+                marks.append((started, gathered, computed))
+    finally:
+        layout.set_gather_ctas(saved_ctas)
     return marks
 
 
