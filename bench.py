@@ -709,7 +709,7 @@ def _overlap_reps(a, wl, lay, g, master, m, v, p16_shard, p16_full, backward, pr
     def hp():
         return zs.AdamW(wl.lr, wl.beta1, wl.beta2, wl.eps, wl.weight_decay, wl.loss_scale, t)
 
-    res = {"bwd": [], "step": [], "pipe": [], "pipe_all": []}
+    res = {"bwd": [], "step": [], "seq": [], "pipe": [], "pipe_all": []}
     warmup = a.warmup if cap else max(a.warmup, 1 + 5 * 2 + 1)   # the plan tuner: a warm-up, 5 plans twice
     for rep in range(warmup + reps):
         torch.cuda.synchronize()
@@ -725,6 +725,17 @@ def _overlap_reps(a, wl, lay, g, master, m, v, p16_shard, p16_full, backward, pr
         e1.record(compute)
         torch.cuda.synchronize()
         t += 1
+        # back to back in one timed region: the whole backward, then the whole step, no
+        # idle gap between them (the same power and clock state the pipelined run sees)
+        s3, e3, done = ev(), ev(), torch.cuda.Event()
+        s3.record(producer)
+        backward()
+        done.record(producer)
+        compute.wait_event(done)
+        zs.step(lay, g, master, m, v, p16_shard, p16_full, hp(), stream=compute)
+        e3.record(compute)
+        torch.cuda.synchronize()
+        t += 1
         ready = [torch.cuda.Event() for _ in range(lay.n_buckets)]
         s2, e2 = ev(), ev()
         s2.record(producer)
@@ -736,14 +747,16 @@ def _overlap_reps(a, wl, lay, g, master, m, v, p16_shard, p16_full, backward, pr
         if rep >= warmup:
             res["bwd"].append(s0.elapsed_time(e0))
             res["step"].append(s1.elapsed_time(e1))
+            res["seq"].append(s3.elapsed_time(e3))
             res["pipe"].append(s2.elapsed_time(e2))
-    tb, ts, tp = (statistics.median(res[k]) for k in ("bwd", "step", "pipe"))
+    tb, ts, tq, tp = (statistics.median(res[k]) for k in ("bwd", "step", "seq", "pipe"))
     print(json.dumps({
         "metric": "bucket-pipelined step behind a simulated backward (overlap)", "workload": wl.name,
         "backward": a.backward, "compute_stream_priority": prio_name,
         "max_ctas": cap if cap else "auto (measured by the library)",
         "bucket_group": group if group else "auto (zero_step_overlapped: launches of >= 2^24 elements)",
-        "t_back_to_back_ms": tb + ts, "pipelined_every_call_ms": res["pipe_all"],
+        "t_back_to_back_ms": tq, "t_backward_plus_step_alone_ms": tb + ts,
+        "pipelined_every_call_ms": res["pipe_all"],
         "buckets": lay.n_buckets,
         "reps": reps, "t_backward_ms": tb, "t_step_ms": ts, "t_pipelined_ms": tp, "exposed_step_ms": tp - tb,
         "overlap_efficiency": (tb + ts - tp) / ts,

@@ -35,8 +35,10 @@ namespace {
 //
 // N = 0 is the runtime rank count (17..kMaxBulkRanks): a stage of (2n + 12) bytes per
 // element grows with n, so the chunk is 1024 elements while two stages of it fit in
-// shared memory and 512 above; 4 consumer warps (one 16-byte vector per thread for a
-// 1024-element chunk).
+// shared memory and 512 above.  Folding that many ranks takes more consumer time per
+// chunk than a few warps have, so this instance runs one group of 4 consumer warps per
+// stage (group g takes the chunks of stage g), and consecutive chunks are folded in
+// parallel; kConsumerWarps is then the size of one group.
 template <int N>
 struct BulkShape {
     static constexpr int kChunk = N <= 4 ? 4096 : 2048;        // elements per stage
@@ -48,9 +50,9 @@ struct BulkShape {
 
 template <>
 struct BulkShape<0> {
-    static constexpr int kConsumerWarps = 4;
-    static constexpr int kThreads = 32 * (1 + kConsumerWarps);
+    static constexpr int kConsumerWarps = 4;      // per group; one group per stage
     static constexpr int kMaxStages = 3;
+    static constexpr int kThreads = 32 * (1 + kConsumerWarps * kMaxStages);
 };
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p)
@@ -182,6 +184,7 @@ __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(co
         n_r = A.n_ranks;
     }
     const uint32_t kStageBytes = (uint32_t)kChunk * (2u * (uint32_t)n_r + 12u);
+    const int groups = N > 0 ? 1 : A.stages;      // consumer groups (see BulkShape<0>)
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem);
     uint64_t *empty = full + A.stages;
@@ -253,7 +256,9 @@ __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(co
     }
 
     // ---------------------------------------------------------------- consumers
-    const int ct = threadIdx.x - 32;            // 0 .. 32 * kConsumerWarps - 1
+    const int grp = (warp - 1) / kConsumerWarps;  // consumer group: takes the chunks of stage grp
+    if (grp >= groups) return;
+    const int ct = threadIdx.x - 32 - grp * 32 * kConsumerWarps;   // 0 .. 32 * kConsumerWarps - 1
     int64_t s = A.w.seg_first;
     uint32_t it = 0;
     for (int64_t t = A.w.tile_first + blockIdx.x; t < t_end; t += gridDim.x) {
@@ -262,6 +267,7 @@ __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(co
         const int64_t va = (tr.a + kVec - 1) / kVec * kVec, vb = tr.b / kVec * kVec;
         int bad = 0;
         for (int64_t q0 = va; q0 < vb; q0 += kChunk, ++it) {
+            if (groups > 1 && (int)(it % (uint32_t)groups) != grp) continue;   // another group's stage
             const uint32_t st = it % (uint32_t)A.stages, ph = (it / (uint32_t)A.stages) & 1u;
             // every lane waits (acquiring the stage's data); the warp leaves together
             const bool got = wait_phase(smem_addr(&full[st]), ph, abort_flag, A.error, A.wait_limit_ns);
@@ -303,7 +309,7 @@ __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(co
         const int64_t head_end = va < tr.b ? va : tr.b;
         const int64_t tail_begin = vb > head_end ? vb : head_end;
         const int64_t n_head = head_end - tr.a, n_tail = tr.b - tail_begin;
-        if (ct < n_head + n_tail) {
+        if (grp == 0 && ct < n_head + n_tail) {
             const int64_t i = ct < n_head ? tr.a + ct : tail_begin + (ct - n_head);
             float acc;
             if constexpr (kWire) {
