@@ -178,6 +178,7 @@ def profiled_traffic(kernel_tag, workload, padded):
 
 
 _NCU_UNITS = {"byte": 1.0, "kbyte": 1e3, "mbyte": 1e6, "gbyte": 1e9, "tbyte": 1e12,
+              "ns": 1e-9, "us": 1e-6, "ms": 1e-3, "s": 1.0,
               "nsecond": 1e-9, "usecond": 1e-6, "msecond": 1e-3, "second": 1.0}
 
 

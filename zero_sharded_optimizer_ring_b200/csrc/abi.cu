@@ -452,9 +452,19 @@ OverlapPlan overlap_plan(const zero_layout *L)
     }
     int pick = T.chosen;
     if (pick < 0 && T.calls++ > 0) {                           // the first call is a warm-up
-        int fewest = 0;
-        for (int i = 1; i < K; ++i)
-            if (T.trials[i] < T.trials[fewest]) fewest = i;
+        // the candidate with the fewest trials; rounds alternate direction (0..K-1, then
+        // K-1..0), so that a steady drift of the clocks while the GPU warms up adds the
+        // same to every candidate's sum
+        int fewest = -1;
+        for (int k = 0; k < K; ++k) {
+            int lo = K;
+            for (int i = 0; i < K; ++i) lo = T.trials[i] < lo ? T.trials[i] : lo;
+            const int i = (lo % 2 == 0) ? k : K - 1 - k;
+            if (T.trials[i] == lo) {
+                fewest = i;
+                break;
+            }
+        }
         if (T.trials[fewest] < zero::OverlapTuner::kTrials) {
             T.pending = fewest;
             p.timed = true;

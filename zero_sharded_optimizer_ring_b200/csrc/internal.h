@@ -80,8 +80,8 @@ struct TileWork {
 // 1, 2/3, 1/2 or 1/3 of the SMs while it follows the backward bucket by bucket, or the
 // whole update deferred to one full-grid launch after the last bucket) are each timed
 // over whole calls (CUDA events on the caller's stream, first wait to last launch),
-// round-robin after one untimed warm-up call, kTrials times each; then the plan with the
-// lowest mean is kept.  Nothing ever waits on these events: a call issued before the
+// round-robin after one untimed warm-up call, kTrials times each, rounds alternating
+// direction; then the plan with the lowest mean is kept.  Nothing ever waits on these events: a call issued before the
 // previous timed call has finished on the GPU is not timed.
 struct OverlapTuner {
     static constexpr int kCands = 5, kTrials = 2;
