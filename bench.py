@@ -62,6 +62,10 @@ def parse():
     ap.add_argument("--dynamic-commit", action="store_true",
                     help="time zero_step_dynamic_commit (one fused pass into a second state set, overflow "
                          "check, swap) instead of the fused step")
+    ap.add_argument("--graph", action="store_true",
+                    help="time steps launched one by one against the same steps replayed from CUDA graphs "
+                         "(zero_step_device_scalars; its own JSON line)")
+    ap.add_argument("--graph-steps", type=int, default=20, help="--graph: steps captured per graph")
     ap.add_argument("--zero3-passes", action="store_true",
                     help="time ZeRO-3's per-layer forward and backward gathers with 1-3 prefetch slots "
                          "against a simulated layer compute (its own JSON line)")
@@ -767,6 +771,78 @@ def _overlap_reps(a, wl, lay, g, master, m, v, p16_shard, p16_full, backward, pr
     return t
 
 
+def run_graph(a, wl):
+    """Launch-bound small models: K fused steps launched one by one (zero_step, scalars
+    passed at launch) against the same K steps replayed from CUDA graphs, each graph
+    holding G captured steps of zero_step_device_scalars that read their scalars from rows
+    of a device table filled before timing.  Both timed with CUDA events on one stream,
+    inputs resident, the same kernels."""
+    import torch
+    import seeded_inputs as si
+    import zero_sharded_optimizer_ring_b200 as zs
+
+    torch.cuda.set_device(dist_env()[1])
+    lay = zs.Layout(list(wl.tensors), wl.n_ranks, wl.stage, wl.bucket_elems, wl.pad_align, list(wl.units))
+    lay.to_device()
+    P, psi, N = lay.padded, lay.psi, wl.n_ranks
+    g = torch.empty((N, P), dtype=torch.int16, device="cuda")
+    si.fill_grads_cuda(g, psi, wl.seed, wl.grad_sigma, wl.loss_scale, wl.heavy_frac, wl.heavy_mult)
+    master = torch.empty(P, dtype=torch.float32, device="cuda")
+    si.fill_f32_cuda(master, psi, wl.seed, si.STREAM_MASTER, wl.master_sigma)
+    m = torch.zeros(P, dtype=torch.float32, device="cuda")
+    v = torch.zeros(P, dtype=torch.float32, device="cuda")
+    p16_full = torch.zeros(P, dtype=torch.int16, device="cuda")
+    p16_shard = torch.zeros(P, dtype=torch.int16, device="cuda") if wl.stage == 3 else None
+    hp = lambda t: zs.AdamW(wl.lr, wl.beta1, wl.beta2, wl.eps, wl.weight_decay, wl.loss_scale, t)
+    G = max(1, min(a.graph_steps, a.steps))
+    K = (a.steps // G) * G
+    st = torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    t = 0
+    with torch.cuda.stream(st):
+        for _ in range(a.warmup):
+            t += 1
+            zs.step(lay, g, master, m, v, p16_shard, p16_full, hp(t))
+        torch.cuda.synchronize()
+        s0, e0 = ev(), ev()
+        s0.record()
+        for _ in range(K):
+            t += 1
+            zs.step(lay, g, master, m, v, p16_shard, p16_full, hp(t))
+        e0.record()
+        torch.cuda.synchronize()
+    plain_ms = s0.elapsed_time(e0) / K
+
+    # the scalars of the next K steps in a device table; graph i holds steps i*G .. i*G+G-1,
+    # each reading its own row (a training loop would refill one table per replay instead)
+    table = torch.empty((K, 9), dtype=torch.float32, device="cuda")
+    table.copy_(torch.from_numpy(np.stack([zs.step_scalars(lay, hp(t + 1 + k)) for k in range(K)])))
+    t += K
+    graphs = []
+    for i in range(K // G):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=st):
+            for j in range(G):
+                zs.step_device_scalars(lay, g, master, m, v, p16_shard, p16_full, table[i * G + j])
+        graphs.append(gr)
+    torch.cuda.synchronize()
+    s1, e1 = ev(), ev()
+    with torch.cuda.stream(st):
+        s1.record()
+        for gr in graphs:
+            gr.replay()
+        e1.record()
+        torch.cuda.synchronize()
+    graph_ms = s1.elapsed_time(e1) / K
+    zs.get_error(lay)
+    del graphs
+    print(json.dumps({"metric": "fused step launched per step vs replayed from a CUDA graph", "workload": wl.name,
+                      "psi": psi, "steps": K, "steps_per_graph": G, "plain_ms_per_step": plain_ms,
+                      "graph_ms_per_step": graph_ms, "plain_params_per_s": psi / (plain_ms / 1e3),
+                      "graph_params_per_s": psi / (graph_ms / 1e3),
+                      "note": "scalars of every step in a device table filled before timing"}), flush=True)
+
+
 def run_zero3_passes(a, wl):
     """ZeRO-3's gather passes over the Llama-shaped list: each layer's parameters are
     gathered (zero_gather_unit) into one of n_slots unit-sized buffers and the layer's
@@ -958,6 +1034,8 @@ def main():
         run_reference(a, wl)
     elif a.overlap:
         run_overlap(a, wl)
+    elif a.graph:
+        run_graph(a, wl)
     elif a.zero3_passes:
         run_zero3_passes(a, wl)
     else:

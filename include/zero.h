@@ -111,6 +111,15 @@ typedef struct {
     int64_t skipped;        /* state: steps skipped for overflow */
 } zero_loss_scaler;
 
+/* The fp32 scalars of one AdamW step as the kernels read them (the update formula of
+ * zero_adamw_shard_step): 1/(N L), 1 - lr wd, beta1, 1 - beta1, beta2, 1 - beta2,
+ * lr / (1 - beta1^t), sqrt(1 - beta2^t), eps; each evaluated in double and rounded once
+ * to fp32.  zero_step_scalars_fill computes them; zero_step_device_scalars reads them from
+ * device memory. */
+typedef struct {
+    float inv_scale, decay, beta1, omb1, beta2, omb2, step_size, sqrt_bc2, eps;
+} zero_step_scalars;
+
 /* Optional CUDA events (cudaEvent_t, created by the caller; any may be NULL) that
  * zero_step records on `stream` around its kernels, for per-kernel timing. */
 typedef struct {
@@ -214,6 +223,28 @@ zero_status zero_step(const zero_layout *layout, const uint16_t *grads, int64_t 
                       float *master, float *m, float *v, uint16_t *p16_shard, uint16_t *p16_full,
                       const zero_adamw_hparams *hp, int32_t *nonfinite,
                       const zero_step_events *events, void *stream);
+
+/* The scalars of step hp->step for this layout's rank count (host only, no CUDA call);
+ * hp as for zero_step. */
+zero_status zero_step_scalars_fill(const zero_layout *layout, const zero_adamw_hparams *hp,
+                                   zero_step_scalars *out);
+
+/* zero_step with the step's scalars read from device memory when the kernels run, instead
+ * of passed at launch: scalars_dev points to a zero_step_scalars in device memory (4-byte
+ * aligned), typically filled by zero_step_scalars_fill and a copy.  Nothing in the launch
+ * then depends on the step number or the hyper-parameters, so the call can be captured
+ * once in a CUDA graph and the graph replayed every step, the caller updating
+ * *scalars_dev before each replay (for instance with a captured cudaMemcpyAsync from a
+ * page-locked host copy it rewrites with zero_step_scalars_fill once the previous replay
+ * has finished).  For small models, whose step is a few tens of microseconds, that
+ * removes the per-step launch work.  Make one ordinary call (or zero_step) on the layout
+ * before capturing, so that the kernels are loaded.  Same results as zero_step with
+ * the same scalars; the same kernels, the same automatic implementation choice.  The
+ * pages have no counterpart. */
+zero_status zero_step_device_scalars(const zero_layout *layout, const uint16_t *grads, int64_t rank_stride,
+                                     float *master, float *m, float *v, uint16_t *p16_shard,
+                                     uint16_t *p16_full, const zero_step_scalars *scalars_dev,
+                                     int32_t *nonfinite, void *stream);
 
 /* One bucket's share of zero_step: the fused reduce-scatter + update of bucket `bucket`
  * only, so that it can start as soon as that bucket's gradients exist (P1 DDP: the first

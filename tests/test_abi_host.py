@@ -188,3 +188,15 @@ def test_scaler_advance_follows_the_oracle_scaler():
         zs.LossScaler(0.0).advance(True)                    # scale must be > 0
     with pytest.raises(zs.ZeroError):
         zs.LossScaler(8.0, factor=1.0).advance(False)       # factor must be > 1
+
+
+def test_step_scalars_fill_equals_the_oracle_scalars():
+    """zero_step_scalars_fill (the library's host computation of a step's nine fp32
+    scalars, the values zero_step_device_scalars reads) against the oracle's, bit for bit."""
+    for wl in reduced_workloads().values():
+        lay = zs.Layout(list(wl.tensors), wl.n_ranks, wl.stage, wl.bucket_elems, wl.pad_align, list(wl.units))
+        for t in (1, 2, 7, 1000):
+            got = zs.step_scalars(lay, zs.AdamW(wl.lr, wl.beta1, wl.beta2, wl.eps, wl.weight_decay, wl.loss_scale, t))
+            want = oracle.adamw_scalars(wl.n_ranks, oracle.Hyper(wl.lr, wl.beta1, wl.beta2, wl.eps, wl.weight_decay,
+                                                                   wl.loss_scale), t)
+            assert got.view(np.uint32).tolist() == want.view(np.uint32).tolist(), (wl.name, t)

@@ -16,7 +16,7 @@ import numpy as np
 from . import _abi
 
 __all__ = ["ZeroError", "Layout", "AdamW", "reduce_scatter", "adamw_shard_step", "allgather", "gather_unit", "gather_unit_ranks",
-           "step", "step_bucket", "step_overlapped", "step_dynamic", "step_dynamic_commit", "LossScaler", "step_host",
+           "step", "step_scalars", "step_device_scalars", "step_bucket", "step_overlapped", "step_dynamic", "step_dynamic_commit", "LossScaler", "step_host",
            "step_noalloc", "step_ranks", "step_shard", "step_shard_commit", "copy_shard", "ipc_handle", "ipc_open", "ipc_close",
            "get_error", "IMPL_AUTO", "IMPL_REGISTER", "IMPL_BULK"]
 
@@ -207,6 +207,26 @@ def step(layout, grads, master, m, v, p16_shard, p16_full, hp, nonfinite=None, e
                                 _ptr(m), _ptr(v), _ptr(p16_shard), _ptr(p16_full), ctypes.byref(h),
                                 _ptr(nonfinite), ctypes.byref(ev) if ev is not None else None,
                                 _stream(stream)), "zero_step")
+
+
+def step_scalars(layout, hp):
+    """The fp32 scalars of step hp.step (zero_step_scalars_fill) as a float32 numpy array
+    of 9, in the order zero_step_device_scalars reads them."""
+    out = _abi.StepScalars()
+    h = hp.c()
+    _check(_abi.lib().zero_step_scalars_fill(layout.handle, ctypes.byref(h), ctypes.byref(out)),
+           "zero_step_scalars_fill")
+    return np.array([getattr(out, f) for f, _ in _abi.StepScalars._fields_], dtype=np.float32)
+
+
+def step_device_scalars(layout, grads, master, m, v, p16_shard, p16_full, scalars_dev, nonfinite=None,
+                        rank_stride=None, stream=None):
+    """zero_step reading its scalars from scalars_dev (a float32 device tensor of 9) when it
+    runs (zero_step_device_scalars): capturable once in a CUDA graph and replayed."""
+    _check(_abi.lib().zero_step_device_scalars(layout.handle, _ptr(grads), _stride(grads, layout, rank_stride),
+                                               _ptr(master), _ptr(m), _ptr(v), _ptr(p16_shard), _ptr(p16_full),
+                                               _ptr(scalars_dev), _ptr(nonfinite), _stream(stream)),
+           "zero_step_device_scalars")
 
 
 def step_bucket(layout, bucket, grads, master, m, v, p16_shard, p16_full, hp, nonfinite=None, rank_stride=None,

@@ -45,6 +45,11 @@ class LossScaler(ctypes.Structure):
                 ("min_scale", ctypes.c_double), ("clean_steps", _i64), ("step", _i64), ("skipped", _i64)]
 
 
+class StepScalars(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_float) for n in ("inv_scale", "decay", "beta1", "omb1", "beta2", "omb2",
+                                              "step_size", "sqrt_bc2", "eps")]
+
+
 class StepEvents(ctypes.Structure):
     _fields_ = [("update_begin", _vp), ("update_end", _vp), ("gather_begin", _vp), ("gather_end", _vp)]
 
@@ -64,6 +69,8 @@ SIGNATURES = {
     "zero_gather_unit": (_i32, [_vp, _i64, _vp, _vp, _vp]),
     "zero_step": (_i32, [_vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(AdamWHparams), _vp,
                          ctypes.POINTER(StepEvents), _vp]),
+    "zero_step_scalars_fill": (_i32, [_vp, ctypes.POINTER(AdamWHparams), ctypes.POINTER(StepScalars)]),
+    "zero_step_device_scalars": (_i32, [_vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "zero_step_bucket": (_i32, [_vp, _i64, _vp, _i64, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(AdamWHparams),
                                 _vp, _vp]),
     "zero_step_overlapped": (_i32, [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(AdamWHparams),

@@ -353,13 +353,15 @@ zero::GradSource strided(const zero_layout *L, const uint16_t *grads, int64_t st
 
 // The fused reduce-scatter + update over the tiles of `w`, in the selected implementation.
 cudaError_t fused(const zero_layout *L, const TileWork &w, const uint16_t *grads, int64_t stride, float *master,
-                  float *m, float *v, uint16_t *p16, const AdamScalars &c, int32_t *nonfinite, cudaStream_t st)
+                  float *m, float *v, uint16_t *p16, const AdamScalars &c, int32_t *nonfinite, cudaStream_t st,
+                  const AdamScalars *c_dev = nullptr)
 {
     const bool bulk = zero::use_bulk(*L);
     if (bulk)
         return zero::launch_bulk_step(*L, w, strided(L, grads, stride), master, m, v, 0, p16, 0, c, nonfinite,
-                                      L->dev.wait_limit_ns, L->dev.skip_first_fill, st);
-    return zero::launch_fused_step(*L, w, grads, stride, master, m, v, p16, c, nonfinite, st);
+                                      L->dev.wait_limit_ns, L->dev.skip_first_fill, st, nullptr, nullptr, nullptr,
+                                      c_dev);
+    return zero::launch_fused_step(*L, w, grads, stride, master, m, v, p16, c, nonfinite, st, c_dev);
 }
 
 }  // namespace
@@ -383,6 +385,39 @@ extern "C" zero_status zero_step(const zero_layout *L, const uint16_t *grads, in
         e = zero::launch_copy_range(*L, 0, L->padded, p16_shard, p16_full, st);
         if (ev) record(ev->gather_end, st);
     }
+    return cuda_status(e);
+}
+
+extern "C" zero_status zero_step_scalars_fill(const zero_layout *L, const zero_adamw_hparams *hp,
+                                              zero_step_scalars *out)
+{
+    ZERO_RANGE("zero_step_scalars_fill");
+    if (!L || !out) return ZERO_ERR_INVALID;
+    zero_status s = check_hparams(hp);
+    if (s != ZERO_OK) return s;
+    const AdamScalars c = step_scalars(L->n_ranks, *hp);
+    memcpy(out, &c, sizeof c);
+    return ZERO_OK;
+}
+
+extern "C" zero_status zero_step_device_scalars(const zero_layout *L, const uint16_t *grads, int64_t rank_stride,
+                                                float *master, float *m, float *v, uint16_t *p16_shard,
+                                                uint16_t *p16_full, const zero_step_scalars *scalars_dev,
+                                                int32_t *nonfinite, void *stream)
+{
+    ZERO_RANGE("zero_step_device_scalars");
+    // the hyper-parameter checks of zero_step apply to whoever filled *scalars_dev
+    zero_adamw_hparams any = {1e-3, 0.9, 0.999, 1e-8, 0.0, 1.0, 1};
+    zero_status s = check_step(L, grads, rank_stride, master, m, v, p16_shard, p16_full, &any);
+    if (s != ZERO_OK || L->padded == 0) return s;
+    if (!scalars_dev) return ZERO_ERR_INVALID;
+    if (((uintptr_t)scalars_dev & 3u) != 0) return ZERO_ERR_ALIGN;
+    cudaStream_t st = (cudaStream_t)stream;
+    const AdamScalars *c_dev = reinterpret_cast<const AdamScalars *>(scalars_dev);
+    uint16_t *p16 = L->stage == 3 ? p16_shard : p16_full;
+    cudaError_t e = fused(L, all_tiles(L), grads, rank_stride, master, m, v, p16, AdamScalars{}, nonfinite, st,
+                          c_dev);
+    if (e == cudaSuccess && L->stage == 3) e = zero::launch_copy_range(*L, 0, L->padded, p16_shard, p16_full, st);
     return cuda_status(e);
 }
 

@@ -131,6 +131,7 @@ struct BulkArgs {
     uint16_t *p16;                // element i at [i - p16_off]
     int64_t p16_off;
     AdamScalars c;
+    const AdamScalars *c_dev;    // non-null: the step's scalars are read from here at run time
     int32_t *nonfinite;
     int32_t *error;
     uint64_t wait_limit_ns;
@@ -259,6 +260,7 @@ __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(co
     const int grp = (warp - 1) / kConsumerWarps;  // consumer group: takes the chunks of stage grp
     if (grp >= groups) return;
     const int ct = threadIdx.x - 32 - grp * 32 * kConsumerWarps;   // 0 .. 32 * kConsumerWarps - 1
+    const AdamScalars c = A.c_dev ? *A.c_dev : A.c;
     int64_t s = A.w.seg_first;
     uint32_t it = 0;
     for (int64_t t = A.w.tile_first + blockIdx.x; t < t_end; t += gridDim.x) {
@@ -290,7 +292,7 @@ __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(co
                 uint32_t h[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) bad += !isfinite(acc[e]);
-                adamw8(acc, A.c, pf, mf, vf, h);
+                adamw8(acc, c, pf, mf, vf, h);
                 const int64_t q = q0 + e0;
                 float4 *pp = reinterpret_cast<float4 *>(A.master + (q - A.state_off));
                 float4 *mp = reinterpret_cast<float4 *>(A.mom1 + (q - A.state_off));
@@ -324,7 +326,7 @@ __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(co
             const int64_t si = i - A.state_off;
             float p = A.master_in[si], m = A.mom1_in[si], v = A.mom2_in[si];
             uint32_t h;
-            adamw_elem(acc, A.c, p, m, v, h);
+            adamw_elem(acc, c, p, m, v, h);
             A.master[si] = p;
             A.mom1[si] = m;
             A.mom2[si] = v;
@@ -388,7 +390,7 @@ cudaError_t launch_bulk_step(const zero_layout &L, const TileWork &w, const Grad
                              float *m, float *v, int64_t state_off, uint16_t *p16, int64_t p16_off,
                              const AdamScalars &c, int32_t *nonfinite, uint64_t wait_limit_ns,
                              int skip_first_fill, cudaStream_t st, const float *master_in,
-                             const float *m_in, const float *v_in)
+                             const float *m_in, const float *v_in, const AdamScalars *c_dev)
 {
     if (w.n_tiles <= 0) return cudaSuccess;
     if ((state_off & 7) != 0 || (p16_off & 7) != 0) return cudaErrorMisalignedAddress;
@@ -405,6 +407,7 @@ cudaError_t launch_bulk_step(const zero_layout &L, const TileWork &w, const Grad
     a.p16 = p16;
     a.p16_off = p16_off;
     a.c = c;
+    a.c_dev = c_dev;
     a.nonfinite = nonfinite;
     a.error = L.dev.error;
     a.wait_limit_ns = wait_limit_ns;

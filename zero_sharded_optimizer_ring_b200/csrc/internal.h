@@ -43,7 +43,8 @@ struct GradSource {
     const uint16_t *rank[kMaxBulkRanks];
 };
 
-// fp32 scalars of one AdamW step, each computed on the host in double and rounded once.
+// fp32 scalars of one AdamW step, each computed on the host in double and rounded once
+// (the layout of zero_step_scalars in zero.h, which the library copies it to and from).
 struct AdamScalars {
     float inv_scale;   // 1 / (N * loss_scale)
     float decay;       // 1 - lr * weight_decay
@@ -53,6 +54,7 @@ struct AdamScalars {
     float sqrt_bc2;    // sqrt(1 - beta2^t)
     float eps;
 };
+static_assert(sizeof(AdamScalars) == sizeof(zero_step_scalars), "same layout as zero_step_scalars");
 
 // What a debug build (ZERO_DEBUG) checks every located tile against; filled by the
 // launch wrappers, read by no release kernel.  A tile that fails the check is skipped and
@@ -149,9 +151,11 @@ cudaError_t launch_copy_range(const zero_layout &L, int64_t lo, int64_t hi, cons
                               uint16_t *dst, cudaStream_t s);
 cudaError_t launch_gather_unit(const uint16_t *src, int64_t lo, int64_t n, uint16_t *dst, int32_t max_ctas,
                                cudaStream_t s);
+// c_dev non-null: the scalars are read from device memory when the kernel runs (c unused)
 cudaError_t launch_fused_step(const zero_layout &L, const TileWork &w, const uint16_t *grads,
                               int64_t stride, float *master, float *m, float *v, uint16_t *p16,
-                              const AdamScalars &c, int32_t *nonfinite, cudaStream_t s);
+                              const AdamScalars &c, int32_t *nonfinite, cudaStream_t s,
+                              const AdamScalars *c_dev = nullptr);
 // The same update out of place (register streaming, any N): state read from *_in,
 // written to master / m / v (buffers that do not overlap the in set).
 cudaError_t launch_fused_step_to(const zero_layout &L, const TileWork &w, const uint16_t *grads,
@@ -169,6 +173,7 @@ cudaError_t launch_bulk_step(const zero_layout &L, const TileWork &w, const Grad
                              float *m, float *v, int64_t state_off, uint16_t *p16, int64_t p16_off,
                              const AdamScalars &c, int32_t *nonfinite, uint64_t wait_limit_ns,
                              int skip_first_fill, cudaStream_t st, const float *master_in = nullptr,
-                             const float *m_in = nullptr, const float *v_in = nullptr);
+                             const float *m_in = nullptr, const float *v_in = nullptr,
+                             const AdamScalars *c_dev = nullptr);
 
 }  // namespace zero

@@ -57,9 +57,10 @@ template <int NT, int U, bool kFused, bool kWire, bool kOut = false>
 __global__ void __launch_bounds__(kThreads)
 tile_kernel(TileWork w, int n_ranks, const uint16_t *__restrict__ grads, int64_t stride,
             float *__restrict__ reduced, float *__restrict__ master, float *__restrict__ mom1,
-            float *__restrict__ mom2, uint16_t *__restrict__ p16, AdamScalars c,
-            int32_t *__restrict__ nonfinite, StateIn in)
+            float *__restrict__ mom2, uint16_t *__restrict__ p16, AdamScalars c_arg,
+            int32_t *__restrict__ nonfinite, StateIn in, const AdamScalars *__restrict__ c_dev)
 {
+    const AdamScalars c = c_dev ? *c_dev : c_arg;     // run-time scalars when given (graph replays)
     const float *__restrict__ master_in = kOut ? in.master : master;
     const float *__restrict__ mom1_in = kOut ? in.mom1 : mom1;
     const float *__restrict__ mom2_in = kOut ? in.mom2 : mom2;
@@ -440,23 +441,24 @@ int grid_for(K kernel, int64_t work_items, int num_sms, int max_ctas = 0)
 template <int NT, int U, bool kFused>
 cudaError_t launch_tiles(const zero_layout &L, const TileWork &w, const uint16_t *grads, int64_t stride,
                          float *reduced, float *master, float *m, float *v, uint16_t *p16,
-                         const AdamScalars &c, int32_t *nonfinite, cudaStream_t st)
+                         const AdamScalars &c, int32_t *nonfinite, cudaStream_t st, const AdamScalars *c_dev)
 {
     auto kern = L.wire16 ? tile_kernel<NT, U, kFused, true> : tile_kernel<NT, U, kFused, false>;
     const int grid = grid_for(kern, w.n_tiles, L.dev.num_sms, w.max_ctas > 0 ? w.max_ctas : L.max_ctas);
     kern<<<grid, kThreads, 0, st>>>(w, L.n_ranks, grads, stride, reduced, master, m, v, p16, c, nonfinite,
-                                    StateIn{nullptr, nullptr, nullptr});
+                                    StateIn{nullptr, nullptr, nullptr}, c_dev);
     return cudaGetLastError();
 }
 
 template <bool kFused>
 cudaError_t dispatch_tiles(const zero_layout &L, const TileWork &w, const uint16_t *grads, int64_t stride,
                            float *reduced, float *master, float *m, float *v, uint16_t *p16,
-                           const AdamScalars &c, int32_t *nonfinite, cudaStream_t st)
+                           const AdamScalars &c, int32_t *nonfinite, cudaStream_t st,
+                           const AdamScalars *c_dev = nullptr)
 {
     if (w.n_tiles <= 0) return cudaSuccess;
 #define ZERO_CASE(NV, UV) \
-    case NV: return launch_tiles<NV, UV, kFused>(L, w, grads, stride, reduced, master, m, v, p16, c, nonfinite, st);
+    case NV: return launch_tiles<NV, UV, kFused>(L, w, grads, stride, reduced, master, m, v, p16, c, nonfinite, st, c_dev);
     switch (L.n_ranks) {
         ZERO_CASE(1, 2)
         ZERO_CASE(2, 2)
@@ -468,7 +470,8 @@ cudaError_t dispatch_tiles(const zero_layout &L, const TileWork &w, const uint16
         ZERO_CASE(8, 1)
         ZERO_CASE(16, 1)
         default:
-            return launch_tiles<0, 1, kFused>(L, w, grads, stride, reduced, master, m, v, p16, c, nonfinite, st);
+            return launch_tiles<0, 1, kFused>(L, w, grads, stride, reduced, master, m, v, p16, c, nonfinite, st,
+                                              c_dev);
     }
 #undef ZERO_CASE
 }
@@ -523,9 +526,9 @@ cudaError_t launch_reduce_scatter(const zero_layout &L, const TileWork &w, const
 
 cudaError_t launch_fused_step(const zero_layout &L, const TileWork &w, const uint16_t *grads,
                               int64_t stride, float *master, float *m, float *v, uint16_t *p16,
-                              const AdamScalars &c, int32_t *nonfinite, cudaStream_t s)
+                              const AdamScalars &c, int32_t *nonfinite, cudaStream_t s, const AdamScalars *c_dev)
 {
-    return dispatch_tiles<true>(L, w, grads, stride, nullptr, master, m, v, p16, c, nonfinite, s);
+    return dispatch_tiles<true>(L, w, grads, stride, nullptr, master, m, v, p16, c, nonfinite, s, c_dev);
 }
 
 cudaError_t launch_fused_step_to(const zero_layout &L, const TileWork &w, const uint16_t *grads,
@@ -537,7 +540,7 @@ cudaError_t launch_fused_step_to(const zero_layout &L, const TileWork &w, const 
     auto kern = L.wire16 ? tile_kernel<0, 1, true, true, true> : tile_kernel<0, 1, true, false, true>;
     const int grid = grid_for(kern, w.n_tiles, L.dev.num_sms, w.max_ctas > 0 ? w.max_ctas : L.max_ctas);
     kern<<<grid, kThreads, 0, s>>>(w, L.n_ranks, grads, stride, nullptr, master, m, v, p16, c, nonfinite,
-                                   StateIn{master_in, m_in, v_in});
+                                   StateIn{master_in, m_in, v_in}, nullptr);
     return cudaGetLastError();
 }
 
