@@ -1,7 +1,8 @@
 /* A plain C99 user of the library on the GPU, with no Python and no PyTorch: the CUDA
  * runtime allocates the buffers, the library runs three fused steps of a small ZeRO-2
- * layout, and the program writes its inputs and outputs to a file for the test to check
- * against the oracle.  Usage: abi_device_check <output file>. */
+ * layout (the first with zero_step, the others with zero_step_device_scalars), and the
+ * program writes its inputs and outputs to a file for the test to check against the
+ * oracle.  Usage: abi_device_check <output file>. */
 #include <stdio.h>
 #include <stdlib.h>
 #include <string.h>
@@ -55,11 +56,23 @@ int main(int argc, char **argv)
     CHECK(cudaMemset(dv, 0, (size_t)P * 4) == cudaSuccess);
     CHECK(cudaMemset(dp16, 0, (size_t)P * 2) == cudaSuccess);
 
+    /* step 1 with its scalars passed at launch (zero_step); steps 2 and 3 with the scalars
+     * filled on the host and read from device memory (zero_step_device_scalars) */
+    zero_step_scalars *dsc;
+    CHECK(cudaMalloc((void **)&dsc, sizeof(zero_step_scalars)) == cudaSuccess);
     for (int64_t t = 1; t <= 3; ++t) {
         zero_adamw_hparams hp = {1e-3, 0.9, 0.999, 1e-8, 0.01, 1024.0, t};
-        CHECK(zero_step(L, dg, P, dmaster, dm, dv, NULL, dp16, &hp, NULL, NULL, NULL) == ZERO_OK);
+        if (t == 1) {
+            CHECK(zero_step(L, dg, P, dmaster, dm, dv, NULL, dp16, &hp, NULL, NULL, NULL) == ZERO_OK);
+        } else {
+            zero_step_scalars sc;
+            CHECK(zero_step_scalars_fill(L, &hp, &sc) == ZERO_OK);
+            CHECK(cudaMemcpy(dsc, &sc, sizeof sc, cudaMemcpyHostToDevice) == cudaSuccess);
+            CHECK(zero_step_device_scalars(L, dg, P, dmaster, dm, dv, NULL, dp16, dsc, NULL, NULL) == ZERO_OK);
+        }
     }
     CHECK(zero_get_error(L, NULL) == ZERO_OK);
+    cudaFree(dsc);
 
     float *out_master = malloc((size_t)P * 4), *out_m = malloc((size_t)P * 4), *out_v = malloc((size_t)P * 4);
     CHECK(out_master && out_m && out_v);
