@@ -761,6 +761,7 @@ def _overlap_reps(a, wl, lay, g, master, m, v, p16_shard, p16_full, backward, pr
         "max_ctas": cap if cap else "auto (measured by the library)",
         "bucket_group": group if group else "auto (zero_step_overlapped: launches of >= 2^24 elements)",
         "t_back_to_back_ms": tq, "t_backward_plus_step_alone_ms": tb + ts,
+        "chosen_plan": dict(zip(("plan", "mean_ms_per_plan"), lay.overlap_plan())),
         "pipelined_every_call_ms": res["pipe_all"],
         "buckets": lay.n_buckets,
         "reps": reps, "t_backward_ms": tb, "t_step_ms": ts, "t_pipelined_ms": tp, "exposed_step_ms": tp - tb,
@@ -944,6 +945,11 @@ def run_zero3_passes(a, wl):
     set_carveout = torch._C._set_sm_carveout_experimental
     passes = (("forward", fwd, order_f), ("backward", bwd, order_b))
     res = {"gathers_only_ms": timed(gathers_only)}
+    for gcap in (8, 16, 32):                       # the 28 gathers alone on a capped grid
+        lay.set_gather_ctas(gcap)
+        res[f"gathers_only_{gcap}ctas_ms"] = timed(gathers_only)
+        res[f"gathers_only_{gcap}ctas_gbs"] = 4 * P / (res[f"gathers_only_{gcap}ctas_ms"] / 1e3) / 1e9
+    lay.set_gather_ctas(0)
     for name, work, order in passes:
         res[f"{name}_compute_only_ms"] = timed(compute_only(work))
         for n in (1, 2, 3):

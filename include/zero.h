@@ -285,6 +285,13 @@ zero_status zero_step_overlapped(const zero_layout *layout, void *const *ready_e
                                  float *v, uint16_t *p16_shard, uint16_t *p16_full,
                                  const zero_adamw_hparams *hp, int32_t *nonfinite, void *stream);
 
+/* The launch plan the overlapped steps settled on for this layout: -1 while the plans
+ * are still being timed (or when zero_set_max_ctas fixed a cap), 0..3 = the update
+ * following the backward with its grid capped at 1, 2/3, 1/2, 1/3 of the SMs, 4 = the
+ * update deferred to one launch after the last bucket.  *mean_ms (optional, [5]) receives
+ * each plan's mean timed call so far (0 where none).  Host only. */
+zero_status zero_overlap_plan(const zero_layout *layout, int32_t *plan, float *mean_ms);
+
 /* zero_step_overlapped with one launch per `group` consecutive buckets (group >= 1; the
  * last group may be shorter; no other coalescing): `stream` waits for the ready events
  * of all the group's buckets, then runs their fused update as one kernel.  With many

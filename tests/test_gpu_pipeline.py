@@ -113,6 +113,9 @@ def test_overlapped_grid_tuner_keeps_results(key):
         torch.cuda.synchronize()                  # the tuner reads the call's events next time
     zs.get_error(lay)
     _check(wl, lay, b, ref)
+    plan, means = lay.overlap_plan()
+    assert 0 <= plan <= 4 and all(x > 0 for x in means)      # every plan timed, one kept
+    assert means[plan] == min(means)
 
 
 def test_overlapped_rejects_unrecorded_events():

@@ -87,6 +87,25 @@ def test_capped_allgather_matches_oracle(aligned, gather_ctas):
     assert (S.to_np(full)[lay.padded:] == 7).all()
 
 
+@pytest.mark.parametrize("gather_ctas", [1, 7])
+def test_capped_gather_of_a_large_unit_matches_oracle(gather_ctas):
+    """One 3,000,017-element unit (ZeRO-3 over the flat list): 123 bulk-copy chunks, many
+    per CTA, so every stage of each CTA's shared-memory ring is reloaded many times."""
+    wl = reduced_workloads()["flat1p3b_n4_zero1"].with_(stage=3, steps=2)
+    lay, shard, ref = _stepped_shards(wl)
+    lay.set_gather_ctas(gather_ctas)
+    dst = torch.full((lay.padded + 24,), 7, dtype=torch.int16, device="cuda")
+    zs.gather_unit(lay, 0, shard, dst)
+    full = torch.full((lay.padded + 24,), 7, dtype=torch.int16, device="cuda")
+    zs.allgather(lay, 0, shard, full[:lay.padded])
+    zs.get_error(lay)
+    torch.cuda.synchronize()
+    for name, buf in (("gather_unit", dst), ("allgather", full)):
+        got = S.to_np(buf)
+        S.assert_bits_equal(got[:lay.padded], ref.p16_full, name)
+        assert (got[lay.padded:] == 7).all(), f"{name}: write past the unit"
+
+
 @pytest.mark.parametrize("gather_ctas", [0, None])
 @pytest.mark.parametrize("n_slots", [1, 2, 3])
 @pytest.mark.parametrize("backward", [False, True])

@@ -145,6 +145,15 @@ class Layout:
     def gather_ctas(self):
         return getattr(self, "_gather_ctas", 0)
 
+    def overlap_plan(self):
+        """(plan, mean ms per plan) the overlapped steps settled on (zero_overlap_plan):
+        plan -1 while still timing, 0-3 = grid capped at 1, 2/3, 1/2, 1/3 of the SMs,
+        4 = deferred to one launch after the last bucket."""
+        plan = ctypes.c_int32()
+        means = np.zeros(5, np.float32)
+        _check(_abi.lib().zero_overlap_plan(self._h, ctypes.byref(plan), means.ctypes.data), "zero_overlap_plan")
+        return int(plan.value), [float(x) for x in means]
+
     def debug_set_wait(self, wait_limit_ns, skip_first_fill=0):
         _check(_abi.lib().zero_debug_set_wait(self._h, int(wait_limit_ns), int(skip_first_fill)),
                "zero_debug_set_wait")

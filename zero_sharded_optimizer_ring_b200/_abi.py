@@ -75,6 +75,7 @@ SIGNATURES = {
                                 _vp, _vp]),
     "zero_step_overlapped": (_i32, [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(AdamWHparams),
                                     _vp, _vp]),
+    "zero_overlap_plan": (_i32, [_vp, ctypes.POINTER(_i32), _vp]),
     "zero_step_overlapped_grouped": (_i32, [_vp, _vp, _i64, _vp, _i64, _vp, _vp, _vp, _vp, _vp,
                                             ctypes.POINTER(AdamWHparams), _vp, _vp]),
     "zero_step_dynamic": (_i32, [_vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(AdamWHparams),

@@ -298,6 +298,7 @@ extern "C" zero_status zero_gather_unit(const zero_layout *L, int64_t unit, cons
     if (!aligned16(p16_shard) || !aligned16(dst)) return ZERO_ERR_ALIGN;
     const int64_t lo = L->unit_lo[(size_t)unit];
     return cuda_status(zero::launch_gather_unit(p16_shard, lo, L->unit_hi[(size_t)unit] - lo, dst, L->gather_ctas,
+                                                L->dev.error, L->dev.wait_limit_ns,
                                                 (cudaStream_t)stream));
 }
 
@@ -555,6 +556,18 @@ zero_status check_overlapped(const zero_layout *L, void *const *ready_events, co
 }
 
 }  // namespace
+
+extern "C" zero_status zero_overlap_plan(const zero_layout *L, int32_t *plan, float *mean_ms)
+{
+    ZERO_RANGE("zero_overlap_plan");
+    if (!L || !plan) return ZERO_ERR_INVALID;
+    const zero::OverlapTuner &T = L->dev.tuner;
+    *plan = L->max_ctas > 0 ? -1 : T.chosen;
+    if (mean_ms)
+        for (int i = 0; i < zero::OverlapTuner::kCands; ++i)
+            mean_ms[i] = T.trials[i] > 0 ? T.sum_ms[i] / (float)T.trials[i] : 0.f;
+    return ZERO_OK;
+}
 
 extern "C" zero_status zero_step_overlapped_grouped(const zero_layout *L, void *const *ready_events, int64_t group,
                                                     const uint16_t *grads, int64_t rank_stride, float *master, float *m,

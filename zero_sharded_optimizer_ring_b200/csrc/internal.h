@@ -149,8 +149,10 @@ cudaError_t launch_adamw_range(const zero_layout &L, int64_t lo, int64_t hi, con
                                const AdamScalars &c, cudaStream_t s);
 cudaError_t launch_copy_range(const zero_layout &L, int64_t lo, int64_t hi, const uint16_t *src,
                               uint16_t *dst, cudaStream_t s);
+// max_ctas > 0 (and lo a multiple of 8): the capped bulk copy, whose bounded waits report
+// to `error` (may be null)
 cudaError_t launch_gather_unit(const uint16_t *src, int64_t lo, int64_t n, uint16_t *dst, int32_t max_ctas,
-                               cudaStream_t s);
+                               int32_t *error, uint64_t limit_ns, cudaStream_t s);
 // c_dev non-null: the scalars are read from device memory when the kernel runs (c unused)
 cudaError_t launch_fused_step(const zero_layout &L, const TileWork &w, const uint16_t *grads,
                               int64_t stride, float *master, float *m, float *v, uint16_t *p16,

@@ -17,6 +17,7 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include "bulk_ptx.cuh"
 #include "device_common.cuh"
 #include "gather_ranks.h"
 
@@ -267,48 +268,87 @@ copy_range_kernel(int64_t lo, int64_t hi, const uint16_t *__restrict__ src, uint
     }
 }
 
-// Copy on a capped grid of persistent CTAs: d[j] = s[j] for j < n (s and d 16-byte
-// aligned), plus hn < 8 head elements hd[j] = hs[j].  Each thread keeps kCapUnroll 16-byte
-// vectors in flight, so one CTA of 1024 threads has 128 KB of loads outstanding: enough to
-// draw a large share of HBM bandwidth from a few SMs while the rest of the GPU computes
-// (the gathers of a ZeRO-3 forward pass beside its GEMMs).
-constexpr int kCapThreads = 1024;
-constexpr int kCapUnroll = 8;
+// Copy on a capped grid of persistent CTAs, through shared memory with bulk copies:
+// d[j] = s[j] for j < n (s and d 16-byte aligned), plus hn < 8 head elements hd[j] = hs[j].
+// One thread per CTA drives a ring of kBulkCopyStages stages of kBulkCopyChunk elements:
+// cp.async.bulk loads (global -> shared, completion on the stage's mbarrier) run
+// kBulkCopyStages - 1 chunks ahead of cp.async.bulk stores (shared -> global); a stage is
+// reloaded only once its store has read it.  With ~144 KB of loads in flight per SM, a
+// few SMs draw a large share of HBM bandwidth while the rest of the GPU computes (the
+// gathers of a ZeRO-3 pass beside the layer GEMMs).  The vector body's last < 8 elements
+// and the head go through other lanes of CTA 0.  Every wait is bounded: on expiry the
+// kernel records ZERO_ERR_TIMEOUT, waits (bounded) for the loads it issued, and returns.
+constexpr int kBulkCopyStages = 4;
+constexpr int64_t kBulkCopyChunk = 24576;                                   // 48 KB
+constexpr size_t kBulkCopySmem = 128 + (size_t)kBulkCopyStages * kBulkCopyChunk * 2;
 
-__global__ void __launch_bounds__(kCapThreads)
-copy_capped_kernel(const uint16_t *__restrict__ s, uint16_t *__restrict__ d, int64_t n,
-                   const uint16_t *__restrict__ hs, uint16_t *__restrict__ hd, int hn)
+__global__ void __launch_bounds__(32, 1)
+copy_bulk_kernel(const uint16_t *__restrict__ s, uint16_t *__restrict__ d, int64_t n,
+                 const uint16_t *__restrict__ hs, uint16_t *__restrict__ hd, int hn, int32_t *error,
+                 uint64_t limit_ns)
 {
-    const int64_t nv = n / kVec;
-    const int64_t step = (int64_t)gridDim.x * kCapThreads * kCapUnroll;
-    for (int64_t base = (int64_t)blockIdx.x * kCapThreads * kCapUnroll; base < nv; base += step) {
-        uint4 x[kCapUnroll];
-#pragma unroll
-        for (int u = 0; u < kCapUnroll; ++u) {
-            const int64_t q = base + (int64_t)u * kCapThreads + threadIdx.x;
-            if (q < nv) x[u] = __ldcs(reinterpret_cast<const uint4 *>(s + q * kVec));
-        }
-#pragma unroll
-        for (int u = 0; u < kCapUnroll; ++u) {
-            const int64_t q = base + (int64_t)u * kCapThreads + threadIdx.x;
-            if (q < nv) __stcs(reinterpret_cast<uint4 *>(d + q * kVec), x[u]);
-        }
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem);
+    unsigned char *ring = smem + 128;
+    const int64_t nv = n / kVec * kVec;                   // the bulk-copied body
+    if (blockIdx.x == 0 && threadIdx.x >= 1) {            // head and tail, element by element
+        const int l = threadIdx.x - 1;
+        if (l < hn) hd[l] = hs[l];
+        if (l < n - nv) d[nv + l] = s[nv + l];
     }
-    if (blockIdx.x == 0) {
-        if (threadIdx.x < n - nv * kVec) d[nv * kVec + threadIdx.x] = s[nv * kVec + threadIdx.x];
-        if (threadIdx.x < hn) hd[threadIdx.x] = hs[threadIdx.x];
+    if (threadIdx.x != 0) return;
+    for (int i = 0; i < kBulkCopyStages; ++i) mbar_init(smem_addr(&full[i]), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+
+    const int64_t n_chunks = (nv + kBulkCopyChunk - 1) / kBulkCopyChunk;
+    const int64_t K = (int64_t)blockIdx.x < n_chunks ? (n_chunks - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    int64_t issued = 0;
+    auto chunk_of = [&](int64_t k) { return (int64_t)blockIdx.x + k * (int64_t)gridDim.x; };
+    auto bytes_of = [&](int64_t c) {
+        const int64_t e = nv - c * kBulkCopyChunk;
+        return (uint32_t)((e < kBulkCopyChunk ? e : kBulkCopyChunk) * 2);
+    };
+    auto issue = [&](int64_t k) {
+        const int st = (int)(k % kBulkCopyStages);
+        const int64_t c = chunk_of(k);
+        const uint32_t bar = smem_addr(&full[st]);
+        mbar_arrive_expect_tx(bar, bytes_of(c));
+        bulk_load(smem_addr(ring + (size_t)st * kBulkCopyChunk * 2), s + c * kBulkCopyChunk, bytes_of(c), bar);
+        issued = k + 1;
+    };
+    for (int64_t k = 0; k < K && k < kBulkCopyStages - 1; ++k) issue(k);
+    int64_t k = 0;
+    for (; k < K; ++k) {
+        const int64_t j = k + kBulkCopyStages - 1;       // the chunk that refills stage (k - 1) % S
+        if (j < K) {
+            if (k >= 1) bulk_wait_read_all();            // the store of chunk k - 1 has read it
+            issue(j);
+        }
+        const int st = (int)(k % kBulkCopyStages);
+        if (!mbar_wait_bounded(smem_addr(&full[st]), (uint32_t)((k / kBulkCopyStages) & 1), limit_ns)) {
+            if (error) atomicExch(error, (int32_t)ZERO_ERR_TIMEOUT);
+            break;
+        }
+        bulk_store(d + chunk_of(k) * kBulkCopyChunk, smem_addr(ring + (size_t)st * kBulkCopyChunk * 2),
+                   bytes_of(chunk_of(k)));
+        bulk_commit_group();
     }
+    for (int64_t i = k + 1; i < issued; ++i)             // after a timeout: loads still in flight
+        mbar_wait_bounded(smem_addr(&full[i % kBulkCopyStages]), (uint32_t)((i / kBulkCopyStages) & 1), limit_ns);
+    bulk_wait_all();                                      // every store complete before the CTA leaves
 }
 
 cudaError_t launch_copy_capped(const uint16_t *s, uint16_t *d, int64_t n, const uint16_t *hs, uint16_t *hd, int hn,
-                               int32_t max_ctas, cudaStream_t st)
+                               int32_t max_ctas, int32_t *error, uint64_t limit_ns, cudaStream_t st)
 {
     if (n <= 0 && hn <= 0) return cudaSuccess;
-    const int64_t per_cta = (int64_t)kCapThreads * kCapUnroll * kVec;
-    int64_t grid = (n + per_cta - 1) / per_cta;
-    if (grid > max_ctas) grid = max_ctas;
+    const int64_t n_chunks = (n / kVec * kVec + kBulkCopyChunk - 1) / kBulkCopyChunk;
+    int64_t grid = n_chunks < max_ctas ? n_chunks : max_ctas;
     if (grid < 1) grid = 1;
-    copy_capped_kernel<<<(unsigned)grid, kCapThreads, 0, st>>>(s, d, n > 0 ? n : 0, hs, hd, hn);
+    cudaError_t e = cudaFuncSetAttribute(copy_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kBulkCopySmem);
+    if (e != cudaSuccess) return e;
+    copy_bulk_kernel<<<(unsigned)grid, 32, kBulkCopySmem, st>>>(s, d, n > 0 ? n : 0, hs, hd, hn, error, limit_ns);
     return cudaGetLastError();
 }
 
@@ -493,10 +533,11 @@ TileBounds tile_bounds(const zero_layout &L, int64_t state_lo, int64_t state_hi)
 }
 
 cudaError_t launch_gather_unit(const uint16_t *src, int64_t lo, int64_t n, uint16_t *dst, int32_t max_ctas,
-                               cudaStream_t s)
+                               int32_t *error, uint64_t limit_ns, cudaStream_t s)
 {
     if (n <= 0) return cudaSuccess;
-    if (max_ctas > 0 && (lo & 7) == 0) return launch_copy_capped(src + lo, dst, n, nullptr, nullptr, 0, max_ctas, s);
+    if (max_ctas > 0 && (lo & 7) == 0)
+        return launch_copy_capped(src + lo, dst, n, nullptr, nullptr, 0, max_ctas, error, limit_ns, s);
     const int64_t per_block = (int64_t)kThreads * kCopyUnroll * kVec;
     gather_unit_kernel<<<(unsigned)((n + per_block - 1) / per_block), kThreads, 0, s>>>(src, lo, n, dst);
     return cudaGetLastError();
@@ -567,7 +608,7 @@ cudaError_t launch_copy_range(const zero_layout &L, int64_t lo, int64_t hi, cons
         // head [lo, min(va, hi)) by one block's scalar pass, then [va, hi) vectorised
         const int64_t head_end = va < hi ? va : hi;
         return launch_copy_capped(src + head_end, dst + head_end, hi - head_end, src + lo, dst + lo,
-                                  (int)(head_end - lo), L.gather_ctas, s);
+                                  (int)(head_end - lo), L.gather_ctas, L.dev.error, L.dev.wait_limit_ns, s);
     }
     const int64_t blocks = vb > va ? (vb - va + per_block - 1) / per_block : 1;
     copy_range_kernel<<<(unsigned)blocks, kThreads, 0, s>>>(lo, hi, src, dst);
