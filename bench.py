@@ -37,9 +37,9 @@ PROFILE_DIR = os.path.join(ROOT, "profiles")
 # sources is stale
 _CSRC = os.path.join(ROOT, "zero_sharded_optimizer_ring_b200", "csrc")
 KERNEL_SOURCES = {tag: [os.path.join(_CSRC, f) for f in files] for tag, files in {
-    "bulk_step": ("bulk_step.cu", "device_common.cuh", "internal.h"),
-    "tile_kernel": ("kernels.cu", "device_common.cuh", "internal.h"),
-    "copy_range": ("kernels.cu", "device_common.cuh", "internal.h"),
+    "bulk_step": ("bulk_step.cu", "bulk_ptx.cuh", "device_common.cuh", "internal.h"),
+    "tile_kernel": ("kernels.cu", "bulk_ptx.cuh", "device_common.cuh", "internal.h"),
+    "copy_range": ("kernels.cu", "bulk_ptx.cuh", "device_common.cuh", "internal.h"),
 }.items()}
 
 
