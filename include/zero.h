@@ -475,9 +475,10 @@ zero_status zero_set_max_ctas(zero_layout *layout, int32_t max_ctas);
 
 /* Grid of the all-gather copies (zero_allgather, zero_gather_unit, and the gather inside
  * the stage-3 steps): 0 (the default) = a grid of short blocks over the whole range, the
- * fastest when a gather has the GPU to itself; k > 0 = k persistent CTAs of 1024 threads,
- * each with 128 KB of loads in flight, so that a gather occupies at most k SMs and can run
- * beside a layer's compute that leaves those SMs free (P1 ZeRO-3: the next layer's
+ * fastest when a gather has the GPU to itself; k > 0 = k persistent CTAs, each moving
+ * 48 KB chunks global -> shared -> global with bulk copies (~144 KB of loads in flight;
+ * bounded waits report ZERO_ERR_TIMEOUT through zero_get_error), so that a gather
+ * occupies at most k SMs and can run beside a layer's compute that leaves those SMs free (P1 ZeRO-3: the next layer's
  * parameters are gathered while the current layer computes).  Results are identical for
  * every k.  Negative k: ZERO_ERR_INVALID.  No counterpart on the pages. */
 zero_status zero_set_gather_ctas(zero_layout *layout, int32_t max_ctas);
