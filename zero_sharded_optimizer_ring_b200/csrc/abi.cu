@@ -324,6 +324,20 @@ extern "C" zero_status zero_gather_unit_ranks(const zero_layout *L, int64_t unit
 
 namespace {
 
+// The buffers of a whole-layout step (hyper-parameters checked separately).
+zero_status check_step_buffers(const zero_layout *L, const uint16_t *grads, int64_t rank_stride, float *master,
+                               float *m, float *v, uint16_t *p16_shard, uint16_t *p16_full)
+{
+    zero_status s = check_device(L);
+    if (s != ZERO_OK) return s;
+    if (L->padded == 0) return ZERO_OK;
+    if ((s = check_grads(L, grads, rank_stride)) != ZERO_OK) return s;
+    if ((s = check_state(master, m, v)) != ZERO_OK) return s;
+    if (!p16_full || (L->stage == 3 && !p16_shard)) return ZERO_ERR_INVALID;
+    if (!aligned16(p16_full) || (p16_shard && !aligned16(p16_shard))) return ZERO_ERR_ALIGN;
+    return ZERO_OK;
+}
+
 zero_status check_step(const zero_layout *L, const uint16_t *grads, int64_t rank_stride, float *master,
                        float *m, float *v, uint16_t *p16_shard, uint16_t *p16_full,
                        const zero_adamw_hparams *hp)
@@ -331,12 +345,7 @@ zero_status check_step(const zero_layout *L, const uint16_t *grads, int64_t rank
     zero_status s = check_device(L);
     if (s != ZERO_OK) return s;
     if ((s = check_hparams(hp)) != ZERO_OK) return s;
-    if (L->padded == 0) return ZERO_OK;
-    if ((s = check_grads(L, grads, rank_stride)) != ZERO_OK) return s;
-    if ((s = check_state(master, m, v)) != ZERO_OK) return s;
-    if (!p16_full || (L->stage == 3 && !p16_shard)) return ZERO_ERR_INVALID;
-    if (!aligned16(p16_full) || (p16_shard && !aligned16(p16_shard))) return ZERO_ERR_ALIGN;
-    return ZERO_OK;
+    return check_step_buffers(L, grads, rank_stride, master, m, v, p16_shard, p16_full);
 }
 
 void record(void *ev, cudaStream_t st)
@@ -407,9 +416,8 @@ extern "C" zero_status zero_step_device_scalars(const zero_layout *L, const uint
                                                 int32_t *nonfinite, void *stream)
 {
     ZERO_RANGE("zero_step_device_scalars");
-    // the hyper-parameter checks of zero_step apply to whoever filled *scalars_dev
-    zero_adamw_hparams any = {1e-3, 0.9, 0.999, 1e-8, 0.0, 1.0, 1};
-    zero_status s = check_step(L, grads, rank_stride, master, m, v, p16_shard, p16_full, &any);
+    // the hyper-parameter rules of zero_step apply to whoever filled *scalars_dev
+    zero_status s = check_step_buffers(L, grads, rank_stride, master, m, v, p16_shard, p16_full);
     if (s != ZERO_OK || L->padded == 0) return s;
     if (!scalars_dev) return ZERO_ERR_INVALID;
     if (((uintptr_t)scalars_dev & 3u) != 0) return ZERO_ERR_ALIGN;
