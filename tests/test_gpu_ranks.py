@@ -7,10 +7,11 @@
 - zero_gather_unit_ranks, reading each rank's own shard buffer as the CUDA step wrote
   it, gives the oracle's gathered layer (vector and element paths, units across shard
   edges, 16 ranks);
-- two processes sharing this GPU, each holding one rank's gradients and one shard's
-  state, run the multi-GPU step (CUDA IPC mappings, host barriers over gloo; no kernel
-  waits on the other process) and end bit-identical to the oracle; for ZeRO-3 each keeps
-  only its parameter shard and gathers every layer from both owners.
+- two or three processes sharing this GPU, each holding one rank's gradients and one
+  shard's state, run the multi-GPU step (CUDA IPC mappings of buffers and phase events,
+  host barriers over gloo; no kernel waits on another process) and end bit-identical to
+  the oracle; for ZeRO-3 each keeps only its parameter shard and gathers every layer
+  from all owners.
 """
 import datetime
 import os
@@ -198,22 +199,26 @@ def _ipc_worker(rank, world, port, wl, steps, out):
     dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("stage", [1, 2, 3])
-def test_two_process_step_over_ipc_matches_oracle(stage):
-    wl = Workload(name="ipc", description="ipc", tensors=(100_003, 77_777, 122_227), units=(0, 1, 2), n_ranks=2,
-                  stage=stage, bucket_elems=50_001, steps=3, loss_scale=1024.0, m_sigma=1e-4, v_sigma=1e-6,
-                  pad_align=8)
+@pytest.mark.parametrize("stage,world", [(1, 2), (2, 2), (3, 2), (1, 3), (3, 3)])
+def test_process_per_rank_step_over_ipc_matches_oracle(stage, world):
+    """One process per rank, all on this GPU: each holds one rank's gradients and one
+    shard's state, maps the others' buffers and phase events over CUDA IPC, and steps
+    through the fenced phases (no kernel waits on another process).  Every process ends
+    with the oracle's shard state and fp16 parameters."""
+    wl = Workload(name="ipc", description="ipc", tensors=(100_003, 77_777, 122_227), units=(0, 1, 2),
+                  n_ranks=world, stage=stage, bucket_elems=50_001, steps=3, loss_scale=1024.0, m_sigma=1e-4,
+                  v_sigma=1e-6, pad_align=8)
     olay = S.oracle_layout(wl)
     g, master, m, v = S.host_inputs(wl, olay.padded)
     ref = oracle.run_steps(olay, stage, g, master, m, v, S.hyper(wl), wl.steps)
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_ipc_worker, args=(r, 2, port, wl, wl.steps, q)) for r in range(2)]
+    procs = [ctx.Process(target=_ipc_worker, args=(r, world, port, wl, wl.steps, q)) for r in range(world)]
     for p in procs:
         p.start()
     try:
-        res = sorted([q.get(timeout=300) for _ in range(2)], key=lambda x: x[0])
+        res = sorted([q.get(timeout=300) for _ in range(world)], key=lambda x: x[0])
     finally:
         for p in procs:
             p.join(60)
