@@ -62,6 +62,8 @@ def parse():
     ap.add_argument("--dynamic-commit", action="store_true",
                     help="time zero_step_dynamic_commit (one fused pass into a second state set, overflow "
                          "check, swap) instead of the fused step")
+    ap.add_argument("--unfused", action="store_true",
+                    help="time the standalone reduce-scatter, shard update and all-gather calls (its own JSON line)")
     ap.add_argument("--graph", action="store_true",
                     help="time steps launched one by one against the same steps replayed from CUDA graphs "
                          "(zero_step_device_scalars; its own JSON line)")
@@ -844,6 +846,62 @@ def run_graph(a, wl):
                       "note": "scalars of every step in a device table filled before timing"}), flush=True)
 
 
+def run_unfused(a, wl):
+    """The three standalone boundary calls of one step, each timed with CUDA events:
+    zero_reduce_scatter of every bucket (2N + 4 bytes per parameter: fp16 grads in, fp32
+    sums out), zero_adamw_shard_step of every shard (4 + 24 + 2: sums, state, fp16
+    parameters) and zero_allgather of every unit (2 + 2).  The fused step moves 2N + 26."""
+    import torch
+    import seeded_inputs as si
+    import zero_sharded_optimizer_ring_b200 as zs
+
+    torch.cuda.set_device(dist_env()[1])
+    lay = zs.Layout(list(wl.tensors), wl.n_ranks, wl.stage, wl.bucket_elems, wl.pad_align, list(wl.units))
+    lay.to_device()
+    if a.kernel:
+        lay.set_impl(a.kernel)
+    P, psi, N = lay.padded, lay.psi, wl.n_ranks
+    g = torch.empty((N, P), dtype=torch.int16, device="cuda")
+    si.fill_grads_cuda(g, psi, wl.seed, wl.grad_sigma, wl.loss_scale, wl.heavy_frac, wl.heavy_mult)
+    master = torch.empty(P, dtype=torch.float32, device="cuda")
+    si.fill_f32_cuda(master, psi, wl.seed, si.STREAM_MASTER, wl.master_sigma)
+    m = torch.zeros(P, dtype=torch.float32, device="cuda")
+    v = torch.zeros(P, dtype=torch.float32, device="cuda")
+    if wl.m_sigma:
+        si.fill_f32_cuda(m, psi, wl.seed, si.STREAM_M, wl.m_sigma)
+    if wl.v_sigma:
+        si.fill_f32_cuda(v, psi, wl.seed, si.STREAM_V, wl.v_sigma, absval=True)
+    red = torch.empty(P, dtype=torch.float32, device="cuda")
+    p16 = torch.zeros(P, dtype=torch.int16, device="cuda")
+    p16_full = torch.zeros(P, dtype=torch.int16, device="cuda")
+    hp = lambda t: zs.AdamW(wl.lr, wl.beta1, wl.beta2, wl.eps, wl.weight_decay, wl.loss_scale, t)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    times = {"reduce_scatter": [], "adamw": [], "allgather": []}
+    for t in range(1, a.warmup + a.steps + 1):
+        e = [ev() for _ in range(4)]
+        e[0].record()
+        zs.reduce_scatter(lay, -1, g, red)
+        e[1].record()
+        zs.adamw_shard_step(lay, -1, red, master, m, v, p16, hp(t))
+        e[2].record()
+        zs.allgather(lay, -1, p16, p16_full)
+        e[3].record()
+        if t > a.warmup:
+            torch.cuda.synchronize()
+            for k, (i, j) in zip(times, ((0, 1), (1, 2), (2, 3))):
+                times[k].append(e[i].elapsed_time(e[j]))
+    zs.get_error(lay)
+    peak, peak_kind = hbm_peak()
+    out = {"metric": "standalone boundary calls of one step", "workload": wl.name, "steps": a.steps,
+           "peak": peak, "peak_kind": peak_kind}
+    for k, per_param in (("reduce_scatter", 2 * N + 4), ("adamw", 4 + 24 + 2), ("allgather", 4)):
+        ms = statistics.median(times[k])
+        gbs = per_param * P / (ms / 1e3) / 1e9
+        out[k] = {"ms": ms, "bytes_per_param": per_param, "achieved_gbs": gbs, "frac": gbs / peak}
+    out["unfused_step_ms"] = sum(out[k]["ms"] for k in times)
+    print(json.dumps(out), flush=True)
+
+
 def run_zero3_passes(a, wl):
     """ZeRO-3's gather passes over the Llama-shaped list: each layer's parameters are
     gathered (zero_gather_unit) into one of n_slots unit-sized buffers and the layer's
@@ -1042,6 +1100,8 @@ def main():
         run_overlap(a, wl)
     elif a.graph:
         run_graph(a, wl)
+    elif a.unfused:
+        run_unfused(a, wl)
     elif a.zero3_passes:
         run_zero3_passes(a, wl)
     else:
