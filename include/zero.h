@@ -452,7 +452,8 @@ zero_status zero_ipc_get_handle(const void *dev_ptr, void *handle_out, int64_t *
 zero_status zero_ipc_open(const void *handle, int64_t offset, void **dev_ptr_out);
 zero_status zero_ipc_close(void *dev_ptr, int64_t offset);
 
-/* Select the fused kernel's implementation: 0 = automatic (the bulk-copy pipeline for
+/* Select the implementation of the fused step and of zero_reduce_scatter (and the
+ * reduce pass of zero_step_dynamic): 0 = automatic (the bulk-copy pipeline for
  * N <= 16, where it has an instance per rank count; register streaming above, where it
  * runs at the copy bandwidth), 1 = register streaming (vectorised 16-byte loads held in
  * registers; any N), 2 = bulk-copy pipeline (cp.async.bulk into a shared-memory ring,

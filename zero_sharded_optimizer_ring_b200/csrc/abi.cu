@@ -32,6 +32,9 @@ zero_status check_device(const zero_layout *L)
 
 zero_status cuda_status(cudaError_t e) { return e == cudaSuccess ? ZERO_OK : ZERO_ERR_CUDA; }
 
+cudaError_t reduce(const zero_layout *L, const TileWork &w, const uint16_t *grads, int64_t stride, float *reduced,
+                   int32_t *nonfinite, cudaStream_t st);   // defined with the step launchers below
+
 TileWork all_tiles(const zero_layout *L)
 {
     TileWork w;
@@ -250,7 +253,7 @@ extern "C" zero_status zero_reduce_scatter(const zero_layout *L, int64_t bucket,
     if (!reduced) return ZERO_ERR_INVALID;
     if (!aligned16(reduced)) return ZERO_ERR_ALIGN;
     const TileWork w = bucket < 0 ? all_tiles(L) : bucket_tiles(L, bucket);
-    return cuda_status(zero::launch_reduce_scatter(*L, w, grads, rank_stride, reduced, nonfinite,
+    return cuda_status(reduce(L, w, grads, rank_stride, reduced, nonfinite,
                                                    (cudaStream_t)stream));
 }
 
@@ -359,6 +362,17 @@ zero::GradSource strided(const zero_layout *L, const uint16_t *grads, int64_t st
     zero::GradSource src = {};
     for (int r = 0; r < L->n_ranks && r < zero::kMaxBulkRanks; ++r) src.rank[r] = grads + (int64_t)r * stride;
     return src;
+}
+
+// The reduce-scatter alone over the tiles of `w`, in the implementation the fused step
+// would use (results identical).
+cudaError_t reduce(const zero_layout *L, const TileWork &w, const uint16_t *grads, int64_t stride, float *reduced,
+                   int32_t *nonfinite, cudaStream_t st)
+{
+    if (zero::use_bulk(*L))
+        return zero::launch_bulk_reduce(*L, w, strided(L, grads, stride), reduced, nonfinite, L->dev.wait_limit_ns,
+                                        st);
+    return zero::launch_reduce_scatter(*L, w, grads, stride, reduced, nonfinite, st);
 }
 
 // The fused reduce-scatter + update over the tiles of `w`, in the selected implementation.
@@ -684,7 +698,7 @@ extern "C" zero_status zero_step_dynamic(const zero_layout *L, const uint16_t *g
     const size_t nb = L->bucket_lo.size();
     int64_t bad = 0;
     cudaError_t e = cudaMemsetAsync(nonfinite, 0, nb * sizeof(int32_t), st);
-    if (e == cudaSuccess) e = zero::launch_reduce_scatter(*L, all_tiles(L), grads, rank_stride, reduced, nonfinite, st);
+    if (e == cudaSuccess) e = reduce(L, all_tiles(L), grads, rank_stride, reduced, nonfinite, st);
     if (e == cudaSuccess) e = total_nonfinite(L, nonfinite, st, &bad);
     if (e != cudaSuccess) return ZERO_ERR_CUDA;
     if (bad == 0) {

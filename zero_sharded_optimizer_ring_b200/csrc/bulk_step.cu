@@ -46,7 +46,6 @@ struct BulkShape {
     static constexpr int kConsumerWarps = N <= 4 ? 16 : 8;
     static constexpr int kThreads = 32 * (1 + kConsumerWarps);
     static constexpr int kMaxStages = 3;
-    static constexpr uint32_t kStageBytes = (uint32_t)kChunk * (2 * N + 12);
 };
 
 template <>
@@ -86,6 +85,7 @@ struct BulkArgs {
     int64_t p16_off;
     AdamScalars c;
     const AdamScalars *c_dev;    // non-null: the step's scalars are read from here at run time
+    float *reduced;              // reduce-only instances: fp32 sums, element i at [i]
     int32_t *nonfinite;
     int32_t *error;
     uint64_t wait_limit_ns;
@@ -125,7 +125,9 @@ __device__ __forceinline__ void fold8(const unsigned char *base, int64_t e0, int
     }
 }
 
-template <int N, bool kWire>
+// kReduce: the reduce-scatter alone (zero_reduce_scatter): only the N gradient slices are
+// staged, and the consumers store the fp32 sums instead of updating the state.
+template <int N, bool kWire, bool kReduce>
 __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(const __grid_constant__ BulkArgs A)
 {
     constexpr int kConsumerWarps = BulkShape<N>::kConsumerWarps;
@@ -138,7 +140,8 @@ __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(co
         kChunk = A.chunk;
         n_r = A.n_ranks;
     }
-    const uint32_t kStageBytes = (uint32_t)kChunk * (2u * (uint32_t)n_r + 12u);
+    const uint32_t kElemBytes = 2u * (uint32_t)n_r + (kReduce ? 0u : 12u);   // staged bytes per element
+    const uint32_t kStageBytes = (uint32_t)kChunk * kElemBytes;
     const int groups = N > 0 ? 1 : A.stages;      // consumer groups (see BulkShape<0>)
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem);
@@ -179,7 +182,7 @@ __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(co
                 const uint32_t n = (uint32_t)((vb - q0) < kChunk ? (vb - q0) : kChunk);
                 const uint32_t bar = smem_addr(&full[st]);
                 unsigned char *base = ring + (size_t)st * kStageBytes;
-                mbar_arrive_expect_tx(bar, n * (2u * (uint32_t)n_r + 12u));
+                mbar_arrive_expect_tx(bar, n * kElemBytes);
                 if constexpr (N > 0) {
 #pragma unroll
                     for (int j = 0; j < N; ++j)
@@ -190,10 +193,12 @@ __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(co
                         bulk_load(smem_addr(base + (size_t)j * kChunk * 2),
                                   A.src.rank[ring_rank(tr.shard, j, n_r)] + q0, n * 2u, bar);
                 }
-                unsigned char *st_base = base + (size_t)n_r * kChunk * 2;
-                bulk_load(smem_addr(st_base), A.master_in + (q0 - A.state_off), n * 4u, bar);
-                bulk_load(smem_addr(st_base + kChunk * 4), A.mom1_in + (q0 - A.state_off), n * 4u, bar);
-                bulk_load(smem_addr(st_base + kChunk * 8), A.mom2_in + (q0 - A.state_off), n * 4u, bar);
+                if constexpr (!kReduce) {
+                    unsigned char *st_base = base + (size_t)n_r * kChunk * 2;
+                    bulk_load(smem_addr(st_base), A.master_in + (q0 - A.state_off), n * 4u, bar);
+                    bulk_load(smem_addr(st_base + kChunk * 4), A.mom1_in + (q0 - A.state_off), n * 4u, bar);
+                    bulk_load(smem_addr(st_base + kChunk * 8), A.mom2_in + (q0 - A.state_off), n * 4u, bar);
+                }
                 posted = it + 1;
             }
         }
@@ -214,7 +219,7 @@ __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(co
     const int grp = (warp - 1) / kConsumerWarps;  // consumer group: takes the chunks of stage grp
     if (grp >= groups) return;
     const int ct = threadIdx.x - 32 - grp * 32 * kConsumerWarps;   // 0 .. 32 * kConsumerWarps - 1
-    const AdamScalars c = A.c_dev ? *A.c_dev : A.c;
+    const AdamScalars c = (!kReduce && A.c_dev) ? *A.c_dev : A.c;
     int64_t s = A.w.seg_first;
     uint32_t it = 0;
     for (int64_t t = A.w.tile_first + blockIdx.x; t < t_end; t += gridDim.x) {
@@ -234,6 +239,14 @@ __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(co
                 const int64_t e0 = vi * kVec;
                 float acc[8];
                 fold8<N, kWire>(base, e0, n_r, kChunk, acc);
+                if constexpr (kReduce) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) bad += !isfinite(acc[e]);
+                    float4 *rp = reinterpret_cast<float4 *>(A.reduced + (q0 + e0));
+                    __stcs(rp, make_float4(acc[0], acc[1], acc[2], acc[3]));
+                    __stcs(rp + 1, make_float4(acc[4], acc[5], acc[6], acc[7]));
+                    continue;
+                }
                 const float *sp = reinterpret_cast<const float *>(base + (size_t)n_r * kChunk * 2);
                 float4 p4[2] = {*reinterpret_cast<const float4 *>(sp + e0), *reinterpret_cast<const float4 *>(sp + e0 + 4)};
                 float4 m4[2] = {*reinterpret_cast<const float4 *>(sp + kChunk + e0),
@@ -277,6 +290,9 @@ __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(co
                 for (int j = 1; j < n_r; ++j) acc = __fadd_rn(acc, h2f(A.src.rank[ring_rank(tr.shard, j, n_r)][i]));
             }
             bad += !isfinite(acc);
+            if constexpr (kReduce) {
+                A.reduced[i] = acc;
+            } else {
             const int64_t si = i - A.state_off;
             float p = A.master_in[si], m = A.mom1_in[si], v = A.mom2_in[si];
             uint32_t h;
@@ -285,6 +301,7 @@ __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(co
             A.mom1[si] = m;
             A.mom2[si] = v;
             A.p16[i - A.p16_off] = (uint16_t)h;
+            }
         }
         if (A.nonfinite) {
             if (__any_sync(0xffffffffu, bad != 0)) {
@@ -295,25 +312,33 @@ __global__ void __launch_bounds__(BulkShape<N>::kThreads, 1) bulk_step_kernel(co
     }
 }
 
-template <int N>
+template <int N, bool kReduce>
 cudaError_t launch_bulk_n(const zero_layout &L, BulkArgs &a, cudaStream_t st)
 {
     const size_t budget = L.dev.smem_optin > 0 ? L.dev.smem_optin : 227 * 1024;
+    const size_t per_elem = 2 * (size_t)L.n_ranks + (kReduce ? 0 : 12);
     size_t stage_bytes;
     if constexpr (N > 0) {
-        stage_bytes = BulkShape<N>::kStageBytes;
+        stage_bytes = (size_t)BulkShape<N>::kChunk * per_elem;
     } else {
-        const size_t per_elem = 2 * (size_t)L.n_ranks + 12;
         a.n_ranks = L.n_ranks;
         a.chunk = 2 * 1024 * per_elem + 256 <= budget ? 1024 : 512;
         stage_bytes = (size_t)a.chunk * per_elem;
     }
     int stages = (int)((budget - 256) / stage_bytes);
-    if (stages > BulkShape<N>::kMaxStages) stages = BulkShape<N>::kMaxStages;
+    int max_stages = BulkShape<N>::kMaxStages;
+    if (kReduce && N > 0) {
+        // the smaller reduce-only stages: as many as keep about 170 KB in flight per SM
+        // (the sweep's sweet spot for the fused step), at most 5
+        const int by_flight = (int)((170 * 1024) / stage_bytes);
+        max_stages = by_flight < 5 ? by_flight : 5;
+        if (max_stages < 2) max_stages = 2;
+    }
+    if (stages > max_stages) stages = max_stages;
     if (stages < 2) return cudaErrorInvalidConfiguration;
     a.stages = stages;
     const size_t smem = ((16 * (size_t)stages + 4 + 127) / 128) * 128 + (size_t)stages * stage_bytes;
-    auto kern = L.wire16 ? bulk_step_kernel<N, true> : bulk_step_kernel<N, false>;
+    auto kern = L.wire16 ? bulk_step_kernel<N, true, kReduce> : bulk_step_kernel<N, false, kReduce>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int64_t grid = L.dev.num_sms > 0 ? L.dev.num_sms : 148;
@@ -322,6 +347,32 @@ cudaError_t launch_bulk_n(const zero_layout &L, BulkArgs &a, cudaStream_t st)
     if (grid > a.w.n_tiles) grid = a.w.n_tiles;
     kern<<<(unsigned)grid, BulkShape<N>::kThreads, smem, st>>>(a);
     return cudaGetLastError();
+}
+
+template <bool kReduce>
+cudaError_t dispatch_bulk(const zero_layout &L, BulkArgs &a, cudaStream_t st)
+{
+    switch (L.n_ranks) {
+        case 1: return launch_bulk_n<1, kReduce>(L, a, st);
+        case 2: return launch_bulk_n<2, kReduce>(L, a, st);
+        case 3: return launch_bulk_n<3, kReduce>(L, a, st);
+        case 4: return launch_bulk_n<4, kReduce>(L, a, st);
+        case 5: return launch_bulk_n<5, kReduce>(L, a, st);
+        case 6: return launch_bulk_n<6, kReduce>(L, a, st);
+        case 7: return launch_bulk_n<7, kReduce>(L, a, st);
+        case 8: return launch_bulk_n<8, kReduce>(L, a, st);
+        case 9: return launch_bulk_n<9, kReduce>(L, a, st);
+        case 10: return launch_bulk_n<10, kReduce>(L, a, st);
+        case 11: return launch_bulk_n<11, kReduce>(L, a, st);
+        case 12: return launch_bulk_n<12, kReduce>(L, a, st);
+        case 13: return launch_bulk_n<13, kReduce>(L, a, st);
+        case 14: return launch_bulk_n<14, kReduce>(L, a, st);
+        case 15: return launch_bulk_n<15, kReduce>(L, a, st);
+        case 16: return launch_bulk_n<16, kReduce>(L, a, st);
+        default:
+            if (L.n_ranks > kMaxBulkRanks || L.n_ranks < 1) return cudaErrorInvalidValue;
+            return launch_bulk_n<0, kReduce>(L, a, st);
+    }
 }
 
 }  // namespace
@@ -369,27 +420,23 @@ cudaError_t launch_bulk_step(const zero_layout &L, const TileWork &w, const Grad
     a.skip_first_fill = skip_first_fill;
     a.n_ranks = L.n_ranks;
     a.chunk = 0;
-    switch (L.n_ranks) {
-        case 1: return launch_bulk_n<1>(L, a, st);
-        case 2: return launch_bulk_n<2>(L, a, st);
-        case 3: return launch_bulk_n<3>(L, a, st);
-        case 4: return launch_bulk_n<4>(L, a, st);
-        case 5: return launch_bulk_n<5>(L, a, st);
-        case 6: return launch_bulk_n<6>(L, a, st);
-        case 7: return launch_bulk_n<7>(L, a, st);
-        case 8: return launch_bulk_n<8>(L, a, st);
-        case 9: return launch_bulk_n<9>(L, a, st);
-        case 10: return launch_bulk_n<10>(L, a, st);
-        case 11: return launch_bulk_n<11>(L, a, st);
-        case 12: return launch_bulk_n<12>(L, a, st);
-        case 13: return launch_bulk_n<13>(L, a, st);
-        case 14: return launch_bulk_n<14>(L, a, st);
-        case 15: return launch_bulk_n<15>(L, a, st);
-        case 16: return launch_bulk_n<16>(L, a, st);
-        default:
-            if (L.n_ranks > kMaxBulkRanks || L.n_ranks < 1) return cudaErrorInvalidValue;
-            return launch_bulk_n<0>(L, a, st);
-    }
+    a.reduced = nullptr;
+    return dispatch_bulk<false>(L, a, st);
+}
+
+cudaError_t launch_bulk_reduce(const zero_layout &L, const TileWork &w, const GradSource &src, float *reduced,
+                               int32_t *nonfinite, uint64_t wait_limit_ns, cudaStream_t st)
+{
+    if (w.n_tiles <= 0) return cudaSuccess;
+    BulkArgs a = {};
+    a.w = w;
+    a.src = src;
+    a.reduced = reduced;
+    a.nonfinite = nonfinite;
+    a.error = L.dev.error;
+    a.wait_limit_ns = wait_limit_ns;
+    a.n_ranks = L.n_ranks;
+    return dispatch_bulk<true>(L, a, st);
 }
 
 }  // namespace zero

@@ -167,6 +167,10 @@ cudaError_t launch_fused_step_to(const zero_layout &L, const TileWork &w, const 
 
 // bulk_step.cu
 bool bulk_supported(int n_ranks);
+// The reduce-scatter alone through the bulk-copy pipeline: reduced[i] = the ring-order
+// fp32 sum of element i, for the tiles of `w` (rank r's gradient of i at src.rank[r][i]).
+cudaError_t launch_bulk_reduce(const zero_layout &L, const TileWork &w, const GradSource &src, float *reduced,
+                               int32_t *nonfinite, uint64_t wait_limit_ns, cudaStream_t st);
 bool use_bulk(const zero_layout &L);   // the fused step's implementation for a strided buffer
 // master / m / v hold flat elements [state_off, ...) and p16 [p16_off, ...): element i is
 // at index i - off (both offsets multiples of 8).  The state is read from master_in /
