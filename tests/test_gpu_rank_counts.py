@@ -84,6 +84,13 @@ def test_every_rank_count_both_kernels(N, wire):
                     nonfinite=b["nonfinite"])
         zs.get_error(lay)
         _check(wl, b, ref, lay.n_buckets)
+        # the reduce-scatter alone, in the same implementation (its reduce-only instances)
+        red = torch.zeros(lay.padded, dtype=torch.float32, device="cuda")
+        b["nonfinite"].zero_()
+        zs.reduce_scatter(lay, -1, g, red, nonfinite=b["nonfinite"])
+        zs.get_error(lay)
+        S.assert_bits_equal(_np(red), ref.reduced, f"reduced, impl {impl}", any_nan=True)
+        assert list(_np(b["nonfinite"])[:lay.n_buckets]) == list(ref.nonfinite)
 
 
 @pytest.mark.parametrize("N", list(range(1, 18)) + [24, 33, 51, 64])
