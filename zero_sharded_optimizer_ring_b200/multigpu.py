@@ -110,7 +110,9 @@ class RankStep:
     def __init__(self, layout, rank, world, grads, master_k, m_k, v_k, p16, group=None, ops=None, spare=None):
         """p16: the full fp16 parameters [P] (stages 0-2) or this rank's shard of them [S]
         (stage 3).  spare: (master_k, m_k, v_k, p16) of the same shapes, the second set
-        that step_dynamic() needs."""
+        that step_dynamic() needs.  group: the process group of the fences' host barriers;
+        a gloo group keeps them on the host (an NCCL group's barrier is itself a GPU
+        collective, queued behind this rank's work, so the GPU would drain at every phase)."""
         import torch.distributed as dist
         if layout.n_ranks != world:
             raise ValueError("the layout's rank count must equal the world size")
