@@ -13,7 +13,6 @@ import numpy as np
 import pytest
 
 import oracle
-import seeded_inputs as si
 from seeded_inputs.workloads import Workload, full_workloads, reduced_workloads
 import zero_sharded_optimizer_ring_b200 as zs
 import support as S
