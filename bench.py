@@ -73,8 +73,8 @@ def parse():
                          "against a simulated layer compute (its own JSON line)")
     ap.add_argument("--tokens", type=int, default=2048, help="--zero3-passes: tokens per rank")
     ap.add_argument("--zero3-configs", default="0:0:0,0:0:1,0:0:2,0:16:2,0:16:3",
-                    help="--zero3-passes sweep: comma-separated carveout:gather_ctas:slots (carveout = SMs the "
-                         "layer GEMMs leave free through cuBLAS's SM-count target; gather_ctas = "
+                    help="--zero3-passes sweep: comma-separated carveout:gather_ctas:slots (carveout = how far "
+                         "below the SM count the matmuls' cuBLAS SM-count target is set; gather_ctas = "
                          "zero_set_gather_ctas, 0 = default grid; slots 0 = the compute alone)")
     ap.add_argument("--zero3-rounds", type=int, default=5, help="--zero3-passes: interleaved rounds of the sweep")
     ap.add_argument("--blas", default="", help="--zero3-passes: torch preferred BLAS library (cublas, cublaslt)")
@@ -1018,9 +1018,10 @@ def run_zero3_passes(a, wl):
         for n in (1, 2):
             res[f"{name}_exposed_gather_{n}slot_ms"] = res[f"{name}_{n}slot_ms"] - res[f"{name}_compute_only_ms"]
 
-    # gathers on a capped grid beside GEMMs that leave SMs free: configurations
-    # "carveout:gather_ctas:slots" (carveout = SMs the matmuls leave free through cuBLAS's
-    # SM-count target; gather_ctas = zero_set_gather_ctas; slots 0 = compute alone), each
+    # gathers on a capped grid beside GEMMs run with a lowered SM-count target: configurations
+    # "carveout:gather_ctas:slots" (carveout = how far below the SM count the matmuls'
+    # cuBLAS SM-count target is set; gather_ctas = zero_set_gather_ctas; slots 0 = compute
+    # alone), each
     # measured once per round, rounds interleaved so that clock drift hits all alike;
     # reported: the median over rounds
     sweep = []

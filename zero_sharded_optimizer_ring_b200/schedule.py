@@ -14,18 +14,19 @@ from . import gather_unit
 
 # How the gathers share the GPU with the layers' GEMMs during a pass (measured on the
 # Llama-shaped list, 2048 tokens, two slots): the gathers run as 16 persistent CTAs
-# (zero_set_gather_ctas) instead of a grid that floods every SM between GEMM waves, and
-# the layer GEMMs leave 16 SMs to them (cuBLAS's SM-count target, honoured on the cuBLASLt
-# path): the compute alone is no slower with 132 SMs, and the gathers then run beside it
-# instead of in its waves' way.
+# (zero_set_gather_ctas) instead of a grid that floods every SM between GEMM waves, and the
+# matmuls run with cuBLAS's SM-count target 16 below the SM count on the cuBLASLt path
+# (torch's matmul carveout).  The target is a hint to the GEMM kernel choice rather than a
+# cap on the SMs a GEMM occupies; with it the layer GEMMs alone are no slower, and beside
+# the capped gathers both passes expose less gather time than without prefetch.
 GATHER_CTAS = 16
 MATMUL_SM_CARVEOUT = 16
 MATMUL_BLAS = "cublaslt"
 
 
 class _MatmulShare:
-    """Within the block, torch's matmuls leave `carveout` SMs free and prefer `blas`
-    (either None: unchanged); both restored on exit."""
+    """Within the block, torch's matmuls run with cuBLAS's SM-count target `carveout` SMs
+    below the SM count and prefer `blas` (either None: unchanged); both restored on exit."""
 
     def __init__(self, carveout, blas):
         self.carveout, self.blas = carveout, blas
@@ -57,8 +58,8 @@ def zero3_pass(layout, p16_shard, slots, units, compute, gather_stream, compute_
     previous occupant units[j - len(slots)] has been computed; compute(unit, buffer) is
     then called with compute_stream current and must enqueue the layer's work there.
     During the pass the gathers run on gather_ctas persistent CTAs (None: the layout's
-    setting) and torch's matmuls leave matmul_sm_carveout SMs free and prefer `blas`
-    (None: unchanged); every setting is restored afterwards.  Returns the list of (gather
+    setting) and torch's matmuls run with the SM-count target matmul_sm_carveout below the
+    SM count and prefer `blas` (None: unchanged); every setting is restored afterwards.  Returns the list of (gather
     started, gathered, computed) torch.cuda.Event triples, one per unit (timing events:
     layer_breakdown reads them)."""
     import torch
