@@ -45,7 +45,11 @@ struct BulkShape {
     static constexpr int kChunk = N <= 4 ? 4096 : 2048;        // elements per stage
     static constexpr int kConsumerWarps = N <= 4 ? 16 : 8;
     static constexpr int kThreads = 32 * (1 + kConsumerWarps);
-    static constexpr int kMaxStages = 3;
+    // stages in flight: two of the 4096-element chunks, three of the 2048-element ones (a
+    // sweep of 2 against 3 on flat lists of 2^28 parameters: the third 4096-element stage,
+    // 56-72 KB at 1-3 ranks, slows the step by 4-5 %; the third 2048-element stage at 8
+    // ranks speeds it up by 7 %)
+    static constexpr int kMaxStages = N <= 4 ? 2 : 3;
 };
 
 template <>
@@ -380,8 +384,9 @@ cudaError_t dispatch_bulk(const zero_layout &L, BulkArgs &a, cudaStream_t st)
 bool bulk_supported(int n_ranks) { return n_ranks >= 1 && n_ranks <= kMaxBulkRanks; }
 
 // The automatic choice (impl 0) for a strided gradient buffer, from B200 measurements of
-// both kernels: the pipeline where it has a compiled instance (N <= 16; ~12 % ahead of
-// register streaming on the flat N=4 list), register streaming above (0.99-1.01 of the
+// both kernels: the pipeline where it has a compiled instance (N <= 16; level with
+// register streaming at 1-4 ranks, 9 % ahead of it on the Llama-shaped list at 8 ranks and
+// 2 % on the ragged list at 16), register streaming above (0.99-1.01 of the
 // measured copy bandwidth at N = 24-64, where the runtime-N pipeline instance reaches
 // 0.48-0.87: its few consumer warps cannot fold that many ranks fast enough).
 bool use_bulk(const zero_layout &L)
