@@ -453,9 +453,10 @@ zero_status zero_ipc_open(const void *handle, int64_t offset, void **dev_ptr_out
 zero_status zero_ipc_close(void *dev_ptr, int64_t offset);
 
 /* Select the implementation of the fused step and of zero_reduce_scatter (and the
- * reduce pass of zero_step_dynamic): 0 = automatic (the bulk-copy pipeline for
- * N <= 16, where it has an instance per rank count; register streaming above, where it
- * runs at the copy bandwidth), 1 = register streaming (vectorised 16-byte loads held in
+ * reduce pass of zero_step_dynamic): 0 = automatic (for the fused step the bulk-copy
+ * pipeline for N <= 16, where it has an instance per rank count, register streaming
+ * above, where it runs at the copy bandwidth; for the reduce-scatter alone the pipeline
+ * for 5 <= N <= 16 and register streaming otherwise, as measured), 1 = register streaming (vectorised 16-byte loads held in
  * registers; any N), 2 = bulk-copy pipeline (cp.async.bulk into a shared-memory ring,
  * warp-specialised; one runtime-N instance serves 17 <= N <= 64; register streaming
  * above).  The per-rank-pointer calls (zero_step_ranks, zero_step_shard*) always use the

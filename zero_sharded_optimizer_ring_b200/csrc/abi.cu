@@ -364,12 +364,12 @@ zero::GradSource strided(const zero_layout *L, const uint16_t *grads, int64_t st
     return src;
 }
 
-// The reduce-scatter alone over the tiles of `w`, in the implementation the fused step
-// would use (results identical).
+// The reduce-scatter alone over the tiles of `w`, in the selected implementation (the
+// automatic choice measured for this pass; results identical either way).
 cudaError_t reduce(const zero_layout *L, const TileWork &w, const uint16_t *grads, int64_t stride, float *reduced,
                    int32_t *nonfinite, cudaStream_t st)
 {
-    if (zero::use_bulk(*L))
+    if (zero::use_bulk_reduce(*L))
         return zero::launch_bulk_reduce(*L, w, strided(L, grads, stride), reduced, nonfinite, L->dev.wait_limit_ns,
                                         st);
     return zero::launch_reduce_scatter(*L, w, grads, stride, reduced, nonfinite, st);

@@ -396,6 +396,18 @@ bool use_bulk(const zero_layout &L)
     return L.n_ranks >= 1 && L.n_ranks <= 16;
 }
 
+// The same for the reduce-scatter alone: the reduce-only pipeline for 5-16 ranks (6 % and
+// 10 % ahead of register streaming at 8 and 16), register streaming for 1-4 ranks (level
+// at 3, 3-12 % ahead at 1, 2 and 4, where the pipeline's 16 consumer warps have little
+// to fold per byte staged) and above 16 (0.97-1.00 of the copy bandwidth at 24-48 ranks,
+// the runtime-N pipeline instance 0.77-0.83).
+bool use_bulk_reduce(const zero_layout &L)
+{
+    if (L.impl == 1) return false;
+    if (L.impl == 2) return bulk_supported(L.n_ranks);
+    return L.n_ranks >= 5 && L.n_ranks <= 16;
+}
+
 cudaError_t launch_bulk_step(const zero_layout &L, const TileWork &w, const GradSource &src, float *master,
                              float *m, float *v, int64_t state_off, uint16_t *p16, int64_t p16_off,
                              const AdamScalars &c, int32_t *nonfinite, uint64_t wait_limit_ns,

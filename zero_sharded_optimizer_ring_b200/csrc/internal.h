@@ -171,7 +171,8 @@ bool bulk_supported(int n_ranks);
 // fp32 sum of element i, for the tiles of `w` (rank r's gradient of i at src.rank[r][i]).
 cudaError_t launch_bulk_reduce(const zero_layout &L, const TileWork &w, const GradSource &src, float *reduced,
                                int32_t *nonfinite, uint64_t wait_limit_ns, cudaStream_t st);
-bool use_bulk(const zero_layout &L);   // the fused step's implementation for a strided buffer
+bool use_bulk(const zero_layout &L);          // the fused step's implementation for a strided buffer
+bool use_bulk_reduce(const zero_layout &L);   // the same for the reduce-scatter alone
 // master / m / v hold flat elements [state_off, ...) and p16 [p16_off, ...): element i is
 // at index i - off (both offsets multiples of 8).  The state is read from master_in /
 // m_in / v_in where given (same indexing; a second buffer set), else from master / m / v.

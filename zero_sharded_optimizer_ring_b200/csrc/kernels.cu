@@ -500,12 +500,18 @@ cudaError_t dispatch_tiles(const zero_layout &L, const TileWork &w, const uint16
                            const AdamScalars *c_dev = nullptr)
 {
     if (w.n_tiles <= 0) return cudaSuccess;
-    // (ranks, vectors in flight per thread, CTAs per SM the registers are held to), from a
-    // sweep on flat lists of 2^28 parameters: for 1-4 ranks one vector per thread at two
-    // CTAs per SM beats two vectors per thread by 3-8 %; at 8 and 16 ranks the compiler's
-    // allocation is as fast or faster
+    // Shapes (vectors in flight per thread, CTAs per SM the registers are held to), from
+    // sweeps on flat lists of 2^28 parameters, one B200.  Fused: for 1-4 ranks one vector
+    // at two CTAs per SM beats two vectors per thread by 3-8 %; at 8 and 16 ranks one
+    // vector with the compiler's allocation is as fast or faster.  Reduce-only: one vector
+    // at two CTAs per SM is the fastest or level at every rank count up to 16 (14-17 %
+    // ahead of the compiler's allocation at 8 and 16 ranks).
 #define ZERO_CASE(NV, UV, BV) \
-    case NV: return launch_tiles<NV, UV, kFused, BV>(L, w, grads, stride, reduced, master, m, v, p16, c, nonfinite, st, c_dev);
+    case NV: \
+        if constexpr (kFused) \
+            return launch_tiles<NV, UV, true, BV>(L, w, grads, stride, reduced, master, m, v, p16, c, nonfinite, st, c_dev); \
+        else \
+            return launch_tiles<NV, 1, false, 2>(L, w, grads, stride, reduced, master, m, v, p16, c, nonfinite, st, c_dev);
     switch (L.n_ranks) {
         ZERO_CASE(1, 1, 2)
         ZERO_CASE(2, 1, 2)
