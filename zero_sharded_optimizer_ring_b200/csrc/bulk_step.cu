@@ -31,7 +31,7 @@ namespace {
 // Pipeline shape per rank count, measured on B200 (kernel GB/s of the full step on the
 // flat N=4, GPT-2 N=8, Llama N=8 and ragged N=16 workloads): larger single copies pay,
 // but more than about 120-170 KB in flight per SM costs DRAM efficiency.  Few ranks:
-// 4096-element chunks (one tile), 16 consumer warps, 2-3 stages.  More ranks: 2048-element
+// 4096-element chunks (one tile), 16 consumer warps, 2 stages.  More ranks: 2048-element
 // chunks, 8 consumer warps, at most 3 stages.
 //
 // N = 0 is the runtime rank count (17..kMaxBulkRanks): a stage of (2n + 12) bytes per
