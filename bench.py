@@ -643,6 +643,8 @@ def run_overlap(a, wl):
     torch.cuda.set_device(dist_env()[1])
     lay = zs.Layout(list(wl.tensors), wl.n_ranks, wl.stage, wl.bucket_elems, wl.pad_align, list(wl.units))
     lay.to_device()
+    if a.kernel:
+        lay.set_impl(a.kernel)
     P, psi, N = lay.padded, lay.psi, wl.n_ranks
     g = torch.zeros((N, P), dtype=torch.int16, device="cuda")
     master = torch.empty(P, dtype=torch.float32, device="cuda")
@@ -700,6 +702,8 @@ def run_overlap(a, wl):
             lay.close()
             lay = zs.Layout(list(wl.tensors), wl.n_ranks, wl.stage, wl.bucket_elems, wl.pad_align, list(wl.units))
             lay.to_device()
+            if a.kernel:
+                lay.set_impl(a.kernel)
         lay.set_max_ctas(cap)
         producer, compute = torch.cuda.Stream(), torch.cuda.Stream(priority=prio)
         make = gemm_backward if a.backward == "gemm" else generator_backward
@@ -717,7 +721,8 @@ def _overlap_reps(a, wl, lay, g, master, m, v, p16_shard, p16_full, backward, pr
         return zs.AdamW(wl.lr, wl.beta1, wl.beta2, wl.eps, wl.weight_decay, wl.loss_scale, t)
 
     res = {"bwd": [], "step": [], "seq": [], "pipe": [], "pipe_all": []}
-    warmup = a.warmup if cap else max(a.warmup, 1 + 5 * 2 + 1)   # the plan tuner: a warm-up, 5 plans twice
+    # the plan tuner: a warm-up call, then every plan timed twice
+    warmup = a.warmup if cap else max(a.warmup, 1 + zs._abi.OVERLAP_PLANS * 2 + 1)
     for rep in range(warmup + reps):
         torch.cuda.synchronize()
         s0, e0 = ev(), ev()
@@ -760,6 +765,7 @@ def _overlap_reps(a, wl, lay, g, master, m, v, p16_shard, p16_full, backward, pr
     print(json.dumps({
         "metric": "bucket-pipelined step behind a simulated backward (overlap)", "workload": wl.name,
         "backward": a.backward, "compute_stream_priority": prio_name,
+        "kernel": {0: "automatic", 1: "register streaming", 2: "bulk-copy pipeline"}[a.kernel],
         "max_ctas": cap if cap else "auto (measured by the library)",
         "bucket_group": group if group else "auto (zero_step_overlapped: launches of >= 2^24 elements)",
         "t_back_to_back_ms": tq, "t_backward_plus_step_alone_ms": tb + ts,

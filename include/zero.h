@@ -273,11 +273,11 @@ zero_status zero_step_bucket(const zero_layout *layout, int64_t bucket, const ui
  * split the SMs depends on the two workloads (and on the power budget they share).
  * Unless zero_set_max_ctas fixed a cap, the library chooses a plan by measurement: after
  * one untimed warm-up call it times whole calls (CUDA events on `stream`, from the first
- * wait to the last launch) under five plans, round-robin, two calls each: the update
- * following the backward bucket by bucket with its grid capped at 1, 2/3, 1/2 or 1/3 of
- * the SMs, or deferred to one full-grid launch after the last bucket's event (the
- * back-to-back order, for workloads where sharing the GPU does not pay); it then keeps
- * the plan with the lowest mean for every later call.  It never waits for these
+ * wait to the last launch) under ZERO_OVERLAP_PLANS plans, round-robin, two calls each:
+ * the update following the backward bucket by bucket with its grid capped at 1, 2/3,
+ * 1/2 or 1/3 of the SMs, or deferred to one full-grid launch after the last bucket's
+ * event (the back-to-back order, for workloads where sharing the GPU does not pay); it
+ * then keeps the plan with the lowest mean for every later call.  It never waits for these
  * events: a call issued before the previous timed call has finished on the GPU is not
  * timed.  The plan never changes a result. */
 zero_status zero_step_overlapped(const zero_layout *layout, void *const *ready_events,
@@ -288,8 +288,10 @@ zero_status zero_step_overlapped(const zero_layout *layout, void *const *ready_e
 /* The launch plan the overlapped steps settled on for this layout: -1 while the plans
  * are still being timed (or when zero_set_max_ctas fixed a cap), 0..3 = the update
  * following the backward with its grid capped at 1, 2/3, 1/2, 1/3 of the SMs, 4 = the
- * update deferred to one launch after the last bucket.  *mean_ms (optional, [5]) receives
- * each plan's mean timed call so far (0 where none).  Host only. */
+ * update deferred to one launch after the last bucket.  *mean_ms (optional, host array
+ * of ZERO_OVERLAP_PLANS) receives each plan's mean timed call so far (0 where none).
+ * Host only. */
+#define ZERO_OVERLAP_PLANS 5
 zero_status zero_overlap_plan(const zero_layout *layout, int32_t *plan, float *mean_ms);
 
 /* zero_step_overlapped with one launch per `group` consecutive buckets (group >= 1; the

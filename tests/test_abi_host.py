@@ -47,6 +47,23 @@ def test_status_codes_named_in_the_binding_and_the_library():
         assert lib.zero_status_string(c).decode() != "unknown status", codes[c]
 
 
+def test_header_constants_mirrored_in_the_binding():
+    """Sizes the binding allocates for the library (the plan-mean array of
+    zero_overlap_plan) and limits it checks must equal the header's."""
+    src = open(os.path.join(ROOT, "include", "zero.h")).read()
+    consts = {k: int(v) for k, v in re.findall(r"#define (ZERO_[A-Z_]+) (\d+)", src)}
+    assert consts["ZERO_OVERLAP_PLANS"] == _abi.OVERLAP_PLANS
+    assert consts["ZERO_NOALLOC_MAX_SEGMENTS"] == _abi.NOALLOC_MAX_SEGMENTS
+
+
+def test_overlap_plan_before_any_overlapped_call():
+    """No plan chosen yet (-1) and every mean 0, in an array of ZERO_OVERLAP_PLANS."""
+    lay = zs.Layout([1000], 2, 1, 0, 128, [0])
+    plan, means = lay.overlap_plan()
+    assert plan == -1 and means == [0.0] * _abi.OVERLAP_PLANS
+    lay.close()
+
+
 def _compare(tensors, N, stage, B, A, units):
     ref = make_layout(tensors, N, B, A, units)
     lay = zs.Layout(tensors, N, stage, B, A, units)

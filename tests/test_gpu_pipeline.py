@@ -114,7 +114,8 @@ def test_overlapped_grid_tuner_keeps_results(key):
     zs.get_error(lay)
     _check(wl, lay, b, ref)
     plan, means = lay.overlap_plan()
-    assert 0 <= plan <= 4 and all(x > 0 for x in means)      # every plan timed, one kept
+    assert 0 <= plan < zs._abi.OVERLAP_PLANS and len(means) == zs._abi.OVERLAP_PLANS
+    assert all(x > 0 for x in means)                         # every plan timed, one kept
     assert means[plan] == min(means)
 
 

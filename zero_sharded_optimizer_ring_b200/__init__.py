@@ -150,7 +150,7 @@ class Layout:
         plan -1 while still timing, 0-3 = grid capped at 1, 2/3, 1/2, 1/3 of the SMs,
         4 = deferred to one launch after the last bucket."""
         plan = ctypes.c_int32()
-        means = np.zeros(5, np.float32)
+        means = np.zeros(_abi.OVERLAP_PLANS, np.float32)
         _check(_abi.lib().zero_overlap_plan(self._h, ctypes.byref(plan), means.ctypes.data), "zero_overlap_plan")
         return int(plan.value), [float(x) for x in means]
 

@@ -14,6 +14,7 @@ _p_i64 = ctypes.POINTER(ctypes.c_int64)
 
 ZERO_OK = 0
 NOALLOC_MAX_SEGMENTS = 8191   # ZERO_NOALLOC_MAX_SEGMENTS in include/zero.h
+OVERLAP_PLANS = 5             # ZERO_OVERLAP_PLANS in include/zero.h
 STATUS_NAMES = {0: "ZERO_OK", 1: "ZERO_ERR_INVALID", 2: "ZERO_ERR_ALIGN", 3: "ZERO_ERR_CUDA",
                 4: "ZERO_ERR_OOM", 5: "ZERO_ERR_TIMEOUT", 6: "ZERO_ERR_STATE", 7: "ZERO_ERR_BOUNDS"}
 

@@ -468,6 +468,8 @@ constexpr int64_t kMinOverlapLaunch = int64_t(1) << 24;
 // update's grid capped at SMs x {1, 2/3, 1/2, 1/3} (0 = no cap); i == 4 defers the whole
 // update to one full-grid launch after the last bucket's event.
 constexpr int kDeferred = 4;
+static_assert(kDeferred + 1 == zero::OverlapTuner::kCands, "one plan per tuner candidate");
+static_assert(zero::OverlapTuner::kCands == ZERO_OVERLAP_PLANS, "zero_overlap_plan fills ZERO_OVERLAP_PLANS means");
 
 int32_t tuner_cap(const zero_layout *L, int i)
 {
