@@ -1004,7 +1004,8 @@ def run_zero3_passes(a, wl):
     def short(bd):
         return {k: round(v, 4) for k, v in bd.items() if k.startswith("sum_")} | {
             "max_wait_ms": round(max(bd["wait_ms"]), 4),
-            "layers_waiting": sum(1 for w in bd["wait_ms"] if w > 0.005)}
+            "layers_waiting": sum(1 for w in bd["wait_ms"] if w > 0.005),
+            "wait_ms_per_unit": [round(w, 3) for w in bd["wait_ms"]]}
 
     set_carveout = torch._C._set_sm_carveout_experimental
     passes = (("forward", fwd, order_f), ("backward", bwd, order_b))

@@ -13,7 +13,8 @@ from . import gather_unit
 
 
 # How the gathers share the GPU with the layers' GEMMs during a pass (measured on the
-# Llama-shaped list, 2048 tokens, two slots): the gathers run as 16 persistent CTAs
+# Llama-shaped list, 2048 tokens, two slots): the gathers issued once layers compute run
+# as 16 persistent CTAs
 # (zero_set_gather_ctas) instead of a grid that floods every SM between GEMM waves, and the
 # matmuls run with cuBLAS's SM-count target 16 below the SM count on the cuBLASLt path
 # (torch's matmul carveout).  The target is a hint to the GEMM kernel choice rather than a
@@ -58,22 +59,25 @@ def zero3_pass(layout, p16_shard, slots, units, compute, gather_stream, compute_
     previous occupant units[j - len(slots)] has been computed; compute(unit, buffer) is
     then called with compute_stream current and must enqueue the layer's work there.
     During the pass the gathers run on gather_ctas persistent CTAs (None: the layout's
-    setting) and torch's matmuls run with the SM-count target matmul_sm_carveout below the
-    SM count and prefer `blas` (None: unchanged); every setting is restored afterwards.  Returns the list of (gather
-    started, gathered, computed) torch.cuda.Event triples, one per unit (timing events:
-    layer_breakdown reads them)."""
+    setting), except the first len(slots), which are issued before any layer has computed
+    and so take the whole GPU; torch's matmuls run with the SM-count target
+    matmul_sm_carveout below the SM count and prefer `blas` (None: unchanged); every
+    setting is restored afterwards.  Returns the list of (gather started, gathered,
+    computed) torch.cuda.Event triples, one per unit (timing events: layer_breakdown reads
+    them)."""
     import torch
     n = len(slots)
     marks = []
     saved_ctas = layout.gather_ctas
-    if gather_ctas is not None:
-        layout.set_gather_ctas(gather_ctas)
     try:
         with _MatmulShare(matmul_sm_carveout, blas):
             for j, u in enumerate(units):
                 started, gathered, computed = (torch.cuda.Event(enable_timing=True) for _ in range(3))
                 if j >= n:
                     gather_stream.wait_event(marks[j - n][2])
+                if gather_ctas is not None:
+                    # the first n gathers have no layer compute to share the GPU with
+                    layout.set_gather_ctas(0 if j < n else gather_ctas)
                 started.record(gather_stream)
                 gather_unit(layout, u, p16_shard, slots[j % n], stream=gather_stream)
                 gathered.record(gather_stream)
