@@ -917,7 +917,7 @@ def run_zero3_passes(a, wl):
     compute alone (parameters already in place) and the gathers alone."""
     import torch
     import zero_sharded_optimizer_ring_b200 as zs
-    from zero_sharded_optimizer_ring_b200.schedule import layer_breakdown, zero3_pass
+    from zero_sharded_optimizer_ring_b200.schedule import GatherWidth, layer_breakdown, zero3_pass
     from seeded_inputs.workloads import llama_tensors
 
     torch.cuda.set_device(dist_env()[1])
@@ -1034,26 +1034,37 @@ def run_zero3_passes(a, wl):
     sweep = []
     # "default" = zero3_pass with its own defaults (capped gathers, matmul SM carveout,
     # cuBLASLt), two slots
-    configs = [("default", "default", 2) if c == "default" else tuple(int(x) for x in c.split(":"))
+    # "width" = the same with the capped gathers' grid chosen per pass kind by feedback
+    # (schedule.GatherWidth, kept across rounds after warm-up passes)
+    configs = [(c, c, 2) if c in ("default", "width") else tuple(int(x) for x in c.split(":"))
                for c in a.zero3_configs.split(",") if c]
+    widths = {name: GatherWidth() for name, _, _ in passes}
     if configs:
         if a.blas:
             torch.backends.cuda.preferred_blas_library(a.blas)
+        if any(c == "width" for c, _, _ in configs):
+            for _ in range(len(widths["forward"].candidates) * widths["forward"].trials + 2):
+                for name, work, order in passes:
+                    zero3_pass(lay, shard, slots[:2], order, work, gs, cs, gather_ctas=widths[name])
+                    torch.cuda.synchronize()
         rounds = {}
         for rnd in range(a.zero3_rounds):
             for c, gcap, n in configs:
-                dflt = c == "default"
+                dflt = c in ("default", "width")
                 set_carveout(None if dflt or c == 0 else c)
                 lay.set_gather_ctas(0 if dflt else gcap)
                 for name, work, order in passes:
                     if n == 0:
                         fn = compute_only(work)
+                    elif c == "width":
+                        fn = (lambda o=order, w=work, k=n, gw=widths[name]: zero3_pass(lay, shard, slots[:k], o, w, gs,
+                                                                                       cs, gather_ctas=gw))
                     elif dflt:
                         fn = (lambda o=order, w=work, k=n: zero3_pass(lay, shard, slots[:k], o, w, gs, cs))
                     else:
-                        fn = (lambda o=order, w=work, k=n: zero3_pass(lay, shard, slots[:k], o, w, gs, cs,
-                                                                      gather_ctas=None, matmul_sm_carveout=None,
-                                                                      blas=None))
+                        fn = (lambda o=order, w=work, k=n, gc=gcap: zero3_pass(lay, shard, slots[:k], o, w, gs, cs,
+                                                                               gather_ctas=gc, matmul_sm_carveout=None,
+                                                                               blas=None))
                     torch.cuda.synchronize()
                     s0, e0 = ev(), ev()
                     s0.record(gs)
@@ -1085,7 +1096,10 @@ def run_zero3_passes(a, wl):
                       "units": lay.n_units, "tokens": T, "gather_bytes_per_pass": gather_bytes,
                       "gather_gbs": gather_bytes / (res["gathers_only_ms"] / 1e3) / 1e9,
                       **{k: (round(v, 4) if isinstance(v, float) else v) for k, v in res.items()},
-                      "sweep": sweep}), flush=True)
+                      "sweep": sweep,
+                      "gather_width": {name: {"chosen_ctas": w.ctas if w.chosen is not None else None,
+                                              "mean_pass_ms": dict(zip(w.candidates, w.means()))}
+                                       for name, w in widths.items() if any(w.count)}}), flush=True)
 
 
 def main():

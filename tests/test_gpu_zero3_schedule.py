@@ -15,7 +15,7 @@ import pytest
 
 from seeded_inputs.workloads import reduced_workloads
 import zero_sharded_optimizer_ring_b200 as zs
-from zero_sharded_optimizer_ring_b200.schedule import zero3_pass
+from zero_sharded_optimizer_ring_b200.schedule import GatherWidth, Zero3Prefetch, zero3_pass
 import support as S
 
 torch = pytest.importorskip("torch")
@@ -106,11 +106,12 @@ def test_capped_gather_of_a_large_unit_matches_oracle(gather_ctas):
         assert (got[lay.padded:] == 7).all(), f"{name}: write past the unit"
 
 
-@pytest.mark.parametrize("gather_ctas", [0, None])
+@pytest.mark.parametrize("gather_ctas", [0, None, "width"])
 @pytest.mark.parametrize("n_slots", [1, 2, 3])
 @pytest.mark.parametrize("backward", [False, True])
 def test_prefetch_schedule_gives_each_layer_its_parameters(n_slots, backward, gather_ctas):
-    """gather_ctas 0: the gathers' default grid; None: the schedule's own setting."""
+    """gather_ctas 0: the gathers' default grid; None: the schedule's own setting;
+    "width": a GatherWidth, over three passes (a warm-up, then two timed ones)."""
     wl = _workload()
     lay, shard, ref = _stepped_shards(wl)
     _, _, _, u = lay.tables()
@@ -128,8 +129,47 @@ def test_prefetch_schedule_gives_each_layer_its_parameters(n_slots, backward, ga
 
     gs, cs = torch.cuda.Stream(), torch.cuda.Stream()
     torch.cuda.synchronize()                        # inputs written on the default stream
-    kw = {} if gather_ctas is None else {"gather_ctas": gather_ctas}
-    zero3_pass(lay, shard, slots, order, compute, gs, cs, **kw)
+    width = GatherWidth() if gather_ctas == "width" else None
+    kw = {} if gather_ctas is None else {"gather_ctas": width if width else gather_ctas}
+    for _ in range(3 if width else 1):
+        out.zero_()
+        torch.cuda.synchronize()
+        zero3_pass(lay, shard, slots, order, compute, gs, cs, **kw)
+        torch.cuda.synchronize()
+        assert lay.gather_ctas == 0                 # the layout's setting is restored
+        S.assert_bits_equal(S.to_np(out), ref.p16_full, "layers as the compute saw them")
+    if width:
+        assert sum(width.count) == 1                # the first pass untimed, the third read the second
+
+
+@pytest.mark.parametrize("n_slots", [2, 3])
+def test_passes_enqueued_back_to_back_reuse_slots_safely(n_slots):
+    """Zero3Prefetch: a forward, a backward and a forward pass enqueued with no host
+    synchronisation between them.  The slots are reused across passes (with three slots
+    the backward pass gathers unit 4 into the slot the forward pass's unit 3 is still
+    being computed from), so each pass's first gathers must wait for the previous pass's
+    layers; every layer of every pass must see exactly its own parameters."""
+    wl = _workload()
+    lay, shard, ref = _stepped_shards(wl)
+    _, _, _, u = lay.tables()
+    width = int(max(hi - lo for lo, hi in u))
+    slots = [torch.zeros(width, dtype=torch.int16, device="cuda") for _ in range(n_slots)]
+    outs = [torch.zeros(lay.padded, dtype=torch.int16, device="cuda") for _ in range(3)]
+
+    def layer(out):
+        def compute(unit, buf):
+            torch.cuda._sleep(400_000)              # a slow layer: a gather into its slot would overtake it
+            lo, hi = int(u[unit][0]), int(u[unit][1])
+            out[lo:hi].copy_(buf[:hi - lo])
+        return compute
+
+    gs, cs = torch.cuda.Stream(), torch.cuda.Stream()
+    pf = Zero3Prefetch(lay, shard, slots, gs, cs, candidates=(2, 16), trials=1)
     torch.cuda.synchronize()
-    assert lay.gather_ctas == 0                     # the layout's setting is restored
-    S.assert_bits_equal(S.to_np(out), ref.p16_full, "layers as the compute saw them")
+    pf.forward(layer(outs[0]))
+    pf.backward(layer(outs[1]))
+    pf.forward(layer(outs[2]))
+    torch.cuda.synchronize()
+    assert lay.gather_ctas == 0
+    for k, out in enumerate(outs):
+        S.assert_bits_equal(S.to_np(out), ref.p16_full, f"pass {k}: layers as the compute saw them")
