@@ -72,10 +72,12 @@ def parse():
                     help="time ZeRO-3's per-layer forward and backward gathers with 1-3 prefetch slots "
                          "against a simulated layer compute (its own JSON line)")
     ap.add_argument("--tokens", type=int, default=2048, help="--zero3-passes: tokens per rank")
-    ap.add_argument("--zero3-configs", default="0:0:0,0:0:1,0:0:2,0:16:2,0:16:3",
+    ap.add_argument("--zero3-configs", default="0:0:0,0:0:1,0:0:2,default,width",
                     help="--zero3-passes sweep: comma-separated carveout:gather_ctas:slots (carveout = how far "
                          "below the SM count the matmuls' cuBLAS SM-count target is set; gather_ctas = "
-                         "zero_set_gather_ctas, 0 = default grid; slots 0 = the compute alone)")
+                         "zero_set_gather_ctas, 0 = default grid; slots 0 = the compute alone), or 'default' "
+                         "(zero3_pass's own settings) or 'width' (those, with the gather width tuned per kind of "
+                         "pass by schedule.GatherWidth)")
     ap.add_argument("--zero3-rounds", type=int, default=5, help="--zero3-passes: interleaved rounds of the sweep")
     ap.add_argument("--blas", default="", help="--zero3-passes: torch preferred BLAS library (cublas, cublaslt)")
     ap.add_argument("--overlap", action="store_true",
