@@ -14,8 +14,8 @@ from . import gather_unit
 
 # How the gathers share the GPU with the layers' GEMMs during a pass (measured on the
 # Llama-shaped list, 2048 tokens, two slots): the gathers issued once layers compute run
-# as 16 persistent CTAs
-# (zero_set_gather_ctas) instead of a grid that floods every SM between GEMM waves, and the
+# as a few persistent CTAs (zero_set_gather_ctas; 16 unless a GatherWidth tunes it per
+# kind of pass) instead of a grid that floods every SM between GEMM waves, and the
 # matmuls run with cuBLAS's SM-count target 16 below the SM count on the cuBLASLt path
 # (torch's matmul carveout).  The target is a hint to the GEMM kernel choice rather than a
 # cap on the SMs a GEMM occupies; with it the layer GEMMs alone are no slower, and beside
