@@ -142,3 +142,30 @@ def test_sampled_path_equals_bucket_simulation():
         assert np.array_equal(r2.view(np.uint32), red.view(np.uint32))
         full = oracle.run_steps(lay, 1, g, master, zeros, zeros, hp, 2)
         assert np.array_equal(p16, full.p16_full)
+
+
+@pytest.mark.parametrize("N", [3, 4, 5])
+def test_a_dropped_or_duplicated_hop_is_caught(N):
+    """Fault injection into the literal ring: one hop fewer leaves every chunk's sum
+    without one rank's value, which the exact-sum invariant and the send counts both
+    catch; one hop more adds a rank twice into a partial that nobody reads (each sum is
+    read from the rank that completed it, which a further send does not change), which
+    only the send counts catch.  The counts are the pages' closed form: (N-1)*S
+    elements sent and received per rank in one scatter-reduce."""
+    S = 8
+    rng = np.random.default_rng(40 + N)
+    # fp16 values on a 2^-10 grid, |x| < 2 (exactly representable): every partial sum
+    # is exact in fp32
+    vals = rng.integers(-2047, 2048, size=(N, N * S)) / 1024.0
+    g = vals.astype(np.float16).view(np.uint16).copy()
+    assert np.all(g.view(np.float16).astype(np.float64) == vals)
+    exact = vals.sum(axis=0)
+    for hops in (N - 1, N - 2, N):
+        red = np.zeros(N * S, dtype=np.float32)
+        sent = np.zeros(N, dtype=np.int64)
+        recv = np.zeros(N, dtype=np.int64)
+        oracle.ring_reduce_scatter(g, S, 0, N * S, hops=hops, reduced=red, sent=sent, recv=recv)
+        sums_exact = bool(np.all(red.astype(np.float64) == exact))
+        counts_closed_form = bool(np.all(sent == (N - 1) * S) and np.all(recv == (N - 1) * S))
+        assert sums_exact == (hops != N - 2), hops
+        assert counts_closed_form == (hops == N - 1), hops
