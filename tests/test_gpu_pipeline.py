@@ -90,6 +90,44 @@ def test_overlapped_step_with_simulated_backward(key, group):
     _check(wl, lay, b, ref)
 
 
+@pytest.mark.parametrize("wire", [False, True])
+@pytest.mark.parametrize("impl", [zs.IMPL_REGISTER, zs.IMPL_BULK])
+@pytest.mark.parametrize("key", ["flat1p3b_n4_zero1", "llama3b_n8_zero3", "ragged2000_n16_zero2"])
+def test_overlapped_step_each_kernel_each_wire(key, impl, wire):
+    """The overlapped step through each implementation, forced, with fp32 sums and with
+    the fp16 wire, gradients arriving bucket by bucket: the oracle's state bit for bit
+    (its fp16-wire run for the fp16 wire), per-bucket non-finite counts included."""
+    import oracle
+    wl = reduced_workloads()[key]
+    olay = S.oracle_layout(wl)
+    g, master, m, v = S.host_inputs(wl, olay.padded)
+    ref = oracle.run_steps(olay, wl.stage, g, master, m, v, S.hyper(wl), STEPS, wire16=wire)
+    lay = zs.Layout(list(wl.tensors), wl.n_ranks, wl.stage, wl.bucket_elems, wl.pad_align, list(wl.units),
+                    wire_fp16=wire).to_device()
+    lay.set_impl(impl)
+    P = lay.padded
+    gd, md, mm, vd = S.device_inputs(wl, P)
+    b = dict(g=gd, master=md, m=mm, v=vd, p16_shard=torch.zeros(P, dtype=torch.int16, device="cuda"),
+             p16_full=torch.zeros(P, dtype=torch.int16, device="cuda"),
+             nonfinite=torch.zeros(max(1, lay.n_buckets), dtype=torch.int32, device="cuda"))
+    _, buckets, _, _ = lay.tables()
+    producer, consumer = torch.cuda.Stream(), torch.cuda.Stream()
+    for t in range(1, STEPS + 1):
+        torch.cuda.synchronize()
+        b["g"].zero_()
+        b["nonfinite"].zero_()
+        torch.cuda.synchronize()
+        ready = [torch.cuda.Event() for _ in range(lay.n_buckets)]
+        for bk, (lo, hi) in enumerate(buckets):
+            si.fill_grads_range_cuda(b["g"], int(lo), int(hi), wl.psi, wl.seed, wl.grad_sigma, wl.loss_scale,
+                                     wl.heavy_frac, wl.heavy_mult, cuda_stream=producer.cuda_stream)
+            ready[bk].record(producer)
+        zs.step_overlapped(lay, ready, b["g"], b["master"], b["m"], b["v"], b["p16_shard"], b["p16_full"],
+                           _hp(wl, t), nonfinite=b["nonfinite"], stream=consumer)
+    zs.get_error(lay)
+    _check(wl, lay, b, ref)
+
+
 @pytest.mark.parametrize("key", ["flat1p3b_n4_zero1", "ragged2000_n16_zero2"])
 def test_overlapped_grid_tuner_keeps_results(key):
     """With no cap set, the overlapped step times several launch plans over its first calls
