@@ -330,13 +330,14 @@ def test_bad_arguments_rejected():
                 zs.AdamW(loss_scale=0.0, step=1))
 
 
-def test_host_buffer_step_matches_oracle():
+@pytest.mark.parametrize("impl", IMPLS)
+def test_host_buffer_step_matches_oracle(impl):
     """zero_step_host: gradients from pinned host memory, fp16 parameters back to pinned
     host memory; the device state and the host parameters equal the oracle's."""
     for key in ("flat1p3b_n4_zero1", "llama3b_n8_zero3", "ragged2000_n16_zero2"):
         wl = reduced_workloads()[key]
         ref, olay = _oracle(wl, 2)
-        lay = _layout(wl)
+        lay = _layout(wl, impl)
         b = _bufs(lay, wl)
         g_host = torch.from_numpy(S.host_inputs(wl, olay.padded)[0].view(np.int16))
         pad = b["g"].shape[1] - g_host.shape[1]

@@ -1,4 +1,4 @@
-"""The allocation-free entry point, zero_step_noalloc, against zero_step.
+"""The allocation-free entry point, zero_step_noalloc, against zero_step and the oracle.
 
 Some callers cannot let a library allocate device memory (their GPU memory belongs to
 another allocator or a reserved pool, or they cannot take the synchronisation an
@@ -7,7 +7,8 @@ segment table and its tile index) in a static device array.  These tests call it
 the C ABI on a layout that was never uploaded (so no library allocation exists at all)
 and check its outputs against zero_step's, within the tolerance of the other parity
 tests and then bit for bit (both kernels follow the same rounded operations), on two
-calls in a row (the second call runs on the array the first one left).
+calls in a row (the second call runs on the array the first one left), and the final
+state against the oracle's two steps.
 
 This file is collected last on purpose: if it fails, every other test has already run.
 """
@@ -48,6 +49,7 @@ def test_noalloc_matches_step_on_two_calls(key):
     uploaded = zs.Layout(*args).to_device()
     host_only = zs.Layout(*args)                  # never uploaded: nothing allocated for it
     assert host_only.n_segments <= _abi.NOALLOC_MAX_SEGMENTS
+    ref, _ = S.oracle_run(wl, 2)
     a = _bufs(uploaded.padded, wl)
     b = _bufs(uploaded.padded, wl)
     guards = S.guard_outputs(b)            # a write past any output buffer shows up here
@@ -69,6 +71,8 @@ def test_noalloc_matches_step_on_two_calls(key):
         names = ("master", "m", "v", "p16_full") + (("p16_shard",) if wl.stage == 3 else ())
         for name in names:
             S.assert_bits_equal(_np(b[name]), _np(a[name]), f"{name} after call {t} (bits)")
+    # and both equal the oracle's two steps
+    S.assert_state_matches_oracle(wl, b, ref, "zero_step_noalloc: ")
 
 
 def test_noalloc_rejects_layouts_beyond_its_table():
