@@ -171,10 +171,13 @@ def test_capped_grid_matches_oracle(key, impl):
 
 
 def test_device_tile_index_matches_host():
+    """The segment table the device builds (with its warp-scanned tile index) against the
+    oracle's layout: the same (bucket, shard, lo, hi) rows, and each segment's first tile
+    = the running count of the kTileElems cells the segments before it overlap."""
     for wl in list(reduced_workloads().values()) + list(full_workloads().values()):
         lay = _layout(wl)
         dev = lay.device_segments()
-        _, _, segs, _ = lay.tables()
+        segs = np.array(S.oracle_layout(wl).segments, dtype=np.int64).reshape(-1, 4)
         T = lay.tile_elems
         assert np.array_equal(dev[:-1, :4], segs)
         counts = [-(-hi // T) - lo // T for _, _, lo, hi in segs]
