@@ -225,6 +225,79 @@ def record_traffic(a, wl):
     print(json.dumps(rec))
 
 
+class NvmlClockSampler:
+    """SM clock and clock-event-reason samples read through NVML (read-only queries) by a
+    polling thread, about every `period` seconds; only those taken between mark_start()
+    and mark_end() (the timed region) are summarised.  `nvml` is the pynvml module (a
+    stand-in in tests); `index` the NVML index of the GPU."""
+    REASON_BITS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+                   ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+                   ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"),
+                   ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+                   ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+
+    def __init__(self, nvml, index, period=0.002):
+        import threading
+        self.nvml, self.period = nvml, period
+        nvml.nvmlInit()
+        self.h = nvml.nvmlDeviceGetHandleByIndex(index)
+        self.max_mhz = float(nvml.nvmlDeviceGetMaxClockInfo(self.h, nvml.NVML_CLOCK_SM))
+        self.t0 = self.t1 = None
+        self.samples = []
+        self._sample()                 # a query that fails, fails here (the caller falls back)
+        self._stop = threading.Event()
+        self._thread = threading.Thread(target=self._poll, daemon=True)
+        self._thread.start()
+
+    def _sample(self):
+        nv = self.nvml
+        t = time.time()
+        self.samples.append((t, float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)),
+                             int(nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))))
+
+    def _poll(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                return
+            self._stop.wait(self.period)
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    def stop(self):
+        self._stop.set()
+        self._thread.join(timeout=5)
+        try:
+            self.nvml.nvmlShutdown()
+        except Exception:
+            pass
+        inside = [x for x in self.samples if self.t0 is not None and self.t0 <= x[0] <= (self.t1 or 1e18)]
+        rows = inside or self.samples
+        if not rows:
+            return None
+        bits = {name: getattr(self.nvml, attr) for name, attr in self.REASON_BITS}
+        reasons = sorted({name for _, _, r in rows for name, bit in bits.items() if r & bit})
+        return {"sm_mhz": statistics.median(sm for _, sm, _ in rows), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(rows), "in_timed_region": bool(inside), "source": "nvml"}
+
+
+def clock_sampler(cuda_index):
+    """NVML polling when the pynvml module and the driver's NVML answer; nvidia-smi
+    otherwise."""
+    try:
+        import pynvml
+        import torch
+        index = torch.cuda._get_nvml_device_index(cuda_index)
+        return NvmlClockSampler(pynvml, index)
+    except Exception:
+        return ClockSampler(cuda_index)
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples; only those taken between mark_start()
     and mark_end() (the timed region) are summarised."""
@@ -280,7 +353,7 @@ class ClockSampler:
         sm = [num(r[2]) for r in rows if num(r[2]) is not None]
         reasons = sorted({self.REASONS[j] for r in rows for j in range(4) if r[6 + j].lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": num(rows[0][3]),
-                "reasons": reasons, "samples": len(rows), "in_timed_region": bool(inside)}
+                "reasons": reasons, "samples": len(rows), "in_timed_region": bool(inside), "source": "nvidia-smi"}
 
 
 def workload_config(wl, world):
@@ -529,7 +602,7 @@ def _measure(a, wl, world, rank, barrier, headline):
     ev = [{k: torch.cuda.Event(enable_timing=True) for k in ("update_begin", "update_end", "gather_begin", "gather_end")}
           for _ in range(K)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    sampler = clock_sampler(torch.cuda.current_device()) if rank == 0 else None
     time.sleep(0.3)
     barrier()
     if sampler:
