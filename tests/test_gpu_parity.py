@@ -390,6 +390,36 @@ def test_full_size_sampled(key, impl):
     assert int(torch.count_nonzero(b["master"][lay.psi:])) == 0
 
 
+@pytest.mark.parametrize("key", ["flat1p3b_n4_zero1", "ragged2000_n16_zero2"])
+def test_full_size_overlapped_sampled(key):
+    """zero_step_overlapped at full size (the flat list's 27 buckets of 5*10^7, each its own
+    launch; the ragged list's 490 buckets of 10^6, coalesced into launches of >= 2^24
+    elements), every bucket's event recorded on a producer stream, through the plan
+    tuner's first calls: the oracle's state at sampled elements, bit for bit."""
+    wl = full_workloads()[key]
+    olay = S.oracle_layout(wl)
+    lay = _layout(wl, zs.IMPL_AUTO)
+    b = _bufs(lay, wl)
+    producer, consumer = torch.cuda.Stream(), torch.cuda.Stream()
+    torch.cuda.synchronize()
+    for t in range(1, wl.steps + 1):
+        ready = [torch.cuda.Event() for _ in range(lay.n_buckets)]
+        for e in ready:
+            e.record(producer)
+        b["nonfinite"].zero_()
+        torch.cuda.synchronize()
+        zs.step_overlapped(lay, ready, b["g"], b["master"], b["m"], b["v"], b["p16_shard"], b["p16_full"],
+                           _hp(wl, t), nonfinite=b["nonfinite"], stream=consumer)
+        torch.cuda.synchronize()
+    zs.get_error(lay)
+    idx = S.sample_indices(olay)
+    it = torch.from_numpy(idx).cuda()
+    _, master, m, v, p16 = S.sampled_oracle(wl, olay, idx, wl.steps)
+    for name, want in (("master", master), ("m", m), ("v", v), ("p16_full", p16)):
+        S.assert_bits_equal(_np(b[name][it]), want, name)
+    assert int(b["nonfinite"].sum()) == 0
+
+
 @pytest.mark.parametrize("impl", IMPLS)
 def test_flat_buffer_beyond_2_32_elements(impl):
     """ψ just above 2^32 (N=2, full fp32 state: 86 GB on the device): element indices,
