@@ -421,6 +421,37 @@ def test_full_size_overlapped_sampled(key):
 
 
 @pytest.mark.parametrize("impl", IMPLS)
+def test_full_size_dynamic_commit_sampled(impl):
+    """zero_step_dynamic_commit at full size (flat list, two state sets and two fp16
+    buffers of 1.3*10^9): with a scale that never overflows here and a window longer than
+    the run, every step applies at the workload's loss scale, so after each commit the
+    current set equals the oracle's plain steps at sampled elements, bit for bit."""
+    wl = full_workloads()["flat1p3b_n4_zero1"]
+    steps = 3
+    olay = S.oracle_layout(wl)
+    lay = _layout(wl, impl)
+    P = lay.padded
+    g, master, m, v = S.device_inputs(wl, P)
+    sets = [[master, m, v], [torch.empty_like(master), torch.empty_like(m), torch.empty_like(v)]]
+    p16s = [torch.zeros(P, dtype=torch.int16, device="cuda"), torch.zeros(P, dtype=torch.int16, device="cuda")]
+    nonfinite = torch.zeros(max(1, lay.n_buckets), dtype=torch.int32, device="cuda")
+    scaler = zs.LossScaler(wl.loss_scale, window=1 << 40)
+    for t in range(1, steps + 1):
+        assert zs.step_dynamic_commit(lay, g, sets[0], sets[1], p16s[1], p16s[1], _hp(wl, t), scaler, nonfinite)
+        sets.reverse()
+        p16s.reverse()
+    zs.get_error(lay)
+    torch.cuda.synchronize()
+    assert scaler.scale == wl.loss_scale
+    idx = S.sample_indices(olay)
+    it = torch.from_numpy(idx).cuda()
+    _, want_master, want_m, want_v, want_p16 = S.sampled_oracle(wl, olay, idx, steps)
+    for name, got, want in (("master", sets[0][0], want_master), ("m", sets[0][1], want_m),
+                            ("v", sets[0][2], want_v), ("p16", p16s[0], want_p16)):
+        S.assert_bits_equal(_np(got[it]), want, name)
+
+
+@pytest.mark.parametrize("impl", IMPLS)
 def test_flat_buffer_beyond_2_32_elements(impl):
     """ψ just above 2^32 (N=2, full fp32 state: 86 GB on the device): element indices,
     byte offsets and tile numbers past 32 bits, sampled against the oracle, including
