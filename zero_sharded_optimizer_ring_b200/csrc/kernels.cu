@@ -50,8 +50,10 @@ __device__ __forceinline__ float fold_scalar(const uint16_t *__restrict__ grads,
 //   loads are in flight together, kWire = fp16 wire (partials rounded to fp16 per hop),
 //   kOut = the fused update reads the state from `in` and writes it to master / mom1 /
 //   mom2 (two buffer sets that do not overlap); otherwise it updates them in place.
-//   kMinBlocks = the resident CTAs per SM the register allocation is held to (0: the
-//   compiler's choice).
+//   kMinBlocks = the launch bound's minimum of resident CTAs per SM, i.e. a register
+//   budget of 65536 / (kThreads * kMinBlocks) per thread (0: no bound, the compiler's
+//   own choice); the grid then takes as many CTAs per SM as the registers actually used
+//   allow.
 struct StateIn {
     const float *master, *mom1, *mom2;
 };
@@ -500,12 +502,13 @@ cudaError_t dispatch_tiles(const zero_layout &L, const TileWork &w, const uint16
                            const AdamScalars *c_dev = nullptr)
 {
     if (w.n_tiles <= 0) return cudaSuccess;
-    // Shapes (vectors in flight per thread, CTAs per SM the registers are held to), from
+    // Shapes (vectors in flight per thread, the launch bound's minimum CTAs per SM), from
     // sweeps on flat lists of 2^28 parameters, one B200.  Fused: for 1-4 ranks one vector
-    // at two CTAs per SM beats two vectors per thread by 3-8 %; at 8 and 16 ranks one
-    // vector with the compiler's allocation is as fast or faster.  Reduce-only: one vector
-    // at two CTAs per SM is the fastest or level at every rank count up to 16 (14-17 %
-    // ahead of the compiler's allocation at 8 and 16 ranks).
+    // with the two-CTA register budget (at 4 ranks 112 registers: two CTAs per SM) beats
+    // two vectors per thread by 3-8 %; at 8 and 16 ranks one vector with no bound is as
+    // fast or faster.  Reduce-only: one vector with the two-CTA budget (at 4 ranks 62
+    // registers instead of 40: four CTAs per SM instead of six) is the fastest or level at
+    // every rank count up to 16, 14-17 % ahead of no bound at 8 and 16 ranks.
 #define ZERO_CASE(NV, UV, BV) \
     case NV: \
         if constexpr (kFused) \
