@@ -477,14 +477,17 @@ zero_status zero_set_impl(zero_layout *layout, int32_t impl);
  * pages. */
 zero_status zero_set_max_ctas(zero_layout *layout, int32_t max_ctas);
 
-/* Grid of the all-gather copies (zero_allgather, zero_gather_unit, and the gather inside
- * the stage-3 steps): 0 (the default) = a grid of short blocks over the whole range, the
- * fastest when a gather has the GPU to itself; k > 0 = k persistent CTAs, each moving
- * 48 KB chunks global -> shared -> global with bulk copies (~144 KB of loads in flight;
- * bounded waits report ZERO_ERR_TIMEOUT through zero_get_error), so that a gather
- * occupies at most k SMs and can run beside a layer's compute that leaves those SMs free (P1 ZeRO-3: the next layer's
- * parameters are gathered while the current layer computes).  Results are identical for
- * every k.  Negative k: ZERO_ERR_INVALID.  No counterpart on the pages. */
+/* Grid of the all-gather copies (zero_allgather, zero_gather_unit, zero_gather_unit_ranks
+ * and the gather inside the stage-3 steps): 0 (the default) = a grid of short blocks over
+ * the whole range, the fastest when a gather has the GPU to itself; k > 0 = k persistent
+ * CTAs, so that a gather occupies at most k SMs and can run beside a layer's compute that
+ * leaves those SMs free (P1 ZeRO-3: the next layer's parameters are gathered while the
+ * current layer computes).  The copies of this GPU's memory then move 48 KB chunks
+ * global -> shared -> global with bulk copies (~144 KB of loads in flight; bounded waits
+ * report ZERO_ERR_TIMEOUT through zero_get_error); the gather from the ranks' shards
+ * (zero_gather_unit_ranks, possibly peers' memory) deals its blocks of 16-byte loads to
+ * the k CTAs by a grid stride.  Results are identical for every k.  Negative k:
+ * ZERO_ERR_INVALID.  No counterpart on the pages. */
 zero_status zero_set_gather_ctas(zero_layout *layout, int32_t max_ctas);
 
 /* Test hook of the bulk-copy pipeline's bounded waits: every in-kernel wait gives up

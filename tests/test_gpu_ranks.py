@@ -121,10 +121,13 @@ def test_copy_shard_copies_exactly_the_shard():
     ((4096, 8192, 40_960, 8), 4, 8, (0, 1, 2, 3)),     # vector path, units across shard edges
     ((1000,) * 16, 16, 8, tuple(range(16))),
 ])
-def test_gather_unit_ranks_matches_oracle(tensors, N, A, units):
+@pytest.mark.parametrize("gather_ctas", [0, 1, 3])
+def test_gather_unit_ranks_matches_oracle(tensors, N, A, units, gather_ctas):
+    """gather_ctas 0: a grid of short blocks; k > 0: k persistent CTAs (grid stride)."""
     wl = Workload(name="gather_ranks", description="stage-3 gather from per-rank shards", tensors=tuple(tensors),
                   units=tuple(units), n_ranks=N, stage=3, bucket_elems=0, steps=2, loss_scale=1024.0, pad_align=A)
     lay, whole, ref = _stepped(wl)
+    lay.set_gather_ctas(gather_ctas)
     S_ = lay.shard
     shards = [whole[k * S_:(k + 1) * S_].clone() for k in range(N)]          # one allocation per rank
     _, _, _, u = lay.tables()
@@ -194,6 +197,26 @@ def _ipc_worker(rank, world, port, wl, steps, out):
             rs.gather_unit(j, buf)
             full[int(lo):int(hi)] = buf
         torch.cuda.synchronize()
+        # the same layers through the prefetching schedule over the owners' shards, with its
+        # gather width tuned per kind of pass (four forward and four backward passes: an
+        # untimed one, one per candidate width, then the chosen width)
+        seen = torch.zeros_like(full)
+        width = int(max(hi - lo for lo, hi in units))
+        pf = rs.prefetch([torch.zeros(width, dtype=torch.int16, device="cuda") for _ in range(2)],
+                         torch.cuda.Stream(), torch.cuda.Stream(), candidates=(1, 4), trials=1)
+
+        def layer(unit, buf):
+            lo, hi = int(units[unit][0]), int(units[unit][1])
+            seen[lo:hi].copy_(buf[:hi - lo])
+
+        for _ in range(4):
+            seen.zero_()
+            torch.cuda.synchronize()               # the layers write `seen` on the compute stream
+            pf.forward(layer)
+            pf.backward(layer)
+            torch.cuda.synchronize()
+            assert torch.equal(seen, full), "prefetched layers differ from the gathered ones"
+        assert all(w.chosen is not None for w in pf.widths.values())
     rs.close()
     out.put((rank, mk.cpu().numpy(), m1.cpu().numpy(), v1.cpu().numpy(), full.cpu().numpy().view(np.uint16)))
     dist.destroy_process_group()

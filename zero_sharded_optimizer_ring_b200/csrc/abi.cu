@@ -322,7 +322,7 @@ extern "C" zero_status zero_gather_unit_ranks(const zero_layout *L, int64_t unit
     if (!aligned16(dst)) return ZERO_ERR_ALIGN;
     const int64_t lo = L->unit_lo[(size_t)unit];
     return cuda_status(zero::launch_gather_ranks(src, L->shard, lo, L->unit_hi[(size_t)unit] - lo, dst,
-                                                 (cudaStream_t)stream));
+                                                 L->gather_ctas, (cudaStream_t)stream));
 }
 
 namespace {

@@ -10,8 +10,9 @@ struct ShardPtrs {
     const uint16_t *rank[kMaxBulkRanks];
 };
 
-// dst[j] = element lo + j of the flat buffer whose shard k (S elements) is src.rank[k]
+// dst[j] = element lo + j of the flat buffer whose shard k (S elements) is src.rank[k];
+// max_ctas > 0: at most that many persistent CTAs (0: a grid of short blocks)
 cudaError_t launch_gather_ranks(const ShardPtrs &src, int64_t S, int64_t lo, int64_t n, uint16_t *dst,
-                                cudaStream_t s);
+                                int32_t max_ctas, cudaStream_t s);
 
 }  // namespace zero

@@ -390,40 +390,48 @@ gather_unit_kernel(const uint16_t *__restrict__ src, int64_t lo, int64_t n, uint
 // Gather of one unit from the ranks' shard buffers: dst[j] = shard k's element lo + j - kS,
 // k = (lo + j) / S, where rank k's buffer holds flat elements [kS, (k+1)S) (on this GPU or a
 // peer's).  With lo and S multiples of 8 no 16-byte vector straddles two shards, so each
-// thread moves 4 vectors, every source and destination 16-byte aligned; otherwise each
-// thread moves 8 scalars.  A grid of short blocks, as for the copy.
+// thread moves 4 vectors per block of work, every source and destination 16-byte aligned;
+// otherwise each thread moves 8 scalars.  Blocks of work are dealt to the CTAs by a grid
+// stride: a grid of one CTA per block of work (short blocks, as for the copy), or a few
+// persistent CTAs (zero_set_gather_ctas) that leave the other SMs to concurrent work.
 __global__ void __launch_bounds__(kThreads)
 gather_ranks_kernel(const __grid_constant__ ShardPtrs src, int64_t S, int64_t lo, int64_t n,
                     uint16_t *__restrict__ dst)
 {
     if ((lo & 7) == 0 && (S & 7) == 0) {
         const int64_t nv = n / kVec;
-        const int64_t base = (int64_t)blockIdx.x * kThreads * kCopyUnroll;
-        uint4 x[kCopyUnroll];
+        const int64_t per = (int64_t)kThreads * kCopyUnroll;              // vectors per block of work
+        for (int64_t blk = blockIdx.x; blk * per < nv; blk += gridDim.x) {
+            const int64_t base = blk * per;
+            uint4 x[kCopyUnroll];
 #pragma unroll
-        for (int u = 0; u < kCopyUnroll; ++u) {
-            const int64_t q = base + (int64_t)u * kThreads + threadIdx.x;
-            if (q < nv) {
-                const int64_t i = lo + q * kVec, k = i / S;
-                x[u] = *reinterpret_cast<const uint4 *>(src.rank[k] + (i - k * S));
+            for (int u = 0; u < kCopyUnroll; ++u) {
+                const int64_t q = base + (int64_t)u * kThreads + threadIdx.x;
+                if (q < nv) {
+                    const int64_t i = lo + q * kVec, k = i / S;
+                    x[u] = *reinterpret_cast<const uint4 *>(src.rank[k] + (i - k * S));
+                }
             }
-        }
 #pragma unroll
-        for (int u = 0; u < kCopyUnroll; ++u) {
-            const int64_t q = base + (int64_t)u * kThreads + threadIdx.x;
-            if (q < nv) *reinterpret_cast<uint4 *>(dst + q * kVec) = x[u];
+            for (int u = 0; u < kCopyUnroll; ++u) {
+                const int64_t q = base + (int64_t)u * kThreads + threadIdx.x;
+                if (q < nv) *reinterpret_cast<uint4 *>(dst + q * kVec) = x[u];
+            }
         }
         if (blockIdx.x == 0 && threadIdx.x < n - nv * kVec) {
             const int64_t j = nv * kVec + threadIdx.x, i = lo + j, k = i / S;
             dst[j] = src.rank[k][i - k * S];
         }
     } else {
-        const int64_t base = (int64_t)blockIdx.x * kThreads * kCopyUnroll * kVec;
-        for (int u = 0; u < kCopyUnroll * kVec; ++u) {
-            const int64_t j = base + (int64_t)u * kThreads + threadIdx.x;
-            if (j < n) {
-                const int64_t i = lo + j, k = i / S;
-                dst[j] = src.rank[k][i - k * S];
+        const int64_t per = (int64_t)kThreads * kCopyUnroll * kVec;      // elements per block of work
+        for (int64_t blk = blockIdx.x; blk * per < n; blk += gridDim.x) {
+            const int64_t base = blk * per;
+            for (int u = 0; u < kCopyUnroll * kVec; ++u) {
+                const int64_t j = base + (int64_t)u * kThreads + threadIdx.x;
+                if (j < n) {
+                    const int64_t i = lo + j, k = i / S;
+                    dst[j] = src.rank[k][i - k * S];
+                }
             }
         }
     }
@@ -560,11 +568,13 @@ cudaError_t launch_gather_unit(const uint16_t *src, int64_t lo, int64_t n, uint1
 }
 
 cudaError_t launch_gather_ranks(const ShardPtrs &src, int64_t S, int64_t lo, int64_t n, uint16_t *dst,
-                                cudaStream_t s)
+                                int32_t max_ctas, cudaStream_t s)
 {
     if (n <= 0) return cudaSuccess;
     const int64_t per_block = (int64_t)kThreads * kCopyUnroll * kVec;
-    gather_ranks_kernel<<<(unsigned)((n + per_block - 1) / per_block), kThreads, 0, s>>>(src, S, lo, n, dst);
+    int64_t grid = (n + per_block - 1) / per_block;
+    if (max_ctas > 0 && grid > max_ctas) grid = max_ctas;
+    gather_ranks_kernel<<<(unsigned)grid, kThreads, 0, s>>>(src, S, lo, n, dst);
     return cudaGetLastError();
 }
 

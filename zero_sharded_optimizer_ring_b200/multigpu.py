@@ -217,6 +217,12 @@ class RankStep:
             self.ops.wait(ev, ("updated", r), stream)
         self.ops.gather_unit_ranks(self.layout, unit, self.peer_p16[self.cur], dst, stream)
 
+    def prefetch(self, slots, gather_stream, compute_stream, **kw):
+        """Stage 3: a schedule.Zero3Prefetch whose gathers are this rank's gather_unit
+        (every owner's shard; the gather width tuned per kind of pass as on one GPU)."""
+        from .schedule import Zero3Prefetch
+        return Zero3Prefetch(self.layout, None, slots, gather_stream, compute_stream, gather=self.gather_unit, **kw)
+
     def close(self):
         """Unmap the peers' buffers (before the process group or the buffers go away)."""
         self._barrier()

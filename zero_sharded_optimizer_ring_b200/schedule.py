@@ -127,19 +127,19 @@ class Zero3Prefetch:
     GatherWidth per kind of pass, kept across steps.  forward() and backward() run
     zero3_pass over the units in ascending and descending order with that kind's width;
     the widths settle on their own over the first steps (candidates x trials + 1 passes
-    of each kind)."""
+    of each kind).  `gather` as for zero3_pass (one GPU per rank: RankStep.prefetch)."""
 
     def __init__(self, layout, p16_shard, slots, gather_stream, compute_stream, candidates=(14, 16, 18, 20),
-                 trials=3, matmul_sm_carveout=MATMUL_SM_CARVEOUT, blas=MATMUL_BLAS):
+                 trials=3, matmul_sm_carveout=MATMUL_SM_CARVEOUT, blas=MATMUL_BLAS, gather=None):
         self.layout, self.p16_shard, self.slots = layout, p16_shard, list(slots)
         self.gather_stream, self.compute_stream = gather_stream, compute_stream
         self.widths = {"forward": GatherWidth(candidates, trials), "backward": GatherWidth(candidates, trials)}
-        self.matmul_sm_carveout, self.blas = matmul_sm_carveout, blas
+        self.matmul_sm_carveout, self.blas, self.gather = matmul_sm_carveout, blas, gather
 
     def _run(self, kind, units, compute):
         return zero3_pass(self.layout, self.p16_shard, self.slots, units, compute, self.gather_stream,
                           self.compute_stream, gather_ctas=self.widths[kind],
-                          matmul_sm_carveout=self.matmul_sm_carveout, blas=self.blas)
+                          matmul_sm_carveout=self.matmul_sm_carveout, blas=self.blas, gather=self.gather)
 
     def forward(self, compute, units=None):
         """The forward pass: units ascending (default: all of the layout's)."""
@@ -151,7 +151,7 @@ class Zero3Prefetch:
 
 
 def zero3_pass(layout, p16_shard, slots, units, compute, gather_stream, compute_stream,
-               gather_ctas=GATHER_CTAS, matmul_sm_carveout=MATMUL_SM_CARVEOUT, blas=MATMUL_BLAS):
+               gather_ctas=GATHER_CTAS, matmul_sm_carveout=MATMUL_SM_CARVEOUT, blas=MATMUL_BLAS, gather=None):
     """Run one pass over `units` (a forward pass: ascending; a backward pass: descending).
 
     Unit units[j] is gathered into slots[j % len(slots)] on gather_stream, once the slot's
@@ -163,12 +163,18 @@ def zero3_pass(layout, p16_shard, slots, units, compute, gather_stream, compute_
     and so take the whole GPU; torch's matmuls run with the SM-count target
     matmul_sm_carveout below the SM count and prefer `blas` (None: unchanged); every
     setting is restored afterwards.  The first gathers wait for the work already on
-    compute_stream (an earlier pass's layers may still read the slots).  Returns the list
+    compute_stream (an earlier pass's layers may still read the slots).  gather(unit, dst,
+    stream) enqueues a unit's parameters into dst (default: zero_gather_unit from
+    p16_shard; with one GPU per rank, RankStep.gather_unit, which reads every owner's
+    shard and honours the same gather width).  Returns the list
     of (gather started, gathered, computed) torch.cuda.Event triples, one per unit (timing
     events: layer_breakdown reads them)."""
     import torch
     n = len(slots)
     marks = []
+    if gather is None:
+        def gather(unit, dst, stream):
+            gather_unit(layout, unit, p16_shard, dst, stream=stream)
     width = gather_ctas if isinstance(gather_ctas, GatherWidth) else None
     if width is not None:
         gather_ctas = width.begin_pass()
@@ -186,7 +192,7 @@ def zero3_pass(layout, p16_shard, slots, units, compute, gather_stream, compute_
                     # the first n gathers have no layer compute to share the GPU with
                     layout.set_gather_ctas(0 if j < n else gather_ctas)
                 started.record(gather_stream)
-                gather_unit(layout, u, p16_shard, slots[j % n], stream=gather_stream)
+                gather(u, slots[j % n], gather_stream)
                 gathered.record(gather_stream)
                 compute_stream.wait_event(gathered)
                 with torch.cuda.stream(compute_stream):
