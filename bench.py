@@ -43,7 +43,8 @@ KERNEL_SOURCES = {tag: [os.path.join(_CSRC, f) for f in files] for tag, files in
 }.items()}
 
 
-def parse():
+def parse(argv=None):
+    """The command line (argv: a list in place of sys.argv[1:])."""
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=400)
@@ -113,7 +114,7 @@ def parse():
     ap.add_argument("--psi", type=int, default=0,
                     help="flat workloads only: run the same shape with this many parameters "
                          "(small cases for profiler captures; not a bench line)")
-    a = ap.parse_args()
+    a = ap.parse_args(argv)
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")
     return a

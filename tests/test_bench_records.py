@@ -96,3 +96,16 @@ def test_record_without_both_dram_metrics_is_refused(sources, tmp_path):
     wl = reduced_workloads()["flat1p3b_n4_zero1"]
     with pytest.raises(SystemExit):
         _record(tmp_path, wl, kernel="other_kernel")
+
+
+def test_default_run_times_both_roofline_workloads():
+    """The plain `bench.py` run adds the Llama-shaped ZeRO-3 list to the flat headline in
+    the same JSON line; variant runs and explicit --also choices do not."""
+    a = bench.parse([])
+    assert a.workload == bench.DEFAULT_WORKLOAD == "flat1p3b_n4_zero1"
+    assert bench.also_workloads(a) == ["llama3b_n8_zero3"]
+    for extra in (["--kernel", "1"], ["--wire-fp16"], ["--psi", "1048576"], ["--also", "none"],
+                  ["--workload", "gpt2_small_n8_zero2"]):
+        assert bench.also_workloads(bench.parse(extra)) == [], extra
+    assert bench.also_workloads(bench.parse(["--also", "gpt2_small_n8_zero2"])) == [
+        "gpt2_small_n8_zero2"]
